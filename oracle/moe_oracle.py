@@ -1,0 +1,282 @@
+"""CPU oracle of the MoE layer forward path (router -> grouping -> SwiGLU experts -> combine).
+
+TEST INFRASTRUCTURE ONLY. Only the test suite, the smoke check in ``__graft_entry__`` and the
+CPU-baseline leg of ``bench.py`` may import this module. The CUDA library never calls it, and
+it shares no code, table or constant with the CUDA sources.
+
+Everything here is plain NumPy in float64 (a matmul and a stable sort are the only library
+primitives used as steps). Inputs arrive as NumPy arrays whose values are exactly the values the
+GPU sees (bf16 values are passed widened to float32, which is exact).
+
+Sources, cited by page title and section:
+
+* [P1] "MoE 模型的 FlashAttention 跟普通模型有什么不一样？" (framerc.cn)
+  - section "FlashAttention 在 MoE 模型里的位置": the five-step flow (route top-k, group tokens
+    by expert, per-expert FFN, merge weighted by the routing weights).
+  - section "融合二：expert 计算的输出 + 合并结果": merge is ``accum += route_weight * expert_output``.
+  - section "手动编译 MoE 融合算子": router weight ``[hidden_dim, num_experts]``, expert weights
+    stacked with a leading expert dimension, ``activation="silu"``.
+* [P4] "MoE Router" on Ascend CANN (2048ai.net)
+  - section "Router 就是一个小型网络": gate = Linear(hidden, E, bias=False); softmax over all E;
+    torch.topk; divide the k selected weights by their sum.
+  - section "昇腾NPU的通信计算重叠": capacity C = (total tokens / E) x 1.25; assignments beyond
+    C are dropped and take the residual path (contribute nothing to the MoE output).
+* [P5] "大模型推理加速200%+？这套国产融合算子库把CUDA/Triton全替换了" (csdn.net)
+  - section "3.1 Moe Fuse Gate & Softmax TopK": exp only over the selected k, which equals the
+    renormalised full softmax in exact arithmetic.
+
+Readings taken where the pages are silent or disagree (each also listed in the design notes):
+
+* "total tokens" in the capacity formula counts assignments, T*k (the preceding section of [P4]
+  counts T*k expert accesses); C = ceil(cf*T*k/E), computed exactly, capped at T; cf <= 0 means
+  no capacity limit (C = T).
+* Drops go in token order: the earliest tokens keep their slot. Survivors are not renormalised;
+  a dropped assignment contributes 0, a fully dropped token has output 0.
+* Top-k ranks float32 logits (softmax is monotone); equal logits (including -0 vs +0) go to the
+  lower expert index; the k indices are listed by descending logit, then ascending index.
+* SwiGLU expert: y = (silu(x Wg) * (x Wu)) Wd, silu(z) = z / (1 + exp(-z)); experts have no bias.
+
+Every function below is pinned by tests that do not re-run its own formula (brute force,
+closed forms, hand-worked fixtures under tests/golden, special cases reducing to a dense FFN).
+"""
+from __future__ import annotations
+
+import math
+from fractions import Fraction
+
+import numpy as np
+
+__all__ = [
+    "router_logits",
+    "select_topk",
+    "route_weights",
+    "route",
+    "capacity",
+    "align",
+    "swiglu_expert",
+    "grouped_ffn_slots",
+    "combine",
+    "layer_forward",
+]
+
+
+def router_logits(x, w_router, logit_bias=None):
+    """Gate logits l[t,e] = sum_h x[t,h] * Wr[h,e] (+ bias[e]), float64, rounded once to float32.
+
+    [P4] "Router 就是一个小型网络": the gate is a bias-free Linear(hidden, E). The optional
+    per-expert bias is an input of the skewed-load workload (not a learned gate bias).
+    """
+    x64 = np.asarray(x, dtype=np.float64)
+    w64 = np.asarray(w_router, dtype=np.float64)
+    logits = x64 @ w64
+    if logit_bias is not None:
+        logits = logits + np.asarray(logit_bias, dtype=np.float64)[None, :]
+    return logits.astype(np.float32)
+
+
+def select_topk(logits, k):
+    """Indices of the k largest float32 logits per row, ordered by (logit desc, index asc).
+
+    [P4] "Router 就是一个小型网络" (torch.topk over the softmax scores; softmax is monotone so
+    ranking logits ranks scores). A stable sort on the negated logits keeps equal values in
+    ascending expert order, which is the tie rule.
+    """
+    l32 = np.asarray(logits, dtype=np.float32)
+    if k < 1 or k > l32.shape[1]:
+        raise ValueError("need 1 <= k <= E")
+    order = np.argsort(-l32, axis=1, kind="stable")
+    return order[:, :k].astype(np.int32)
+
+
+def route_weights(logits, topk_idx):
+    """Renormalised routing weights, float64.
+
+    [P4] "Router 就是一个小型网络": p = softmax(l) over all E experts, then the k selected
+    probabilities are divided by their sum so that they add to 1.
+    """
+    l64 = np.asarray(logits, dtype=np.float32).astype(np.float64)
+    m = l64.max(axis=1, keepdims=True)
+    p = np.exp(l64 - m)
+    p = p / p.sum(axis=1, keepdims=True)
+    sel = np.take_along_axis(p, np.asarray(topk_idx, dtype=np.int64), axis=1)
+    return sel / sel.sum(axis=1, keepdims=True)
+
+
+def route(x, w_router, k, logit_bias=None, logits=None):
+    """Router step: returns (logits f32 [T,E], topk_idx i32 [T,k], topk_w f64 [T,k])."""
+    if logits is None:
+        logits = router_logits(x, w_router, logit_bias)
+    idx = select_topk(logits, k)
+    return np.asarray(logits, dtype=np.float32), idx, route_weights(logits, idx)
+
+
+def capacity(T, k, E, capacity_factor):
+    """Per-expert capacity C = ceil(cf * T * k / E), exact rational arithmetic, capped at T.
+
+    [P4] "昇腾NPU的通信计算重叠": C = (total_tokens / num_experts) x 1.25, with total tokens read
+    as the T*k assignments. cf is taken as the float32 value the C ABI receives. cf <= 0: no limit.
+    """
+    cf = Fraction(float(np.float32(capacity_factor)))
+    if cf <= 0:
+        return int(T)
+    c = math.ceil(cf * int(T) * int(k) / int(E))
+    return int(min(c, int(T)))
+
+
+def align(topk_idx, E, C):
+    """Capacity-limited grouping of assignments by expert, token order first.
+
+    [P1] "FlashAttention 在 MoE 模型里的位置" step 3 (pick the tokens that go to the same
+    expert) and [P4] "昇腾NPU的通信计算重叠" (at most C per expert, overflow dropped).
+
+    Assignment a = t*k + j goes to expert idx[t,j]. Its rank is the number of earlier
+    assignments (smaller t) to the same expert. Kept iff rank < C.
+
+    Returns dict with counts [E], offsets [E+1], sorted_ids [T*k] (slot -> a, -1 past the kept
+    total), slot_of [T*k] (a -> slot or -1), drop_mask [T*k] (1 = dropped), raw [E], rank [T*k].
+    """
+    idx = np.asarray(topk_idx, dtype=np.int64)
+    T, k = idx.shape
+    A = T * k
+    seen = [0] * E
+    rank = [0] * A
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            rank[t * k + j] = seen[e]
+            seen[e] += 1
+    counts = [min(r, C) for r in seen]
+    offsets = [0]
+    for e in range(E):
+        offsets.append(offsets[-1] + counts[e])
+    sorted_ids = np.full(A, -1, dtype=np.int32)
+    slot_of = np.full(A, -1, dtype=np.int32)
+    drop_mask = np.zeros(A, dtype=np.uint8)
+    for t in range(T):
+        for j in range(k):
+            a = t * k + j
+            e = int(idx[t, j])
+            if rank[a] < C:
+                slot = offsets[e] + rank[a]
+                sorted_ids[slot] = a
+                slot_of[a] = slot
+            else:
+                drop_mask[a] = 1
+    return {
+        "counts": np.asarray(counts, dtype=np.int32),
+        "offsets": np.asarray(offsets, dtype=np.int32),
+        "sorted_ids": sorted_ids,
+        "slot_of": slot_of,
+        "drop_mask": drop_mask,
+        "raw": np.asarray(seen, dtype=np.int64),
+        "rank": np.asarray(rank, dtype=np.int64),
+    }
+
+
+def swiglu_expert(x_rows, w_gate_e, w_up_e, w_down_e):
+    """One expert's FFN on a block of rows: (silu(x Wg) * (x Wu)) Wd, all in float64.
+
+    [P1] "手动编译 MoE 融合算子" (activation="silu", weights [hidden, ffn] per expert);
+    silu(z) = z * sigmoid(z) = z / (1 + exp(-z)).
+    """
+    xr = np.asarray(x_rows, dtype=np.float64)
+    g = xr @ np.asarray(w_gate_e, dtype=np.float64)
+    u = xr @ np.asarray(w_up_e, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        h = g * u / (1.0 + np.exp(-g))
+    return h @ np.asarray(w_down_e, dtype=np.float64)
+
+
+def grouped_ffn_slots(x, sorted_ids, offsets, k, w_gate, w_up, w_down, slots=None):
+    """Expert output per kept slot: y[s] = expert_e(x[sorted_ids[s] // k]) for s in expert e's range.
+
+    [P1] "FlashAttention 在 MoE 模型里的位置" step 4. ``w_*`` may be arrays or any object whose
+    ``[e]`` returns expert e's matrix. ``slots`` restricts the evaluation to a subset (returned
+    as a dict slot -> row); by default every kept slot is evaluated into a [A_kept, H] array.
+    """
+    offsets = np.asarray(offsets, dtype=np.int64)
+    E = len(offsets) - 1
+    sorted_ids = np.asarray(sorted_ids, dtype=np.int64)
+    x = np.asarray(x)
+    want = None if slots is None else set(int(s) for s in slots)
+    result = {}
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        sl = [s for s in range(lo, hi) if want is None or s in want]
+        if not sl:
+            continue
+        toks = sorted_ids[sl] // k
+        y = swiglu_expert(x[toks], w_gate[e], w_up[e], w_down[e])
+        for i, s in enumerate(sl):
+            result[s] = y[i]
+    if slots is not None:
+        return result
+    a_kept = int(offsets[-1])
+    H = np.asarray(w_down[0]).shape[1] if a_kept else 0
+    out = np.zeros((a_kept, H), dtype=np.float64)
+    for s, row in result.items():
+        out[s] = row
+    return out
+
+
+def combine(y_slots, slot_of, topk_w, tokens=None):
+    """Weighted merge back to token order: out[t] = sum_{kept j} w[t,j] * y[slot_of[t*k+j]].
+
+    [P1] "融合二：expert 计算的输出 + 合并结果" (accum += route_weight * expert_output).
+    A dropped assignment (slot -1) contributes nothing; a fully dropped token gives 0.
+    ``y_slots`` may be an array or a dict slot -> row.
+    """
+    w = np.asarray(topk_w, dtype=np.float64)
+    T, k = w.shape
+    slot_of = np.asarray(slot_of, dtype=np.int64).reshape(T, k)
+    toks = range(T) if tokens is None else tokens
+    H = None
+    rows = {}
+    for t in toks:
+        acc = None
+        for j in range(k):
+            s = int(slot_of[t, j])
+            if s < 0:
+                continue
+            y = np.asarray(y_slots[s], dtype=np.float64)
+            acc = w[t, j] * y if acc is None else acc + w[t, j] * y
+            H = y.shape[0]
+        rows[t] = acc
+    if H is None:
+        H = np.asarray(y_slots[0]).shape[-1] if len(y_slots) else 0
+    out = np.zeros((len(rows), H), dtype=np.float64)
+    for i, t in enumerate(toks):
+        if rows[t] is not None:
+            out[i] = rows[t]
+    return out
+
+
+def layer_forward(x, w_router, w_gate, w_up, w_down, k, capacity_factor,
+                  logit_bias=None, logits=None, tokens=None):
+    """Whole MoE layer: route -> align -> experts -> combine, float64 throughout.
+
+    [P1] "FlashAttention 在 MoE 模型里的位置" steps 2-5. ``logits`` (float32) may be supplied
+    to route from given gate logits. ``tokens`` restricts the expert FFN and the combine to a
+    subset of tokens (routing and capacity still see every token, since ranks depend on all).
+    Returns dict with out [len(tokens) or T, H] and all routing intermediates.
+    """
+    x = np.asarray(x)
+    T = x.shape[0]
+    logits, idx, w = route(x, w_router, k, logit_bias=logit_bias, logits=logits)
+    E = logits.shape[1]
+    C = capacity(T, k, E, capacity_factor)
+    al = align(idx, E, C)
+    tok_list = list(range(T)) if tokens is None else [int(t) for t in tokens]
+    need = set()
+    for t in tok_list:
+        for j in range(k):
+            s = int(al["slot_of"][t * k + j])
+            if s >= 0:
+                need.add(s)
+    y = grouped_ffn_slots(x, al["sorted_ids"], al["offsets"], k, w_gate, w_up, w_down,
+                          slots=sorted(need))
+    out = combine(y, al["slot_of"], w, tokens=tok_list)
+    res = dict(al)
+    res.update({"logits": logits, "topk_idx": idx, "topk_w": w, "C": C, "out": out,
+                "tokens": tok_list})
+    return res

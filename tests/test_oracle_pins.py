@@ -1,0 +1,308 @@
+"""Pins for the CPU oracle: each check rests on something other than the oracle's own formula
+(brute force, closed forms, hand-worked fixtures, textbook special cases)."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as orc
+from expert_dispatch_gate_b200 import workloads as wlm
+
+
+def _load(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- router logits
+
+def test_router_logits_match_scalar_dot_products():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((5, 7)).astype(np.float32)
+    w = rng.standard_normal((7, 3)).astype(np.float32)
+    b = rng.standard_normal(3).astype(np.float32)
+    got = orc.router_logits(x, w, b)
+    assert got.dtype == np.float32 and got.shape == (5, 3)
+    for t in range(5):
+        for e in range(3):
+            ref = math.fsum(float(x[t, h]) * float(w[h, e]) for h in range(7)) + float(b[e])
+            assert got[t, e] == np.float32(ref)
+
+
+# ---------------------------------------------------------------- top-k selection
+
+def _valid_topk_sets(l, k):
+    """Every k-subset S with: for i in S, j not in S, l_i > l_j or (l_i == l_j and i < j)."""
+    E = len(l)
+    found = []
+    for S in itertools.combinations(range(E), k):
+        ok = all((l[i] > l[j]) or (l[i] == l[j] and i < j)
+                 for i in S for j in range(E) if j not in S)
+        if ok:
+            found.append(set(S))
+    return found
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_brute_force_with_ties(seed):
+    rng = np.random.default_rng(seed)
+    for E in range(1, 8):
+        for k in range(1, E + 1):
+            l = rng.integers(-2, 3, size=(6, E)).astype(np.float32) * 0.5
+            # plant signed zeros
+            l[rng.random(l.shape) < 0.2] = -0.0
+            idx = orc.select_topk(l, k)
+            for t in range(l.shape[0]):
+                sets = _valid_topk_sets(list(l[t]), k)
+                assert len(sets) == 1
+                assert set(idx[t].tolist()) == sets[0]
+                # listed by descending logit, then ascending index
+                for a, b in zip(idx[t][:-1], idx[t][1:]):
+                    assert l[t, a] > l[t, b] or (l[t, a] == l[t, b] and a < b)
+
+
+def test_topk_is_max_sum_subset_for_distinct_logits():
+    rng = np.random.default_rng(7)
+    for _ in range(20):
+        E = int(rng.integers(2, 9))
+        k = int(rng.integers(1, E + 1))
+        l = rng.permutation(E).astype(np.float32) + rng.random(E).astype(np.float32) * 0.1
+        best = max(itertools.combinations(range(E), k), key=lambda S: sum(float(l[i]) for i in S))
+        assert set(orc.select_topk(l[None, :], k)[0].tolist()) == set(best)
+
+
+def test_routing_golden(golden_dir):
+    g = _load(golden_dir, "routing_tiny.json")
+    logits = np.asarray(g["logits"], dtype=np.float32)
+    # the fixture's -0.0 must survive json
+    assert math.copysign(1.0, float(logits[2, 1])) == -1.0
+    _, idx, w = orc.route(None, None, g["k"], logits=logits)
+    assert idx.tolist() == g["topk_idx"]
+    np.testing.assert_allclose(w, np.asarray(g["topk_w"]), atol=g["tolerance"], rtol=0)
+
+
+# ---------------------------------------------------------------- routing weights
+
+def test_weights_sum_to_one_and_k1_is_exactly_one():
+    l = wlm.random_logits(200, 16, seed=3).numpy()
+    for k in (1, 2, 5, 16):
+        idx = orc.select_topk(l, k)
+        w = orc.route_weights(l, idx)
+        assert np.all(w > 0)
+        np.testing.assert_allclose(w.sum(axis=1), 1.0, atol=1e-14, rtol=0)
+        if k == 1:
+            assert np.all(w == 1.0)
+
+
+def test_weights_two_experts_logistic_closed_form():
+    rng = np.random.default_rng(11)
+    l = (rng.standard_normal((50, 2)) * 3).astype(np.float32)
+    idx = orc.select_topk(l, 2)
+    w = orc.route_weights(l, idx)
+    for t in range(50):
+        a, b = idx[t]
+        da = float(l[t, a]) - float(l[t, b])
+        assert abs(w[t, 0] - 1.0 / (1.0 + math.exp(-da))) < 1e-14
+        assert abs(w[t, 1] - 1.0 / (1.0 + math.exp(da))) < 1e-14
+
+
+def test_weights_ratio_and_independence_from_unselected():
+    rng = np.random.default_rng(12)
+    l = rng.standard_normal((40, 12)).astype(np.float32)
+    idx = orc.select_topk(l, 4)
+    w = orc.route_weights(l, idx)
+    # w_i / w_j = exp(l_i - l_j) for selected i, j
+    for t in range(40):
+        for a in range(4):
+            for b in range(4):
+                r = w[t, a] / w[t, b]
+                assert abs(r - math.exp(float(l[t, idx[t, a]]) - float(l[t, idx[t, b]]))) < 1e-12 * max(1, r)
+    # lowering an unselected logit changes the full softmax but not the renormalised weights
+    l2 = l.copy()
+    for t in range(40):
+        for e in range(12):
+            if e not in idx[t]:
+                l2[t, e] -= 3.0
+    idx2 = orc.select_topk(l2, 4)
+    assert np.array_equal(idx, idx2)
+    np.testing.assert_allclose(orc.route_weights(l2, idx2), w, atol=1e-14, rtol=0)
+
+
+def test_routing_shift_invariance():
+    l = wlm.random_logits(100, 32, seed=5).numpy()
+    idx = orc.select_topk(l, 6)
+    w = orc.route_weights(l, idx)
+    l2 = (l.astype(np.float64) + 0.5).astype(np.float32)  # exact: |l| < 8, step 2^-20
+    assert np.array_equal(orc.select_topk(l2, 6), idx)
+    np.testing.assert_allclose(orc.route_weights(l2, idx), w, atol=1e-6, rtol=0)
+
+
+# ---------------------------------------------------------------- capacity
+
+def test_capacity_golden(golden_dir):
+    g = _load(golden_dir, "capacity_cases.json")
+    for c in g["cases"]:
+        assert orc.capacity(c["T"], c["k"], c["E"], c["cf"]) == c["C"], c
+
+
+# ---------------------------------------------------------------- align
+
+def test_align_golden(golden_dir):
+    g = _load(golden_dir, "align_tiny.json")
+    al = orc.align(np.asarray(g["topk_idx"]), g["E"], g["C"])
+    for key in ("counts", "offsets", "sorted_ids", "slot_of", "drop_mask"):
+        assert al[key].tolist() == g[key], key
+
+
+def _check_align_invariants(idx, E, C, al):
+    T, k = idx.shape
+    A = T * k
+    counts, offsets = al["counts"], al["offsets"]
+    sid, slot_of, drop = al["sorted_ids"], al["slot_of"], al["drop_mask"]
+    raw = np.bincount(idx.reshape(-1), minlength=E)
+    assert np.array_equal(counts, np.minimum(raw, C))
+    assert np.all(counts <= C)
+    assert offsets[0] == 0 and np.array_equal(np.diff(offsets), counts)
+    kept = int(offsets[-1])
+    assert kept == A - int(drop.sum())
+    # bijection between slots [0, kept) and kept assignments
+    assert np.all(sid[kept:] == -1)
+    assert sorted(sid[:kept].tolist()) == sorted(np.nonzero(drop == 0)[0].tolist())
+    for s in range(kept):
+        assert slot_of[sid[s]] == s
+    assert np.all((slot_of == -1) == (drop == 1))
+    # each slot sits inside its expert's range
+    flat = idx.reshape(-1)
+    for s in range(kept):
+        e = flat[sid[s]]
+        assert offsets[e] <= s < offsets[e + 1]
+    # token order, checked by listing each expert's tokens: the first C of them are kept,
+    # in ascending token order
+    for e in range(E):
+        toks = [a for a in range(A) if flat[a] == e]
+        keep = toks[:C]
+        assert sid[offsets[e]:offsets[e + 1]].tolist() == keep
+        assert all(drop[a] == 1 for a in toks[C:])
+
+
+@pytest.mark.parametrize("mode", ["uniform", "zipf", "one"])
+def test_align_invariants(mode):
+    for (T, E, k, cf) in [(50, 8, 2, 1.25), (97, 16, 4, 1.0), (64, 4, 4, 0.0), (33, 64, 6, 1.25)]:
+        idx = wlm.random_topk_idx(T, E, k, seed=T + E, mode=mode).numpy()
+        C = orc.capacity(T, k, E, cf)
+        al = orc.align(idx, E, C)
+        _check_align_invariants(idx, E, C, al)
+        if cf <= 0:
+            assert al["drop_mask"].sum() == 0
+
+
+def test_align_all_to_one_expert_keeps_first_C():
+    T, E, k = 40, 8, 1
+    idx = np.zeros((T, 1), dtype=np.int32)
+    C = orc.capacity(T, k, E, 1.25)  # ceil(50/8) = 7
+    assert C == 7
+    al = orc.align(idx, E, C)
+    assert al["counts"].tolist() == [7] + [0] * 7
+    assert al["sorted_ids"][:7].tolist() == list(range(7))
+    assert al["drop_mask"].tolist() == [0] * 7 + [1] * 33
+
+
+# ---------------------------------------------------------------- expert FFN + combine
+
+def test_layer_golden(golden_dir):
+    g = _load(golden_dir, "layer_tiny.json")
+    arr = lambda key: np.asarray(g[key], dtype=np.float64)
+    res = orc.layer_forward(arr("x"), arr("w_router"), arr("w_gate"), arr("w_up"), arr("w_down"),
+                            g["k"], g["capacity_factor"])
+    assert res["topk_idx"].tolist() == g["topk_idx"]
+    np.testing.assert_allclose(res["out"], arr("out"), atol=g["tolerance"], rtol=0)
+
+
+def _dense_swiglu_torch(x, wg, wu, wd):
+    x, wg, wu, wd = (torch.as_tensor(np.asarray(a, dtype=np.float64)) for a in (x, wg, wu, wd))
+    return (torch.nn.functional.silu(x @ wg) * (x @ wu) @ wd).numpy()
+
+
+def test_single_expert_top1_is_dense_swiglu():
+    wl = wlm.Workload("t", 0, 37, 24, 1, 1, 40, "f32", 1.25)
+    inp = wlm.make_inputs(wl)
+    a = {k_: (v.numpy() if v is not None else None) for k_, v in inp.items()}
+    res = orc.layer_forward(a["x"], a["w_router"], a["w_gate"], a["w_up"], a["w_down"], 1, 1.25)
+    assert res["C"] == 37 and res["drop_mask"].sum() == 0
+    assert np.all(res["topk_w"] == 1.0)
+    ref = _dense_swiglu_torch(a["x"], a["w_gate"][0], a["w_up"][0], a["w_down"][0])
+    np.testing.assert_allclose(res["out"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_identical_experts_equal_dense_ffn_for_any_routing():
+    wl = wlm.Workload("t", 0, 29, 16, 6, 3, 20, "f32", 0.0)
+    inp = wlm.make_inputs(wl)
+    a = {k_: (v.numpy() if v is not None else None) for k_, v in inp.items()}
+    wg = np.repeat(a["w_gate"][:1], 6, axis=0)
+    wu = np.repeat(a["w_up"][:1], 6, axis=0)
+    wd = np.repeat(a["w_down"][:1], 6, axis=0)
+    res = orc.layer_forward(a["x"], a["w_router"], wg, wu, wd, 3, 0.0)
+    ref = _dense_swiglu_torch(a["x"], wg[0], wu[0], wd[0])
+    np.testing.assert_allclose(res["out"], ref, rtol=1e-10, atol=1e-10)
+
+
+def test_one_hot_routing_linearity_and_drops():
+    wl = wlm.Workload("t", 0, 24, 16, 4, 1, 12, "f32", 1.0)
+    inp = wlm.make_inputs(wl)
+    a = {k_: (v.numpy() if v is not None else None) for k_, v in inp.items()}
+    # force every token to expert 2 through the logits; C = ceil(24/4) = 6
+    logits = np.zeros((24, 4), dtype=np.float32)
+    logits[:, 2] = 1.0
+    res = orc.layer_forward(a["x"], None, a["w_gate"], a["w_up"], a["w_down"], 1, 1.0, logits=logits)
+    assert res["C"] == 6
+    ref = _dense_swiglu_torch(a["x"], a["w_gate"][2], a["w_up"][2], a["w_down"][2])
+    np.testing.assert_allclose(res["out"][:6], ref[:6], rtol=1e-12, atol=1e-12)
+    assert np.all(res["out"][6:] == 0.0)  # dropped tokens take the residual path only
+    # linear in the down projection
+    res2 = orc.layer_forward(a["x"], None, a["w_gate"], a["w_up"], 2.0 * a["w_down"], 1, 1.0,
+                             logits=logits)
+    np.testing.assert_allclose(res2["out"], 2.0 * res["out"], rtol=1e-12, atol=1e-12)
+
+
+def test_token_subset_matches_full_layer():
+    wl = wlm.Workload("t", 0, 31, 16, 8, 2, 24, "f32", 1.25)
+    inp = wlm.make_inputs(wl)
+    a = {k_: (v.numpy() if v is not None else None) for k_, v in inp.items()}
+    full = orc.layer_forward(a["x"], a["w_router"], a["w_gate"], a["w_up"], a["w_down"], 2, 1.25)
+    sub = orc.layer_forward(a["x"], a["w_router"], a["w_gate"], a["w_up"], a["w_down"], 2, 1.25,
+                            tokens=[30, 3, 17])
+    # same values up to the BLAS blocking of the matmul (rows batched differently)
+    np.testing.assert_allclose(sub["out"], full["out"][[30, 3, 17]], rtol=1e-13, atol=1e-15)
+
+
+def test_silu_textbook_values():
+    # silu(0) = 0 kills the gate: zero x rows give zero output for every expert
+    x = np.zeros((3, 4))
+    rng = np.random.default_rng(2)
+    y = orc.swiglu_expert(x, rng.standard_normal((4, 5)), rng.standard_normal((4, 5)),
+                          rng.standard_normal((5, 4)))
+    assert np.all(y == 0.0)
+    # large positive gate: silu(z) -> z; very negative: -> 0 without overflow warnings
+    one = np.ones((1, 1))
+    assert abs(orc.swiglu_expert(one * 40.0, one, one, one)[0, 0] - 1600.0) < 1e-9
+    assert abs(orc.swiglu_expert(one * -800.0, one, one, one)[0, 0]) < 1e-300
+
+
+# ---------------------------------------------------------------- sizes printed on the pages
+
+def test_page_sizes(golden_dir):
+    g = _load(golden_dir, "page_sizes.json")
+    r = g["router_params"]
+    assert r["H"] * r["E"] == 1048576  # "about 1M"
+    d = g["dispatch_volume"]
+    assert d["T"] * d["k"] == d["page_accesses"]
+    assert d["H"] * d["bytes_per_elem"] == 8192  # 8 KB per access
+    assert d["T"] * d["k"] * d["H"] * d["bytes_per_elem"] == 256 * 1024 * 1024  # "about 256MB"
+    fine = wlm.WORKLOADS["fine"]
+    assert (fine.T, fine.k, fine.H, fine.E) == (d["T"], d["k"], d["H"], r["E"])
+    mix = wlm.WORKLOADS["mixtral"]
+    assert (mix.E, mix.k) == (g["mixtral_active"]["E"], g["mixtral_active"]["k"])
