@@ -1,0 +1,485 @@
+"""Benchmark of the MoE layer forward hot path (libmoe.so) on B200.
+
+Default workload: the fine-grained MoE layer (T=4096, H=4096, E=256, k=8, I=2048, bf16,
+capacity factor 1.25), the configuration the headline metric is quoted on. One step = one
+moe_layer_forward (route -> align -> GEMM1 -> GEMM2 -> combine) over the whole batch.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun as independent replicas (one process per GPU, no data-path
+collective); timing is the max over ranks. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from expert_dispatch_gate_b200 import _lib as L  # noqa: E402
+from expert_dispatch_gate_b200 import layer as M  # noqa: E402
+from expert_dispatch_gate_b200 import workloads as W  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (E=256,k=8,T=4096,1 GPU); route+align+combine HBM GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+STAGES = ["route", "align", "gemm1", "gemm2", "combine"]
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        kw = {"timeout": datetime.timedelta(seconds=120)}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, **kw)
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value, world, device="cpu"):
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world == 1:
+        return float(value)
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank, n_ranks, max_seconds):
+    """Whole-job throughput: units processed by all ranks / the slowest rank's time."""
+    return units_per_rank * n_ranks / max_seconds
+
+
+# ------------------------------------------------------------------ clocks (NVML)
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every few ms while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index, period_s=0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: clocks reported as unavailable
+            self.ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ algorithmic cost model
+
+def stage_costs(wl, counts, hbm_peak, tc_peak):
+    """Algorithmic bytes/flops per stage for one step, from the step's routing counts."""
+    es = 2 if wl.dtype == "bf16" else 4
+    T, H, E, k, I = wl.T, wl.H, wl.E, wl.k, wl.I
+    A = T * k
+    a_kept = int(counts.sum())
+    used = int((counts > 0).sum())
+    bias = E * 4 if wl.zipf_s > 0 else 0
+    c = {
+        "route": {"bytes": T * H * es + H * E * es + bias + T * k * 8, "flops": 2 * T * H * E},
+        "align": {"bytes": T * k * 4 * 3 + A * (4 + 4 + 1) + E * 8, "flops": 0},
+        "gemm1": {"bytes": used * 2 * H * I * es + a_kept * H * es + a_kept * I * es,
+                  "flops": 4 * a_kept * H * I},
+        "gemm2": {"bytes": used * I * H * es + a_kept * I * es + a_kept * H * es,
+                  "flops": 2 * a_kept * I * H},
+        "combine": {"bytes": a_kept * H * es + T * k * 8 + T * H * es, "flops": 2 * a_kept * H},
+    }
+    for v in c.values():
+        v["t_hbm_us"] = v["bytes"] / (hbm_peak * 1e9) * 1e6
+        v["t_tc_us"] = v["flops"] / (tc_peak * 1e12) * 1e6
+    return c
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("ffn_tc.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "expert_dispatch_gate_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on this source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(f"{kernel}@{workload}")
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def oracle_sample_time(wl, host, weights, n_tokens, seed=0):
+    """Time the oracle on a bounded sample: routing + capacity grouping over all T tokens
+    (the grouping depends on every token), the expert FFN + combine on n_tokens sampled
+    tokens. Returns (seconds_route_align, seconds_ffn_combine, tokens_sampled)."""
+    from oracle import moe_oracle as orc
+    t0 = time.perf_counter()
+    logits = orc.router_logits(host["x"], host["w_router"], host["logit_bias"])
+    idx = orc.select_topk(logits, wl.k)
+    w = orc.route_weights(logits, idx)
+    C = orc.capacity(wl.T, wl.k, wl.E, wl.capacity_factor)
+    al = orc.align(idx, wl.E, C)
+    t1 = time.perf_counter()
+    rng = np.random.default_rng(seed)
+    toks = sorted(rng.choice(wl.T, size=min(n_tokens, wl.T), replace=False).tolist())
+    need = sorted({int(al["slot_of"][t * wl.k + j]) for t in toks for j in range(wl.k)
+                   if al["slot_of"][t * wl.k + j] >= 0})
+    y = orc.grouped_ffn_slots(host["x"], al["sorted_ids"], al["offsets"], wl.k, weights[0],
+                              weights[1], weights[2], slots=need)
+    orc.combine(y, al["slot_of"], w, tokens=toks)
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1, len(toks)
+
+
+class HostExperts:
+    """Expert matrices of the sampled experts, copied to host memory in their own dtype before
+    timing; the widening to float64 happens on access, inside the timed oracle call."""
+
+    def __init__(self, w, experts):
+        self.m = {int(e): w[int(e)].cpu() for e in experts}
+
+    def __getitem__(self, e):
+        return self.m[int(e)].double().numpy()
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_baseline(wl, dev, n_tokens, reps=1):
+    from oracle import moe_oracle as orc
+    host = {"x": dev["x"].float().cpu().numpy(), "w_router": dev["w_router"].float().cpu().numpy(),
+            "logit_bias": None if dev["logit_bias"] is None else dev["logit_bias"].cpu().numpy()}
+    # which experts the sample touches (routing recomputed inside the timed call)
+    logits = orc.router_logits(host["x"], host["w_router"], host["logit_bias"])
+    idx = orc.select_topk(logits, wl.k)
+    rng = np.random.default_rng(0)
+    toks = rng.choice(wl.T, size=min(n_tokens, wl.T), replace=False)
+    experts = sorted(set(idx[toks].reshape(-1).tolist()))
+    weights = [HostExperts(dev[n], experts) for n in ("w_gate", "w_up", "w_down")]
+    best = None
+    for _ in range(reps):
+        r = oracle_sample_time(wl, host, weights, n_tokens)
+        best = r if best is None or sum(r[:2]) < sum(best[:2]) else best
+    t_ra, t_ffn, s = best
+    per_token = t_ra / wl.T + t_ffn / s
+    return {"value": 1.0 / per_token, "unit": "tokens/s", "cores": cpu_threads(),
+            "kind": "oracle",
+            "sample": (f"float64 NumPy oracle: routing + capacity grouping timed over all {wl.T} "
+                       f"tokens ({t_ra:.2f} s), expert SwiGLU FFN + combine timed on {s} sampled "
+                       f"tokens ({t_ffn:.2f} s); tokens/s = 1 / (t_route_align/T + t_ffn/{s})")}
+
+
+# ------------------------------------------------------------------ the GPU arm
+
+def run_ours(args, world, rank, local):
+    wl = W.WORKLOADS[args.workload]
+    if args.tokens:
+        wl = wl.with_tokens(args.tokens)
+    dev = torch.device("cuda", local)
+    inp = W.make_inputs(wl, dev)
+    peaks, peaks_src = load_peaks()
+    shape = M.shape_of(wl.T, wl.H, wl.E, wl.k, wl.I, wl.capacity_factor, wl.dtype)
+    ws = M.Workspace(shape, dev)
+    out = torch.empty((wl.T, wl.H), dtype=wl.torch_dtype, device=dev)
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+    wts = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
+    counts = torch.empty(wl.E, dtype=torch.int32, device=dev)
+    drop = torch.empty(wl.T * wl.k, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(x=inp["x"]):
+        L.moe_layer_forward(shape, x, inp["w_router"], inp["logit_bias"], inp["w_gate"],
+                            inp["w_up"], inp["w_down"], out, None, idx, wts, counts, drop, ws.buf,
+                            ws.nbytes, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ws.check()
+
+    # per-stage events: one set per timed step
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in STAGES] for _ in range(args.steps)]
+    for e in ev:
+        for x in e:
+            x.record(stream)
+    for s in starts:
+        s.record(stream)
+    torch.cuda.synchronize()
+
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            L.moe_set_stage_events(ev[i])
+            step()
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    L.moe_set_stage_events(None)
+    barrier(world)
+    ms = t_start.elapsed_time(t_end)
+    ws.check()
+    ms_max = max_over_ranks(ms, world, "cuda")
+    secs = ms_max / 1e3
+    value = aggregate_throughput(wl.T * args.steps, world, secs)
+
+    # per-stage durations (ms), averaged over the timed steps
+    st_ms = {s: 0.0 for s in STAGES}
+    for i in range(args.steps):
+        prev = starts[i]
+        for j, s in enumerate(STAGES):
+            st_ms[s] += prev.elapsed_time(ev[i][j]) / args.steps
+            prev = ev[i][j]
+    cnt = counts.cpu().numpy()
+    cost = stage_costs(wl, cnt, peaks["hbm_gbs"], peaks["bf16_tflops_sustained"])
+    kernels = {}
+    for s in STAGES:
+        t = st_ms[s] * 1e-3
+        kernels[s] = {"us": round(st_ms[s] * 1e3, 2),
+                      "gbs": round(cost[s]["bytes"] / t / 1e9, 1),
+                      "tflops": round(cost[s]["flops"] / t / 1e12, 1),
+                      "bytes": cost[s]["bytes"], "flops": cost[s]["flops"],
+                      "frac_hbm": round(cost[s]["bytes"] / t / 1e9 / peaks["hbm_gbs"], 3)}
+    dom = max(["gemm1", "gemm2"], key=lambda s: st_ms[s])
+    t_dom = st_ms[dom] * 1e-3
+    bound = "hbm" if cost[dom]["t_hbm_us"] >= cost[dom]["t_tc_us"] else "tensor"
+    if bound == "hbm":
+        ach, peak, unit = cost[dom]["bytes"] / t_dom / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        ach, peak, unit = cost[dom]["flops"] / t_dom / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+    rac_bytes = sum(cost[s]["bytes"] for s in ("route", "align", "combine"))
+    rac_t = sum(st_ms[s] for s in ("route", "align", "combine")) * 1e-3
+
+    # end to end through the C ABI with host buffers: H2D x, forward, D2H of the outputs
+    x_host = inp["x"].cpu().pin_memory()
+    outs_dev = [out, idx, wts, counts, drop]
+    outs_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs_dev]
+    x_dev = torch.empty_like(inp["x"])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        for h, d in zip(outs_host, outs_dev):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
+    h2d = x_host.numel() * x_host.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in outs_host)
+
+    launches_route = 2 if (wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0) else 1
+    per_step = launches_route + 3 + 2 + 1
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": wl.dtype,
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights; no dataset)",
+        "config": {"workload": wl.describe(), "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k,
+                   "I": wl.I, "capacity": int(L.moe_capacity(shape)),
+                   "kept_assignments": int(cnt.sum()), "experts_used": int((cnt > 0).sum()),
+                   "parallelism": "replicas" if world > 1 else "single-gpu",
+                   "l2": "inputs larger than L2: %.1f GB of expert weights streamed per step"
+                         % (3 * wl.E * wl.H * wl.I * (2 if wl.dtype == "bf16" else 4) / 1e9)},
+        "roofline": {"kernel": dom, "bound": bound, "achieved": round(ach, 1),
+                     "peak": peak, "unit": unit, "frac": round(ach / peak, 3),
+                     "peak_source": f"{peaks_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
+                     "traffic": recorded_traffic(dom, args.workload),
+                     "algorithmic_bytes": cost[dom]["bytes"],
+                     "tensor_frac": round(cost[dom]["flops"] / t_dom / 1e12 / peaks["bf16_tflops_sustained"], 3)},
+        "route_align_combine_gbs": round(rac_bytes / rac_t / 1e9, 1),
+        "route_align_combine_frac": round(rac_bytes / rac_t / 1e9 / peaks["hbm_gbs"], 3),
+        "kernels": kernels,
+        "e2e": {"value": round(aggregate_throughput(wl.T * args.steps, world, e2e_ms / 1e3), 1),
+                "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_baseline(wl, inp, args.cpu_sample_tokens)
+    return line
+
+
+def run_reference(args, world, rank, local):
+    """The reference arm: the CPU oracle itself, on the same workload, bounded samples."""
+    if rank != 0:
+        return None
+    wl = W.WORKLOADS[args.workload]
+    if args.tokens:
+        wl = wl.with_tokens(args.tokens)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = W.make_inputs(wl, dev)
+    n_tok = max(1, args.cpu_sample_tokens // 4)
+    from oracle import moe_oracle as orc
+    host = {"x": inp["x"].float().cpu().numpy(), "w_router": inp["w_router"].float().cpu().numpy(),
+            "logit_bias": None if inp["logit_bias"] is None else inp["logit_bias"].cpu().numpy()}
+    logits = orc.router_logits(host["x"], host["w_router"], host["logit_bias"])
+    idx = orc.select_topk(logits, wl.k)
+    rng = np.random.default_rng(0)
+    toks = rng.choice(wl.T, size=min(n_tok, wl.T), replace=False)
+    experts = sorted(set(idx[toks].reshape(-1).tolist()))
+    weights = [HostExperts(inp[n], experts) for n in ("w_gate", "w_up", "w_down")]
+    for _ in range(args.warmup):
+        oracle_sample_time(wl, host, weights, n_tok)
+    per = []
+    for _ in range(args.steps):
+        t_ra, t_ffn, s = oracle_sample_time(wl, host, weights, n_tok)
+        per.append(t_ra / wl.T + t_ffn / s)
+    per_token = sum(per) / len(per)
+    value = 1.0 / per_token
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(per_token * wl.T * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.describe(), "T": wl.T},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cpu_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step: routing + grouping over all {wl.T} tokens, FFN + "
+                                   f"combine on {n_tok} sampled tokens, extrapolated to T"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="fine", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=0, help="override T (decode sweep)")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, world, rank, local)
+        else:
+            line = run_ours(args, world, rank, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,512 @@
+// ffn_tc.cu — grouped expert GEMMs (and the E >= 64 router GEMM) on the B200 tensor cores.
+//
+// [P1] "MoE 模型的 FlashAttention 跟普通模型有什么不一样？", section "FlashAttention 在 MoE 模型里的位置",
+// step 4: each expert runs its FFN on the tokens grouped to it. Here the FFN is SwiGLU,
+// h = silu(x Wg) * (x Wu), y = h Wd ([P1] section "手动编译 MoE 融合算子": activation="silu").
+//
+// Design (sm_100a):
+//   * swap-AB: the weight matrix is the MMA's A operand (M = 128 output features per tile) and
+//     the expert's tokens are the B operand (N = tokens of the tile, padded to 16). An expert's
+//     weights are streamed from HBM once per tile, whatever its token count; a decode step with
+//     one token per expert pays for N = 16 columns of MMA, not 128 rows.
+//   * A (weights, MN-major: features contiguous) arrives by 3-D TMA tiles of 64x64 bf16 with
+//     128-byte swizzle; B (token rows, K-major) arrives by TMA tile::gather4 straight from the
+//     unpermuted activations using the grouping's slot -> token map, so no permuted copy of x is
+//     ever written.
+//   * tcgen05.mma accumulates in TMEM (fp32); GEMM1 keeps gate and up accumulators side by side
+//     so one epilogue thread owns both values of a (feature, token) pair and applies SwiGLU.
+//   * Persistent CTAs (one per SM), warp-specialised: warp 0 issues TMA, warp 1 issues MMAs,
+//     warps 2-5 drain TMEM. Tiles are ordered (expert, feature block, token block) so the token
+//     blocks that share a weight slice run at the same time and hit it in L2.
+//   * Every mbarrier wait is bounded; on timeout the CTA raises an error word and winds down.
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;        // MMA M: output features per tile
+constexpr int kBK = 64;         // K per pipeline stage: one 128-byte swizzle row of bf16
+constexpr int kThreads = 192;   // 6 warps
+constexpr int kMaxStages = 8;
+constexpr int kMaxGroups = 256;
+constexpr int kTmemCols = 512;
+constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory per block
+constexpr int kCtrlBytes = 2560;    // barriers + group tables
+
+enum EpiMode { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2 };
+
+struct TcParams {
+  int K;          // reduction length (multiple of 64)
+  int num_fb;     // feature blocks of 128
+  int m_rows_a;   // extent of A along M (a 64-wide chunk starting past it is not loaded)
+  int m_valid;    // features stored by the epilogue
+  int TB;         // max tokens per tile, multiple of 32, <= 256
+  int groups;     // experts (ignored when offsets == nullptr)
+  int k_top;      // GEMM1: B row = sorted_ids[slot] / k_top
+  int rows_b;     // rows of the B tensor
+  const int32_t* sorted_ids;
+  const int32_t* offsets;     // [groups+1] slot offsets, or nullptr: one group of n_static rows
+  const int32_t* blk_prefix;  // [groups+1] token blocks before each group
+  int n_static;
+  void* out;
+  int64_t ldo;
+  const float* bias;
+  int* err;
+  int stages;
+  int nbuf;       // TMEM accumulator buffers (1 or 2, 256 columns apart)
+};
+
+struct Tile {
+  int group, fb, n, row0;
+};
+
+__device__ __forceinline__ Tile decode_tile(int tile, int num_fb, int groups, int TB,
+                                            const int* s_off, const int* s_blk) {
+  int lo = 0, hi = groups;  // largest lo with num_fb * s_blk[lo] <= tile
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (num_fb * s_blk[mid] <= tile) lo = mid; else hi = mid;
+  }
+  Tile t;
+  t.group = lo;
+  const int nb = s_blk[lo + 1] - s_blk[lo];
+  const int local = tile - num_fb * s_blk[lo];
+  t.fb = local / nb;
+  const int b = local - t.fb * nb;
+  const int cnt = s_off[lo + 1] - s_off[lo];
+  t.n = min(TB, cnt - b * TB);
+  t.row0 = s_off[lo] + b * TB;
+  return t;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0,
+                    const __grid_constant__ CUtensorMap tmA1,
+                    const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+  constexpr bool kSwiGLU = (MODE == kEpiSwiGLU);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int a_bytes = kSwiGLU ? 32768 : 16384;
+  const int stage_bytes = a_bytes + p.TB * 128;
+  const int S = p.stages;
+  uint8_t* ctrl = smem + static_cast<size_t>(S) * stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* tfull = empty + kMaxStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* s_off = reinterpret_cast<int*>(ctrl + 256);
+  int* s_blk = s_off + (kMaxGroups + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int groups = (p.offsets != nullptr) ? p.groups : 1;
+
+  if (p.offsets != nullptr) {
+    for (int i = threadIdx.x; i <= groups; i += blockDim.x) {
+      s_off[i] = p.offsets[i];
+      s_blk[i] = p.blk_prefix[i];
+    }
+  } else if (threadIdx.x == 0) {
+    s_off[0] = 0;
+    s_off[1] = p.n_static;
+    s_blk[0] = 0;
+    s_blk[1] = (p.n_static + p.TB - 1) / p.TB;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&tfull[b]), 1);
+      mbar_init(smem_u32(&tempty[b]), 128);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int num_tiles = p.num_fb * s_blk[groups];
+  const int kblocks = p.K / kBK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk);
+      const int npad = (t.n + 15) & ~15;
+      int rows[8];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int nn = (lane + 32 * q) * 4 + r;
+          const int src = t.row0 + min(nn, t.n - 1);
+          int row = (p.sorted_ids != nullptr) ? (p.sorted_ids[src] / p.k_top) : src;
+          rows[q * 4 + r] = min(max(row, 0), p.rows_b - 1);
+        }
+      }
+      const int m0 = t.fb * kBM;
+      const bool hi_chunk = (m0 + 64) < p.m_rows_a;
+      const uint32_t tx = (hi_chunk ? 16384u : 8192u) * (kSwiGLU ? 2u : 1u) +
+                          static_cast<uint32_t>(npad) * 128u;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = it % S;
+        const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+        int got = 1;
+        if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          ok = false;
+          break;
+        }
+        const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+        const uint32_t sb = sa + a_bytes;
+        const uint32_t fbar = smem_u32(&full[s]);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(fbar, tx);
+          tma_load_3d(sa, &tmA0, m0, kb * kBK, t.group, fbar);
+          if (hi_chunk) tma_load_3d(sa + 8192, &tmA0, m0 + 64, kb * kBK, t.group, fbar);
+          if (kSwiGLU) {
+            tma_load_3d(sa + 16384, &tmA1, m0, kb * kBK, t.group, fbar);
+            if (hi_chunk) tma_load_3d(sa + 16384 + 8192, &tmA1, m0 + 64, kb * kBK, t.group, fbar);
+          }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int grp = lane + 32 * q;
+          if (grp * 4 < npad)
+            tma_gather4(sb + grp * 512, &tmB, kb * kBK, rows[q * 4], rows[q * 4 + 1],
+                        rows[q * 4 + 2], rows[q * 4 + 3], fbar);
+        }
+        ++it;
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) flag_error(p.err, kDevWaitTimeout);
+    }
+    // Every load issued must land before the CTA may exit.
+    if (lane == 0) {
+      for (int i = max(0, it - S); i < it; ++i)
+        mbar_wait(smem_u32(&full[i % S]), static_cast<uint32_t>(i / S) & 1u, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (one thread)
+    if (lane == 0) {
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk);
+        const int npad = (t.n + 15) & ~15;
+        const int buf = tc % p.nbuf;
+        const uint32_t use = static_cast<uint32_t>(tc / p.nbuf);
+        if (!mbar_wait(smem_u32(&tempty[buf]), (use & 1u) ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * 256);
+        const uint32_t idesc = idesc_bf16(kBM, npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          const int s = it % S;
+          const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+          if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+          const uint32_t sb = sa + a_bytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(sa + kk * 2048, 8192, 1024);
+            const uint64_t bd = smem_desc_sw128(sb + kk * 32, 16, 1024);
+            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+            tc_mma_bf16(d0, ad, bd, idesc, acc);
+            if (kSwiGLU) {
+              const uint64_t ad1 = smem_desc_sw128(sa + 16384 + kk * 2048, 8192, 1024);
+              tc_mma_bf16(d0 + static_cast<uint32_t>(p.TB), ad1, bd, idesc, acc);
+            }
+          }
+          tc_commit(smem_u32(&empty[s]));
+          ++it;
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&tfull[buf]));
+        ++tc;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        flag_error(p.err, kDevWaitTimeout);
+      }
+      // Every MMA issued must complete before TMEM is released.
+      tc_commit(smem_u32(drain));
+      mbar_wait(smem_u32(drain), 0u, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lane quadrant this warp may read
+    int tc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk);
+      const int buf = tc % p.nbuf;
+      const uint32_t use = static_cast<uint32_t>(tc / p.nbuf);
+      int got = 1;
+      if (lane == 0) got = mbar_wait(smem_u32(&tfull[buf]), use & 1u, abort_flag) ? 1 : 0;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int m = t.fb * kBM + q * 32 + lane;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                          static_cast<uint32_t>(buf * 256);
+      float bias_m = 0.f;
+      if constexpr (MODE == kEpiF32) {
+        if (p.bias != nullptr && m < p.m_valid) bias_m = p.bias[m];
+      }
+      for (int c0 = 0; c0 < t.n; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tb + static_cast<uint32_t>(c0), v);
+        uint32_t u[32];
+        if constexpr (kSwiGLU) tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), u);
+        tmem_wait_ld();
+        const int cmax = min(32, t.n - c0);
+        if constexpr (MODE == kEpiSwiGLU) {
+          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                             static_cast<size_t>(t.row0 + c0) * p.ldo + m;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (j < cmax) {
+              const float g = __uint_as_float(v[j]);
+              const float h = g / (1.0f + __expf(-g)) * __uint_as_float(u[j]);
+              o[static_cast<size_t>(j) * p.ldo] = __float2bfloat16_rn(h);
+            }
+          }
+        } else if constexpr (MODE == kEpiBF16) {
+          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                             static_cast<size_t>(t.row0 + c0) * p.ldo + m;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < cmax) o[static_cast<size_t>(j) * p.ldo] = __float2bfloat16_rn(__uint_as_float(v[j]));
+        } else {
+          if (m < p.m_valid) {
+            float* o = reinterpret_cast<float*>(p.out) + static_cast<size_t>(t.row0 + c0) * p.ldo + m;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < cmax) o[static_cast<size_t>(j) * p.ldo] = __uint_as_float(v[j]) + bias_m;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&tempty[buf]));
+      ++tc;
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) flag_error(p.err, kDevWaitTimeout);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 [rows, cols] row-major, box = {64 columns, 1 row}, 128-byte swizzle: for tile::gather4.
+bool map_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, std::string* d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) {
+    if (d) *d = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && d) *d = "cuTensorMapEncodeTiled(rows) failed with code " + std::to_string(r);
+  return r == CUDA_SUCCESS;
+}
+
+// bf16 [groups, kdim, mdim] (mdim contiguous), box = {64, 64, 1}, 128-byte swizzle.
+bool map_weights(CUtensorMap* m, const void* base, uint64_t mdim, uint64_t kdim, uint64_t groups,
+                 std::string* d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) {
+    if (d) *d = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  cuuint64_t dims[3] = {mdim, kdim, groups};
+  cuuint64_t strides[2] = {mdim * 2, mdim * kdim * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && d) *d = "cuTensorMapEncodeTiled(weights) failed with code " + std::to_string(r);
+  return r == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+                        TcParams p, int64_t tiles_ub, int num_sms, cudaStream_t stream,
+                        std::string* d) {
+  const int a_bytes = (MODE == kEpiSwiGLU) ? 32768 : 16384;
+  const int stage_bytes = a_bytes + p.TB * 128;
+  int stages = (kSmemLimit - 1024 - kCtrlBytes) / stage_bytes;
+  if (stages > kMaxStages) stages = kMaxStages;
+  if (stages < 2) {
+    if (d) *d = "tile too large for shared memory";
+    return cudaErrorInvalidValue;
+  }
+  p.stages = stages;
+  p.nbuf = (((MODE == kEpiSwiGLU) ? 2 : 1) * p.TB <= 256) ? 2 : 1;
+  const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + kCtrlBytes;
+  int64_t grid = tiles_ub < num_sms ? tiles_ub : num_sms;
+  if (grid < 1) grid = 1;
+  cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  tc_grouped_gemm<MODE><<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(a0, a1, b, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, const float* bias, int T,
+                                 int H, int E, float* logits, int* err, int num_sms,
+                                 cudaStream_t stream, std::string* detail) {
+  CUtensorMap a0, b;
+  if (!map_weights(&a0, w_router, static_cast<uint64_t>(E), static_cast<uint64_t>(H), 1, detail) ||
+      !map_rows(&b, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), detail))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.K = H;
+  p.num_fb = (E + kBM - 1) / kBM;
+  p.m_rows_a = E;
+  p.m_valid = E;
+  p.TB = T >= 64 ? 64 : ((T + 31) / 32) * 32;
+  p.groups = 1;
+  p.k_top = 1;
+  p.rows_b = T;
+  p.sorted_ids = nullptr;
+  p.offsets = nullptr;
+  p.blk_prefix = nullptr;
+  p.n_static = T;
+  p.out = logits;
+  p.ldo = E;
+  p.bias = bias;
+  p.err = err;
+  const int64_t tiles = static_cast<int64_t>(p.num_fb) * ((T + p.TB - 1) / p.TB);
+  return launch_mode<kEpiF32>(a0, a0, b, p, tiles, num_sms, stream, detail);
+}
+
+cudaError_t launch_gemm1_tc(const void* x, int T, const int32_t* sorted_ids,
+                            const int32_t* offsets, const int32_t* blk_prefix, const void* w_gate,
+                            const void* w_up, void* hbuf, int64_t hbuf_rows, int H, int E, int k,
+                            int I, int TB, int64_t ub_blocks, int* err, int num_sms,
+                            cudaStream_t stream, std::string* detail) {
+  (void)hbuf_rows;
+  CUtensorMap a0, a1, b;
+  if (!map_weights(&a0, w_gate, I, H, E, detail) || !map_weights(&a1, w_up, I, H, E, detail) ||
+      !map_rows(&b, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), detail))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.K = H;
+  p.num_fb = I / kBM;
+  p.m_rows_a = I;
+  p.m_valid = I;
+  p.TB = TB;
+  p.groups = E;
+  p.k_top = k;
+  p.rows_b = T;
+  p.sorted_ids = sorted_ids;
+  p.offsets = offsets;
+  p.blk_prefix = blk_prefix;
+  p.out = hbuf;
+  p.ldo = I;
+  p.bias = nullptr;
+  p.err = err;
+  return launch_mode<kEpiSwiGLU>(a0, a1, b, p, static_cast<int64_t>(p.num_fb) * ub_blocks,
+                                 num_sms, stream, detail);
+}
+
+cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* offsets,
+                            const int32_t* blk_prefix, const void* w_down, void* y, int H, int E,
+                            int I, int TB, int64_t ub_blocks, int* err, int num_sms,
+                            cudaStream_t stream, std::string* detail) {
+  CUtensorMap a0, b;
+  if (!map_weights(&a0, w_down, H, I, E, detail) ||
+      !map_rows(&b, hbuf, static_cast<uint64_t>(I), static_cast<uint64_t>(hbuf_rows), detail))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.K = I;
+  p.num_fb = H / kBM;
+  p.m_rows_a = H;
+  p.m_valid = H;
+  p.TB = TB;
+  p.groups = E;
+  p.k_top = 1;
+  p.rows_b = static_cast<int>(hbuf_rows);
+  p.sorted_ids = nullptr;
+  p.offsets = offsets;
+  p.blk_prefix = blk_prefix;
+  p.out = y;
+  p.ldo = H;
+  p.bias = nullptr;
+  p.err = err;
+  return launch_mode<kEpiBF16>(a0, a0, b, p, static_cast<int64_t>(p.num_fb) * ub_blocks, num_sms,
+                               stream, detail);
+}
+
+}  // namespace moe

@@ -1,0 +1,60 @@
+// internal.h — launchers shared between the C-ABI layer (moe_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+
+namespace moe {
+
+// ---- route.cu
+// Fused gate GEMM (CUDA cores) + top-k + renormalise, one warp per token; E <= 64.
+cudaError_t launch_route_simt(int dtype, const void* x, const void* w_router, const float* bias,
+                              int64_t T, int H, int E, int k, float* logits_out, int32_t* topk_idx,
+                              float* topk_w, cudaStream_t stream);
+// Top-k + renormalise from float32 logits [T,E], one warp per token; E <= 256.
+cudaError_t launch_topk_from_logits(const float* logits, int64_t T, int E, int k,
+                                    int32_t* topk_idx, float* topk_w, cudaStream_t stream);
+
+// ---- ffn_tc.cu (tcgen05 / TMEM / TMA, bf16)
+// Gate logits [T,E] = x @ w_router (+ bias) on the tensor cores (swap-AB: experts on MMA M).
+cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, const float* bias, int T,
+                                 int H, int E, float* logits, int* err, int num_sms,
+                                 cudaStream_t stream, std::string* detail);
+// Expert GEMM1: h[s, :] = silu(x[t] Wg[e]) * (x[t] Wu[e]) for kept slots; h rows = hbuf_rows.
+cudaError_t launch_gemm1_tc(const void* x, int T, const int32_t* sorted_ids,
+                            const int32_t* offsets, const int32_t* blk_prefix, const void* w_gate,
+                            const void* w_up, void* hbuf, int64_t hbuf_rows, int H, int E, int k,
+                            int I, int TB, int64_t ub_blocks, int* err, int num_sms,
+                            cudaStream_t stream, std::string* detail);
+// Expert GEMM2: y[s, :] = h[s] Wd[e].
+cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* offsets,
+                            const int32_t* blk_prefix, const void* w_down, void* y, int H, int E,
+                            int I, int TB, int64_t ub_blocks, int* err, int num_sms,
+                            cudaStream_t stream, std::string* detail);
+
+// ---- ffn_simt.cu (float32 CUDA-core path)
+cudaError_t launch_gemm1_simt(const float* x, const int32_t* sorted_ids, const int32_t* offsets,
+                              const float* w_gate, const float* w_up, float* hbuf, int64_t A,
+                              int H, int E, int k, int I, cudaStream_t stream);
+cudaError_t launch_gemm2_simt(const float* hbuf, const int32_t* offsets, const float* w_down,
+                              float* y, int64_t A, int H, int E, int I, cudaStream_t stream);
+
+// ---- align.cu
+constexpr int kAlignChunk = 2048;  // assignments per align block
+cudaError_t launch_align(const int32_t* topk_idx, int64_t A, int E, int C, int TB,
+                         int32_t* blk_hist, int32_t* counts, int32_t* offsets,
+                         int32_t* blk_prefix, int32_t* sorted_ids, int32_t* slot_of,
+                         uint8_t* drop_mask, int* err, cudaStream_t stream);
+// blk_prefix[e] = sum over e' < e of ceil(count[e'] / TB), count from offsets.
+cudaError_t launch_plan_from_offsets(const int32_t* offsets, int E, int TB, int32_t* blk_prefix,
+                                     cudaStream_t stream);
+
+// ---- combine.cu
+cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_of,
+                           const float* topk_w, void* out, int64_t T, int H, int k,
+                           cudaStream_t stream);
+
+}  // namespace moe

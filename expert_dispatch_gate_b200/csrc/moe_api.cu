@@ -1,0 +1,444 @@
+// moe_api.cu — the C ABI of libmoe.so (declared in include/moe.h): host-side validation,
+// workspace layout and the launch sequence of the MoE layer forward path.
+//
+// Nothing here allocates, frees or synchronises device memory (moe_check_error excepted).
+// Invalid calls fail loudly with a status and a detail string and launch nothing; there is no
+// fallback path.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <cmath>
+#include <mutex>
+#include <string>
+
+#include "../../include/moe.h"
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_detail = "";
+
+std::mutex g_events_mu;
+void* g_events[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+bool g_events_on = false;
+
+moe_status fail(moe_status s, const std::string& why) {
+  g_detail = why;
+  return s;
+}
+
+moe_status cuda_fail(cudaError_t e, const char* where, const std::string& extra = "") {
+  g_detail = std::string(where) + ": " + cudaGetErrorString(e) + (extra.empty() ? "" : " (" + extra + ")");
+  return MOE_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(int32_t dtype) { return dtype == MOE_F32 ? 4 : 2; }
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+// Shape checks shared by every entry point.
+moe_status check_shape(const moe_shape* s) {
+  if (s == nullptr) return fail(MOE_ERR_INVALID_ARG, "shape is NULL");
+  if (s->T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+  if (s->T >= (int64_t(1) << 24)) return fail(MOE_ERR_UNSUPPORTED, "T >= 2^24");
+  if (s->H < 1 || s->I < 1) return fail(MOE_ERR_INVALID_ARG, "H and I must be >= 1");
+  if (s->E < 1) return fail(MOE_ERR_INVALID_ARG, "E must be >= 1");
+  if (s->E > 256) return fail(MOE_ERR_UNSUPPORTED, "E > 256");
+  if (s->k < 1 || s->k > s->E) return fail(MOE_ERR_INVALID_ARG, "need 1 <= k <= E");
+  if (s->k > 16) return fail(MOE_ERR_UNSUPPORTED, "k > 16");
+  if (s->dtype != MOE_F32 && s->dtype != MOE_BF16)
+    return fail(MOE_ERR_INVALID_ARG, "dtype must be MOE_F32 or MOE_BF16");
+  if (!(s->capacity_factor == s->capacity_factor))
+    return fail(MOE_ERR_INVALID_ARG, "capacity_factor is NaN");
+  if (s->H % 8 != 0) return fail(MOE_ERR_UNSUPPORTED, "H % 8 != 0");
+  if (s->dtype == MOE_BF16) {
+    if (s->H % 128 != 0 || s->I % 128 != 0)
+      return fail(MOE_ERR_UNSUPPORTED, "bf16 needs H % 128 == 0 and I % 128 == 0");
+    if (s->E > 64 && s->E % 8 != 0) return fail(MOE_ERR_UNSUPPORTED, "bf16 with E > 64 needs E % 8 == 0");
+  } else {
+    if (s->E > 64) return fail(MOE_ERR_UNSUPPORTED, "f32 needs E <= 64");
+  }
+  return MOE_OK;
+}
+
+// Capacity C = ceil(cf*T*k/E), cf taken exactly as the float32 it is, capped at T.
+int32_t capacity_of(const moe_shape& s) {
+  if (!(s.capacity_factor > 0.0f)) return static_cast<int32_t>(s.T);
+  int exp2 = 0;
+  const double frac = frexp(static_cast<double>(s.capacity_factor), &exp2);  // cf = frac*2^exp2
+  // frac in [0.5, 1) has a 24-bit mantissa: cf = m * 2^(exp2-24), m integer
+  const unsigned __int128 m = static_cast<unsigned __int128>(ldexp(frac, 24));
+  const int sh = exp2 - 24;
+  unsigned __int128 num = m * static_cast<unsigned __int128>(s.T) * static_cast<unsigned>(s.k);
+  unsigned __int128 den = static_cast<unsigned>(s.E);
+  if (sh >= 0) {
+    if (sh > 60) return static_cast<int32_t>(s.T);
+    num <<= sh;
+  } else {
+    if (-sh > 60) return s.T > 0 ? 1 : 0;  // positive but tiny: ceil of a tiny positive value
+    den <<= -sh;
+  }
+  const unsigned __int128 c = (num + den - 1) / den;
+  return c >= static_cast<unsigned __int128>(s.T) ? static_cast<int32_t>(s.T) : static_cast<int32_t>(c);
+}
+
+// Rows per token block of the expert GEMMs: a multiple of 32 in [32, 256] that splits the
+// largest possible expert group (min(C, T) rows) into equal-sized blocks.
+int token_block(const moe_shape& s, int32_t C) {
+  int64_t maxrows = C < s.T ? C : s.T;
+  if (maxrows < 1) maxrows = 1;
+  const int64_t nblk = (maxrows + 255) / 256;
+  int64_t tb = (maxrows + nblk - 1) / nblk;
+  tb = ((tb + 31) / 32) * 32;
+  if (tb < 32) tb = 32;
+  if (tb > 256) tb = 256;
+  return static_cast<int>(tb);
+}
+
+struct Layout {
+  size_t err, logits, blk_hist, offsets, blk_prefix, sorted_ids, slot_of, hbuf, yslots, total;
+  int64_t A, a_cap;
+  int nblk;
+  int32_t C;
+  int TB;
+};
+
+Layout layout_of(const moe_shape& s) {
+  Layout L{};
+  L.C = capacity_of(s);
+  L.TB = token_block(s, L.C);
+  L.A = s.T * s.k;
+  const int64_t ec = static_cast<int64_t>(s.E) * L.C;
+  L.a_cap = L.A < ec ? L.A : ec;
+  L.nblk = static_cast<int>((L.A + moe::kAlignChunk - 1) / moe::kAlignChunk);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  const size_t es = elem_size(s.dtype);
+  L.err = take(256);
+  L.logits = take(static_cast<size_t>(s.T) * s.E * 4);
+  L.blk_hist = take(static_cast<size_t>(L.nblk) * s.E * 4);
+  L.offsets = take(static_cast<size_t>(s.E + 1) * 4);
+  L.blk_prefix = take(static_cast<size_t>(s.E + 1) * 4);
+  L.sorted_ids = take(static_cast<size_t>(L.A) * 4);
+  L.slot_of = take(static_cast<size_t>(L.A) * 4);
+  L.hbuf = take(static_cast<size_t>(L.a_cap) * s.I * es);
+  L.yslots = take(static_cast<size_t>(L.a_cap) * s.H * es);
+  L.total = off;
+  return L;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+    return 148;
+  return n;
+}
+
+#define REQUIRE_PTR(p, name)                                                  \
+  do {                                                                        \
+    if ((p) == nullptr) return fail(MOE_ERR_INVALID_ARG, name " is NULL");    \
+    if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, name " is not 16-byte aligned"); \
+  } while (0)
+
+#define OPT_PTR(p, name)                                                      \
+  do {                                                                        \
+    if ((p) != nullptr && !aligned16(p))                                      \
+      return fail(MOE_ERR_INVALID_ARG, name " is not 16-byte aligned");       \
+  } while (0)
+
+moe_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+  if (!aligned16(ws)) return fail(MOE_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+  if (ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "workspace too small: need " + std::to_string(need) +
+                                       " bytes, got " + std::to_string(ws_bytes));
+  return MOE_OK;
+}
+
+template <typename P>
+P* at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<char*>(ws) + off);
+}
+
+void record_stage(int i, cudaStream_t st) {
+  std::lock_guard<std::mutex> lk(g_events_mu);
+  if (g_events_on && g_events[i] != nullptr)
+    cudaEventRecord(static_cast<cudaEvent_t>(g_events[i]), st);
+}
+
+// ---- stage bodies (arguments already validated)
+
+moe_status do_route(const moe_shape& s, const Layout& L, const void* x, const void* w_router,
+                    const float* bias, float* logits_out, int32_t* topk_idx, float* topk_w,
+                    void* ws, cudaStream_t st) {
+  cudaError_t e;
+  if (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0) {
+    float* logits = logits_out != nullptr ? logits_out : at<float>(ws, L.logits);
+    std::string d;
+    e = moe::launch_route_gemm_tc(x, w_router, bias, static_cast<int>(s.T), s.H, s.E, logits,
+                                  at<int>(ws, L.err), num_sms(), st, &d);
+    if (e != cudaSuccess) return cuda_fail(e, "router gate GEMM (tcgen05)", d);
+    e = moe::launch_topk_from_logits(logits, s.T, s.E, s.k, topk_idx, topk_w, st);
+    if (e != cudaSuccess) return cuda_fail(e, "router top-k");
+  } else {
+    e = moe::launch_route_simt(s.dtype, x, w_router, bias, s.T, s.H, s.E, s.k, logits_out,
+                               topk_idx, topk_w, st);
+    if (e != cudaSuccess) return cuda_fail(e, "router (CUDA cores)");
+  }
+  return MOE_OK;
+}
+
+moe_status do_ffn(const moe_shape& s, const Layout& L, const void* x, const int32_t* sorted_ids,
+                  const int32_t* offsets, const void* w_gate, const void* w_up, const void* w_down,
+                  void* y, void* ws, cudaStream_t st, bool stage_events) {
+  cudaError_t e;
+  if (s.dtype == MOE_BF16) {
+    const int64_t ub_blocks = (s.E < L.a_cap ? s.E : L.a_cap) + L.a_cap / L.TB;
+    std::string d;
+    e = moe::launch_gemm1_tc(x, static_cast<int>(s.T), sorted_ids, offsets,
+                             at<int32_t>(ws, L.blk_prefix), w_gate, w_up, at<void>(ws, L.hbuf),
+                             L.a_cap, s.H, s.E, s.k, s.I, L.TB, ub_blocks, at<int>(ws, L.err),
+                             num_sms(), st, &d);
+    if (e != cudaSuccess) return cuda_fail(e, "expert GEMM1 (tcgen05)", d);
+    if (stage_events) record_stage(2, st);
+    e = moe::launch_gemm2_tc(at<void>(ws, L.hbuf), L.a_cap, offsets, at<int32_t>(ws, L.blk_prefix),
+                             w_down, y, s.H, s.E, s.I, L.TB, ub_blocks, at<int>(ws, L.err),
+                             num_sms(), st, &d);
+    if (e != cudaSuccess) return cuda_fail(e, "expert GEMM2 (tcgen05)", d);
+  } else {
+    e = moe::launch_gemm1_simt(static_cast<const float*>(x), sorted_ids, offsets,
+                               static_cast<const float*>(w_gate), static_cast<const float*>(w_up),
+                               at<float>(ws, L.hbuf), L.a_cap, s.H, s.E, s.k, s.I, st);
+    if (e != cudaSuccess) return cuda_fail(e, "expert GEMM1 (CUDA cores)");
+    if (stage_events) record_stage(2, st);
+    e = moe::launch_gemm2_simt(at<float>(ws, L.hbuf), offsets, static_cast<const float*>(w_down),
+                               static_cast<float*>(y), L.a_cap, s.H, s.E, s.I, st);
+    if (e != cudaSuccess) return cuda_fail(e, "expert GEMM2 (CUDA cores)");
+  }
+  if (stage_events) record_stage(3, st);
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_shape* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  return layout_of(*shape).total;
+}
+
+int32_t moe_capacity(const moe_shape* shape) {
+  if (check_shape(shape) != MOE_OK) return -1;
+  return capacity_of(*shape);
+}
+
+moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router,
+                     const float* logit_bias, float* logits_out, int32_t* topk_idx,
+                     float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->T == 0) return MOE_OK;
+  REQUIRE_PTR(x, "x");
+  REQUIRE_PTR(w_router, "w_router");
+  REQUIRE_PTR(topk_idx, "topk_idx");
+  REQUIRE_PTR(topk_w, "topk_w");
+  OPT_PTR(logit_bias, "logit_bias");
+  OPT_PTR(logits_out, "logits_out");
+  const Layout L = layout_of(*shape);
+  st = check_ws(ws, ws_bytes, L.logits + static_cast<size_t>(shape->T) * shape->E * 4);
+  if (st != MOE_OK) return st;
+  return do_route(*shape, L, x, w_router, logit_bias, logits_out, topk_idx, topk_w, ws,
+                  static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_route_from_logits(const moe_shape* shape, const float* logits, int32_t* topk_idx,
+                                 float* topk_w, void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->T == 0) return MOE_OK;
+  REQUIRE_PTR(logits, "logits");
+  REQUIRE_PTR(topk_idx, "topk_idx");
+  REQUIRE_PTR(topk_w, "topk_w");
+  cudaError_t e = moe::launch_topk_from_logits(logits, shape->T, shape->E, shape->k, topk_idx,
+                                               topk_w, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "router top-k");
+  return MOE_OK;
+}
+
+moe_status moe_align(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts,
+                     int32_t* offsets, int32_t* sorted_ids, int32_t* slot_of, uint8_t* drop_mask,
+                     void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  REQUIRE_PTR(counts, "counts");
+  REQUIRE_PTR(offsets, "offsets");
+  const Layout L = layout_of(*shape);
+  st = check_ws(ws, ws_bytes, L.blk_prefix + static_cast<size_t>(shape->E + 1) * 4);
+  if (st != MOE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (shape->T == 0) {
+    // empty batch: zero counts and offsets, nothing else to write
+    cudaError_t e = cudaMemsetAsync(counts, 0, static_cast<size_t>(shape->E) * 4, cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, static_cast<size_t>(shape->E + 1) * 4, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "align (empty batch)");
+    return MOE_OK;
+  }
+  REQUIRE_PTR(topk_idx, "topk_idx");
+  REQUIRE_PTR(sorted_ids, "sorted_ids");
+  REQUIRE_PTR(slot_of, "slot_of");
+  REQUIRE_PTR(drop_mask, "drop_mask");
+  cudaError_t e = moe::launch_align(topk_idx, L.A, shape->E, L.C, L.TB, at<int32_t>(ws, L.blk_hist),
+                                    counts, offsets, at<int32_t>(ws, L.blk_prefix), sorted_ids,
+                                    slot_of, drop_mask, at<int>(ws, L.err), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "align");
+  return MOE_OK;
+}
+
+moe_status moe_grouped_ffn(const moe_shape* shape, const void* x, const int32_t* sorted_ids,
+                           const int32_t* offsets, const void* w_gate, const void* w_up,
+                           const void* w_down, void* y_slots, void* ws, size_t ws_bytes,
+                           void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->T == 0) return MOE_OK;
+  REQUIRE_PTR(x, "x");
+  REQUIRE_PTR(sorted_ids, "sorted_ids");
+  REQUIRE_PTR(offsets, "offsets");
+  REQUIRE_PTR(w_gate, "w_gate");
+  REQUIRE_PTR(w_up, "w_up");
+  REQUIRE_PTR(w_down, "w_down");
+  REQUIRE_PTR(y_slots, "y_slots");
+  const Layout L = layout_of(*shape);
+  st = check_ws(ws, ws_bytes, L.yslots);
+  if (st != MOE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (shape->dtype == MOE_BF16) {
+    cudaError_t e = moe::launch_plan_from_offsets(offsets, shape->E, L.TB,
+                                                  at<int32_t>(ws, L.blk_prefix), cs);
+    if (e != cudaSuccess) return cuda_fail(e, "expert GEMM tile plan");
+  }
+  return do_ffn(*shape, L, x, sorted_ids, offsets, w_gate, w_up, w_down, y_slots, ws, cs, false);
+}
+
+moe_status moe_combine(const moe_shape* shape, const void* y_slots, const int32_t* slot_of,
+                       const float* topk_w, void* out, void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->T == 0) return MOE_OK;
+  REQUIRE_PTR(y_slots, "y_slots");
+  REQUIRE_PTR(slot_of, "slot_of");
+  REQUIRE_PTR(topk_w, "topk_w");
+  REQUIRE_PTR(out, "out");
+  cudaError_t e = moe::launch_combine(shape->dtype, y_slots, slot_of, topk_w, out, shape->T,
+                                      shape->H, shape->k, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "combine");
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward(const moe_shape* shape, const void* x, const void* w_router,
+                             const float* logit_bias, const void* w_gate, const void* w_up,
+                             const void* w_down, void* out, float* logits_out, int32_t* topk_idx,
+                             float* topk_w, int32_t* counts, uint8_t* drop_mask, void* ws,
+                             size_t ws_bytes, void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  const moe_shape& s = *shape;
+  REQUIRE_PTR(counts, "counts");
+  const Layout L = layout_of(s);
+  st = check_ws(ws, ws_bytes, L.total);
+  if (st != MOE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (s.T == 0) {
+    cudaError_t e = cudaMemsetAsync(counts, 0, static_cast<size_t>(s.E) * 4, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "layer (empty batch)");
+    return MOE_OK;
+  }
+  REQUIRE_PTR(x, "x");
+  REQUIRE_PTR(w_router, "w_router");
+  REQUIRE_PTR(w_gate, "w_gate");
+  REQUIRE_PTR(w_up, "w_up");
+  REQUIRE_PTR(w_down, "w_down");
+  REQUIRE_PTR(out, "out");
+  REQUIRE_PTR(topk_idx, "topk_idx");
+  REQUIRE_PTR(topk_w, "topk_w");
+  REQUIRE_PTR(drop_mask, "drop_mask");
+  OPT_PTR(logit_bias, "logit_bias");
+  OPT_PTR(logits_out, "logits_out");
+
+  st = do_route(s, L, x, w_router, logit_bias, logits_out, topk_idx, topk_w, ws, cs);
+  if (st != MOE_OK) return st;
+  record_stage(0, cs);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* sorted_ids = at<int32_t>(ws, L.sorted_ids);
+  int32_t* slot_of = at<int32_t>(ws, L.slot_of);
+  cudaError_t e = moe::launch_align(topk_idx, L.A, s.E, L.C, L.TB, at<int32_t>(ws, L.blk_hist),
+                                    counts, offsets, at<int32_t>(ws, L.blk_prefix), sorted_ids,
+                                    slot_of, drop_mask, at<int>(ws, L.err), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "align");
+  record_stage(1, cs);
+  void* y = at<void>(ws, L.yslots);
+  st = do_ffn(s, L, x, sorted_ids, offsets, w_gate, w_up, w_down, y, ws, cs, true);
+  if (st != MOE_OK) return st;
+  e = moe::launch_combine(s.dtype, y, slot_of, topk_w, out, s.T, s.H, s.k, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "combine");
+  record_stage(4, cs);
+  return MOE_OK;
+}
+
+moe_status moe_check_error(void* ws, void* stream) {
+  if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(int), cudaMemcpyDeviceToHost, cs);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_check_error");
+  if (word != 0) {
+    e = cudaMemsetAsync(ws, 0, sizeof(int), cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_check_error (clear)");
+    const char* what = word == 1 ? "an expert id outside [0, E) in topk_idx"
+                       : word == 2 ? "a bounded pipeline wait ran out in an expert GEMM"
+                                   : "unknown device error";
+    return fail(MOE_ERR_DEVICE, std::string("device error ") + std::to_string(word) + ": " + what);
+  }
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape outside the supported limits";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing or too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA runtime or launch failure";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE: a kernel reported a device-side fault";
+  }
+  return "unknown moe_status";
+}
+
+const char* moe_last_error_detail(void) { return g_detail.c_str(); }
+
+moe_status moe_set_stage_events(void** events, int32_t n_events) {
+  std::lock_guard<std::mutex> lk(g_events_mu);
+  if (events == nullptr) {
+    if (n_events != 0) return fail(MOE_ERR_INVALID_ARG, "events is NULL but n_events != 0");
+    for (int i = 0; i < 5; ++i) g_events[i] = nullptr;
+    g_events_on = false;
+    return MOE_OK;
+  }
+  if (n_events != 5) return fail(MOE_ERR_INVALID_ARG, "n_events must be 5");
+  for (int i = 0; i < 5; ++i) g_events[i] = events[i];
+  g_events_on = true;
+  return MOE_OK;
+}
+
+}  // extern "C"

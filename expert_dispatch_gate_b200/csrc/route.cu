@@ -1,0 +1,228 @@
+// route.cu — router: gate logits, top-k selection and renormalised weights.
+//
+// [P4] "MoE Router" (2048ai.net), section "Router 就是一个小型网络": logits = x Wr (bias-free
+// Linear), softmax, top-k, divide the k selected weights by their sum.
+// [P5] "大模型推理加速200%+？…", section "3.1 Moe Fuse Gate & Softmax TopK": gate + softmax + top-k
+// in one kernel, warp-shuffle arg-max with the winner erased each round, exp evaluated only for
+// the k selected logits (exp(l - m) / sum over the selection equals the renormalised softmax).
+//
+// Selection rule: the k largest float32 logits, ties to the lower expert index (-0 == +0);
+// listed by descending logit then ascending index. Logits must be finite.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+
+// Winner of (value desc, index asc) across the warp; every lane ends with the same pair.
+__device__ __forceinline__ void warp_argmax(float& bv, int& bi) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+    if (ov > bv || (ov == bv && oi < bi)) {
+      bv = ov;
+      bi = oi;
+    }
+  }
+}
+
+// Lane j < k holds the j-th selected (value, index); `top` is the largest logit. Writes
+// topk_idx and the weights exp(l_j - top) / sum_i exp(l_i - top).
+__device__ __forceinline__ void write_selection(int lane, int k, float my_v, int my_i, float top,
+                                                int32_t* idx_row, float* w_row) {
+  const float ex = (lane < k) ? expf(my_v - top) : 0.0f;
+  float s = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (lane < k) {
+    idx_row[lane] = my_i;
+    w_row[lane] = ex / s;
+  }
+}
+
+// Logits distributed over lanes: lane holds experts lane, lane+32, ... (VPL per lane).
+template <int VPL>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+    topk_from_logits_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
+                            int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float* row = logits + t * E;
+  float v[VPL];
+  uint32_t taken = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = (e < E) ? row[e] : -INFINITY;
+    if (e >= E) taken |= 1u << i;
+  }
+  float my_v = 0.f, top = 0.f;
+  int my_i = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane + 32 * i;
+      if (!((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < bi))) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+    warp_argmax(bv, bi);
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == j) {
+      my_v = bv;
+      my_i = bi;
+    }
+    if (j == 0) top = bv;
+  }
+  write_selection(lane, k, my_v, my_i, top, topk_idx + t * k, topk_w + t * k);
+}
+
+template <typename Tin>
+__device__ __forceinline__ float ld_f(const Tin* p);
+template <>
+__device__ __forceinline__ float ld_f<float>(const float* p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float ld_f<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+
+template <typename Tin>
+__device__ __forceinline__ void load8(const Tin* p, float (&o)[8]);
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float (&o)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&o)[8]) {
+  const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    o[2 * i] = __uint_as_float(w[i] << 16);
+    o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Gate GEMM on CUDA cores + selection, one warp per token; E <= EMAX <= 64, H % 8 == 0.
+// Every lane accumulates all E partial dot products over its slice of H (8 consecutive
+// elements per 128-bit load); a butterfly reduction gives every lane all E logits.
+template <typename Tin, int EMAX>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+    route_simt_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr,
+                      const float* __restrict__ bias, int64_t T, int H, int E, int k,
+                      float* __restrict__ logits_out, int32_t* __restrict__ topk_idx,
+                      float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
+  if (t >= T) return;
+  float acc[EMAX];
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) acc[e] = 0.f;
+  const Tin* xr = x + t * H;
+  for (int h0 = lane * 8; h0 < H; h0 += 256) {
+    float xv[8];
+    load8<Tin>(xr + h0, xv);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const Tin* wrow = wr + static_cast<size_t>(h0 + u) * E;
+#pragma unroll
+      for (int e = 0; e < EMAX; ++e)
+        if (e < E) acc[e] = fmaf(xv[u], ld_f<Tin>(wrow + e), acc[e]);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+    if (bias != nullptr && e < E) acc[e] += __ldg(bias + e);
+  }
+  if (logits_out != nullptr) {
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e)
+      if (e < E && (e & 31) == lane) logits_out[t * E + e] = acc[e];
+  }
+  // Every lane holds the same E logits: select redundantly, lane j keeps the j-th pick.
+  uint64_t taken = 0;
+  float my_v = 0.f, top = 0.f;
+  int my_i = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) {
+      if (e < E && !((taken >> e) & 1ull) && (acc[e] > bv || (acc[e] == bv && e < bi))) {
+        bv = acc[e];
+        bi = e;
+      }
+    }
+    taken |= 1ull << bi;
+    if (lane == j) {
+      my_v = bv;
+      my_i = bi;
+    }
+    if (j == 0) top = bv;
+  }
+  write_selection(lane, k, my_v, my_i, top, topk_idx + t * k, topk_w + t * k);
+}
+
+template <typename Tin>
+cudaError_t route_simt_dispatch(const Tin* x, const Tin* wr, const float* bias, int64_t T, int H,
+                                int E, int k, float* logits_out, int32_t* idx, float* w,
+                                cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
+  const unsigned block = kWarpsPerBlock * 32;
+  if (E <= 8)
+    route_simt_kernel<Tin, 8><<<grid, block, 0, st>>>(x, wr, bias, T, H, E, k, logits_out, idx, w);
+  else if (E <= 16)
+    route_simt_kernel<Tin, 16><<<grid, block, 0, st>>>(x, wr, bias, T, H, E, k, logits_out, idx, w);
+  else if (E <= 32)
+    route_simt_kernel<Tin, 32><<<grid, block, 0, st>>>(x, wr, bias, T, H, E, k, logits_out, idx, w);
+  else
+    route_simt_kernel<Tin, 64><<<grid, block, 0, st>>>(x, wr, bias, T, H, E, k, logits_out, idx, w);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route_simt(int dtype, const void* x, const void* w_router, const float* bias,
+                              int64_t T, int H, int E, int k, float* logits_out, int32_t* topk_idx,
+                              float* topk_w, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  if (dtype == 0)
+    return route_simt_dispatch<float>(static_cast<const float*>(x),
+                                      static_cast<const float*>(w_router), bias, T, H, E, k,
+                                      logits_out, topk_idx, topk_w, stream);
+  return route_simt_dispatch<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x),
+                                            static_cast<const __nv_bfloat16*>(w_router), bias, T,
+                                            H, E, k, logits_out, topk_idx, topk_w, stream);
+}
+
+cudaError_t launch_topk_from_logits(const float* logits, int64_t T, int E, int k,
+                                    int32_t* topk_idx, float* topk_w, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
+  const unsigned block = kWarpsPerBlock * 32;
+  if (E <= 32)
+    topk_from_logits_kernel<1><<<grid, block, 0, stream>>>(logits, T, E, k, topk_idx, topk_w);
+  else if (E <= 64)
+    topk_from_logits_kernel<2><<<grid, block, 0, stream>>>(logits, T, E, k, topk_idx, topk_w);
+  else if (E <= 128)
+    topk_from_logits_kernel<4><<<grid, block, 0, stream>>>(logits, T, E, k, topk_idx, topk_w);
+  else
+    topk_from_logits_kernel<8><<<grid, block, 0, stream>>>(logits, T, E, k, topk_idx, topk_w);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

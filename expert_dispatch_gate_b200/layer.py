@@ -1,0 +1,116 @@
+"""Tensor-level wrappers over the C ABI: allocate outputs and workspace with PyTorch (device
+memory is PyTorch's job), then make one library call. No arithmetic happens here."""
+from __future__ import annotations
+
+import torch
+
+from . import _lib as L
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return L.MOE_F32
+    if t.dtype == torch.bfloat16:
+        return L.MOE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: the layer takes float32 or bfloat16")
+
+
+def shape_of(T, H, E, k, I, capacity_factor, dtype):
+    return L.make_shape(T, H, E, k, I, capacity_factor, dtype)
+
+
+class Workspace:
+    """A device byte buffer sized by moe_workspace_bytes, reused across calls of one shape."""
+
+    def __init__(self, shape, device):
+        self.nbytes = max(int(L.moe_workspace_bytes(shape)), 256)
+        self.buf = torch.zeros(self.nbytes, dtype=torch.uint8, device=device)
+
+    def check(self, stream=None):
+        return L.moe_check_error(self.buf, stream)
+
+
+def route(x, w_router, k, logit_bias=None, logits_out=True, ws=None, stream=None):
+    T, H = x.shape
+    E = w_router.shape[1]
+    shape = shape_of(T, H, E, k, 128, 0.0, _dtype_code(x))
+    ws = ws or Workspace(shape, x.device)
+    idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    logits = torch.empty((T, E), dtype=torch.float32, device=x.device) if logits_out else None
+    L.moe_route(shape, x, w_router, logit_bias, logits, idx, w, ws.buf, ws.nbytes, stream)
+    return idx, w, logits
+
+
+def route_from_logits(logits, k, stream=None):
+    T, E = logits.shape
+    shape = shape_of(T, 128, E, k, 128, 0.0, L.MOE_BF16 if E <= 64 or E % 8 == 0 else L.MOE_F32)
+    idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    L.moe_route_from_logits(shape, logits, idx, w, stream)
+    return idx, w
+
+
+def align(topk_idx, E, capacity_factor, H=128, I=128, dtype=L.MOE_BF16, ws=None, stream=None):
+    T, k = topk_idx.shape
+    shape = shape_of(T, H, E, k, I, capacity_factor, dtype)
+    dev = topk_idx.device
+    ws = ws or Workspace(shape, dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    sorted_ids = torch.empty(T * k, dtype=torch.int32, device=dev)
+    slot_of = torch.empty(T * k, dtype=torch.int32, device=dev)
+    drop = torch.empty(T * k, dtype=torch.uint8, device=dev)
+    L.moe_align(shape, topk_idx, counts, offsets, sorted_ids, slot_of, drop, ws.buf, ws.nbytes,
+                stream)
+    return {"counts": counts, "offsets": offsets, "sorted_ids": sorted_ids, "slot_of": slot_of,
+            "drop_mask": drop, "C": L.moe_capacity(shape), "ws": ws}
+
+
+def grouped_ffn(x, sorted_ids, offsets, w_gate, w_up, w_down, k, capacity_factor, ws=None,
+                stream=None):
+    T, H = x.shape
+    E, _, I = w_gate.shape
+    shape = shape_of(T, H, E, k, I, capacity_factor, _dtype_code(x))
+    ws = ws or Workspace(shape, x.device)
+    y = torch.empty((T * k, H), dtype=x.dtype, device=x.device)
+    L.moe_grouped_ffn(shape, x, sorted_ids, offsets, w_gate, w_up, w_down, y, ws.buf, ws.nbytes,
+                      stream)
+    return y
+
+
+def combine(y_slots, slot_of, topk_w, E, stream=None):
+    T, k = topk_w.shape
+    H = y_slots.shape[1]
+    shape = shape_of(T, H, E, k, 128, 0.0, _dtype_code(y_slots))
+    out = torch.empty((T, H), dtype=y_slots.dtype, device=y_slots.device)
+    L.moe_combine(shape, y_slots, slot_of, topk_w, out, stream)
+    return out
+
+
+class MoELayerOutputs(dict):
+    pass
+
+
+def layer_forward(x, w_router, w_gate, w_up, w_down, k, capacity_factor, logit_bias=None,
+                  logits_out=True, ws=None, out=None, stream=None):
+    """Whole layer through moe_layer_forward. Returns out, topk_idx, topk_w, counts, drop_mask
+    (and logits when requested)."""
+    T, H = x.shape
+    E, _, I = w_gate.shape
+    dev = x.device
+    shape = shape_of(T, H, E, k, I, capacity_factor, _dtype_code(x))
+    ws = ws or Workspace(shape, dev)
+    res = MoELayerOutputs()
+    res["out"] = out if out is not None else torch.empty((T, H), dtype=x.dtype, device=dev)
+    res["topk_idx"] = torch.empty((T, k), dtype=torch.int32, device=dev)
+    res["topk_w"] = torch.empty((T, k), dtype=torch.float32, device=dev)
+    res["counts"] = torch.empty(E, dtype=torch.int32, device=dev)
+    res["drop_mask"] = torch.empty(T * k, dtype=torch.uint8, device=dev)
+    res["logits"] = torch.empty((T, E), dtype=torch.float32, device=dev) if logits_out else None
+    L.moe_layer_forward(shape, x, w_router, logit_bias, w_gate, w_up, w_down, res["out"],
+                        res["logits"], res["topk_idx"], res["topk_w"], res["counts"],
+                        res["drop_mask"], ws.buf, ws.nbytes, stream)
+    res["ws"] = ws
+    res["C"] = L.moe_capacity(shape)
+    return res

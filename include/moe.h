@@ -1,0 +1,163 @@
+/*
+ * moe.h — C ABI of libmoe.so: the MoE layer forward hot path on one NVIDIA B200 (sm_100a).
+ *
+ * The layer (router gate -> softmax/top-k/renormalise -> capacity-limited grouping by expert
+ * -> grouped SwiGLU expert FFN -> weighted combine) follows these pages:
+ *   [P1] "MoE 模型的 FlashAttention 跟普通模型有什么不一样？" (framerc.cn):
+ *        section "FlashAttention 在 MoE 模型里的位置" (the five steps), section
+ *        "融合二：expert 计算的输出 + 合并结果" (accum += route_weight * expert_output),
+ *        section "手动编译 MoE 融合算子" (npu_moe_fusion(x, router_weight[H,E],
+ *        expert_weights[E,...], num_experts, top_k, activation="silu")).
+ *   [P4] "MoE Router" on Ascend CANN (2048ai.net): section "Router 就是一个小型网络" (gate
+ *        Linear(H,E,bias=False), softmax, topk, renormalise), section "Token 分发的通信瓶颈"
+ *        (per-destination counts), section "昇腾NPU的通信计算重叠" (capacity C = total/E x 1.25,
+ *        overflow dropped to the residual path).
+ *   [P5] "大模型推理加速200%+？这套国产融合算子库把CUDA/Triton全替换了" (csdn.net): sections
+ *        "3.1 Moe Fuse Gate & Softmax TopK" and "3.2 Fuse RMS RoPE & MoE Align & MoE Sum".
+ *
+ * Conventions (all entry points):
+ *   - Notation: T tokens, H hidden size, E experts, k experts per token, I SwiGLU intermediate
+ *     size, C per-expert capacity (moe_capacity), A = T*k assignments; assignment a = t*k + j.
+ *   - Pointers named x, w_*, out, y_slots, logits*, topk_*, counts, offsets, sorted_ids,
+ *     slot_of, drop_mask and ws are DEVICE pointers owned by the caller; the library never
+ *     allocates, frees or synchronises (except moe_check_error). Every device pointer must be
+ *     16-byte aligned; tensors are dense row-major with the shapes given below.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). All calls are
+ *     asynchronous on that stream; outputs are valid once the stream reaches them.
+ *   - Arguments are validated on the host before any launch; an invalid call returns an error
+ *     status and launches nothing. A failed launch returns MOE_ERR_CUDA. Device-side faults
+ *     that the kernels detect (an expert id out of range, a bounded wait that ran out) are
+ *     recorded in the first word of `ws` and reported by moe_check_error.
+ *   - Float dtype: MOE_F32 or MOE_BF16 for x, the weights, y_slots and out. Gate logits,
+ *     routing weights and the logit bias are always float32.
+ *   - Weight layout (x @ W convention): w_router [H,E]; w_gate, w_up [E,H,I]; w_down [E,I,H]
+ *     (one tensor per kind with a leading expert dimension, [P1] "手动编译 MoE 融合算子").
+ *   - Outputs are the MoE contribution only; the residual add belongs to the caller.
+ *   - Limits: 1 <= E <= 256, 1 <= k <= min(E,16), 0 <= T < 2^24, H % 8 == 0, I >= 1.
+ *     BF16: H % 128 == 0 and I % 128 == 0 (tensor-core expert GEMMs); E <= 64 or E % 8 == 0.
+ *     F32: E <= 64.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, k > E ... */
+  MOE_ERR_UNSUPPORTED = 2, /* valid layer, but outside the limits listed above */
+  MOE_ERR_WORKSPACE = 3,   /* ws missing or ws_bytes below the required size */
+  MOE_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+  MOE_ERR_DEVICE = 5       /* a kernel reported a fault through the workspace error word */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+typedef struct {
+  int64_t T;             /* tokens (rows of x); 0 is valid and launches nothing */
+  int32_t H;             /* hidden size */
+  int32_t E;             /* number of experts */
+  int32_t k;             /* experts per token */
+  int32_t I;             /* SwiGLU intermediate size per expert */
+  float capacity_factor; /* C = ceil(cf*T*k/E) capped at T; cf <= 0 means no limit (C = T) */
+  int32_t dtype;         /* moe_dtype */
+} moe_shape;
+
+/* Workspace bytes that moe_layer_forward needs for `shape`; it also covers every other call
+ * on the same shape. 0 if the shape is invalid. */
+size_t moe_workspace_bytes(const moe_shape* shape);
+
+/* Per-expert capacity C, [P4] section "昇腾NPU的通信计算重叠", reading "total tokens" as the
+ * T*k assignments: C = ceil(cf*T*k/E) in exact integer arithmetic on the float32 cf, capped at
+ * T; cf <= 0 gives T. Returns -1 for an invalid shape. */
+int32_t moe_capacity(const moe_shape* shape);
+
+/* Router, [P4] section "Router 就是一个小型网络" and [P5] section "3.1 Moe Fuse Gate &
+ * Softmax TopK": logits[t,e] = sum_h x[t,h]*w_router[h,e] (+ logit_bias[e]) accumulated in
+ * float32; topk_idx[t,:] = the k largest logits in (logit desc, index asc) order, ties to the
+ * lower index; topk_w[t,j] = exp(l_j - m) / sum over the selected i of exp(l_i - m), m = row
+ * max (the renormalised softmax over the selected experts).
+ *   x [T,H] dtype; w_router [H,E] dtype; logit_bias [E] float32 or NULL;
+ *   logits_out [T,E] float32 or NULL (when given, receives the logits the selection used);
+ *   topk_idx [T,k] int32; topk_w [T,k] float32; ws/ws_bytes: workspace (moe_workspace_bytes). */
+moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router,
+                     const float* logit_bias, float* logits_out, int32_t* topk_idx,
+                     float* topk_w, void* ws, size_t ws_bytes, void* stream);
+
+/* Selection only, from given float32 logits [T,E] (same rule as moe_route). No workspace.
+ * Logits must be finite. */
+moe_status moe_route_from_logits(const moe_shape* shape, const float* logits,
+                                 int32_t* topk_idx, float* topk_w, void* stream);
+
+/* Capacity-limited grouping, [P1] section "FlashAttention 在 MoE 模型里的位置" step 3, [P4]
+ * sections "Token 分发的通信瓶颈" and "昇腾NPU的通信计算重叠", [P5] "MoE Align". The rank of
+ * assignment a = t*k+j within expert e = idx[t,j] counts earlier tokens routed to e; a is kept
+ * iff rank < C. counts[e] = min(#assignments to e, C); offsets = exclusive scan of counts
+ * (offsets[E] = kept total); slot = offsets[e] + rank; sorted_ids[slot] = a (slots past the
+ * kept total hold -1); slot_of[a] = slot or -1; drop_mask[a] = 1 iff dropped.
+ *   topk_idx [T,k] int32 (distinct experts per token; an id outside [0,E) is treated as
+ *   dropped and flagged in the error word); counts [E], offsets [E+1], sorted_ids [T*k],
+ *   slot_of [T*k] int32; drop_mask [T*k] uint8. */
+moe_status moe_align(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts,
+                     int32_t* offsets, int32_t* sorted_ids, int32_t* slot_of,
+                     uint8_t* drop_mask, void* ws, size_t ws_bytes, void* stream);
+
+/* Grouped SwiGLU expert FFN, [P1] section "FlashAttention 在 MoE 模型里的位置" step 4 and
+ * section "手动编译 MoE 融合算子" (activation "silu"): for every kept slot s of expert e (offsets[e]
+ * <= s < offsets[e+1]) with token t = sorted_ids[s] / k:
+ *   y_slots[s,:] = (silu(x[t] @ w_gate[e]) * (x[t] @ w_up[e])) @ w_down[e], silu(z) = z*sigmoid(z),
+ * float32 accumulation; BF16 rounds the intermediate and y to bf16. Rows of y_slots past
+ * offsets[E] are not written.
+ *   x [T,H]; sorted_ids [T*k], offsets [E+1] as produced by moe_align; w_gate, w_up [E,H,I];
+ *   w_down [E,I,H]; y_slots [T*k,H] dtype. */
+moe_status moe_grouped_ffn(const moe_shape* shape, const void* x, const int32_t* sorted_ids,
+                           const int32_t* offsets, const void* w_gate, const void* w_up,
+                           const void* w_down, void* y_slots, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Weighted combine, [P1] section "融合二：expert 计算的输出 + 合并结果" and [P5] "MoE Sum":
+ * out[t,:] = sum over j with slot_of[t*k+j] >= 0 of topk_w[t,j] * y_slots[slot_of[t*k+j],:],
+ * accumulated in float32 and rounded once; a fully dropped token gives a zero row.
+ *   y_slots [T*k,H] dtype; slot_of [T*k] int32; topk_w [T,k] float32; out [T,H] dtype. */
+moe_status moe_combine(const moe_shape* shape, const void* y_slots, const int32_t* slot_of,
+                       const float* topk_w, void* out, void* stream);
+
+/* The whole layer on one stream: moe_route -> moe_align -> moe_grouped_ffn -> moe_combine,
+ * with the intermediates (logits unless logits_out is given, offsets, sorted_ids, slot_of, the
+ * SwiGLU intermediate, y_slots) in the workspace. Outputs: out [T,H] dtype, topk_idx [T,k],
+ * topk_w [T,k], counts [E], drop_mask [T*k]; logits_out [T,E] float32 or NULL. No host
+ * synchronisation: launch grids come from upper bounds and kernels read counts on the device. */
+moe_status moe_layer_forward(const moe_shape* shape, const void* x, const void* w_router,
+                             const float* logit_bias, const void* w_gate, const void* w_up,
+                             const void* w_down, void* out, float* logits_out,
+                             int32_t* topk_idx, float* topk_w, int32_t* counts,
+                             uint8_t* drop_mask, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, reads and clears the device error word at the start of `ws`.
+ * Returns MOE_OK, MOE_ERR_DEVICE (a kernel flagged a fault; see moe_last_error_detail) or
+ * MOE_ERR_CUDA. */
+moe_status moe_check_error(void* ws, void* stream);
+
+/* Static description of a status code. */
+const char* moe_status_string(moe_status status);
+
+/* Human-readable detail of the last error returned on the calling thread (which argument
+ * failed validation, the CUDA error string, the device error code). Never NULL. */
+const char* moe_last_error_detail(void);
+
+/* Profiling hook. When `events` is non-NULL, moe_layer_forward records events[i] (cudaEvent_t
+ * passed as void*) on its stream after stage i: 0 route, 1 align, 2 expert GEMM1 (gate/up +
+ * SwiGLU), 3 expert GEMM2 (down projection), 4 combine. n_events must be 5 (or 0 with NULL to
+ * switch recording off). The setting is process-wide. */
+moe_status moe_set_stage_events(void** events, int32_t n_events);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,124 @@
+"""Helpers for the GPU-vs-oracle parity tests: input marshalling and comparison rules.
+
+Inputs always flow from the seeded generators (or from the oracle) into the CUDA library,
+never from the CUDA library into the oracle. Where floating point decides an integer (the top-k
+choice from gate logits that both sides compute in their own summation order), tokens whose
+decision is fragile are identified from the oracle's logits and compared for validity only.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import moe_oracle as orc
+
+# Layer-output tolerances: max-abs error relative to max |reference|.
+TOL_OUT = {"f32": 1e-4, "bf16": 2e-2}
+# Gate-logit tolerances (relative to max |reference logit|).
+TOL_LOGITS = {"f32": 1e-5, "bf16": 1e-3}
+# Routing weights from identical float32 logits: a few float32 ulp of values <= 1.
+TOL_W = 1e-6
+
+
+def np32(t):
+    """Tensor -> float32 numpy (exact for bf16 and f32)."""
+    return t.detach().float().cpu().numpy()
+
+
+def npi(t):
+    return t.detach().cpu().numpy()
+
+
+class ExpertWeights:
+    """Expert e's matrix as float64 numpy, copied from a (device) [E, a, b] tensor on demand
+    (not cached: the oracle visits each expert once, and the workload weights are large)."""
+
+    def __init__(self, w):
+        self.w = w
+
+    def __getitem__(self, e):
+        return self.w[int(e)].detach().cpu().double().numpy()
+
+    def __len__(self):
+        return self.w.shape[0]
+
+
+def rel_err(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    scale = float(np.max(np.abs(ref))) if ref.size else 0.0
+    err = float(np.max(np.abs(got - ref))) if ref.size else 0.0
+    return err / scale if scale > 0 else err, err, scale
+
+
+def assert_close_rel(got, ref, tol, what=""):
+    r, err, scale = rel_err(got, ref)
+    assert r <= tol, f"{what}: max|err| = {err:.3e}, max|ref| = {scale:.3e}, ratio {r:.3e} > {tol}"
+    return r
+
+
+def decided_tokens(logits_ref, k, delta):
+    """Tokens whose top-k list (set and order) cannot change under a perturbation of every logit
+    by at most delta: every gap among the k+1 largest logits exceeds 2*delta (ties decided by
+    index need exactly equal values, which a perturbation can break, so they count as fragile
+    unless delta == 0)."""
+    l = np.asarray(logits_ref, dtype=np.float64)
+    T, E = l.shape
+    kk = min(k + 1, E)
+    top = -np.sort(-l, axis=1)[:, :kk]
+    if kk < 2:
+        return np.ones(T, dtype=bool)
+    gaps = top[:, :-1] - top[:, 1:]
+    if delta == 0:
+        return np.ones(T, dtype=bool)
+    return np.all(gaps > 2.0 * delta, axis=1)
+
+
+def check_topk_valid(logits_ref, idx_gpu, k, delta, rows):
+    """Fragile tokens: the GPU's set must be a top-k of some perturbation within delta."""
+    l = np.asarray(logits_ref, dtype=np.float64)
+    for t in rows:
+        sel = set(int(e) for e in idx_gpu[t])
+        assert len(sel) == k
+        kth = -np.sort(-l[t])[k - 1]
+        for e in range(l.shape[1]):
+            if e in sel:
+                assert l[t, e] >= kth - 2 * delta - 1e-30
+            else:
+                assert l[t, e] <= kth + 2 * delta + 1e-30
+
+
+def check_align_valid(idx, E, C, counts, offsets, sorted_ids, slot_of, drop):
+    """Align invariants on any routing (no oracle call): counts = min(raw, C); offsets scan;
+    slots are a bijection onto kept assignments; the kept ones of each expert are its first C
+    assignments in token order and occupy its slot range in that order."""
+    idx = np.asarray(idx).reshape(-1)
+    A = idx.size
+    raw = np.bincount(idx, minlength=E)
+    assert np.array_equal(counts, np.minimum(raw, C))
+    assert offsets[0] == 0 and np.array_equal(np.diff(offsets), counts)
+    kept = int(offsets[-1])
+    assert np.all(sorted_ids[kept:] == -1)
+    order = np.argsort(idx, kind="stable")  # assignments grouped by expert, token order inside
+    pos = 0
+    for e in range(E):
+        mine = order[pos:pos + raw[e]]
+        pos += raw[e]
+        keep = mine[:C]
+        assert np.array_equal(sorted_ids[offsets[e]:offsets[e + 1]], keep)
+        assert np.all(slot_of[keep] == np.arange(offsets[e], offsets[e + 1]))
+        assert np.all(drop[keep] == 0)
+        assert np.all(slot_of[mine[C:]] == -1) and np.all(drop[mine[C:]] == 1)
+
+
+def inputs_np(inp):
+    """Host copies of the activations/router inputs (weights stay lazy)."""
+    return {
+        "x": np32(inp["x"]),
+        "w_router": np32(inp["w_router"]),
+        "logit_bias": None if inp.get("logit_bias") is None else np32(inp["logit_bias"]),
+    }
+
+
+def to_dev(a, dtype=torch.int32, device="cuda"):
+    return torch.as_tensor(np.ascontiguousarray(a)).to(device=device, dtype=dtype)

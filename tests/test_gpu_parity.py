@@ -1,0 +1,322 @@
+"""CUDA path vs the CPU oracle, through the C ABI (libmoe.so), on one B200.
+
+Every stage is tested on oracle-produced inputs (bit-exact for integer outputs, tolerance for
+floating point), then the whole layer is compared, at small sizes in full and at the workload
+sizes on sampled tokens/slots.
+"""
+import numpy as np
+import pytest
+import torch
+
+from expert_dispatch_gate_b200 import _lib as L
+from expert_dispatch_gate_b200 import layer as M
+from expert_dispatch_gate_b200 import workloads as W
+from oracle import moe_oracle as orc
+from tests.parity import (TOL_LOGITS, TOL_OUT, TOL_W, ExpertWeights, assert_close_rel,
+                          check_topk_valid, decided_tokens, inputs_np, np32, npi, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+# Parity sizes: several tiles and ragged tails, oracle-friendly.
+SMALL = {
+    "tiny": W.WORKLOADS["tiny"],
+    "e8_two_token_blocks": W.Workload("e8", 10, 1500, 128, 8, 2, 256, "bf16", 1.25),
+    "e32_ragged": W.Workload("e32", 11, 517, 256, 32, 4, 384, "bf16", 1.25),
+    "e64_zipf": W.Workload("e64z", 12, 300, 256, 64, 6, 256, "bf16", 1.25, zipf_s=1.2),
+    "e256_k8": W.Workload("e256", 13, 200, 128, 256, 8, 128, "bf16", 1.25),
+    "e16_nocap": W.Workload("e16n", 14, 97, 256, 16, 4, 256, "bf16", 0.0),
+    "dense_e1": W.Workload("e1", 15, 130, 128, 1, 1, 128, "bf16", 1.25),
+    "e64_k16_f32": W.Workload("e64f", 16, 77, 64, 64, 16, 96, "f32", 1.0),
+}
+
+
+@pytest.fixture(scope="session", autouse=True)
+def cuda_ready():
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    L.lib()  # fails loudly when libmoe.so is missing
+
+
+_cache = {}
+
+
+def small_inputs(name):
+    if name not in _cache:
+        wl = SMALL[name]
+        cpu = W.make_inputs(wl, "cpu")
+        dev = {k: (None if v is None else v.cuda()) for k, v in cpu.items()}
+        _cache[name] = (wl, cpu, dev)
+    return _cache[name]
+
+
+def oracle_routing(wl, cpu):
+    host = inputs_np(cpu)
+    logits = orc.router_logits(host["x"], host["w_router"], host["logit_bias"])
+    idx = orc.select_topk(logits, wl.k)
+    w = orc.route_weights(logits, idx)
+    C = orc.capacity(wl.T, wl.k, wl.E, wl.capacity_factor)
+    return logits, idx, w, C, orc.align(idx, wl.E, C)
+
+
+# ----------------------------------------------------------------- route (selection only)
+
+@pytest.mark.parametrize("T,E,k,ties", [
+    (1, 8, 2, False), (300, 8, 1, True), (300, 64, 6, True), (1000, 256, 8, True),
+    (257, 256, 16, False), (33, 16, 16, True), (4096, 256, 8, False), (129, 128, 4, True),
+])
+def test_route_from_logits_bitexact(T, E, k, ties):
+    logits = W.random_logits(T, E, seed=T * 7 + E + k, ties=ties)
+    idx_g, w_g = M.route_from_logits(logits.cuda(), k)
+    torch.cuda.synchronize()
+    l32 = logits.numpy()
+    idx_o = orc.select_topk(l32, k)
+    w_o = orc.route_weights(l32, idx_o)
+    assert np.array_equal(npi(idx_g), idx_o)
+    np.testing.assert_allclose(npi(w_g), w_o, atol=TOL_W, rtol=0)
+    np.testing.assert_allclose(npi(w_g).astype(np.float64).sum(1), 1.0, atol=k * 2.0 ** -23 * 2)
+
+
+# ----------------------------------------------------------------- route (gate GEMM + selection)
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_router(name):
+    wl, cpu, dev = small_inputs(name)
+    idx_g, w_g, logits_g = M.route(dev["x"], dev["w_router"], wl.k, dev["logit_bias"])
+    torch.cuda.synchronize()
+    L_o, idx_o, w_o, _, _ = oracle_routing(wl, cpu)
+    L_g = np32(logits_g)
+    tol = TOL_LOGITS[wl.dtype] * max(1.0, float(np.abs(L_o).max()))
+    delta = float(np.abs(L_g - L_o).max())
+    assert delta <= tol, (delta, tol)
+    dec = decided_tokens(L_o, wl.k, delta)
+    idx_g = npi(idx_g)
+    assert np.array_equal(idx_g[dec], idx_o[dec])
+    check_topk_valid(L_o, idx_g, wl.k, delta, np.nonzero(~dec)[0])
+    np.testing.assert_allclose(npi(w_g)[dec], w_o[dec], atol=TOL_W + wl.k * delta, rtol=0)
+    # the selection the kernel made is exactly the rule applied to the logits it exported
+    # (checked by the selection-only kernel on the same values, bit for bit)
+    idx_s, w_s = M.route_from_logits(logits_g, wl.k)
+    assert torch.equal(idx_s.cpu(), torch.as_tensor(idx_g))
+
+
+# ----------------------------------------------------------------- align
+
+@pytest.mark.parametrize("T,E,k,cf,mode", [
+    (1, 256, 8, 1.25, "uniform"), (64, 8, 2, 0.0, "uniform"), (5000, 8, 2, 1.25, "zipf"),
+    (4096, 256, 8, 1.25, "uniform"), (4096, 256, 8, 1.25, "zipf"), (3000, 64, 6, 1.25, "zipf"),
+    (2500, 16, 4, 1.0, "one"), (777, 32, 3, 0.5, "uniform"), (2049, 1, 1, 1.25, "one"),
+    (20000, 64, 6, 1.25, "zipf"),
+])
+def test_align_bitexact(T, E, k, cf, mode):
+    idx = W.random_topk_idx(T, E, k, seed=T + 31 * E + k, mode=mode)
+    res = M.align(idx.cuda(), E, cf)
+    torch.cuda.synchronize()
+    C = orc.capacity(T, k, E, cf)
+    assert res["C"] == C
+    al = orc.align(idx.numpy(), E, C)
+    for key in ("counts", "offsets", "sorted_ids", "slot_of", "drop_mask"):
+        assert np.array_equal(npi(res[key]), al[key]), key
+    assert res["ws"].check() == L.MOE_OK
+
+
+def test_align_every_expert_exactly_at_capacity():
+    # T = 64, E = 8, k = 1, cf = 1: C = 8 and each expert gets exactly 8 tokens: no drops
+    idx = torch.arange(64, dtype=torch.int32).remainder(8).reshape(64, 1)
+    res = M.align(idx.cuda(), 8, 1.0)
+    al = orc.align(idx.numpy(), 8, 8)
+    assert npi(res["drop_mask"]).sum() == 0
+    for key in ("counts", "offsets", "sorted_ids", "slot_of", "drop_mask"):
+        assert np.array_equal(npi(res[key]), al[key]), key
+
+
+def test_align_flags_out_of_range_expert_ids():
+    idx = W.random_topk_idx(100, 16, 2, seed=3)
+    idx[7, 1] = 16
+    idx[50, 0] = -3
+    res = M.align(idx.cuda(), 16, 0.0)
+    with pytest.raises(L.MoeError) as ei:
+        res["ws"].check()
+    assert ei.value.status == L.MOE_ERR_DEVICE
+    drop = npi(res["drop_mask"])
+    assert drop[7 * 2 + 1] == 1 and drop[50 * 2] == 1
+    assert res["ws"].check() == L.MOE_OK  # the error word was cleared
+
+
+# ----------------------------------------------------------------- grouped FFN
+
+def _ffn_check(wl, x_dev, weights_dev, al, slots, x_host=None):
+    y = M.grouped_ffn(x_dev, to_dev(al["sorted_ids"]), to_dev(al["offsets"]), weights_dev[0],
+                      weights_dev[1], weights_dev[2], wl.k, wl.capacity_factor)
+    torch.cuda.synchronize()
+    xh = np32(x_dev) if x_host is None else x_host
+    ref = orc.grouped_ffn_slots(xh, al["sorted_ids"], al["offsets"], wl.k,
+                                ExpertWeights(weights_dev[0]), ExpertWeights(weights_dev[1]),
+                                ExpertWeights(weights_dev[2]), slots=slots)
+    got = np32(y[torch.as_tensor(sorted(ref), dtype=torch.long, device=y.device)])
+    want = np.stack([ref[s] for s in sorted(ref)])
+    return assert_close_rel(got, want, TOL_OUT[wl.dtype], "expert outputs")
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_grouped_ffn(name):
+    wl, cpu, dev = small_inputs(name)
+    _, _, _, _, al = oracle_routing(wl, cpu)
+    kept = int(al["offsets"][-1])
+    _ffn_check(wl, dev["x"], (dev["w_gate"], dev["w_up"], dev["w_down"]), al, list(range(kept)))
+
+
+# ----------------------------------------------------------------- combine
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_combine(name):
+    wl, cpu, dev = small_inputs(name)
+    _, _, w_o, _, al = oracle_routing(wl, cpu)
+    y = W.make_y_slots(wl, "cpu")
+    w32 = w_o.astype(np.float32)
+    out = M.combine(y.cuda(), to_dev(al["slot_of"]), to_dev(w32, torch.float32), wl.E)
+    torch.cuda.synchronize()
+    ref = orc.combine(np32(y), al["slot_of"], w32)
+    got = np32(out)
+    assert_close_rel(got, ref, TOL_OUT[wl.dtype], "combine")
+    # arithmetic bound: fp32 accumulation, one final rounding to the output type
+    ulp = 2.0 ** -8 if wl.dtype == "bf16" else 2.0 ** -22
+    assert np.all(np.abs(got - ref) <= ulp * np.abs(ref) + 1e-6 * np.abs(ref).max())
+    dropped_all = np.all(al["slot_of"].reshape(wl.T, wl.k) < 0, axis=1)
+    assert np.all(got[dropped_all] == 0.0)
+
+
+# ----------------------------------------------------------------- whole layer
+
+def compare_layer(wl, cpu_or_dev, dev, res, sample=None, seed=0):
+    """Compare moe_layer_forward's outputs with the oracle (see module docstring of parity)."""
+    host = inputs_np(cpu_or_dev)
+    T, E, k = wl.T, wl.E, wl.k
+    L_o = orc.router_logits(host["x"], host["w_router"], host["logit_bias"])
+    L_g = np32(res["logits"])
+    tol = TOL_LOGITS[wl.dtype] * max(1.0, float(np.abs(L_o).max()))
+    delta = float(np.abs(L_g - L_o).max())
+    assert delta <= tol, (delta, tol)
+    idx_o = orc.select_topk(L_o, k)
+    w_o = orc.route_weights(L_o, idx_o)
+    idx_g, w_g = npi(res["topk_idx"]), npi(res["topk_w"])
+    dec = decided_tokens(L_o, k, delta)
+    assert np.array_equal(idx_g[dec], idx_o[dec])
+    check_topk_valid(L_o, idx_g, k, delta, np.nonzero(~dec)[0])
+    np.testing.assert_allclose(w_g[dec], w_o[dec], atol=TOL_W + k * delta, rtol=0)
+    C = orc.capacity(T, k, E, wl.capacity_factor)
+    assert res["C"] == C
+    al = orc.align(idx_o, E, C)
+    counts_g, drop_g = npi(res["counts"]), npi(res["drop_mask"])
+    # the GPU's grouping is valid for the GPU's own routing (invariants, no oracle call)
+    raw_g = np.bincount(idx_g.reshape(-1), minlength=E)
+    assert np.array_equal(counts_g, np.minimum(raw_g, C))
+    flat_g = idx_g.reshape(-1)
+    order = np.argsort(flat_g, kind="stable")
+    pos = 0
+    for e in range(E):
+        mine = order[pos:pos + raw_g[e]]
+        pos += raw_g[e]
+        assert np.all(drop_g[mine[:C]] == 0) and np.all(drop_g[mine[C:]] == 1)
+    # experts untouched by fragile tokens: identical counts and drops
+    tainted = set(idx_o[~dec].reshape(-1).tolist()) | set(idx_g[~dec].reshape(-1).tolist())
+    clean = np.array([e not in tainted for e in range(E)])
+    assert np.array_equal(counts_g[clean], al["counts"][clean])
+    flat_o = idx_o.reshape(-1)
+    sel = clean[flat_o]
+    assert np.array_equal(drop_g[sel], al["drop_mask"][sel])
+    # outputs on tokens whose routing and ranks are the same on both sides
+    comparable = [t for t in range(T) if dec[t] and not (set(idx_o[t].tolist()) & tainted)]
+    assert len(comparable) >= min(T, 1)
+    if sample is not None and len(comparable) > sample:
+        rng = np.random.default_rng(seed)
+        comparable = sorted(rng.choice(comparable, size=sample, replace=False).tolist())
+    ref = orc.layer_forward(host["x"], host["w_router"], ExpertWeights(dev["w_gate"]),
+                            ExpertWeights(dev["w_up"]), ExpertWeights(dev["w_down"]), k,
+                            wl.capacity_factor, logit_bias=host["logit_bias"], tokens=comparable)
+    got = np32(res["out"])[comparable]
+    r = assert_close_rel(got, ref["out"], TOL_OUT[wl.dtype], "layer output")
+    return {"delta_logits": delta, "fragile": int((~dec).sum()), "compared": len(comparable),
+            "rel_err": r}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_small(name):
+    wl, cpu, dev = small_inputs(name)
+    res = M.layer_forward(dev["x"], dev["w_router"], dev["w_gate"], dev["w_up"], dev["w_down"],
+                          wl.k, wl.capacity_factor, logit_bias=dev["logit_bias"])
+    torch.cuda.synchronize()
+    assert res["ws"].check() == L.MOE_OK
+    compare_layer(wl, cpu, dev, res)
+    # determinism: a second run gives the same bits
+    res2 = M.layer_forward(dev["x"], dev["w_router"], dev["w_gate"], dev["w_up"], dev["w_down"],
+                           wl.k, wl.capacity_factor, logit_bias=dev["logit_bias"], ws=res["ws"])
+    torch.cuda.synchronize()
+    for key in ("out", "topk_idx", "topk_w", "counts", "drop_mask", "logits"):
+        assert torch.equal(res[key], res2[key]), key
+
+
+def test_layer_empty_batch():
+    wl = SMALL["e8_two_token_blocks"].with_tokens(0)
+    dev = {k: (None if v is None else v.cuda()) for k, v in W.make_inputs(wl, "cpu").items()}
+    res = M.layer_forward(dev["x"], dev["w_router"], dev["w_gate"], dev["w_up"], dev["w_down"],
+                          wl.k, wl.capacity_factor)
+    torch.cuda.synchronize()
+    assert res["out"].shape == (0, wl.H)
+    assert int(res["counts"].sum()) == 0
+
+
+def test_layer_heavy_drops_give_zero_rows():
+    # cf = 0.05 -> C = ceil(0.05*400*2/8) = 5: most assignments dropped, many tokens fully
+    wl = W.Workload("drops", 17, 400, 128, 8, 2, 128, "bf16", 0.05)
+    cpu = W.make_inputs(wl, "cpu")
+    dev = {k: (None if v is None else v.cuda()) for k, v in cpu.items()}
+    res = M.layer_forward(dev["x"], dev["w_router"], dev["w_gate"], dev["w_up"], dev["w_down"],
+                          wl.k, wl.capacity_factor)
+    torch.cuda.synchronize()
+    assert res["C"] == 5
+    drop = npi(res["drop_mask"]).reshape(wl.T, wl.k)
+    assert int(npi(res["counts"]).sum()) <= 5 * wl.E
+    out = np32(res["out"])
+    assert np.all(out[np.all(drop == 1, axis=1)] == 0.0)
+    compare_layer(wl, cpu, dev, res)
+
+
+# ----------------------------------------------------------------- workload sizes (sampled)
+
+FULL = [("mixtral", None), ("fine", None), ("skewed", None), ("decode", 1), ("decode", 16),
+        ("decode", 64), ("decode", 256)]
+
+
+def _full_inputs(name, T):
+    wl = W.WORKLOADS[name] if T is None else W.WORKLOADS[name].with_tokens(T)
+    dev = W.make_inputs(wl, "cuda")
+    return wl, dev
+
+
+@pytest.mark.parametrize("name,T", FULL)
+def test_layer_workload_sizes(name, T):
+    wl, dev = _full_inputs(name, T)
+    res = M.layer_forward(dev["x"], dev["w_router"], dev["w_gate"], dev["w_up"], dev["w_down"],
+                          wl.k, wl.capacity_factor, logit_bias=dev["logit_bias"])
+    torch.cuda.synchronize()
+    assert res["ws"].check() == L.MOE_OK
+    info = compare_layer(wl, dev, dev, res, sample=12 if wl.E > 8 else 24)
+    print(name, T, info)
+    # per-stage checks on oracle-made inputs at this size
+    host = inputs_np(dev)
+    L_o = orc.router_logits(host["x"], host["w_router"], host["logit_bias"])
+    idx_s, w_s = M.route_from_logits(torch.as_tensor(L_o).cuda(), wl.k)
+    idx_o = orc.select_topk(L_o, wl.k)
+    assert np.array_equal(npi(idx_s), idx_o)
+    np.testing.assert_allclose(npi(w_s), orc.route_weights(L_o, idx_o), atol=TOL_W, rtol=0)
+    C = orc.capacity(wl.T, wl.k, wl.E, wl.capacity_factor)
+    al_o = orc.align(idx_o, wl.E, C)
+    al_g = M.align(to_dev(idx_o), wl.E, wl.capacity_factor, H=wl.H, I=wl.I)
+    for key in ("counts", "offsets", "sorted_ids", "slot_of", "drop_mask"):
+        assert np.array_equal(npi(al_g[key]), al_o[key]), key
+    # expert outputs for every slot of a few experts: the fullest, a ragged one, the last
+    counts = al_o["counts"]
+    nz = np.nonzero(counts)[0]
+    pick = sorted({int(nz[np.argmax(counts[nz])]), int(nz[len(nz) // 2]), int(nz[-1])})
+    slots = [s for e in pick for s in range(al_o["offsets"][e], al_o["offsets"][e + 1])]
+    _ffn_check(wl, dev["x"], (dev["w_gate"], dev["w_up"], dev["w_down"]), al_o, slots,
+               x_host=host["x"])
