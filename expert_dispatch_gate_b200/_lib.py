@@ -52,6 +52,7 @@ def _signatures(lib):
         "moe_route": (st, [S, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
         "moe_route_from_logits": (st, [S, _P, _P, _P, _P]),
         "moe_align": (st, [S, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
+        "moe_align_noalloc": (st, [S, _P, _P, _P, _P, _P, _P, _P]),
         "moe_grouped_ffn": (st, [S, _P, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
         "moe_combine": (st, [S, _P, _P, _P, _P, _P]),
         "moe_layer_forward": (st, [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
@@ -154,6 +155,13 @@ def moe_align(shape, topk_idx, counts, offsets, sorted_ids, slot_of, drop_mask, 
     s = lib().moe_align(ctypes.byref(shape), ptr(topk_idx), ptr(counts), ptr(offsets),
                         ptr(sorted_ids), ptr(slot_of), ptr(drop_mask), ptr(ws), int(ws_bytes),
                         _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_align_noalloc(shape, topk_idx, counts, offsets, sorted_ids, slot_of, drop_mask,
+                      stream=None, check=True):
+    s = lib().moe_align_noalloc(ctypes.byref(shape), ptr(topk_idx), ptr(counts), ptr(offsets),
+                                ptr(sorted_ids), ptr(slot_of), ptr(drop_mask), _stream(stream))
     return _check(s) if check else s
 
 

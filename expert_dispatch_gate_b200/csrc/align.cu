@@ -16,6 +16,8 @@
 //               plan blk_prefix used by the expert GEMMs.
 //   3. scatter: per chunk, stable in-chunk ranks (warp __match_any_sync + per-warp prefix),
 //               then slot = offsets[e] + rank for kept assignments; fills the -1 tail.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -201,6 +203,55 @@ cudaError_t launch_align(const int32_t* topk_idx, int64_t A, int E, int C, int T
   align_scatter_kernel<<<nblk, kThreads, 0, stream>>>(topk_idx, A, E, C, blk_hist, offsets,
                                                       sorted_ids, slot_of, drop_mask);
   return cudaGetLastError();
+}
+
+// ---- grouping without a caller workspace
+//
+// Scratch of moe_align_noalloc, a variant of the launch sequence above for callers that may
+// not allocate device memory. It holds the per-chunk histograms of up to
+// kNoAllocMaxAssignments assignments for up to 256 experts, the token-block plan and an
+// error word: about 130 KB, resident on every device that loads the library until the
+// process exits. All calls share it, so calls that overlap on the GPU (different streams,
+// different host threads) race on it and must be serialised by the caller.
+namespace {
+struct NoAllocScratch {
+  int err[64];
+  int blk_prefix[320];
+  int blk_hist[(kNoAllocMaxAssignments / kAlignChunk) * 256];
+};
+static __device__ __align__(256) NoAllocScratch g_noalloc_scratch;
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+}  // namespace
+
+cudaError_t launch_align_noalloc(const int32_t* topk_idx, int64_t A, int E, int C, int TB,
+                                 int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
+                                 int32_t* slot_of, uint8_t* drop_mask, cudaStream_t stream) {
+  if (A > kNoAllocMaxAssignments || E > 256) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  void* base = nullptr;
+  {
+    // In host code g_noalloc_scratch names a host-side stand-in, not device memory: the
+    // device address is looked up once per device, with that device current.
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return e;
+      g_noalloc_ptr[dev] = p;
+    }
+    base = g_noalloc_ptr[dev];
+  }
+  NoAllocScratch* sc = static_cast<NoAllocScratch*>(base);
+  // The error word must start at zero; the histograms and the plan are fully rewritten.
+  e = cudaMemsetAsync(sc->err, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return e;
+  return launch_align(topk_idx, A, E, C, TB, sc->blk_hist, counts, offsets, sc->blk_prefix,
+                      sorted_ids, slot_of, drop_mask, sc->err, stream);
 }
 
 cudaError_t launch_plan_from_offsets(const int32_t* offsets, int E, int TB, int32_t* blk_prefix,

@@ -48,6 +48,12 @@ cudaError_t launch_align(const int32_t* topk_idx, int64_t A, int E, int C, int T
                          int32_t* blk_hist, int32_t* counts, int32_t* offsets,
                          int32_t* blk_prefix, int32_t* sorted_ids, int32_t* slot_of,
                          uint8_t* drop_mask, int* err, cudaStream_t stream);
+// Same grouping with its scratch in a file-scope device array instead of a workspace;
+// at most kNoAllocMaxAssignments assignments and 256 experts.
+constexpr int64_t kNoAllocMaxAssignments = 262144;
+cudaError_t launch_align_noalloc(const int32_t* topk_idx, int64_t A, int E, int C, int TB,
+                                 int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
+                                 int32_t* slot_of, uint8_t* drop_mask, cudaStream_t stream);
 // blk_prefix[e] = sum over e' < e of ceil(count[e'] / TB), count from offsets.
 cudaError_t launch_plan_from_offsets(const int32_t* offsets, int E, int TB, int32_t* blk_prefix,
                                      cudaStream_t stream);

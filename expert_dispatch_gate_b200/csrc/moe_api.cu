@@ -303,6 +303,36 @@ moe_status moe_align(const moe_shape* shape, const int32_t* topk_idx, int32_t* c
   return MOE_OK;
 }
 
+moe_status moe_align_noalloc(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts,
+                             int32_t* offsets, int32_t* sorted_ids, int32_t* slot_of,
+                             uint8_t* drop_mask, void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  REQUIRE_PTR(counts, "counts");
+  REQUIRE_PTR(offsets, "offsets");
+  const Layout L = layout_of(*shape);
+  if (L.A > moe::kNoAllocMaxAssignments)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "moe_align_noalloc handles at most " + std::to_string(moe::kNoAllocMaxAssignments) +
+                    " assignments (T*k); got " + std::to_string(L.A) +
+                    ": use moe_align with a workspace");
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (shape->T == 0) {
+    cudaError_t e = cudaMemsetAsync(counts, 0, static_cast<size_t>(shape->E) * 4, cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, static_cast<size_t>(shape->E + 1) * 4, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "align without workspace (empty batch)");
+    return MOE_OK;
+  }
+  REQUIRE_PTR(topk_idx, "topk_idx");
+  REQUIRE_PTR(sorted_ids, "sorted_ids");
+  REQUIRE_PTR(slot_of, "slot_of");
+  REQUIRE_PTR(drop_mask, "drop_mask");
+  cudaError_t e = moe::launch_align_noalloc(topk_idx, L.A, shape->E, L.C, L.TB, counts, offsets,
+                                            sorted_ids, slot_of, drop_mask, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "align without workspace");
+  return MOE_OK;
+}
+
 moe_status moe_grouped_ffn(const moe_shape* shape, const void* x, const int32_t* sorted_ids,
                            const int32_t* offsets, const void* w_gate, const void* w_up,
                            const void* w_down, void* y_slots, void* ws, size_t ws_bytes,

@@ -107,6 +107,26 @@ moe_status moe_align(const moe_shape* shape, const int32_t* topk_idx, int32_t* c
                      int32_t* offsets, int32_t* sorted_ids, int32_t* slot_of,
                      uint8_t* drop_mask, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_align without a workspace, for callers that cannot allocate device memory: code that
+ * runs inside another framework's memory planner, which hands out only the tensors it owns,
+ * or on a latency-critical path where a cudaMalloc could stall the device or fail under memory
+ * pressure. The pages have no counterpart to this call: it is a deployment variant of
+ * moe_align with identical arguments and results, minus ws/ws_bytes.
+ *   Its scratch (per-chunk histograms, the token-block plan, an error word; about 130 KB) is
+ *   a file-scope __device__ array inside libmoe.so that every device loading the library keeps
+ *   until the process exits. The first call on a device looks up that array's device address
+ *   (cudaGetSymbolAddress) with the device current; make that first call before any stream
+ *   capture. The call itself allocates nothing: no cudaMalloc, cudaFree or allocating library
+ *   routine.
+ *   Limits: T*k <= 262144 assignments and E <= 256; larger batches return MOE_ERR_UNSUPPORTED
+ *   (use moe_align with a workspace). All calls share the one scratch array, which keeps the
+ *   last call's contents: calls that overlap on the GPU (other streams or host threads) race on
+ *   it and must be serialised by the caller. Expert ids outside [0,E) are treated as dropped;
+ *   this call does not report them (moe_check_error reads a workspace, which it has none of). */
+moe_status moe_align_noalloc(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts,
+                             int32_t* offsets, int32_t* sorted_ids, int32_t* slot_of,
+                             uint8_t* drop_mask, void* stream);
+
 /* Grouped SwiGLU expert FFN, [P1] section "FlashAttention 在 MoE 模型里的位置" step 4 and
  * section "手动编译 MoE 融合算子" (activation "silu"): for every kept slot s of expert e (offsets[e]
  * <= s < offsets[e+1]) with token t = sorted_ids[s] / k:
