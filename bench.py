@@ -262,10 +262,13 @@ def oracle_baseline(wl, dev, n_tokens, reps=1):
 
 # ------------------------------------------------------------------ the GPU arm
 
+def workload_of(args):
+    wl = W.WORKLOADS.get(args.workload) or W.PROFILE_WORKLOADS[args.workload]
+    return wl.with_tokens(args.tokens) if args.tokens else wl
+
+
 def run_ours(args, world, rank, local):
-    wl = W.WORKLOADS[args.workload]
-    if args.tokens:
-        wl = wl.with_tokens(args.tokens)
+    wl = workload_of(args)
     dev = torch.device("cuda", local)
     inp = W.make_inputs(wl, dev)
     peaks, peaks_src = load_peaks()
@@ -415,9 +418,7 @@ def run_reference(args, world, rank, local):
     """The reference arm: the CPU oracle itself, on the same workload, bounded samples."""
     if rank != 0:
         return None
-    wl = W.WORKLOADS[args.workload]
-    if args.tokens:
-        wl = wl.with_tokens(args.tokens)
+    wl = workload_of(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = W.make_inputs(wl, dev)
     n_tok = max(1, args.cpu_sample_tokens // 4)
@@ -459,7 +460,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="fine", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="fine",
+                    choices=sorted(W.WORKLOADS) + sorted(W.PROFILE_WORKLOADS))
     ap.add_argument("--tokens", type=int, default=0, help="override T (decode sweep)")
     ap.add_argument("--cpu-sample-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -10,9 +10,12 @@
 //     weights are streamed from HBM once per tile, whatever its token count; a decode step with
 //     one token per expert pays for N = 16 columns of MMA, not 128 rows.
 //   * A (weights, MN-major: features contiguous) arrives by 3-D TMA tiles of 64x64 bf16 with
-//     128-byte swizzle; B (token rows, K-major) arrives by TMA tile::gather4 straight from the
-//     unpermuted activations using the grouping's slot -> token map, so no permuted copy of x is
-//     ever written.
+//     128-byte swizzle. B (token rows, K-major, same swizzle) arrives in one of three ways:
+//       - contiguous rows (router: x rows; GEMM2: slot-major h rows): 2-D TMA boxes of 32 rows;
+//       - gathered rows by cp.async from four producer warps that read the grouping's
+//         slot -> token map and write the swizzled layout themselves (GEMM1: x rows straight
+//         from the unpermuted activations, so no permuted copy of x is ever written);
+//       - gathered rows by TMA tile::gather4 (four rows per instruction; kept as an option).
 //   * tcgen05.mma accumulates in TMEM (fp32); GEMM1 keeps gate and up accumulators side by side
 //     so one epilogue thread owns both values of a (feature, token) pair and applies SwiGLU.
 //   * Persistent CTAs (one per SM), warp-specialised: warp 0 issues TMA, warp 1 issues MMAs,
@@ -29,7 +32,7 @@ namespace {
 
 constexpr int kBM = 128;        // MMA M: output features per tile
 constexpr int kBK = 64;         // K per pipeline stage: one 128-byte swizzle row of bf16
-constexpr int kThreads = 192;   // 6 warps
+constexpr int kRowBox = 32;     // rows per 2-D TMA box of B in the contiguous-rows mode
 constexpr int kMaxStages = 8;
 constexpr int kMaxGroups = 256;
 constexpr int kTmemCols = 512;
@@ -37,6 +40,12 @@ constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory per b
 constexpr int kCtrlBytes = 2560;    // barriers + group tables
 
 enum EpiMode { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2 };
+// How the B operand (token rows) reaches shared memory.
+enum BMode { kBGather4 = 0, kBTiled = 1, kBCpAsync = 2 };
+
+// Warps: 0 TMA producer, 1 MMA issuer, 2-5 epilogue, 6-9 cp.async row gatherers (kBCpAsync).
+template <int BMODE>
+constexpr int threads_of() { return BMODE == kBCpAsync ? 320 : 192; }
 
 struct TcParams {
   int K;          // reduction length (multiple of 64)
@@ -47,6 +56,7 @@ struct TcParams {
   int groups;     // experts (ignored when offsets == nullptr)
   int k_top;      // GEMM1: B row = sorted_ids[slot] / k_top
   int rows_b;     // rows of the B tensor
+  const __nv_bfloat16* b_ptr;  // B tensor [rows_b, K] (cp.async gather)
   const int32_t* sorted_ids;
   const int32_t* offsets;     // [groups+1] slot offsets, or nullptr: one group of n_static rows
   const int32_t* blk_prefix;  // [groups+1] token blocks before each group
@@ -82,12 +92,13 @@ __device__ __forceinline__ Tile decode_tile(int tile, int num_fb, int groups, in
   return t;
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int MODE, int BMODE>
+__global__ void __launch_bounds__(threads_of<BMODE>(), 1)
     tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0,
                     const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB, const TcParams p) {
   constexpr bool kSwiGLU = (MODE == kEpiSwiGLU);
+  constexpr uint32_t kFullCount = (BMODE == kBCpAsync) ? 1u + 128u : 1u;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -122,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&full[s]), kFullCount);
       mbar_init(smem_u32(&empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -151,21 +162,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk);
       const int npad = (t.n + 15) & ~15;
+      const int nbox = (t.n + kRowBox - 1) / kRowBox;
       int rows[8];
+      if constexpr (BMODE == kBGather4) {
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < 2; ++q) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int nn = (lane + 32 * q) * 4 + r;
-          const int src = t.row0 + min(nn, t.n - 1);
-          int row = (p.sorted_ids != nullptr) ? (p.sorted_ids[src] / p.k_top) : src;
-          rows[q * 4 + r] = min(max(row, 0), p.rows_b - 1);
+          for (int r = 0; r < 4; ++r) {
+            const int nn = (lane + 32 * q) * 4 + r;
+            const int src = t.row0 + min(nn, t.n - 1);
+            int row = (p.sorted_ids != nullptr) ? (p.sorted_ids[src] / p.k_top) : src;
+            rows[q * 4 + r] = min(max(row, 0), p.rows_b - 1);
+          }
         }
       }
       const int m0 = t.fb * kBM;
       const bool hi_chunk = (m0 + 64) < p.m_rows_a;
-      const uint32_t tx = (hi_chunk ? 16384u : 8192u) * (kSwiGLU ? 2u : 1u) +
-                          static_cast<uint32_t>(npad) * 128u;
+      uint32_t tx = (hi_chunk ? 16384u : 8192u) * (kSwiGLU ? 2u : 1u);
+      if constexpr (BMODE == kBGather4) tx += static_cast<uint32_t>(npad) * 128u;
+      if constexpr (BMODE == kBTiled) tx += static_cast<uint32_t>(nbox) * (kRowBox * 128u);
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = it % S;
         const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
@@ -188,13 +203,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (hi_chunk) tma_load_3d(sa + 16384 + 8192, &tmA1, m0 + 64, kb * kBK, t.group, fbar);
           }
         }
+        if constexpr (BMODE == kBTiled) {
+          if (lane == 0)
+            for (int j = 0; j < nbox; ++j)
+              tma_load_2d(sb + j * (kRowBox * 128), &tmB, kb * kBK, t.row0 + j * kRowBox, fbar);
+        }
         __syncwarp();
+        if constexpr (BMODE == kBGather4) {
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int grp = lane + 32 * q;
-          if (grp * 4 < npad)
-            tma_gather4(sb + grp * 512, &tmB, kb * kBK, rows[q * 4], rows[q * 4 + 1],
-                        rows[q * 4 + 2], rows[q * 4 + 3], fbar);
+          for (int q = 0; q < 2; ++q) {
+            const int grp = lane + 32 * q;
+            if (grp * 4 < npad)
+              tma_gather4(sb + grp * 512, &tmB, kb * kBK, rows[q * 4], rows[q * 4 + 1],
+                          rows[q * 4 + 2], rows[q * 4 + 3], fbar);
+          }
         }
         ++it;
       }
@@ -263,6 +285,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(smem_u32(drain), 0u, nullptr);
     }
     __syncwarp();
+  } else if (BMODE == kBCpAsync && warp >= 6) {
+    // ------------------------------------------------------------ cp.async row gatherers
+    // Thread g (0..127) copies 16-byte chunk (g % 8) of rows g/8, g/8 + 16, ... of each
+    // stage's B tile, writing the 128-byte-swizzled K-major layout the MMA descriptor expects.
+    const int g = threadIdx.x - 6 * 32;
+    const int chunk = g & 7;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk);
+      const int npad = (t.n + 15) & ~15;
+      const int iters = npad >> 4;  // rows per thread
+      const __nv_bfloat16* src[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = (g >> 3) + 16 * i;
+        const int slot = t.row0 + min(r, t.n - 1);
+        int row = (p.sorted_ids != nullptr) ? (p.sorted_ids[slot] / p.k_top) : slot;
+        row = min(max(row, 0), p.rows_b - 1);
+        src[i] = p.b_ptr + static_cast<size_t>(row) * p.K + chunk * 8;
+      }
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = it % S;
+        const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+        int got = 1;
+        if (lane == 0) got = mbar_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          ok = false;
+          break;
+        }
+        const uint32_t sb = smem_u32(smem + static_cast<size_t>(s) * stage_bytes) + a_bytes;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (i < iters) {
+            const int r = (g >> 3) + 16 * i;
+            cp_async_16(sb + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * kBK);
+          }
+        }
+        cp_async_arrive_noinc(smem_u32(&full[s]));
+        ++it;
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) flag_error(p.err, kDevWaitTimeout);
+    }
+    cp_async_wait_all();
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;  // TMEM lane quadrant this warp may read
@@ -377,6 +447,24 @@ bool map_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, st
   return r == CUDA_SUCCESS;
 }
 
+// bf16 [rows, cols] row-major, box = {64 columns, 32 rows}, 128-byte swizzle: contiguous rows.
+bool map_row_boxes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, std::string* d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) {
+    if (d) *d = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, kRowBox};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && d) *d = "cuTensorMapEncodeTiled(row boxes) failed with code " + std::to_string(r);
+  return r == CUDA_SUCCESS;
+}
+
 // bf16 [groups, kdim, mdim] (mdim contiguous), box = {64, 64, 1}, 128-byte swizzle.
 bool map_weights(CUtensorMap* m, const void* base, uint64_t mdim, uint64_t kdim, uint64_t groups,
                  std::string* d) {
@@ -396,7 +484,7 @@ bool map_weights(CUtensorMap* m, const void* base, uint64_t mdim, uint64_t kdim,
   return r == CUDA_SUCCESS;
 }
 
-template <int MODE>
+template <int MODE, int BMODE>
 cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                         TcParams p, int64_t tiles_ub, int num_sms, cudaStream_t stream,
                         std::string* d) {
@@ -413,11 +501,12 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + kCtrlBytes;
   int64_t grid = tiles_ub < num_sms ? tiles_ub : num_sms;
   if (grid < 1) grid = 1;
-  cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE>,
+  cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE, BMODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  tc_grouped_gemm<MODE><<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(a0, a1, b, p);
+  tc_grouped_gemm<MODE, BMODE><<<static_cast<unsigned>(grid), threads_of<BMODE>(), smem, stream>>>(
+      a0, a1, b, p);
   return cudaGetLastError();
 }
 
@@ -428,7 +517,7 @@ cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, const floa
                                  cudaStream_t stream, std::string* detail) {
   CUtensorMap a0, b;
   if (!map_weights(&a0, w_router, static_cast<uint64_t>(E), static_cast<uint64_t>(H), 1, detail) ||
-      !map_rows(&b, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), detail))
+      !map_row_boxes(&b, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), detail))
     return cudaErrorInvalidValue;
   TcParams p{};
   p.K = H;
@@ -448,7 +537,7 @@ cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, const floa
   p.bias = bias;
   p.err = err;
   const int64_t tiles = static_cast<int64_t>(p.num_fb) * ((T + p.TB - 1) / p.TB);
-  return launch_mode<kEpiF32>(a0, a0, b, p, tiles, num_sms, stream, detail);
+  return launch_mode<kEpiF32, kBTiled>(a0, a0, b, p, tiles, num_sms, stream, detail);
 }
 
 cudaError_t launch_gemm1_tc(const void* x, int T, const int32_t* sorted_ids,
@@ -461,6 +550,11 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const int32_t* sorted_ids,
   if (!map_weights(&a0, w_gate, I, H, E, detail) || !map_weights(&a1, w_up, I, H, E, detail) ||
       !map_rows(&b, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), detail))
     return cudaErrorInvalidValue;
+#ifdef MOE_GEMM1_GATHER4
+  const bool use_gather4 = true;   // TMA tile::gather4 row gather (build-time choice)
+#else
+  const bool use_gather4 = false;  // cp.async row gather
+#endif
   TcParams p{};
   p.K = H;
   p.num_fb = I / kBM;
@@ -477,8 +571,11 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const int32_t* sorted_ids,
   p.ldo = I;
   p.bias = nullptr;
   p.err = err;
-  return launch_mode<kEpiSwiGLU>(a0, a1, b, p, static_cast<int64_t>(p.num_fb) * ub_blocks,
-                                 num_sms, stream, detail);
+  p.b_ptr = static_cast<const __nv_bfloat16*>(x);
+  const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
+  if (use_gather4)
+    return launch_mode<kEpiSwiGLU, kBGather4>(a0, a1, b, p, tiles, num_sms, stream, detail);
+  return launch_mode<kEpiSwiGLU, kBCpAsync>(a0, a1, b, p, tiles, num_sms, stream, detail);
 }
 
 cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* offsets,
@@ -487,7 +584,7 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
                             cudaStream_t stream, std::string* detail) {
   CUtensorMap a0, b;
   if (!map_weights(&a0, w_down, H, I, E, detail) ||
-      !map_rows(&b, hbuf, static_cast<uint64_t>(I), static_cast<uint64_t>(hbuf_rows), detail))
+      !map_row_boxes(&b, hbuf, static_cast<uint64_t>(I), static_cast<uint64_t>(hbuf_rows), detail))
     return cudaErrorInvalidValue;
   TcParams p{};
   p.K = I;
@@ -505,8 +602,8 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
   p.ldo = H;
   p.bias = nullptr;
   p.err = err;
-  return launch_mode<kEpiBF16>(a0, a0, b, p, static_cast<int64_t>(p.num_fb) * ub_blocks, num_sms,
-                               stream, detail);
+  return launch_mode<kEpiBF16, kBTiled>(a0, a0, b, p, static_cast<int64_t>(p.num_fb) * ub_blocks,
+                                        num_sms, stream, detail);
 }
 
 }  // namespace moe

@@ -66,6 +66,15 @@ WORKLOADS = {
 }
 DECODE_TOKENS = (1, 16, 64, 256)
 
+# Profiling stand-in for the fine-grained layer: same per-expert shapes and load (C = 160,
+# about 128 tokens per expert) with 32 experts, so a profiler capture holds 1.6 GB of weights
+# (still far larger than L2) instead of 12.9 GB.
+PROFILE_WORKLOADS = {
+    "fine_e32": Workload("fine_e32", 5, 512, 4096, 32, 8, 2048, "bf16", 1.25),
+    # the fine-grained router (T, H, E, k identical) with a small expert FFN
+    "route_fine": Workload("route_fine", 6, 4096, 4096, 256, 8, 128, "bf16", 1.25),
+}
+
 
 def _gen(device, seed):
     g = torch.Generator(device=device)
