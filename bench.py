@@ -262,6 +262,15 @@ def oracle_baseline(wl, dev, n_tokens, reps=1):
 
 # ------------------------------------------------------------------ the GPU arm
 
+def launches_per_step(wl):
+    """Kernels one moe_layer_forward launches: router (tensor-core GEMM + top-k, or one fused
+    CUDA-core kernel), align (one kernel up to 2048 assignments, else three), two expert
+    GEMMs, combine."""
+    route = 2 if (wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0) else 1
+    align = 1 if wl.T * wl.k <= 2048 else 3
+    return route + align + 2 + 1
+
+
 def workload_of(args):
     wl = W.WORKLOADS.get(args.workload) or W.PROFILE_WORKLOADS[args.workload]
     return wl.with_tokens(args.tokens) if args.tokens else wl
@@ -374,8 +383,7 @@ def run_ours(args, world, rank, local):
     h2d = x_host.numel() * x_host.element_size()
     d2h = sum(t.numel() * t.element_size() for t in outs_host)
 
-    launches_route = 2 if (wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0) else 1
-    per_step = launches_route + 3 + 2 + 1
+    per_step = launches_per_step(wl)
     line = {
         "metric": METRIC,
         "value": round(value, 1),

@@ -176,6 +176,86 @@ __global__ void __launch_bounds__(kThreads)
     sorted_ids[s] = -1;
 }
 
+// Whole grouping in one block when every assignment fits one chunk (A <= kAlignChunk): the
+// histogram, scan and stable scatter of the three kernels above, without two launches.
+__global__ void __launch_bounds__(kThreads)
+    align_single_chunk_kernel(const int32_t* __restrict__ idx, int64_t A, int E, int C, int TB,
+                              int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                              int32_t* __restrict__ blk_prefix, int32_t* __restrict__ sorted_ids,
+                              int32_t* __restrict__ slot_of, uint8_t* __restrict__ drop_mask,
+                              int* err) {
+  __shared__ int wrun[kWarps][kMaxE];
+  __shared__ int s_off[kMaxE + 1];
+  __shared__ int sh[kWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kWarps * kMaxE; i += kThreads) (&wrun[0][0])[i] = 0;
+  __syncthreads();
+  const int64_t wbase = static_cast<int64_t>(warp) * kPerWarp;
+  // per-warp per-expert counts
+  for (int step = 0; step < kPerWarp / 32; ++step) {
+    const int64_t a = wbase + step * 32 + lane;
+    const int e = (a < A) ? idx[a] : -1;
+    const bool ok = (e >= 0 && e < E);
+    if (a < A && !ok) flag_error(err, kDevBadExpert);
+    const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : (E + lane));
+    if (ok && lane == __ffs(peers) - 1) wrun[warp][e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // per expert: exclusive prefix across warps and the raw total
+  const int e = threadIdx.x;
+  int raw = 0;
+  if (e < E) {
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = wrun[w][e];
+      wrun[w][e] = raw;
+      raw += c;
+    }
+  }
+  const int cnt = (e < E) ? min(raw, C) : 0;
+  const int nb = (cnt + TB - 1) / TB;
+  int tot_cnt, tot_nb;
+  const int off = block_exclusive_scan(cnt, sh, tot_cnt);
+  const int bp = block_exclusive_scan(nb, sh, tot_nb);
+  if (e < E) {
+    counts[e] = cnt;
+    offsets[e] = off;
+    s_off[e] = off;
+    if (blk_prefix != nullptr) blk_prefix[e] = bp;
+  }
+  if (e == 0) {
+    offsets[E] = tot_cnt;
+    if (blk_prefix != nullptr) blk_prefix[E] = tot_nb;
+  }
+  __syncthreads();
+  // stable ranks in assignment order, then the scatter
+  for (int step = 0; step < kPerWarp / 32; ++step) {
+    const int64_t a = wbase + step * 32 + lane;
+    const bool in = a < A;
+    const int ea = in ? idx[a] : -1;
+    const bool ok = (ea >= 0 && ea < E);
+    const uint32_t peers = __match_any_sync(0xffffffffu, ok ? ea : (E + lane));
+    int rank = 0;
+    if (ok) rank = wrun[warp][ea] + __popc(peers & lanemask_lt());
+    __syncwarp();
+    if (ok && lane == __ffs(peers) - 1) wrun[warp][ea] += __popc(peers);
+    __syncwarp();
+    if (in) {
+      if (ok && rank < C) {
+        const int slot = s_off[ea] + rank;
+        sorted_ids[slot] = static_cast<int32_t>(a);
+        slot_of[a] = slot;
+        drop_mask[a] = 0;
+      } else {
+        slot_of[a] = -1;
+        drop_mask[a] = 1;
+      }
+    }
+  }
+  for (int64_t sl = tot_cnt + threadIdx.x; sl < A; sl += kThreads) sorted_ids[sl] = -1;
+}
+
 __global__ void __launch_bounds__(kThreads)
     plan_from_offsets_kernel(const int32_t* __restrict__ offsets, int E, int TB,
                              int32_t* __restrict__ blk_prefix) {
@@ -197,6 +277,12 @@ cudaError_t launch_align(const int32_t* topk_idx, int64_t A, int E, int C, int T
                          uint8_t* drop_mask, int* err, cudaStream_t stream) {
   if (A == 0) return cudaSuccess;
   const int nblk = static_cast<int>((A + kAlignChunk - 1) / kAlignChunk);
+  if (nblk == 1) {
+    align_single_chunk_kernel<<<1, kThreads, 0, stream>>>(topk_idx, A, E, C, TB, counts, offsets,
+                                                          blk_prefix, sorted_ids, slot_of,
+                                                          drop_mask, err);
+    return cudaGetLastError();
+  }
   align_hist_kernel<<<nblk, kThreads, 0, stream>>>(topk_idx, A, E, blk_hist, err);
   align_scan_kernel<<<1, kThreads, 0, stream>>>(blk_hist, nblk, E, C, TB, counts, offsets,
                                                 blk_prefix);

@@ -5,8 +5,7 @@
 // MoE Align & MoE Sum" (128-bit vector reads/writes).
 //
 // out[t,:] = sum over kept j of topk_w[t,j] * y_slots[slot_of[t*k+j],:], fp32 accumulation in
-// ascending j, rounded once. One block per token; each thread owns 16-byte chunks of the row
-// and issues the (up to 16) expert-row loads of a chunk back to back before accumulating.
+// ascending j, rounded once.
 #include "common.cuh"
 #include "internal.h"
 
@@ -14,7 +13,6 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kMaxK = 16;
 
 template <typename T>
 struct Vec;  // a 16-byte chunk of T: raw load, widen to float, narrow-and-store
@@ -51,43 +49,67 @@ struct Vec<__nv_bfloat16> {
   }
 };
 
+// One warp per (token, row segment of 32*kG 16-byte chunks). Lane j < k holds slot_of/topk_w
+// of assignment j (broadcast by shuffle); lane l owns chunks l, l+32, ... of the segment, and
+// every expert row's loads for those chunks are issued before they are accumulated.
+constexpr int kWarps = kThreads / 32;
+constexpr int kG = 4;
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
     combine_kernel(const T* __restrict__ y, const int32_t* __restrict__ slot_of,
                    const float* __restrict__ topk_w, T* __restrict__ out, int64_t Ttok, int H,
-                   int k) {
+                   int k, int segs) {
   constexpr int N = Vec<T>::N;
-  __shared__ int s_slot[kMaxK];
-  __shared__ float s_w[kMaxK];
-  for (int64_t t = blockIdx.x; t < Ttok; t += gridDim.x) {
-    if (threadIdx.x < k) {
-      s_slot[threadIdx.x] = slot_of[t * k + threadIdx.x];
-      s_w[threadIdx.x] = topk_w[t * k + threadIdx.x];
-    }
-    __syncthreads();
-    for (int c = threadIdx.x * N; c < H; c += kThreads * N) {
-      uint4 raw[kMaxK];
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  const int64_t t = wid / segs;
+  if (t >= Ttok) return;
+  const int seg = static_cast<int>(wid - t * segs);
+  const int my_slot = (lane < k) ? slot_of[t * k + lane] : -1;
+  const float my_w = (lane < k) ? topk_w[t * k + lane] : 0.f;
+  const int nchunk = H / N;
+  T* orow = out + static_cast<size_t>(t) * H;
+  {
+    const int c0 = seg * 32 * kG + lane;
+    float acc[kG][N];
 #pragma unroll
-      for (int j = 0; j < kMaxK; ++j) {
-        if (j < k && s_slot[j] >= 0)
-          raw[j] = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(s_slot[j]) * H + c));
-      }
-      float acc[N];
+    for (int g = 0; g < kG; ++g)
 #pragma unroll
-      for (int i = 0; i < N; ++i) acc[i] = 0.f;
+      for (int i = 0; i < N; ++i) acc[g][i] = 0.f;
+    for (int j0 = 0; j0 < k; j0 += 4) {
+      uint4 raw[4][kG];
+      int sl[4];
+      float wj[4];
 #pragma unroll
-      for (int j = 0; j < kMaxK; ++j) {
-        if (j < k && s_slot[j] >= 0) {
-          const float wj = s_w[j];
-          float v[N];
-          Vec<T>::widen(raw[j], v);
+      for (int jj = 0; jj < 4; ++jj) {
+        sl[jj] = __shfl_sync(0xffffffffu, my_slot, (j0 + jj) & 31);
+        wj[jj] = __shfl_sync(0xffffffffu, my_w, (j0 + jj) & 31);
+        if (j0 + jj >= k) sl[jj] = -1;
 #pragma unroll
-          for (int i = 0; i < N; ++i) acc[i] = fmaf(wj, v[i], acc[i]);
+        for (int g = 0; g < kG; ++g) {
+          const int c = c0 + 32 * g;
+          if (sl[jj] >= 0 && c < nchunk)
+            raw[jj][g] = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(sl[jj]) * H) + c);
         }
       }
-      Vec<T>::store(out + static_cast<size_t>(t) * H + c, acc);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        if (sl[jj] < 0) continue;
+#pragma unroll
+        for (int g = 0; g < kG; ++g) {
+          float v[N];
+          Vec<T>::widen(raw[jj][g], v);
+#pragma unroll
+          for (int i = 0; i < N; ++i) acc[g][i] = fmaf(wj[jj], v[i], acc[g][i]);
+        }
+      }
     }
-    __syncthreads();
+#pragma unroll
+    for (int g = 0; g < kG; ++g) {
+      const int c = c0 + 32 * g;
+      if (c < nchunk) Vec<T>::store(orow + static_cast<size_t>(c) * N, acc[g]);
+    }
   }
 }
 
@@ -97,14 +119,17 @@ cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_o
                            const float* topk_w, void* out, int64_t T, int H, int k,
                            cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  const int64_t blocks = T < 65535 * 8 ? T : 65535 * 8;
+  const int n = (dtype == 0) ? 4 : 8;  // elements per 16-byte chunk
+  const int segs = static_cast<int>((H / n + 32 * kG - 1) / (32 * kG));
+  const int64_t blocks = (T * segs + kWarps - 1) / kWarps;
   if (dtype == 0)
     combine_kernel<float><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
-        static_cast<const float*>(y_slots), slot_of, topk_w, static_cast<float*>(out), T, H, k);
+        static_cast<const float*>(y_slots), slot_of, topk_w, static_cast<float*>(out), T, H, k,
+        segs);
   else
     combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(y_slots), slot_of, topk_w,
-        static_cast<__nv_bfloat16*>(out), T, H, k);
+        static_cast<__nv_bfloat16*>(out), T, H, k, segs);
   return cudaGetLastError();
 }
 

@@ -39,7 +39,17 @@ constexpr int kTmemCols = 512;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory per block
 constexpr int kCtrlBytes = 2560;    // barriers + group tables
 
-enum EpiMode { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2 };
+// Epilogue / operand modes:
+//   kEpiSwiGLU: two A operands (gate, up) of the same 128 features; h = silu(g) * u (bf16).
+//   kEpiBF16:   one A operand, 128 features; y stored as bf16.
+//   kEpiBF16x2: two A operands = features [m0, m0+128) and [m0+128, m0+256) of one weight; both
+//               accumulators share the B tile, halving B traffic per weight byte; bf16 out.
+//   kEpiF32:    one A operand, fp32 out plus an optional per-feature bias (router logits).
+enum EpiMode { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2, kEpiBF16x2 = 3 };
+template <int MODE>
+constexpr bool dual_a() { return MODE == kEpiSwiGLU || MODE == kEpiBF16x2; }
+template <int MODE>
+constexpr int tile_features() { return MODE == kEpiBF16x2 ? 256 : 128; }
 // How the B operand (token rows) reaches shared memory.
 enum BMode { kBGather4 = 0, kBTiled = 1, kBCpAsync = 2 };
 
@@ -61,6 +71,8 @@ struct TcParams {
   const int32_t* offsets;     // [groups+1] slot offsets, or nullptr: one group of n_static rows
   const int32_t* blk_prefix;  // [groups+1] token blocks before each group
   int n_static;
+  int ksplit;            // K split into ksplit equal ranges (router only; partial sums)
+  int64_t split_stride;  // elements between the partial-sum slabs of consecutive K ranges
   void* out;
   int64_t ldo;
   const float* bias;
@@ -70,11 +82,15 @@ struct TcParams {
 };
 
 struct Tile {
-  int group, fb, n, row0;
+  int group, fb, n, row0, ks, kb0, kb1;
 };
 
+// Tile order: K range fastest, then token block, then feature block, then group (expert).
 __device__ __forceinline__ Tile decode_tile(int tile, int num_fb, int groups, int TB,
-                                            const int* s_off, const int* s_blk) {
+                                            const int* s_off, const int* s_blk, int ksplit,
+                                            int kblocks) {
+  const int ks = tile % ksplit;
+  tile /= ksplit;
   int lo = 0, hi = groups;  // largest lo with num_fb * s_blk[lo] <= tile
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -89,6 +105,10 @@ __device__ __forceinline__ Tile decode_tile(int tile, int num_fb, int groups, in
   const int cnt = s_off[lo + 1] - s_off[lo];
   t.n = min(TB, cnt - b * TB);
   t.row0 = s_off[lo] + b * TB;
+  const int per = kblocks / ksplit;
+  t.ks = ks;
+  t.kb0 = ks * per;
+  t.kb1 = t.kb0 + per;
   return t;
 }
 
@@ -98,11 +118,12 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
                     const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB, const TcParams p) {
   constexpr bool kSwiGLU = (MODE == kEpiSwiGLU);
+  constexpr bool kDual = dual_a<MODE>();
   constexpr uint32_t kFullCount = (BMODE == kBCpAsync) ? 1u + 128u : 1u;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int a_bytes = kSwiGLU ? 32768 : 16384;
+  const int a_bytes = kDual ? 32768 : 16384;
   const int stage_bytes = a_bytes + p.TB * 128;
   const int S = p.stages;
   uint8_t* ctrl = smem + static_cast<size_t>(S) * stage_bytes;
@@ -152,7 +173,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int num_tiles = p.num_fb * s_blk[groups];
+  const int num_tiles = p.num_fb * s_blk[groups] * p.ksplit;
   const int kblocks = p.K / kBK;
 
   if (warp == 0) {
@@ -160,7 +181,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk);
+      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
       const int npad = (t.n + 15) & ~15;
       const int nbox = (t.n + kRowBox - 1) / kRowBox;
       int rows[8];
@@ -176,12 +197,12 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
           }
         }
       }
-      const int m0 = t.fb * kBM;
+      const int m0 = t.fb * tile_features<MODE>();
       const bool hi_chunk = (m0 + 64) < p.m_rows_a;
-      uint32_t tx = (hi_chunk ? 16384u : 8192u) * (kSwiGLU ? 2u : 1u);
+      uint32_t tx = (hi_chunk ? 16384u : 8192u) * (kDual ? 2u : 1u);
       if constexpr (BMODE == kBGather4) tx += static_cast<uint32_t>(npad) * 128u;
       if constexpr (BMODE == kBTiled) tx += static_cast<uint32_t>(nbox) * (kRowBox * 128u);
-      for (int kb = 0; kb < kblocks; ++kb) {
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
         const int s = it % S;
         const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
         int got = 1;
@@ -198,9 +219,12 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
           mbar_arrive_expect_tx(fbar, tx);
           tma_load_3d(sa, &tmA0, m0, kb * kBK, t.group, fbar);
           if (hi_chunk) tma_load_3d(sa + 8192, &tmA0, m0 + 64, kb * kBK, t.group, fbar);
-          if (kSwiGLU) {
+          if constexpr (kSwiGLU) {
             tma_load_3d(sa + 16384, &tmA1, m0, kb * kBK, t.group, fbar);
             if (hi_chunk) tma_load_3d(sa + 16384 + 8192, &tmA1, m0 + 64, kb * kBK, t.group, fbar);
+          } else if constexpr (kDual) {
+            tma_load_3d(sa + 16384, &tmA0, m0 + 128, kb * kBK, t.group, fbar);
+            tma_load_3d(sa + 16384 + 8192, &tmA0, m0 + 192, kb * kBK, t.group, fbar);
           }
         }
         if constexpr (BMODE == kBTiled) {
@@ -237,7 +261,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
       int it = 0, tc = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk);
+        const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
         const int npad = (t.n + 15) & ~15;
         const int buf = tc % p.nbuf;
         const uint32_t use = static_cast<uint32_t>(tc / p.nbuf);
@@ -248,7 +272,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
         tc_fence_after();
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * 256);
         const uint32_t idesc = idesc_bf16(kBM, npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
           const int s = it % S;
           const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
           if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) {
@@ -262,9 +286,9 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t ad = smem_desc_sw128(sa + kk * 2048, 8192, 1024);
             const uint64_t bd = smem_desc_sw128(sb + kk * 32, 16, 1024);
-            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t acc = (kb > t.kb0 || kk > 0) ? 1u : 0u;
             tc_mma_bf16(d0, ad, bd, idesc, acc);
-            if (kSwiGLU) {
+            if constexpr (kDual) {
               const uint64_t ad1 = smem_desc_sw128(sa + 16384 + kk * 2048, 8192, 1024);
               tc_mma_bf16(d0 + static_cast<uint32_t>(p.TB), ad1, bd, idesc, acc);
             }
@@ -294,7 +318,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk);
+      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
       const int npad = (t.n + 15) & ~15;
       const int iters = npad >> 4;  // rows per thread
       const __nv_bfloat16* src[16];
@@ -306,7 +330,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
         row = min(max(row, 0), p.rows_b - 1);
         src[i] = p.b_ptr + static_cast<size_t>(row) * p.K + chunk * 8;
       }
-      for (int kb = 0; kb < kblocks; ++kb) {
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
         const int s = it % S;
         const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
         int got = 1;
@@ -339,7 +363,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
     int tc = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk);
+      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
       const int buf = tc % p.nbuf;
       const uint32_t use = static_cast<uint32_t>(tc / p.nbuf);
       int got = 1;
@@ -350,18 +374,14 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
         break;
       }
       tc_fence_after();
-      const int m = t.fb * kBM + q * 32 + lane;
+      const int m = t.fb * tile_features<MODE>() + q * 32 + lane;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(buf * 256);
-      float bias_m = 0.f;
-      if constexpr (MODE == kEpiF32) {
-        if (p.bias != nullptr && m < p.m_valid) bias_m = p.bias[m];
-      }
       for (int c0 = 0; c0 < t.n; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tb + static_cast<uint32_t>(c0), v);
         uint32_t u[32];
-        if constexpr (kSwiGLU) tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), u);
+        if constexpr (kDual) tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), u);
         tmem_wait_ld();
         const int cmax = min(32, t.n - c0);
         if constexpr (MODE == kEpiSwiGLU) {
@@ -375,18 +395,24 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
               o[static_cast<size_t>(j) * p.ldo] = __float2bfloat16_rn(h);
             }
           }
-        } else if constexpr (MODE == kEpiBF16) {
+        } else if constexpr (MODE == kEpiBF16 || MODE == kEpiBF16x2) {
           __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) +
                              static_cast<size_t>(t.row0 + c0) * p.ldo + m;
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j < cmax) o[static_cast<size_t>(j) * p.ldo] = __float2bfloat16_rn(__uint_as_float(v[j]));
+          for (int j = 0; j < 32; ++j) {
+            if (j < cmax) {
+              o[static_cast<size_t>(j) * p.ldo] = __float2bfloat16_rn(__uint_as_float(v[j]));
+              if constexpr (kDual)
+                o[static_cast<size_t>(j) * p.ldo + 128] = __float2bfloat16_rn(__uint_as_float(u[j]));
+            }
+          }
         } else {
           if (m < p.m_valid) {
-            float* o = reinterpret_cast<float*>(p.out) + static_cast<size_t>(t.row0 + c0) * p.ldo + m;
+            float* o = reinterpret_cast<float*>(p.out) + t.ks * p.split_stride +
+                       static_cast<size_t>(t.row0 + c0) * p.ldo + m;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (j < cmax) o[static_cast<size_t>(j) * p.ldo] = __uint_as_float(v[j]) + bias_m;
+              if (j < cmax) o[static_cast<size_t>(j) * p.ldo] = __uint_as_float(v[j]);
           }
         }
       }
@@ -488,7 +514,7 @@ template <int MODE, int BMODE>
 cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                         TcParams p, int64_t tiles_ub, int num_sms, cudaStream_t stream,
                         std::string* d) {
-  const int a_bytes = (MODE == kEpiSwiGLU) ? 32768 : 16384;
+  const int a_bytes = dual_a<MODE>() ? 32768 : 16384;
   const int stage_bytes = a_bytes + p.TB * 128;
   int stages = (kSmemLimit - 1024 - kCtrlBytes) / stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
@@ -497,7 +523,7 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
     return cudaErrorInvalidValue;
   }
   p.stages = stages;
-  p.nbuf = (((MODE == kEpiSwiGLU) ? 2 : 1) * p.TB <= 256) ? 2 : 1;
+  p.nbuf = ((dual_a<MODE>() ? 2 : 1) * p.TB <= 256) ? 2 : 1;
   const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + kCtrlBytes;
   int64_t grid = tiles_ub < num_sms ? tiles_ub : num_sms;
   if (grid < 1) grid = 1;
@@ -512,8 +538,20 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
 
 }  // namespace
 
-cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, const float* bias, int T,
-                                 int H, int E, float* logits, int* err, int num_sms,
+int route_token_block(int64_t T) { return T >= 64 ? 64 : static_cast<int>(((T + 31) / 32) * 32); }
+
+int route_ksplit(int64_t T, int H, int E) {
+  const int64_t kb_total = H / kBK;
+  const int64_t base = ((E + kBM - 1) / kBM) * ((T + route_token_block(T) - 1) / route_token_block(T));
+  int ks = 1;
+  // at most 8 ranges: the top-k kernel sums the partials of a token in one warp
+  while (ks * 2 <= 8 && ks * 2 <= kb_total && kb_total % (ks * 2) == 0 && base * ks * 2 <= 128)
+    ks *= 2;
+  return ks;
+}
+
+cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int H, int E,
+                                 float* partials, int ksplit, int* err, int num_sms,
                                  cudaStream_t stream, std::string* detail) {
   CUtensorMap a0, b;
   if (!map_weights(&a0, w_router, static_cast<uint64_t>(E), static_cast<uint64_t>(H), 1, detail) ||
@@ -524,7 +562,7 @@ cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, const floa
   p.num_fb = (E + kBM - 1) / kBM;
   p.m_rows_a = E;
   p.m_valid = E;
-  p.TB = T >= 64 ? 64 : ((T + 31) / 32) * 32;
+  p.TB = route_token_block(T);
   p.groups = 1;
   p.k_top = 1;
   p.rows_b = T;
@@ -532,11 +570,13 @@ cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, const floa
   p.offsets = nullptr;
   p.blk_prefix = nullptr;
   p.n_static = T;
-  p.out = logits;
+  p.ksplit = ksplit;
+  p.split_stride = static_cast<int64_t>(T) * E;
+  p.out = partials;
   p.ldo = E;
-  p.bias = bias;
+  p.bias = nullptr;
   p.err = err;
-  const int64_t tiles = static_cast<int64_t>(p.num_fb) * ((T + p.TB - 1) / p.TB);
+  const int64_t tiles = static_cast<int64_t>(p.num_fb) * ((T + p.TB - 1) / p.TB) * ksplit;
   return launch_mode<kEpiF32, kBTiled>(a0, a0, b, p, tiles, num_sms, stream, detail);
 }
 
@@ -572,6 +612,7 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const int32_t* sorted_ids,
   p.bias = nullptr;
   p.err = err;
   p.b_ptr = static_cast<const __nv_bfloat16*>(x);
+  p.ksplit = 1;
   const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
   if (use_gather4)
     return launch_mode<kEpiSwiGLU, kBGather4>(a0, a1, b, p, tiles, num_sms, stream, detail);
@@ -587,8 +628,10 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
       !map_row_boxes(&b, hbuf, static_cast<uint64_t>(I), static_cast<uint64_t>(hbuf_rows), detail))
     return cudaErrorInvalidValue;
   TcParams p{};
+  const bool dual = (H % 256) == 0;
+  p.ksplit = 1;
   p.K = I;
-  p.num_fb = H / kBM;
+  p.num_fb = dual ? H / 256 : H / kBM;
   p.m_rows_a = H;
   p.m_valid = H;
   p.TB = TB;
@@ -602,8 +645,9 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
   p.ldo = H;
   p.bias = nullptr;
   p.err = err;
-  return launch_mode<kEpiBF16, kBTiled>(a0, a0, b, p, static_cast<int64_t>(p.num_fb) * ub_blocks,
-                                        num_sms, stream, detail);
+  const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
+  if (dual) return launch_mode<kEpiBF16x2, kBTiled>(a0, a0, b, p, tiles, num_sms, stream, detail);
+  return launch_mode<kEpiBF16, kBTiled>(a0, a0, b, p, tiles, num_sms, stream, detail);
 }
 
 }  // namespace moe

@@ -14,14 +14,20 @@ namespace moe {
 cudaError_t launch_route_simt(int dtype, const void* x, const void* w_router, const float* bias,
                               int64_t T, int H, int E, int k, float* logits_out, int32_t* topk_idx,
                               float* topk_w, cudaStream_t stream);
-// Top-k + renormalise from float32 logits [T,E], one warp per token; E <= 256.
-cudaError_t launch_topk_from_logits(const float* logits, int64_t T, int E, int k,
-                                    int32_t* topk_idx, float* topk_w, cudaStream_t stream);
+// Top-k + renormalise, one warp per token, E <= 256: logits[t,e] = sum over ks of
+// partials[ks * split_stride + t*E + e] (ascending ks) + bias[e] (bias optional); the logits
+// are written to logits_out when it is non-null.
+cudaError_t launch_topk(const float* partials, int ksplit, int64_t split_stride,
+                        const float* bias, float* logits_out, int64_t T, int E, int k,
+                        int32_t* topk_idx, float* topk_w, cudaStream_t stream);
 
 // ---- ffn_tc.cu (tcgen05 / TMEM / TMA, bf16)
-// Gate logits [T,E] = x @ w_router (+ bias) on the tensor cores (swap-AB: experts on MMA M).
-cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, const float* bias, int T,
-                                 int H, int E, float* logits, int* err, int num_sms,
+// Gate logits on the tensor cores (swap-AB: experts on MMA M), K split into `ksplit` ranges:
+// partials[ks][t][e] = sum over h in range ks of x[t,h] * w_router[h,e].
+int route_token_block(int64_t T);
+int route_ksplit(int64_t T, int H, int E);
+cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int H, int E,
+                                 float* partials, int ksplit, int* err, int num_sms,
                                  cudaStream_t stream, std::string* detail);
 // Expert GEMM1: h[s, :] = silu(x[t] Wg[e]) * (x[t] Wu[e]) for kept slots; h rows = hbuf_rows.
 cudaError_t launch_gemm1_tc(const void* x, int T, const int32_t* sorted_ids,

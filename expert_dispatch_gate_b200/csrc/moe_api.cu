@@ -12,7 +12,7 @@
 #include <mutex>
 #include <string>
 
-#include "../../include/moe.h"
+#include "moe.h"
 #include "internal.h"
 
 namespace {
@@ -104,6 +104,7 @@ struct Layout {
   int nblk;
   int32_t C;
   int TB;
+  int ksplit;  // router K split (tensor-core router only)
 };
 
 Layout layout_of(const moe_shape& s) {
@@ -122,7 +123,9 @@ Layout layout_of(const moe_shape& s) {
   };
   const size_t es = elem_size(s.dtype);
   L.err = take(256);
-  L.logits = take(static_cast<size_t>(s.T) * s.E * 4);
+  L.ksplit = (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0 && s.T > 0)
+                 ? moe::route_ksplit(s.T, s.H, s.E) : 1;
+  L.logits = take(static_cast<size_t>(s.T) * s.E * 4 * L.ksplit);
   L.blk_hist = take(static_cast<size_t>(L.nblk) * s.E * 4);
   L.offsets = take(static_cast<size_t>(s.E + 1) * 4);
   L.blk_prefix = take(static_cast<size_t>(s.E + 1) * 4);
@@ -181,12 +184,13 @@ moe_status do_route(const moe_shape& s, const Layout& L, const void* x, const vo
                     void* ws, cudaStream_t st) {
   cudaError_t e;
   if (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0) {
-    float* logits = logits_out != nullptr ? logits_out : at<float>(ws, L.logits);
+    float* partials = at<float>(ws, L.logits);
     std::string d;
-    e = moe::launch_route_gemm_tc(x, w_router, bias, static_cast<int>(s.T), s.H, s.E, logits,
-                                  at<int>(ws, L.err), num_sms(), st, &d);
+    e = moe::launch_route_gemm_tc(x, w_router, static_cast<int>(s.T), s.H, s.E, partials,
+                                  L.ksplit, at<int>(ws, L.err), num_sms(), st, &d);
     if (e != cudaSuccess) return cuda_fail(e, "router gate GEMM (tcgen05)", d);
-    e = moe::launch_topk_from_logits(logits, s.T, s.E, s.k, topk_idx, topk_w, st);
+    e = moe::launch_topk(partials, L.ksplit, s.T * s.E, bias, logits_out, s.T, s.E, s.k,
+                         topk_idx, topk_w, st);
     if (e != cudaSuccess) return cuda_fail(e, "router top-k");
   } else {
     e = moe::launch_route_simt(s.dtype, x, w_router, bias, s.T, s.H, s.E, s.k, logits_out,
@@ -254,7 +258,7 @@ moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router
   OPT_PTR(logit_bias, "logit_bias");
   OPT_PTR(logits_out, "logits_out");
   const Layout L = layout_of(*shape);
-  st = check_ws(ws, ws_bytes, L.logits + static_cast<size_t>(shape->T) * shape->E * 4);
+  st = check_ws(ws, ws_bytes, L.logits + static_cast<size_t>(shape->T) * shape->E * 4 * L.ksplit);
   if (st != MOE_OK) return st;
   return do_route(*shape, L, x, w_router, logit_bias, logits_out, topk_idx, topk_w, ws,
                   static_cast<cudaStream_t>(stream));
@@ -268,8 +272,8 @@ moe_status moe_route_from_logits(const moe_shape* shape, const float* logits, in
   REQUIRE_PTR(logits, "logits");
   REQUIRE_PTR(topk_idx, "topk_idx");
   REQUIRE_PTR(topk_w, "topk_w");
-  cudaError_t e = moe::launch_topk_from_logits(logits, shape->T, shape->E, shape->k, topk_idx,
-                                               topk_w, static_cast<cudaStream_t>(stream));
+  cudaError_t e = moe::launch_topk(logits, 1, 0, nullptr, nullptr, shape->T, shape->E, shape->k,
+                                   topk_idx, topk_w, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "router top-k");
   return MOE_OK;
 }

@@ -45,22 +45,31 @@ __device__ __forceinline__ void write_selection(int lane, int k, float my_v, int
   }
 }
 
-// Logits distributed over lanes: lane holds experts lane, lane+32, ... (VPL per lane).
+// Logits distributed over lanes: lane holds experts lane, lane+32, ... (VPL per lane). Each
+// logit is the sum of the K-range partials in ascending order plus the optional bias.
 template <int VPL>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
-    topk_from_logits_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
-                            int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+    topk_kernel(const float* __restrict__ partials, int ksplit, int64_t split_stride,
+                const float* __restrict__ bias, float* __restrict__ logits_out, int64_t T, int E,
+                int k, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   const int lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
   if (t >= T) return;
-  const float* row = logits + t * E;
   float v[VPL];
   uint32_t taken = 0;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = lane + 32 * i;
-    v[i] = (e < E) ? row[e] : -INFINITY;
-    if (e >= E) taken |= 1u << i;
+    if (e < E) {
+      float acc = partials[t * E + e];
+      for (int ks = 1; ks < ksplit; ++ks) acc += partials[ks * split_stride + t * E + e];
+      if (bias != nullptr) acc += bias[e];
+      v[i] = acc;
+      if (logits_out != nullptr) logits_out[t * E + e] = acc;
+    } else {
+      v[i] = -INFINITY;
+      taken |= 1u << i;
+    }
   }
   float my_v = 0.f, top = 0.f;
   int my_i = 0;
@@ -76,7 +85,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
       }
     }
     warp_argmax(bv, bi);
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if ((bi & 31) == lane) taken |= 1u << ((bi >> 5) & 31);
     if (lane == j) {
       my_v = bv;
       my_i = bi;
@@ -115,15 +124,43 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, flo
   }
 }
 
+// 16 bytes of Tin widened to float.
+template <typename Tin>
+struct Vec16;
+template <>
+struct Vec16<float> {
+  static constexpr int N = 4;
+  __device__ static void load(const float* p, float (&o)[4]) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+  }
+};
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load(const __nv_bfloat16* p, float (&o)[8]) {
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      o[2 * i] = __uint_as_float(w[i] << 16);
+      o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
+
 // Gate GEMM on CUDA cores + selection, one warp per token; E <= EMAX <= 64, H % 8 == 0.
-// Every lane accumulates all E partial dot products over its slice of H (8 consecutive
-// elements per 128-bit load); a butterfly reduction gives every lane all E logits.
-template <typename Tin, int EMAX>
+// Lane l owns x[h] for h in [8l + 256i, 8l + 256i + 8): one 128-bit x load, then the matching
+// 8 rows of Wr (contiguous, 8*E values) as 128-bit loads when a row is a whole number of
+// 16-byte vectors (VEC), else element by element. Every lane accumulates all E partial dot
+// products; a butterfly reduction gives every lane all E logits.
+template <typename Tin, int EMAX, bool VEC>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     route_simt_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr,
                       const float* __restrict__ bias, int64_t T, int H, int E, int k,
                       float* __restrict__ logits_out, int32_t* __restrict__ topk_idx,
                       float* __restrict__ topk_w) {
+  constexpr int VN = Vec16<Tin>::N;
   const int lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -134,12 +171,24 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   for (int h0 = lane * 8; h0 < H; h0 += 256) {
     float xv[8];
     load8<Tin>(xr + h0, xv);
+    const Tin* wb = wr + static_cast<size_t>(h0) * E;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const Tin* wrow = wr + static_cast<size_t>(h0 + u) * E;
+      if constexpr (VEC) {
 #pragma unroll
-      for (int e = 0; e < EMAX; ++e)
-        if (e < E) acc[e] = fmaf(xv[u], ld_f<Tin>(wrow + e), acc[e]);
+        for (int e0 = 0; e0 < EMAX; e0 += VN) {
+          if (e0 < E) {
+            float wv[VN];
+            Vec16<Tin>::load(wb + u * E + e0, wv);
+#pragma unroll
+            for (int i = 0; i < VN; ++i) acc[e0 + i] = fmaf(xv[u], wv[i], acc[e0 + i]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e)
+          if (e < E) acc[e] = fmaf(xv[u], ld_f<Tin>(wb + u * E + e), acc[e]);
+      }
     }
   }
 #pragma unroll
@@ -167,7 +216,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         bi = e;
       }
     }
-    taken |= 1ull << bi;
+    taken |= 1ull << (bi & 63);
     if (lane == j) {
       my_v = bv;
       my_i = bi;
@@ -177,20 +226,29 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   write_selection(lane, k, my_v, my_i, top, topk_idx + t * k, topk_w + t * k);
 }
 
+template <typename Tin, int EMAX>
+void route_simt_launch(const Tin* x, const Tin* wr, const float* bias, int64_t T, int H, int E,
+                       int k, float* logits_out, int32_t* idx, float* w, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
+  const unsigned block = kWarpsPerBlock * 32;
+  if ((E * sizeof(Tin)) % 16 == 0)
+    route_simt_kernel<Tin, EMAX, true><<<grid, block, 0, st>>>(x, wr, bias, T, H, E, k, logits_out, idx, w);
+  else
+    route_simt_kernel<Tin, EMAX, false><<<grid, block, 0, st>>>(x, wr, bias, T, H, E, k, logits_out, idx, w);
+}
+
 template <typename Tin>
 cudaError_t route_simt_dispatch(const Tin* x, const Tin* wr, const float* bias, int64_t T, int H,
                                 int E, int k, float* logits_out, int32_t* idx, float* w,
                                 cudaStream_t st) {
-  const unsigned grid = static_cast<unsigned>((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
-  const unsigned block = kWarpsPerBlock * 32;
   if (E <= 8)
-    route_simt_kernel<Tin, 8><<<grid, block, 0, st>>>(x, wr, bias, T, H, E, k, logits_out, idx, w);
+    route_simt_launch<Tin, 8>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
   else if (E <= 16)
-    route_simt_kernel<Tin, 16><<<grid, block, 0, st>>>(x, wr, bias, T, H, E, k, logits_out, idx, w);
+    route_simt_launch<Tin, 16>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
   else if (E <= 32)
-    route_simt_kernel<Tin, 32><<<grid, block, 0, st>>>(x, wr, bias, T, H, E, k, logits_out, idx, w);
+    route_simt_launch<Tin, 32>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
   else
-    route_simt_kernel<Tin, 64><<<grid, block, 0, st>>>(x, wr, bias, T, H, E, k, logits_out, idx, w);
+    route_simt_launch<Tin, 64>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
   return cudaGetLastError();
 }
 
@@ -209,19 +267,20 @@ cudaError_t launch_route_simt(int dtype, const void* x, const void* w_router, co
                                             H, E, k, logits_out, topk_idx, topk_w, stream);
 }
 
-cudaError_t launch_topk_from_logits(const float* logits, int64_t T, int E, int k,
-                                    int32_t* topk_idx, float* topk_w, cudaStream_t stream) {
+cudaError_t launch_topk(const float* partials, int ksplit, int64_t split_stride,
+                        const float* bias, float* logits_out, int64_t T, int E, int k,
+                        int32_t* topk_idx, float* topk_w, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
   const unsigned block = kWarpsPerBlock * 32;
   if (E <= 32)
-    topk_from_logits_kernel<1><<<grid, block, 0, stream>>>(logits, T, E, k, topk_idx, topk_w);
+    topk_kernel<1><<<grid, block, 0, stream>>>(partials, ksplit, split_stride, bias, logits_out, T, E, k, topk_idx, topk_w);
   else if (E <= 64)
-    topk_from_logits_kernel<2><<<grid, block, 0, stream>>>(logits, T, E, k, topk_idx, topk_w);
+    topk_kernel<2><<<grid, block, 0, stream>>>(partials, ksplit, split_stride, bias, logits_out, T, E, k, topk_idx, topk_w);
   else if (E <= 128)
-    topk_from_logits_kernel<4><<<grid, block, 0, stream>>>(logits, T, E, k, topk_idx, topk_w);
+    topk_kernel<4><<<grid, block, 0, stream>>>(partials, ksplit, split_stride, bias, logits_out, T, E, k, topk_idx, topk_w);
   else
-    topk_from_logits_kernel<8><<<grid, block, 0, stream>>>(logits, T, E, k, topk_idx, topk_w);
+    topk_kernel<8><<<grid, block, 0, stream>>>(partials, ksplit, split_stride, bias, logits_out, T, E, k, topk_idx, topk_w);
   return cudaGetLastError();
 }
 
