@@ -268,7 +268,9 @@ def launches_per_step(wl):
     GEMMs, combine."""
     route = 2 if (wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0) else 1
     align = 1 if wl.T * wl.k <= 2048 else 3
-    return route + align + 2 + 1
+    # expert-major copy of the token rows before GEMM1 (when CTA pairs run GEMM1)
+    copy = 1 if (wl.dtype == "bf16" and wl.I % 256 == 0) else 0
+    return route + align + copy + 2 + 1
 
 
 def workload_of(args):

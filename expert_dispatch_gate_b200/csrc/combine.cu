@@ -113,7 +113,39 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// xs[s, :] = x[sorted_ids[s] / k, :] for every kept slot s < offsets[E]: the token rows in
+// expert-major order, so a GEMM can stream them as contiguous rows. One warp per slot row.
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+    dispatch_rows_kernel(const T* __restrict__ x, const int32_t* __restrict__ sorted_ids,
+                         const int32_t* __restrict__ offsets, int E, int k, int H, int64_t rows,
+                         T* __restrict__ xs) {
+  const int lane = threadIdx.x & 31;
+  const int64_t s = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  if (s >= rows || s >= offsets[E]) return;
+  const int64_t t = sorted_ids[s] / k;
+  const uint4* src = reinterpret_cast<const uint4*>(x + t * H);
+  uint4* dst = reinterpret_cast<uint4*>(xs + s * H);
+  const int n = H * static_cast<int>(sizeof(T)) / 16;
+  for (int c = lane; c < n; c += 32) dst[c] = __ldg(src + c);
+}
+
 }  // namespace
+
+cudaError_t launch_dispatch_rows(int dtype, const void* x, const int32_t* sorted_ids,
+                                 const int32_t* offsets, int E, int k, int H, int64_t rows,
+                                 void* xs, cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>((rows + kWarps - 1) / kWarps);
+  if (dtype == 0)
+    dispatch_rows_kernel<float><<<grid, kThreads, 0, stream>>>(
+        static_cast<const float*>(x), sorted_ids, offsets, E, k, H, rows, static_cast<float*>(xs));
+  else
+    dispatch_rows_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), sorted_ids, offsets, E, k, H, rows,
+        static_cast<__nv_bfloat16*>(xs));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_of,
                            const float* topk_w, void* out, int64_t T, int H, int k,

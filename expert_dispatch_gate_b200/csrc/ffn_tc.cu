@@ -53,9 +53,12 @@ constexpr int tile_features() { return MODE == kEpiBF16x2 ? 256 : 128; }
 // How the B operand (token rows) reaches shared memory.
 enum BMode { kBGather4 = 0, kBTiled = 1, kBCpAsync = 2 };
 
-// Warps: 0 TMA producer, 1 MMA issuer, 2-5 epilogue, 6-9 cp.async row gatherers (kBCpAsync).
+// Warps: 0 TMA producer, 1 MMA issuer, 2-9 epilogue (two warps per TMEM lane quadrant, each
+// draining half of the token columns), 10-13 cp.async row gatherers (kBCpAsync).
+constexpr int kEpiWarps = 8;
+constexpr int kGatherWarp0 = 2 + kEpiWarps;
 template <int BMODE>
-constexpr int threads_of() { return BMODE == kBCpAsync ? 320 : 192; }
+constexpr int threads_of() { return 32 * (kGatherWarp0 + (BMODE == kBCpAsync ? 4 : 0)); }
 
 struct TcParams {
   int K;          // reduction length (multiple of 64)
@@ -112,14 +115,28 @@ __device__ __forceinline__ Tile decode_tile(int tile, int num_fb, int groups, in
   return t;
 }
 
-template <int MODE, int BMODE>
+// PAIR: two CTAs of a cluster cooperate on each tile with tcgen05.mma.cta_group::2 (M = 256).
+// Each CTA holds its own feature rows of A (its 128 features, or 256 in kEpiBF16x2) and half of
+// the tile's token rows of B; the even CTA issues the MMAs, every CTA reads back its own TMEM
+// rows. B traffic per weight byte halves. Stage bookkeeping lives in the even CTA: its full[s]
+// counts both CTAs' A bytes (TMA completes there), and its tempty[b] counts both epilogues;
+// MMA completions are signalled to both CTAs at once (commit with a two-CTA mask).
+template <int MODE, int BMODE, bool PAIR>
 __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
     tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0,
                     const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB, const TcParams p) {
   constexpr bool kSwiGLU = (MODE == kEpiSwiGLU);
   constexpr bool kDual = dual_a<MODE>();
-  constexpr uint32_t kFullCount = (BMODE == kBCpAsync) ? 1u + 128u : 1u;
+  constexpr bool kCp = (BMODE == kBCpAsync);
+  // full[s] arrivals: the producer's expect_tx (+ one completion-tracked arrival per cp.async
+  // gatherer thread). Pairs stream B by TMA only.
+  static_assert(!(PAIR && BMODE != kBTiled), "CTA pairs take the B operand by TMA boxes");
+  constexpr uint32_t kFullCount = 1u + (kCp ? 128u : 0u);
+  // one arrival per epilogue warp (both CTAs' warps in PAIR mode)
+  constexpr uint32_t kTemptyCount = PAIR ? 2u * kEpiWarps : kEpiWarps;
+  constexpr int kCtaFeatures = tile_features<MODE>();
+  constexpr int kTileFeatures = kCtaFeatures * (PAIR ? 2 : 1);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -140,6 +157,8 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int groups = (p.offsets != nullptr) ? p.groups : 1;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = (rank == 0);
 
   if (p.offsets != nullptr) {
     for (int i = threadIdx.x; i <= groups; i += blockDim.x) {
@@ -159,31 +178,43 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&tfull[b]), 1);
-      mbar_init(smem_u32(&tempty[b]), 128);
+      mbar_init(smem_u32(&tempty[b]), kTemptyCount);
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_holder), kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // barriers of both CTAs are initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int num_tiles = p.num_fb * s_blk[groups] * p.ksplit;
   const int kblocks = p.K / kBK;
+  const int tile0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int tstep = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  // B rows of a tile held by this CTA: all npad rows, or half of them per CTA in PAIR mode
+  auto b_rows = [&](int npad) { return PAIR ? (npad >> 1) : npad; };
+  auto b_first = [&](int npad) { return PAIR ? static_cast<int>(rank) * (npad >> 1) : 0; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+    for (int tile = tile0; ok && tile < num_tiles; tile += tstep) {
       const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
       const int npad = (t.n + 15) & ~15;
-      const int nbox = (t.n + kRowBox - 1) / kRowBox;
+      const int bn = b_rows(npad);
+      const int nbox = (bn + kRowBox - 1) / kRowBox;
       int rows[8];
       if constexpr (BMODE == kBGather4) {
 #pragma unroll
@@ -197,11 +228,13 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
           }
         }
       }
-      const int m0 = t.fb * tile_features<MODE>();
+      const int m0 = t.fb * kTileFeatures + static_cast<int>(rank) * kCtaFeatures;
       const bool hi_chunk = (m0 + 64) < p.m_rows_a;
       uint32_t tx = (hi_chunk ? 16384u : 8192u) * (kDual ? 2u : 1u);
       if constexpr (BMODE == kBGather4) tx += static_cast<uint32_t>(npad) * 128u;
       if constexpr (BMODE == kBTiled) tx += static_cast<uint32_t>(nbox) * (kRowBox * 128u);
+      if constexpr (PAIR) tx *= 2u;  // both CTAs' loads complete on the even CTA's barrier
+      const int brow0 = t.row0 + b_first(npad);
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
         const int s = it % S;
         const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
@@ -214,32 +247,53 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
         }
         const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
         const uint32_t sb = sa + a_bytes;
-        const uint32_t fbar = smem_u32(&full[s]);
-        if (lane == 0) {
-          mbar_arrive_expect_tx(fbar, tx);
-          tma_load_3d(sa, &tmA0, m0, kb * kBK, t.group, fbar);
-          if (hi_chunk) tma_load_3d(sa + 8192, &tmA0, m0 + 64, kb * kBK, t.group, fbar);
-          if constexpr (kSwiGLU) {
-            tma_load_3d(sa + 16384, &tmA1, m0, kb * kBK, t.group, fbar);
-            if (hi_chunk) tma_load_3d(sa + 16384 + 8192, &tmA1, m0 + 64, kb * kBK, t.group, fbar);
-          } else if constexpr (kDual) {
-            tma_load_3d(sa + 16384, &tmA0, m0 + 128, kb * kBK, t.group, fbar);
-            tma_load_3d(sa + 16384 + 8192, &tmA0, m0 + 192, kb * kBK, t.group, fbar);
+        if constexpr (PAIR) {
+          const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
+          if (lane == 0) {
+            if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), tx);
+            tma_load_3d_pair(sa, &tmA0, m0, kb * kBK, t.group, fbar);
+            if (hi_chunk) tma_load_3d_pair(sa + 8192, &tmA0, m0 + 64, kb * kBK, t.group, fbar);
+            if constexpr (kSwiGLU) {
+              tma_load_3d_pair(sa + 16384, &tmA1, m0, kb * kBK, t.group, fbar);
+              if (hi_chunk)
+                tma_load_3d_pair(sa + 16384 + 8192, &tmA1, m0 + 64, kb * kBK, t.group, fbar);
+            } else if constexpr (kDual) {
+              tma_load_3d_pair(sa + 16384, &tmA0, m0 + 128, kb * kBK, t.group, fbar);
+              tma_load_3d_pair(sa + 16384 + 8192, &tmA0, m0 + 192, kb * kBK, t.group, fbar);
+            }
+            if constexpr (BMODE == kBTiled)
+              for (int j = 0; j < nbox; ++j)
+                tma_load_2d_pair(sb + j * (kRowBox * 128), &tmB, kb * kBK, brow0 + j * kRowBox,
+                                 fbar);
           }
-        }
-        if constexpr (BMODE == kBTiled) {
-          if (lane == 0)
-            for (int j = 0; j < nbox; ++j)
-              tma_load_2d(sb + j * (kRowBox * 128), &tmB, kb * kBK, t.row0 + j * kRowBox, fbar);
-        }
-        __syncwarp();
-        if constexpr (BMODE == kBGather4) {
+          __syncwarp();
+        } else {
+          const uint32_t fbar = smem_u32(&full[s]);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(fbar, tx);
+            tma_load_3d(sa, &tmA0, m0, kb * kBK, t.group, fbar);
+            if (hi_chunk) tma_load_3d(sa + 8192, &tmA0, m0 + 64, kb * kBK, t.group, fbar);
+            if constexpr (kSwiGLU) {
+              tma_load_3d(sa + 16384, &tmA1, m0, kb * kBK, t.group, fbar);
+              if (hi_chunk)
+                tma_load_3d(sa + 16384 + 8192, &tmA1, m0 + 64, kb * kBK, t.group, fbar);
+            } else if constexpr (kDual) {
+              tma_load_3d(sa + 16384, &tmA0, m0 + 128, kb * kBK, t.group, fbar);
+              tma_load_3d(sa + 16384 + 8192, &tmA0, m0 + 192, kb * kBK, t.group, fbar);
+            }
+            if constexpr (BMODE == kBTiled)
+              for (int j = 0; j < nbox; ++j)
+                tma_load_2d(sb + j * (kRowBox * 128), &tmB, kb * kBK, brow0 + j * kRowBox, fbar);
+          }
+          __syncwarp();
+          if constexpr (BMODE == kBGather4) {
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int grp = lane + 32 * q;
-            if (grp * 4 < npad)
-              tma_gather4(sb + grp * 512, &tmB, kb * kBK, rows[q * 4], rows[q * 4 + 1],
-                          rows[q * 4 + 2], rows[q * 4 + 3], fbar);
+            for (int q = 0; q < 2; ++q) {
+              const int grp = lane + 32 * q;
+              if (grp * 4 < npad)
+                tma_gather4(sb + grp * 512, &tmB, kb * kBK, rows[q * 4], rows[q * 4 + 1],
+                            rows[q * 4 + 2], rows[q * 4 + 3], fbar);
+            }
           }
         }
         ++it;
@@ -249,33 +303,35 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
       *abort_flag = 1;
       if (lane == 0) flag_error(p.err, kDevWaitTimeout);
     }
-    // Every load issued must land before the CTA may exit.
-    if (lane == 0) {
+    // Every load issued must land before the CTA may exit. In PAIR mode the loads complete on
+    // the even CTA's barriers; the cluster barrier at the end covers the odd CTA.
+    if (lane == 0 && (!PAIR || leader)) {
       for (int i = max(0, it - S); i < it; ++i)
-        mbar_wait(smem_u32(&full[i % S]), static_cast<uint32_t>(i / S) & 1u, nullptr);
+        mbar_wait_cluster(smem_u32(&full[i % S]), static_cast<uint32_t>(i / S) & 1u, nullptr);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (one thread)
-    if (lane == 0) {
+    if (lane == 0 && leader) {
+      // ---------------------------------------------------------- MMA issuer (one thread)
       int it = 0, tc = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      for (int tile = tile0; ok && tile < num_tiles; tile += tstep) {
         const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
         const int npad = (t.n + 15) & ~15;
         const int buf = tc % p.nbuf;
         const uint32_t use = static_cast<uint32_t>(tc / p.nbuf);
-        if (!mbar_wait(smem_u32(&tempty[buf]), (use & 1u) ^ 1u, abort_flag)) {
+        if (!mbar_wait_cluster(smem_u32(&tempty[buf]), (use & 1u) ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * 256);
-        const uint32_t idesc = idesc_bf16(kBM, npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
+        const uint32_t idesc =
+            idesc_bf16(PAIR ? 2 * kBM : kBM, npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           const int s = it % S;
           const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
-          if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) {
+          if (!mbar_wait_cluster(smem_u32(&full[s]), ph, abort_flag)) {
             ok = false;
             break;
           }
@@ -287,17 +343,23 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
             const uint64_t ad = smem_desc_sw128(sa + kk * 2048, 8192, 1024);
             const uint64_t bd = smem_desc_sw128(sb + kk * 32, 16, 1024);
             const uint32_t acc = (kb > t.kb0 || kk > 0) ? 1u : 0u;
-            tc_mma_bf16(d0, ad, bd, idesc, acc);
+            if constexpr (PAIR) tc_mma_bf16_pair(d0, ad, bd, idesc, acc);
+            else tc_mma_bf16(d0, ad, bd, idesc, acc);
             if constexpr (kDual) {
               const uint64_t ad1 = smem_desc_sw128(sa + 16384 + kk * 2048, 8192, 1024);
-              tc_mma_bf16(d0 + static_cast<uint32_t>(p.TB), ad1, bd, idesc, acc);
+              if constexpr (PAIR)
+                tc_mma_bf16_pair(d0 + static_cast<uint32_t>(p.TB), ad1, bd, idesc, acc);
+              else
+                tc_mma_bf16(d0 + static_cast<uint32_t>(p.TB), ad1, bd, idesc, acc);
             }
           }
-          tc_commit(smem_u32(&empty[s]));
+          if constexpr (PAIR) tc_commit_pair_mc(smem_u32(&empty[s]), 0x3);
+          else tc_commit(smem_u32(&empty[s]));
           ++it;
         }
         if (!ok) break;
-        tc_commit(smem_u32(&tfull[buf]));
+        if constexpr (PAIR) tc_commit_pair_mc(smem_u32(&tfull[buf]), 0x3);
+        else tc_commit(smem_u32(&tfull[buf]));
         ++tc;
       }
       if (!ok) {
@@ -305,27 +367,29 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
         flag_error(p.err, kDevWaitTimeout);
       }
       // Every MMA issued must complete before TMEM is released.
-      tc_commit(smem_u32(drain));
+      if constexpr (PAIR) tc_commit_pair_mc(smem_u32(drain), 0x3);
+      else tc_commit(smem_u32(drain));
       mbar_wait(smem_u32(drain), 0u, nullptr);
     }
     __syncwarp();
-  } else if (BMODE == kBCpAsync && warp >= 6) {
+  } else if (kCp && warp >= kGatherWarp0) {
     // ------------------------------------------------------------ cp.async row gatherers
-    // Thread g (0..127) copies 16-byte chunk (g % 8) of rows g/8, g/8 + 16, ... of each
-    // stage's B tile, writing the 128-byte-swizzled K-major layout the MMA descriptor expects.
-    const int g = threadIdx.x - 6 * 32;
+    // Thread g (0..127) copies 16-byte chunk (g % 8) of rows g/8, g/8 + 16, ... of this CTA's
+    // B rows of each stage, writing the 128-byte-swizzled K-major layout the MMA expects.
+    const int g = threadIdx.x - kGatherWarp0 * 32;
     const int chunk = g & 7;
     int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+    for (int tile = tile0; ok && tile < num_tiles; tile += tstep) {
       const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
       const int npad = (t.n + 15) & ~15;
-      const int iters = npad >> 4;  // rows per thread
+      const int bn = b_rows(npad);
+      const int first = b_first(npad);
       const __nv_bfloat16* src[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int r = (g >> 3) + 16 * i;
-        const int slot = t.row0 + min(r, t.n - 1);
+        const int slot = t.row0 + min(first + r, t.n - 1);
         int row = (p.sorted_ids != nullptr) ? (p.sorted_ids[slot] / p.k_top) : slot;
         row = min(max(row, 0), p.rows_b - 1);
         src[i] = p.b_ptr + static_cast<size_t>(row) * p.K + chunk * 8;
@@ -343,10 +407,8 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
         const uint32_t sb = smem_u32(smem + static_cast<size_t>(s) * stage_bytes) + a_bytes;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          if (i < iters) {
-            const int r = (g >> 3) + 16 * i;
-            cp_async_16(sb + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * kBK);
-          }
+          const int r = (g >> 3) + 16 * i;
+          if (r < bn) cp_async_16(sb + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * kBK);
         }
         cp_async_arrive_noinc(smem_u32(&full[s]));
         ++it;
@@ -358,26 +420,27 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
     }
     cp_async_wait_all();
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
-    const int q = warp & 3;  // TMEM lane quadrant this warp may read
+    // ------------------------------------------------------------ epilogue (warps 2..9)
+    const int q = warp & 3;               // TMEM lane quadrant this warp may read
+    const int half = (warp - 2) >> 2;     // which alternate 32-column chunks it drains
     int tc = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = tile0; tile < num_tiles; tile += tstep) {
       const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
       const int buf = tc % p.nbuf;
       const uint32_t use = static_cast<uint32_t>(tc / p.nbuf);
       int got = 1;
-      if (lane == 0) got = mbar_wait(smem_u32(&tfull[buf]), use & 1u, abort_flag) ? 1 : 0;
+      if (lane == 0) got = mbar_wait_cluster(smem_u32(&tfull[buf]), use & 1u, abort_flag) ? 1 : 0;
       got = __shfl_sync(0xffffffffu, got, 0);
       if (!got) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int m = t.fb * tile_features<MODE>() + q * 32 + lane;
+      const int m = t.fb * kTileFeatures + static_cast<int>(rank) * kCtaFeatures + q * 32 + lane;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(buf * 256);
-      for (int c0 = 0; c0 < t.n; c0 += 32) {
+      for (int c0 = 32 * half; c0 < t.n; c0 += 64) {
         uint32_t v[32];
         tmem_ld32(tb + static_cast<uint32_t>(c0), v);
         uint32_t u[32];
@@ -417,7 +480,11 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&tempty[buf]));
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
+        else mbar_arrive(smem_u32(&tempty[buf]));
+      }
       ++tc;
     }
     if (!ok) {
@@ -428,9 +495,11 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // no CTA leaves while its peer may still signal it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -510,7 +579,7 @@ bool map_weights(CUtensorMap* m, const void* base, uint64_t mdim, uint64_t kdim,
   return r == CUDA_SUCCESS;
 }
 
-template <int MODE, int BMODE>
+template <int MODE, int BMODE, bool PAIR>
 cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                         TcParams p, int64_t tiles_ub, int num_sms, cudaStream_t stream,
                         std::string* d) {
@@ -525,18 +594,46 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   p.stages = stages;
   p.nbuf = ((dual_a<MODE>() ? 2 : 1) * p.TB <= 256) ? 2 : 1;
   const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + kCtrlBytes;
-  int64_t grid = tiles_ub < num_sms ? tiles_ub : num_sms;
+  const int64_t units = PAIR ? num_sms / 2 : num_sms;  // CTA pairs or CTAs, one per SM
+  int64_t grid = tiles_ub < units ? tiles_ub : units;
   if (grid < 1) grid = 1;
-  cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE, BMODE>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (PAIR) grid *= 2;
+  auto kernel = tc_grouped_gemm<MODE, BMODE, PAIR>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  tc_grouped_gemm<MODE, BMODE><<<static_cast<unsigned>(grid), threads_of<BMODE>(), smem, stream>>>(
-      a0, a1, b, p);
+  if constexpr (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(threads_of<BMODE>(), 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, a0, a1, b, p);
+    if (e != cudaSuccess) return e;
+  } else {
+    kernel<<<static_cast<unsigned>(grid), threads_of<BMODE>(), smem, stream>>>(a0, a1, b, p);
+  }
   return cudaGetLastError();
 }
 
+// CTA pairs (cta_group::2) for the expert GEMMs unless the build opts out.
+constexpr bool kUsePairs =
+#ifdef MOE_NO_CTA_PAIRS
+    false;
+#else
+    true;
+#endif
+
 }  // namespace
+
+bool gemm1_uses_row_copy(int I) { return kUsePairs && (I % 256) == 0; }
 
 int route_token_block(int64_t T) { return T >= 64 ? 64 : static_cast<int>(((T + 31) / 32) * 32); }
 
@@ -577,18 +674,47 @@ cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int
   p.bias = nullptr;
   p.err = err;
   const int64_t tiles = static_cast<int64_t>(p.num_fb) * ((T + p.TB - 1) / p.TB) * ksplit;
-  return launch_mode<kEpiF32, kBTiled>(a0, a0, b, p, tiles, num_sms, stream, detail);
+  return launch_mode<kEpiF32, kBTiled, false>(a0, a0, b, p, tiles, num_sms, stream, detail);
 }
 
-cudaError_t launch_gemm1_tc(const void* x, int T, const int32_t* sorted_ids,
+cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t* sorted_ids,
                             const int32_t* offsets, const int32_t* blk_prefix, const void* w_gate,
                             const void* w_up, void* hbuf, int64_t hbuf_rows, int H, int E, int k,
                             int I, int TB, int64_t ub_blocks, int* err, int num_sms,
                             cudaStream_t stream, std::string* detail) {
-  (void)hbuf_rows;
   CUtensorMap a0, a1, b;
-  if (!map_weights(&a0, w_gate, I, H, E, detail) || !map_weights(&a1, w_up, I, H, E, detail) ||
-      !map_rows(&b, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), detail))
+  if (!map_weights(&a0, w_gate, I, H, E, detail) || !map_weights(&a1, w_up, I, H, E, detail))
+    return cudaErrorInvalidValue;
+  if (xs != nullptr) {
+    // token rows already in expert-major order: contiguous rows like GEMM2's B operand, so
+    // both CTAs of a pair can take their halves by TMA
+    if (!map_row_boxes(&b, xs, static_cast<uint64_t>(H), static_cast<uint64_t>(hbuf_rows), detail))
+      return cudaErrorInvalidValue;
+    const bool pair = kUsePairs && (I % 256) == 0;
+    TcParams p{};
+    p.K = H;
+    p.num_fb = pair ? I / 256 : I / kBM;
+    p.m_rows_a = I;
+    p.m_valid = I;
+    p.TB = TB;
+    p.groups = E;
+    p.k_top = 1;
+    p.rows_b = static_cast<int>(hbuf_rows);
+    p.sorted_ids = nullptr;
+    p.offsets = offsets;
+    p.blk_prefix = blk_prefix;
+    p.out = hbuf;
+    p.ldo = I;
+    p.bias = nullptr;
+    p.err = err;
+    p.b_ptr = nullptr;
+    p.ksplit = 1;
+    const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
+    if (pair)
+      return launch_mode<kEpiSwiGLU, kBTiled, true>(a0, a1, b, p, tiles, num_sms, stream, detail);
+    return launch_mode<kEpiSwiGLU, kBTiled, false>(a0, a1, b, p, tiles, num_sms, stream, detail);
+  }
+  if (!map_rows(&b, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), detail))
     return cudaErrorInvalidValue;
 #ifdef MOE_GEMM1_GATHER4
   const bool use_gather4 = true;   // TMA tile::gather4 row gather (build-time choice)
@@ -615,8 +741,8 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const int32_t* sorted_ids,
   p.ksplit = 1;
   const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
   if (use_gather4)
-    return launch_mode<kEpiSwiGLU, kBGather4>(a0, a1, b, p, tiles, num_sms, stream, detail);
-  return launch_mode<kEpiSwiGLU, kBCpAsync>(a0, a1, b, p, tiles, num_sms, stream, detail);
+    return launch_mode<kEpiSwiGLU, kBGather4, false>(a0, a1, b, p, tiles, num_sms, stream, detail);
+  return launch_mode<kEpiSwiGLU, kBCpAsync, false>(a0, a1, b, p, tiles, num_sms, stream, detail);
 }
 
 cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* offsets,
@@ -629,9 +755,10 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
     return cudaErrorInvalidValue;
   TcParams p{};
   const bool dual = (H % 256) == 0;
+  const bool pair = kUsePairs && (H % 512) == 0;
   p.ksplit = 1;
   p.K = I;
-  p.num_fb = dual ? H / 256 : H / kBM;
+  p.num_fb = pair ? H / 512 : (dual ? H / 256 : H / kBM);
   p.m_rows_a = H;
   p.m_valid = H;
   p.TB = TB;
@@ -646,8 +773,11 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
   p.bias = nullptr;
   p.err = err;
   const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
-  if (dual) return launch_mode<kEpiBF16x2, kBTiled>(a0, a0, b, p, tiles, num_sms, stream, detail);
-  return launch_mode<kEpiBF16, kBTiled>(a0, a0, b, p, tiles, num_sms, stream, detail);
+  if (pair)
+    return launch_mode<kEpiBF16x2, kBTiled, true>(a0, a0, b, p, tiles, num_sms, stream, detail);
+  if (dual)
+    return launch_mode<kEpiBF16x2, kBTiled, false>(a0, a0, b, p, tiles, num_sms, stream, detail);
+  return launch_mode<kEpiBF16, kBTiled, false>(a0, a0, b, p, tiles, num_sms, stream, detail);
 }
 
 }  // namespace moe

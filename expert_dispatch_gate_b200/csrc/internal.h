@@ -30,7 +30,11 @@ cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int
                                  float* partials, int ksplit, int* err, int num_sms,
                                  cudaStream_t stream, std::string* detail);
 // Expert GEMM1: h[s, :] = silu(x[t] Wg[e]) * (x[t] Wu[e]) for kept slots; h rows = hbuf_rows.
-cudaError_t launch_gemm1_tc(const void* x, int T, const int32_t* sorted_ids,
+// With xs != nullptr the token rows come from the expert-major copy xs (contiguous per expert,
+// streamed by TMA, CTA pairs when I % 256 == 0); otherwise they are gathered from x through
+// sorted_ids by cp.async (single CTAs).
+bool gemm1_uses_row_copy(int I);
+cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t* sorted_ids,
                             const int32_t* offsets, const int32_t* blk_prefix, const void* w_gate,
                             const void* w_up, void* hbuf, int64_t hbuf_rows, int H, int E, int k,
                             int I, int TB, int64_t ub_blocks, int* err, int num_sms,
@@ -65,6 +69,10 @@ cudaError_t launch_plan_from_offsets(const int32_t* offsets, int E, int TB, int3
                                      cudaStream_t stream);
 
 // ---- combine.cu
+// Expert-major copy of the token rows: xs[s,:] = x[sorted_ids[s]/k,:] for kept slots.
+cudaError_t launch_dispatch_rows(int dtype, const void* x, const int32_t* sorted_ids,
+                                 const int32_t* offsets, int E, int k, int H, int64_t rows,
+                                 void* xs, cudaStream_t stream);
 cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_of,
                            const float* topk_w, void* out, int64_t T, int H, int k,
                            cudaStream_t stream);

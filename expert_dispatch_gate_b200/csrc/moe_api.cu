@@ -98,8 +98,15 @@ int token_block(const moe_shape& s, int32_t C) {
   return static_cast<int>(tb);
 }
 
+// GEMM1 reads the token rows from an expert-major copy made right after the grouping when
+// CTA pairs can share it (I % 256 == 0): the copy is streamed by TMA, half per CTA. Otherwise
+// GEMM1 gathers the rows straight from x.
+bool gemm1_from_copy(const moe_shape& s) {
+  return s.dtype == MOE_BF16 && moe::gemm1_uses_row_copy(s.I);
+}
+
 struct Layout {
-  size_t err, logits, blk_hist, offsets, blk_prefix, sorted_ids, slot_of, hbuf, yslots, total;
+  size_t err, logits, blk_hist, offsets, blk_prefix, sorted_ids, slot_of, hbuf, yslots, xs, total;
   int64_t A, a_cap;
   int nblk;
   int32_t C;
@@ -133,6 +140,7 @@ Layout layout_of(const moe_shape& s) {
   L.slot_of = take(static_cast<size_t>(L.A) * 4);
   L.hbuf = take(static_cast<size_t>(L.a_cap) * s.I * es);
   L.yslots = take(static_cast<size_t>(L.a_cap) * s.H * es);
+  L.xs = gemm1_from_copy(s) ? take(static_cast<size_t>(L.a_cap) * s.H * es) : 0;
   L.total = off;
   return L;
 }
@@ -207,7 +215,13 @@ moe_status do_ffn(const moe_shape& s, const Layout& L, const void* x, const int3
   if (s.dtype == MOE_BF16) {
     const int64_t ub_blocks = (s.E < L.a_cap ? s.E : L.a_cap) + L.a_cap / L.TB;
     std::string d;
-    e = moe::launch_gemm1_tc(x, static_cast<int>(s.T), sorted_ids, offsets,
+    void* xs = nullptr;
+    if (gemm1_from_copy(s)) {
+      xs = at<void>(ws, L.xs);
+      e = moe::launch_dispatch_rows(s.dtype, x, sorted_ids, offsets, s.E, s.k, s.H, L.a_cap, xs, st);
+      if (e != cudaSuccess) return cuda_fail(e, "expert-major row copy");
+    }
+    e = moe::launch_gemm1_tc(x, static_cast<int>(s.T), xs, sorted_ids, offsets,
                              at<int32_t>(ws, L.blk_prefix), w_gate, w_up, at<void>(ws, L.hbuf),
                              L.a_cap, s.H, s.E, s.k, s.I, L.TB, ub_blocks, at<int>(ws, L.err),
                              num_sms(), st, &d);
@@ -352,7 +366,7 @@ moe_status moe_grouped_ffn(const moe_shape* shape, const void* x, const int32_t*
   REQUIRE_PTR(w_down, "w_down");
   REQUIRE_PTR(y_slots, "y_slots");
   const Layout L = layout_of(*shape);
-  st = check_ws(ws, ws_bytes, L.yslots);
+  st = check_ws(ws, ws_bytes, L.total);
   if (st != MOE_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (shape->dtype == MOE_BF16) {
