@@ -60,6 +60,12 @@ constexpr int kGatherWarp0 = 2 + kEpiWarps;
 template <int BMODE>
 constexpr int threads_of() { return 32 * (kGatherWarp0 + (BMODE == kBCpAsync ? 4 : 0)); }
 
+// Token rows of B one CTA keeps per stage: all TB, or the half it holds in a CTA pair (rounded
+// up to whole 32-row TMA boxes).
+__host__ __device__ constexpr int b_rows_smem(bool pair, int TB) {
+  return pair ? (((TB >> 1) + 31) & ~31) : TB;
+}
+
 struct TcParams {
   int K;          // reduction length (multiple of 64)
   int num_fb;     // feature blocks of 128
@@ -105,9 +111,12 @@ __device__ __forceinline__ Tile decode_tile(int tile, int num_fb, int groups, in
   const int local = tile - num_fb * s_blk[lo];
   t.fb = local / nb;
   const int b = local - t.fb * nb;
+  // nb = ceil(cnt / TB) blocks of equal size bs = ceil(cnt / nb) <= TB; every block is non-empty
+  // because (nb - 1) * bs <= (nb - 1) * TB < cnt
   const int cnt = s_off[lo + 1] - s_off[lo];
-  t.n = min(TB, cnt - b * TB);
-  t.row0 = s_off[lo] + b * TB;
+  const int bs = (cnt + nb - 1) / nb;
+  t.n = min(bs, cnt - b * bs);
+  t.row0 = s_off[lo] + b * bs;
   const int per = kblocks / ksplit;
   t.ks = ks;
   t.kb0 = ks * per;
@@ -141,7 +150,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int a_bytes = kDual ? 32768 : 16384;
-  const int stage_bytes = a_bytes + p.TB * 128;
+  const int stage_bytes = a_bytes + b_rows_smem(PAIR, p.TB) * 128;
   const int S = p.stages;
   uint8_t* ctrl = smem + static_cast<size_t>(S) * stage_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
@@ -584,7 +593,7 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
                         TcParams p, int64_t tiles_ub, int num_sms, cudaStream_t stream,
                         std::string* d) {
   const int a_bytes = dual_a<MODE>() ? 32768 : 16384;
-  const int stage_bytes = a_bytes + p.TB * 128;
+  const int stage_bytes = a_bytes + b_rows_smem(PAIR, p.TB) * 128;
   int stages = (kSmemLimit - 1024 - kCtrlBytes) / stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) {

@@ -85,15 +85,17 @@ int32_t capacity_of(const moe_shape& s) {
   return c >= static_cast<unsigned __int128>(s.T) ? static_cast<int32_t>(s.T) : static_cast<int32_t>(c);
 }
 
-// Rows per token block of the expert GEMMs: a multiple of 32 in [32, 256] that splits the
-// largest possible expert group (min(C, T) rows) into equal-sized blocks.
+// Largest token block of the expert GEMMs (a multiple of 32 in [32, 256]). It only shapes the
+// work: an expert with n kept tokens runs as ceil(n / TB) blocks of equal size, whatever n is.
+// Sized from the largest expected group, min(C, T, 2 * T*k/E): the shared-memory stages and
+// TMEM accumulators are reserved for TB rows, so a TB far above the real groups (decode) wastes
+// pipeline depth, and one far below splits experts and re-reads their weights.
 int token_block(const moe_shape& s, int32_t C) {
-  int64_t maxrows = C < s.T ? C : s.T;
-  if (maxrows < 1) maxrows = 1;
-  const int64_t nblk = (maxrows + 255) / 256;
-  int64_t tb = (maxrows + nblk - 1) / nblk;
-  tb = ((tb + 31) / 32) * 32;
-  if (tb < 32) tb = 32;
+  int64_t rows = C < s.T ? C : s.T;
+  const int64_t mean2 = 2 * ((s.T * s.k + s.E - 1) / s.E);
+  if (mean2 < rows) rows = mean2;
+  if (rows < 1) rows = 1;
+  int64_t tb = ((rows + 31) / 32) * 32;
   if (tb > 256) tb = 256;
   return static_cast<int>(tb);
 }
