@@ -55,8 +55,9 @@ struct Vec<__nv_bfloat16> {
 constexpr int kWarps = kThreads / 32;
 constexpr int kG = 4;
 
+// Two blocks per SM (registers capped accordingly) keep enough row loads in flight.
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
     combine_kernel(const T* __restrict__ y, const int32_t* __restrict__ slot_of,
                    const float* __restrict__ topk_w, T* __restrict__ out, int64_t Ttok, int H,
                    int k, int segs) {

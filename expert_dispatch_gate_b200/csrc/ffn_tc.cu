@@ -88,6 +88,8 @@ struct TcParams {
   int* err;
   int stages;
   int nbuf;       // TMEM accumulator buffers (1 or 2, 256 columns apart)
+  int a_wide;     // A maps are 4-D: one box = all 64-feature chunks of a CTA's feature rows
+  int b_box_rows; // rows per B box (contiguous-rows mode)
 };
 
 struct Tile {
@@ -223,7 +225,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
       const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
       const int npad = (t.n + 15) & ~15;
       const int bn = b_rows(npad);
-      const int nbox = (bn + kRowBox - 1) / kRowBox;
+      const int nbox = p.a_wide ? 1 : (bn + kRowBox - 1) / kRowBox;
       int rows[8];
       if constexpr (BMODE == kBGather4) {
 #pragma unroll
@@ -238,10 +240,11 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
         }
       }
       const int m0 = t.fb * kTileFeatures + static_cast<int>(rank) * kCtaFeatures;
-      const bool hi_chunk = (m0 + 64) < p.m_rows_a;
+      const bool hi_chunk = p.a_wide || (m0 + 64) < p.m_rows_a;
       uint32_t tx = (hi_chunk ? 16384u : 8192u) * (kDual ? 2u : 1u);
       if constexpr (BMODE == kBGather4) tx += static_cast<uint32_t>(npad) * 128u;
-      if constexpr (BMODE == kBTiled) tx += static_cast<uint32_t>(nbox) * (kRowBox * 128u);
+      if constexpr (BMODE == kBTiled)
+        tx += static_cast<uint32_t>(nbox) * static_cast<uint32_t>(p.b_box_rows) * 128u;
       if constexpr (PAIR) tx *= 2u;  // both CTAs' loads complete on the even CTA's barrier
       const int brow0 = t.row0 + b_first(npad);
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
@@ -258,7 +261,14 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
         const uint32_t sb = sa + a_bytes;
         if constexpr (PAIR) {
           const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
-          if (lane == 0) {
+          if (lane == 0 && p.a_wide) {
+            // one box per weight operand: all feature chunks of this CTA's rows
+            if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), tx);
+            tma_load_4d_pair(sa, &tmA0, 0, kb * kBK, m0 >> 6, t.group, fbar);
+            if constexpr (kSwiGLU) tma_load_4d_pair(sa + 16384, &tmA1, 0, kb * kBK, m0 >> 6, t.group, fbar);
+            if constexpr (BMODE == kBTiled)
+              tma_load_2d_pair(sb, &tmB, kb * kBK, brow0, fbar);
+          } else if (lane == 0) {
             if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), tx);
             tma_load_3d_pair(sa, &tmA0, m0, kb * kBK, t.group, fbar);
             if (hi_chunk) tma_load_3d_pair(sa + 8192, &tmA0, m0 + 64, kb * kBK, t.group, fbar);
@@ -278,7 +288,12 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
           __syncwarp();
         } else {
           const uint32_t fbar = smem_u32(&full[s]);
-          if (lane == 0) {
+          if (lane == 0 && p.a_wide) {
+            mbar_arrive_expect_tx(fbar, tx);
+            tma_load_4d(sa, &tmA0, 0, kb * kBK, m0 >> 6, t.group, fbar);
+            if constexpr (kSwiGLU) tma_load_4d(sa + 16384, &tmA1, 0, kb * kBK, m0 >> 6, t.group, fbar);
+            if constexpr (BMODE == kBTiled) tma_load_2d(sb, &tmB, kb * kBK, brow0, fbar);
+          } else if (lane == 0) {
             mbar_arrive_expect_tx(fbar, tx);
             tma_load_3d(sa, &tmA0, m0, kb * kBK, t.group, fbar);
             if (hi_chunk) tma_load_3d(sa + 8192, &tmA0, m0 + 64, kb * kBK, t.group, fbar);
@@ -552,7 +567,8 @@ bool map_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, st
 }
 
 // bf16 [rows, cols] row-major, box = {64 columns, 32 rows}, 128-byte swizzle: contiguous rows.
-bool map_row_boxes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, std::string* d) {
+bool map_row_boxes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, std::string* d,
+                   uint32_t box_rows = kRowBox) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) {
     if (d) *d = "cuTensorMapEncodeTiled is not available from the driver";
@@ -560,12 +576,33 @@ bool map_row_boxes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t row
   }
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, kRowBox};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t es[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS && d) *d = "cuTensorMapEncodeTiled(row boxes) failed with code " + std::to_string(r);
+  return r == CUDA_SUCCESS;
+}
+
+// bf16 [groups, kdim, mdim] (mdim contiguous) seen as 4-D {64, kdim, mdim/64, groups}, so that one
+// box {64, 64, chunks, 1} brings `chunks` consecutive 64-feature chunks of 64 K rows, laid out
+// chunk after chunk (8 KB apart) as the MN-major operand expects. 128-byte swizzle.
+bool map_weights_wide(CUtensorMap* m, const void* base, uint64_t mdim, uint64_t kdim,
+                      uint64_t groups, uint32_t chunks, std::string* d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) {
+    if (d) *d = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  cuuint64_t dims[4] = {64, kdim, mdim / 64, groups};
+  cuuint64_t strides[3] = {mdim * 2, 128, mdim * kdim * 2};
+  cuuint32_t box[4] = {64, 64, chunks, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && d) *d = "cuTensorMapEncodeTiled(wide weights) failed with code " + std::to_string(r);
   return r == CUDA_SUCCESS;
 }
 
@@ -682,6 +719,8 @@ cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int
   p.ldo = E;
   p.bias = nullptr;
   p.err = err;
+  p.a_wide = 0;
+  p.b_box_rows = kRowBox;
   const int64_t tiles = static_cast<int64_t>(p.num_fb) * ((T + p.TB - 1) / p.TB) * ksplit;
   return launch_mode<kEpiF32, kBTiled, false>(a0, a0, b, p, tiles, num_sms, stream, detail);
 }
@@ -692,15 +731,21 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
                             int I, int TB, int64_t ub_blocks, int* err, int num_sms,
                             cudaStream_t stream, std::string* detail) {
   CUtensorMap a0, a1, b;
-  if (!map_weights(&a0, w_gate, I, H, E, detail) || !map_weights(&a1, w_up, I, H, E, detail))
+  // gate and up slices of a CTA's 128 features arrive as one box each
+  if (!map_weights_wide(&a0, w_gate, I, H, E, 2, detail) ||
+      !map_weights_wide(&a1, w_up, I, H, E, 2, detail))
     return cudaErrorInvalidValue;
   if (xs != nullptr) {
     // token rows already in expert-major order: contiguous rows like GEMM2's B operand, so
-    // both CTAs of a pair can take their halves by TMA
-    if (!map_row_boxes(&b, xs, static_cast<uint64_t>(H), static_cast<uint64_t>(hbuf_rows), detail))
-      return cudaErrorInvalidValue;
+    // both CTAs of a pair can take their halves by TMA, one box per stage
     const bool pair = kUsePairs && (I % 256) == 0;
+    const int box_rows = b_rows_smem(pair, TB);
+    if (!map_row_boxes(&b, xs, static_cast<uint64_t>(H), static_cast<uint64_t>(hbuf_rows), detail,
+                       static_cast<uint32_t>(box_rows)))
+      return cudaErrorInvalidValue;
     TcParams p{};
+    p.a_wide = 1;
+    p.b_box_rows = box_rows;
     p.K = H;
     p.num_fb = pair ? I / 256 : I / kBM;
     p.m_rows_a = I;
@@ -731,6 +776,8 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
   const bool use_gather4 = false;  // cp.async row gather
 #endif
   TcParams p{};
+  p.a_wide = 1;
+  p.b_box_rows = 0;
   p.K = H;
   p.num_fb = I / kBM;
   p.m_rows_a = I;
@@ -759,12 +806,17 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
                             int I, int TB, int64_t ub_blocks, int* err, int num_sms,
                             cudaStream_t stream, std::string* detail) {
   CUtensorMap a0, b;
-  if (!map_weights(&a0, w_down, H, I, E, detail) ||
-      !map_row_boxes(&b, hbuf, static_cast<uint64_t>(I), static_cast<uint64_t>(hbuf_rows), detail))
-    return cudaErrorInvalidValue;
-  TcParams p{};
   const bool dual = (H % 256) == 0;
   const bool pair = kUsePairs && (H % 512) == 0;
+  const int box_rows = b_rows_smem(pair, TB);
+  // a CTA's 256 (dual) or 128 feature rows of Wd arrive as one box; its token rows as another
+  if (!map_weights_wide(&a0, w_down, H, I, E, dual ? 4 : 2, detail) ||
+      !map_row_boxes(&b, hbuf, static_cast<uint64_t>(I), static_cast<uint64_t>(hbuf_rows), detail,
+                     static_cast<uint32_t>(box_rows)))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.a_wide = 1;
+  p.b_box_rows = box_rows;
   p.ksplit = 1;
   p.K = I;
   p.num_fb = pair ? H / 512 : (dual ? H / 256 : H / kBM);
