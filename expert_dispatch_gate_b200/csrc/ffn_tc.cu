@@ -56,6 +56,10 @@ enum BMode { kBGather4 = 0, kBTiled = 1, kBCpAsync = 2 };
 // Warps: 0 TMA producer, 1 MMA issuer, 2-9 epilogue (two warps per TMEM lane quadrant, each
 // draining half of the token columns), 10-13 cp.async row gatherers (kBCpAsync).
 constexpr int kEpiWarps = 8;
+// 32-column chunks one epilogue warp drains per tile: columns 32*half + 64*i, i < 4, cover
+// every token block of up to 256 rows.
+constexpr int kEpiChunks = 4;
+constexpr int kMaxTokenBlock = 256;
 constexpr int kGatherWarp0 = 2 + kEpiWarps;
 template <int BMODE>
 constexpr int threads_of() { return 32 * (kGatherWarp0 + (BMODE == kBCpAsync ? 4 : 0)); }
@@ -124,6 +128,15 @@ __device__ __forceinline__ Tile decode_tile(int tile, int num_fb, int groups, in
   t.kb0 = ks * per;
   t.kb1 = t.kb0 + per;
   return t;
+}
+
+// Round two floats to bf16 (nearest-even) and pack them, the first in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ uint16_t bf16_half(uint32_t w, int hi) {
+  return static_cast<uint16_t>(hi ? (w >> 16) : (w & 0xffffu));
 }
 
 // PAIR: two CTAs of a cluster cooperate on each tile with tcgen05.mma.cta_group::2 (M = 256).
@@ -335,64 +348,81 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0 && leader) {
-      // ---------------------------------------------------------- MMA issuer (one thread)
-      int it = 0, tc = 0;
+    if (leader) {
+      // ---------------------------------------------------------- MMA issuer (one warp)
+      // The whole warp runs this loop so that its control flow, counters and descriptors stay
+      // warp-uniform; one elected lane issues each tcgen05.mma / commit. Stage index, phase and
+      // stage byte offset advance incrementally, and the smem descriptors are the stage-0 ones
+      // plus the offset (in 16-byte units), so nothing but the MMAs sits between two MMAs.
+      constexpr uint32_t kFull = 0xffffffffu;
+      const uint32_t S = static_cast<uint32_t>(p.stages);
+      const uint32_t sbase = smem_u32(smem);
+      const uint64_t adesc0 = smem_desc_sw128(sbase, 8192, 1024);
+      const uint64_t bdesc0 = smem_desc_sw128(sbase + a_bytes, 16, 1024);
+      uint32_t s = 0, ph = 0, soff = 0;
+      int tc = 0;
       bool ok = true;
       for (int tile = tile0; ok && tile < num_tiles; tile += tstep) {
         const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
         const int npad = (t.n + 15) & ~15;
         const int buf = tc % p.nbuf;
         const uint32_t use = static_cast<uint32_t>(tc / p.nbuf);
-        if (!mbar_wait_cluster(smem_u32(&tempty[buf]), (use & 1u) ^ 1u, abort_flag)) {
+        if (!__all_sync(kFull, mbar_wait_cluster(smem_u32(&tempty[buf]), (use & 1u) ^ 1u,
+                                                 abort_flag))) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * 256);
+        const uint32_t d1 = d0 + static_cast<uint32_t>(p.TB);
         const uint32_t idesc =
             idesc_bf16(PAIR ? 2 * kBM : kBM, npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
+        uint32_t acc = 0;
+#pragma unroll 2
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          const int s = it % S;
-          const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
-          if (!mbar_wait_cluster(smem_u32(&full[s]), ph, abort_flag)) {
+          if (!__all_sync(kFull, mbar_wait_cluster(smem_u32(&full[s]), ph, abort_flag))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
-          const uint32_t sb = sa + a_bytes;
+          const uint64_t ad = adesc0 + (soff >> 4);
+          const uint64_t bd = bdesc0 + (soff >> 4);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(sa + kk * 2048, 8192, 1024);
-            const uint64_t bd = smem_desc_sw128(sb + kk * 32, 16, 1024);
-            const uint32_t acc = (kb > t.kb0 || kk > 0) ? 1u : 0u;
-            if constexpr (PAIR) tc_mma_bf16_pair(d0, ad, bd, idesc, acc);
-            else tc_mma_bf16(d0, ad, bd, idesc, acc);
+            // A advances 16 K-rows (2 KB), B 16 K-columns (32 B) per step; the second A
+            // operand sits 16 KB after the first
+            if constexpr (PAIR) tc_mma_bf16_pair_elect(d0, ad + kk * 128, bd + kk * 2, idesc, acc);
+            else tc_mma_bf16_elect(d0, ad + kk * 128, bd + kk * 2, idesc, acc);
             if constexpr (kDual) {
-              const uint64_t ad1 = smem_desc_sw128(sa + 16384 + kk * 2048, 8192, 1024);
               if constexpr (PAIR)
-                tc_mma_bf16_pair(d0 + static_cast<uint32_t>(p.TB), ad1, bd, idesc, acc);
+                tc_mma_bf16_pair_elect(d1, ad + 1024 + kk * 128, bd + kk * 2, idesc, acc);
               else
-                tc_mma_bf16(d0 + static_cast<uint32_t>(p.TB), ad1, bd, idesc, acc);
+                tc_mma_bf16_elect(d1, ad + 1024 + kk * 128, bd + kk * 2, idesc, acc);
             }
+            acc = 1u;
           }
-          if constexpr (PAIR) tc_commit_pair_mc(smem_u32(&empty[s]), 0x3);
-          else tc_commit(smem_u32(&empty[s]));
-          ++it;
+          if constexpr (PAIR) tc_commit_pair_mc_elect(smem_u32(&empty[s]), 0x3);
+          else tc_commit_elect(smem_u32(&empty[s]));
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+            soff = 0;
+          } else {
+            soff += static_cast<uint32_t>(stage_bytes);
+          }
         }
         if (!ok) break;
-        if constexpr (PAIR) tc_commit_pair_mc(smem_u32(&tfull[buf]), 0x3);
-        else tc_commit(smem_u32(&tfull[buf]));
+        if constexpr (PAIR) tc_commit_pair_mc_elect(smem_u32(&tfull[buf]), 0x3);
+        else tc_commit_elect(smem_u32(&tfull[buf]));
         ++tc;
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         *abort_flag = 1;
         flag_error(p.err, kDevWaitTimeout);
       }
       // Every MMA issued must complete before TMEM is released.
-      if constexpr (PAIR) tc_commit_pair_mc(smem_u32(drain), 0x3);
-      else tc_commit(smem_u32(drain));
+      if constexpr (PAIR) tc_commit_pair_mc_elect(smem_u32(drain), 0x3);
+      else tc_commit_elect(smem_u32(drain));
       mbar_wait(smem_u32(drain), 0u, nullptr);
     }
     __syncwarp();
@@ -464,36 +494,13 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
       const int m = t.fb * kTileFeatures + static_cast<int>(rank) * kCtaFeatures + q * 32 + lane;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(buf * 256);
-      for (int c0 = 32 * half; c0 < t.n; c0 += 64) {
-        uint32_t v[32];
-        tmem_ld32(tb + static_cast<uint32_t>(c0), v);
-        uint32_t u[32];
-        if constexpr (kDual) tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), u);
-        tmem_wait_ld();
-        const int cmax = min(32, t.n - c0);
-        if constexpr (MODE == kEpiSwiGLU) {
-          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                             static_cast<size_t>(t.row0 + c0) * p.ldo + m;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (j < cmax) {
-              const float g = __uint_as_float(v[j]);
-              const float h = g / (1.0f + __expf(-g)) * __uint_as_float(u[j]);
-              o[static_cast<size_t>(j) * p.ldo] = __float2bfloat16_rn(h);
-            }
-          }
-        } else if constexpr (MODE == kEpiBF16 || MODE == kEpiBF16x2) {
-          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                             static_cast<size_t>(t.row0 + c0) * p.ldo + m;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (j < cmax) {
-              o[static_cast<size_t>(j) * p.ldo] = __float2bfloat16_rn(__uint_as_float(v[j]));
-              if constexpr (kDual)
-                o[static_cast<size_t>(j) * p.ldo + 128] = __float2bfloat16_rn(__uint_as_float(u[j]));
-            }
-          }
-        } else {
+      if constexpr (MODE == kEpiF32) {
+        // router partial logits: fp32 stores straight from TMEM (token blocks of <= 64 rows)
+        for (int c0 = 32 * half; c0 < t.n; c0 += 64) {
+          uint32_t v[32];
+          tmem_ld32(tb + static_cast<uint32_t>(c0), v);
+          tmem_wait_ld();
+          const int cmax = min(32, t.n - c0);
           if (m < p.m_valid) {
             float* o = reinterpret_cast<float*>(p.out) + t.ks * p.split_stride +
                        static_cast<size_t>(t.row0 + c0) * p.ldo + m;
@@ -502,12 +509,75 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
               if (j < cmax) o[static_cast<size_t>(j) * p.ldo] = __uint_as_float(v[j]);
           }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
-        else mbar_arrive(smem_u32(&tempty[buf]));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
+          else mbar_arrive(smem_u32(&tempty[buf]));
+        }
+      } else {
+        // Read every accumulator chunk this warp owns into registers, already rounded to bf16
+        // (two values per word), hand the TMEM buffer back to the MMA issuer, and only then
+        // write the rows out: the next tile's MMAs run under these stores.
+        constexpr int kW = (MODE == kEpiBF16x2) ? 32 : 16;  // words held per 32-column chunk
+        uint32_t pk[kEpiChunks][kW];
+#pragma unroll
+        for (int i = 0; i < kEpiChunks; ++i) {
+          const int c0 = 32 * half + 64 * i;
+          if (c0 < t.n) {
+            uint32_t v[32];
+            tmem_ld32(tb + static_cast<uint32_t>(c0), v);
+            if constexpr (kSwiGLU) {
+              uint32_t u[32];
+              tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), u);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const float g0 = __uint_as_float(v[2 * j]);
+                const float g1 = __uint_as_float(v[2 * j + 1]);
+                const float h0 = g0 / (1.0f + __expf(-g0)) * __uint_as_float(u[2 * j]);
+                const float h1 = g1 / (1.0f + __expf(-g1)) * __uint_as_float(u[2 * j + 1]);
+                pk[i][j] = pack_bf16x2(h0, h1);
+              }
+            } else {
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                pk[i][j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+              if constexpr (kDual) {
+                tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                  pk[i][16 + j] =
+                      pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
+          else mbar_arrive(smem_u32(&tempty[buf]));
+        }
+#pragma unroll
+        for (int i = 0; i < kEpiChunks; ++i) {
+          const int c0 = 32 * half + 64 * i;
+          if (c0 < t.n) {
+            const int cmax = min(32, t.n - c0);
+            uint16_t* o = reinterpret_cast<uint16_t*>(p.out) +
+                          static_cast<size_t>(t.row0 + c0) * p.ldo + m;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j < cmax) {
+                o[static_cast<size_t>(j) * p.ldo] = bf16_half(pk[i][j >> 1], j & 1);
+                if constexpr (MODE == kEpiBF16x2)
+                  o[static_cast<size_t>(j) * p.ldo + 128] = bf16_half(pk[i][16 + (j >> 1)], j & 1);
+              }
+            }
+          }
+        }
       }
       ++tc;
     }
@@ -635,6 +705,10 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) {
     if (d) *d = "tile too large for shared memory";
+    return cudaErrorInvalidValue;
+  }
+  if (p.TB < 32 || p.TB > kMaxTokenBlock || (p.TB & 31) != 0) {
+    if (d) *d = "token block must be a multiple of 32 in [32, 256]";
     return cudaErrorInvalidValue;
   }
   p.stages = stages;
