@@ -130,6 +130,13 @@ __device__ __forceinline__ Tile decode_tile(int tile, int num_fb, int groups, in
   return t;
 }
 
+// SiLU(g) = g * sigmoid(g) = g / (1 + e^-g), with the fast-division intrinsic (at most 2 ulp
+// in fp32; the result is rounded to bf16 right after). The IEEE-exact division made the
+// SwiGLU epilogue hold the accumulator several times longer on tensor-bound shapes. For
+// g below about -85 the denominator reaches 2^126 or overflows and the quotient is 0, where
+// SiLU itself is below 1e-35 in magnitude.
+__device__ __forceinline__ float silu_f32(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
 // Round two floats to bf16 (nearest-even) and pack them, the first in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -532,13 +539,10 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
               tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), u);
               tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const float g0 = __uint_as_float(v[2 * j]);
-                const float g1 = __uint_as_float(v[2 * j + 1]);
-                const float h0 = g0 / (1.0f + __expf(-g0)) * __uint_as_float(u[2 * j]);
-                const float h1 = g1 / (1.0f + __expf(-g1)) * __uint_as_float(u[2 * j + 1]);
-                pk[i][j] = pack_bf16x2(h0, h1);
-              }
+              for (int j = 0; j < 16; ++j)
+                pk[i][j] = pack_bf16x2(
+                    silu_f32(__uint_as_float(v[2 * j])) * __uint_as_float(u[2 * j]),
+                    silu_f32(__uint_as_float(v[2 * j + 1])) * __uint_as_float(u[2 * j + 1]));
             } else {
               tmem_wait_ld();
 #pragma unroll
@@ -561,10 +565,14 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
           if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
           else mbar_arrive(smem_u32(&tempty[buf]));
         }
+        // The last tile of a CTA pair may reach past the weight's feature extent (the second
+        // CTA's rows were loaded as zeros): those feature rows have no output.
+        const bool keep0 = m < p.m_valid;
+        const bool keep1 = (MODE == kEpiBF16x2) && (m + 128 < p.m_valid);
 #pragma unroll
         for (int i = 0; i < kEpiChunks; ++i) {
           const int c0 = 32 * half + 64 * i;
-          if (c0 < t.n) {
+          if (c0 < t.n && keep0) {
             const int cmax = min(32, t.n - c0);
             uint16_t* o = reinterpret_cast<uint16_t*>(p.out) +
                           static_cast<size_t>(t.row0 + c0) * p.ldo + m;
@@ -573,7 +581,8 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
               if (j < cmax) {
                 o[static_cast<size_t>(j) * p.ldo] = bf16_half(pk[i][j >> 1], j & 1);
                 if constexpr (MODE == kEpiBF16x2)
-                  o[static_cast<size_t>(j) * p.ldo + 128] = bf16_half(pk[i][16 + (j >> 1)], j & 1);
+                  if (keep1)
+                    o[static_cast<size_t>(j) * p.ldo + 128] = bf16_half(pk[i][16 + (j >> 1)], j & 1);
               }
             }
           }
@@ -753,7 +762,7 @@ constexpr bool kUsePairs =
 
 }  // namespace
 
-bool gemm1_uses_row_copy(int I) { return kUsePairs && (I % 256) == 0; }
+bool gemm1_uses_row_copy(int /*I*/) { return kUsePairs; }
 
 int route_token_block(int64_t T) { return T >= 64 ? 64 : static_cast<int>(((T + 31) / 32) * 32); }
 
@@ -812,7 +821,9 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
   if (xs != nullptr) {
     // token rows already in expert-major order: contiguous rows like GEMM2's B operand, so
     // both CTAs of a pair can take their halves by TMA, one box per stage
-    const bool pair = kUsePairs && (I % 256) == 0;
+    // CTA pairs cover 256 features; when I % 256 == 128 the last pair tile's second CTA reads
+    // only zero-filled weight rows and stores nothing
+    const bool pair = kUsePairs;
     const int box_rows = b_rows_smem(pair, TB);
     if (!map_row_boxes(&b, xs, static_cast<uint64_t>(H), static_cast<uint64_t>(hbuf_rows), detail,
                        static_cast<uint32_t>(box_rows)))
@@ -821,7 +832,7 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
     p.a_wide = 1;
     p.b_box_rows = box_rows;
     p.K = H;
-    p.num_fb = pair ? I / 256 : I / kBM;
+    p.num_fb = pair ? (I + 255) / 256 : I / kBM;
     p.m_rows_a = I;
     p.m_valid = I;
     p.TB = TB;
@@ -881,7 +892,7 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
                             cudaStream_t stream, std::string* detail) {
   CUtensorMap a0, b;
   const bool dual = (H % 256) == 0;
-  const bool pair = kUsePairs && (H % 512) == 0;
+  const bool pair = kUsePairs && dual;  // 512 features per pair tile; a partial last tile is masked
   const int box_rows = b_rows_smem(pair, TB);
   // a CTA's 256 (dual) or 128 feature rows of Wd arrive as one box; its token rows as another
   if (!map_weights_wide(&a0, w_down, H, I, E, dual ? 4 : 2, detail) ||
@@ -893,7 +904,7 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
   p.b_box_rows = box_rows;
   p.ksplit = 1;
   p.K = I;
-  p.num_fb = pair ? H / 512 : (dual ? H / 256 : H / kBM);
+  p.num_fb = pair ? (H + 511) / 512 : (dual ? H / 256 : H / kBM);
   p.m_rows_a = H;
   p.m_valid = H;
   p.TB = TB;
