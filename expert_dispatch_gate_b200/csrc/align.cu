@@ -32,6 +32,7 @@ constexpr int kMaxE = 256;
 __global__ void __launch_bounds__(kThreads)
     align_hist_kernel(const int32_t* __restrict__ idx, int64_t A, int E,
                       int32_t* __restrict__ blk_hist, int* err) {
+  pdl_enter<false>();
   __shared__ int h[kMaxE];
   for (int e = threadIdx.x; e < E; e += kThreads) h[e] = 0;
   __syncthreads();
@@ -78,6 +79,7 @@ __global__ void __launch_bounds__(kThreads)
     align_scan_kernel(int32_t* __restrict__ blk_hist, int nblk, int E, int C, int TB,
                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                       int32_t* __restrict__ blk_prefix) {
+  pdl_enter<false>();
   __shared__ int sh[kWarps];
   const int e = threadIdx.x;
   int run = 0;
@@ -116,6 +118,7 @@ __global__ void __launch_bounds__(kThreads)
                          const int32_t* __restrict__ blk_base, const int32_t* __restrict__ offsets,
                          int32_t* __restrict__ sorted_ids, int32_t* __restrict__ slot_of,
                          uint8_t* __restrict__ drop_mask) {
+  pdl_enter<false>();
   __shared__ int wrun[kWarps][kMaxE];
   __shared__ int s_off[kMaxE];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -184,6 +187,7 @@ __global__ void __launch_bounds__(kThreads)
                               int32_t* __restrict__ blk_prefix, int32_t* __restrict__ sorted_ids,
                               int32_t* __restrict__ slot_of, uint8_t* __restrict__ drop_mask,
                               int* err) {
+  pdl_enter<false>();
   __shared__ int wrun[kWarps][kMaxE];
   __shared__ int s_off[kMaxE + 1];
   __shared__ int sh[kWarps];
@@ -259,6 +263,7 @@ __global__ void __launch_bounds__(kThreads)
 __global__ void __launch_bounds__(kThreads)
     plan_from_offsets_kernel(const int32_t* __restrict__ offsets, int E, int TB,
                              int32_t* __restrict__ blk_prefix) {
+  pdl_enter<false>();
   __shared__ int sh[kWarps];
   const int e = threadIdx.x;
   const int cnt = (e < E) ? (offsets[e + 1] - offsets[e]) : 0;
@@ -277,18 +282,19 @@ cudaError_t launch_align(const int32_t* topk_idx, int64_t A, int E, int C, int T
                          uint8_t* drop_mask, int* err, cudaStream_t stream) {
   if (A == 0) return cudaSuccess;
   const int nblk = static_cast<int>((A + kAlignChunk - 1) / kAlignChunk);
-  if (nblk == 1) {
-    align_single_chunk_kernel<<<1, kThreads, 0, stream>>>(topk_idx, A, E, C, TB, counts, offsets,
-                                                          blk_prefix, sorted_ids, slot_of,
-                                                          drop_mask, err);
-    return cudaGetLastError();
-  }
-  align_hist_kernel<<<nblk, kThreads, 0, stream>>>(topk_idx, A, E, blk_hist, err);
-  align_scan_kernel<<<1, kThreads, 0, stream>>>(blk_hist, nblk, E, C, TB, counts, offsets,
-                                                blk_prefix);
-  align_scatter_kernel<<<nblk, kThreads, 0, stream>>>(topk_idx, A, E, C, blk_hist, offsets,
-                                                      sorted_ids, slot_of, drop_mask);
-  return cudaGetLastError();
+  if (nblk == 1)
+    return launch_kernel(align_single_chunk_kernel, dim3(1), dim3(kThreads), 0, stream, 1,
+                         topk_idx, A, E, C, TB, counts, offsets, blk_prefix, sorted_ids, slot_of,
+                         drop_mask, err);
+  cudaError_t e = launch_kernel(align_hist_kernel, dim3(nblk), dim3(kThreads), 0, stream, 1,
+                                topk_idx, A, E, blk_hist, err);
+  if (e == cudaSuccess)
+    e = launch_kernel(align_scan_kernel, dim3(1), dim3(kThreads), 0, stream, 1, blk_hist, nblk, E,
+                      C, TB, counts, offsets, blk_prefix);
+  if (e == cudaSuccess)
+    e = launch_kernel(align_scatter_kernel, dim3(nblk), dim3(kThreads), 0, stream, 1, topk_idx, A,
+                      E, C, blk_hist, offsets, sorted_ids, slot_of, drop_mask);
+  return e;
 }
 
 // ---- grouping without a caller workspace
@@ -342,8 +348,8 @@ cudaError_t launch_align_noalloc(const int32_t* topk_idx, int64_t A, int E, int 
 
 cudaError_t launch_plan_from_offsets(const int32_t* offsets, int E, int TB, int32_t* blk_prefix,
                                      cudaStream_t stream) {
-  plan_from_offsets_kernel<<<1, kThreads, 0, stream>>>(offsets, E, TB, blk_prefix);
-  return cudaGetLastError();
+  return launch_kernel(plan_from_offsets_kernel, dim3(1), dim3(kThreads), 0, stream, 1, offsets, E,
+                       TB, blk_prefix);
 }
 
 }  // namespace moe

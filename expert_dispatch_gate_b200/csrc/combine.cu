@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     combine_kernel(const T* __restrict__ y, const int32_t* __restrict__ slot_of,
                    const float* __restrict__ topk_w, T* __restrict__ out, int64_t Ttok, int H,
                    int k, int segs) {
+  pdl_enter<false>();
   constexpr int N = Vec<T>::N;
   const int lane = threadIdx.x & 31;
   const int64_t wid = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
@@ -121,6 +122,7 @@ __global__ void __launch_bounds__(kThreads)
     dispatch_rows_kernel(const T* __restrict__ x, const int32_t* __restrict__ sorted_ids,
                          const int32_t* __restrict__ offsets, int E, int k, int H, int64_t rows,
                          T* __restrict__ xs) {
+  pdl_enter<false>();
   const int lane = threadIdx.x & 31;
   const int64_t s = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   if (s >= rows || s >= offsets[E]) return;
@@ -139,13 +141,12 @@ cudaError_t launch_dispatch_rows(int dtype, const void* x, const int32_t* sorted
   if (rows == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((rows + kWarps - 1) / kWarps);
   if (dtype == 0)
-    dispatch_rows_kernel<float><<<grid, kThreads, 0, stream>>>(
-        static_cast<const float*>(x), sorted_ids, offsets, E, k, H, rows, static_cast<float*>(xs));
-  else
-    dispatch_rows_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), sorted_ids, offsets, E, k, H, rows,
-        static_cast<__nv_bfloat16*>(xs));
-  return cudaGetLastError();
+    return launch_kernel(dispatch_rows_kernel<float>, dim3(grid), dim3(kThreads), 0, stream, 1,
+                         static_cast<const float*>(x), sorted_ids, offsets, E, k, H, rows,
+                         static_cast<float*>(xs));
+  return launch_kernel(dispatch_rows_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), 0, stream,
+                       1, static_cast<const __nv_bfloat16*>(x), sorted_ids, offsets, E, k, H, rows,
+                       static_cast<__nv_bfloat16*>(xs));
 }
 
 cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_of,
@@ -155,15 +156,14 @@ cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_o
   const int n = (dtype == 0) ? 4 : 8;  // elements per 16-byte chunk
   const int segs = static_cast<int>((H / n + 32 * kG - 1) / (32 * kG));
   const int64_t blocks = (T * segs + kWarps - 1) / kWarps;
+  const dim3 grid(static_cast<unsigned>(blocks));
   if (dtype == 0)
-    combine_kernel<float><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
-        static_cast<const float*>(y_slots), slot_of, topk_w, static_cast<float*>(out), T, H, k,
-        segs);
-  else
-    combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(y_slots), slot_of, topk_w,
-        static_cast<__nv_bfloat16*>(out), T, H, k, segs);
-  return cudaGetLastError();
+    return launch_kernel(combine_kernel<float>, grid, dim3(kThreads), 0, stream, 1,
+                         static_cast<const float*>(y_slots), slot_of, topk_w,
+                         static_cast<float*>(out), T, H, k, segs);
+  return launch_kernel(combine_kernel<__nv_bfloat16>, grid, dim3(kThreads), 0, stream, 1,
+                       static_cast<const __nv_bfloat16*>(y_slots), slot_of, topk_w,
+                       static_cast<__nv_bfloat16*>(out), T, H, k, segs);
 }
 
 }  // namespace moe

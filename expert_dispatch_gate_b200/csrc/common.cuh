@@ -41,6 +41,22 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Every kernel of the library is launched with programmatic stream serialization (see
+// launch_kernel): it may be scheduled while the kernel before it in the stream is still
+// running, and on entry it waits until every kernel it depends on has completed and their
+// writes are visible. Nothing before this call may touch global memory that another kernel
+// writes or reads. With early_trigger the kernel also lets the next kernel be scheduled right
+// away (used by the persistent GEMMs, whose successor's CTAs then take over SMs one by one as
+// the GEMM's CTAs finish); otherwise the successor is scheduled once every CTA has exited,
+// which measured faster for chains of short kernels.
+template <bool early_trigger>
+__device__ __forceinline__ void pdl_enter() {
+  if constexpr (early_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -352,6 +368,43 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
   return m;
+}
+
+// ------------------------------------------------------------------ host: kernel launch
+
+#ifdef MOE_NO_PDL
+constexpr bool kUsePdl = false;
+#else
+constexpr bool kUsePdl = true;  // programmatic dependent launch between the library's kernels
+#endif
+
+// cudaLaunchKernelEx with programmatic stream serialization (unless built with MOE_NO_PDL) and,
+// when cluster_x > 1, clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t stream, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (kUsePdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
 }
 
 }  // namespace moe

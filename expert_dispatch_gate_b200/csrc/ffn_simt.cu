@@ -29,6 +29,7 @@ __global__ void __launch_bounds__(kThreads)
                       const int32_t* __restrict__ offsets, const float* __restrict__ wg,
                       const float* __restrict__ wu, float* __restrict__ hbuf, int H, int E, int k,
                       int I) {
+  pdl_enter<false>();
   extern __shared__ float xs[];
   const int s = blockIdx.x;
   if (s >= offsets[E]) return;  // uniform across the block
@@ -51,6 +52,7 @@ __global__ void __launch_bounds__(kThreads)
 __global__ void __launch_bounds__(kThreads)
     gemm2_simt_kernel(const float* __restrict__ hbuf, const int32_t* __restrict__ offsets,
                       const float* __restrict__ wd, float* __restrict__ y, int H, int E, int I) {
+  pdl_enter<false>();
   extern __shared__ float hs[];
   const int s = blockIdx.x;
   if (s >= offsets[E]) return;
@@ -79,9 +81,8 @@ cudaError_t launch_gemm1_simt(const float* x, const int32_t* sorted_ids, const i
     if (e != cudaSuccess) return e;
   }
   dim3 grid(static_cast<unsigned>(A), static_cast<unsigned>((I + kThreads - 1) / kThreads));
-  gemm1_simt_kernel<<<grid, kThreads, smem, stream>>>(x, sorted_ids, offsets, w_gate, w_up, hbuf,
-                                                      H, E, k, I);
-  return cudaGetLastError();
+  return launch_kernel(gemm1_simt_kernel, grid, dim3(kThreads), smem, stream, 1, x, sorted_ids,
+                       offsets, w_gate, w_up, hbuf, H, E, k, I);
 }
 
 cudaError_t launch_gemm2_simt(const float* hbuf, const int32_t* offsets, const float* w_down,
@@ -95,8 +96,8 @@ cudaError_t launch_gemm2_simt(const float* hbuf, const int32_t* offsets, const f
     if (e != cudaSuccess) return e;
   }
   dim3 grid(static_cast<unsigned>(A), static_cast<unsigned>((H + kThreads - 1) / kThreads));
-  gemm2_simt_kernel<<<grid, kThreads, smem, stream>>>(hbuf, offsets, w_down, y, H, E, I);
-  return cudaGetLastError();
+  return launch_kernel(gemm2_simt_kernel, grid, dim3(kThreads), smem, stream, 1, hbuf, offsets,
+                       w_down, y, H, E, I);
 }
 
 }  // namespace moe

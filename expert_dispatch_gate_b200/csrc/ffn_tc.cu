@@ -191,17 +191,6 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const bool leader = (rank == 0);
 
-  if (p.offsets != nullptr) {
-    for (int i = threadIdx.x; i <= groups; i += blockDim.x) {
-      s_off[i] = p.offsets[i];
-      s_blk[i] = p.blk_prefix[i];
-    }
-  } else if (threadIdx.x == 0) {
-    s_off[0] = 0;
-    s_off[1] = p.n_static;
-    s_blk[0] = 0;
-    s_blk[1] = (p.n_static + p.TB - 1) / p.TB;
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(&full[s]), kFullCount);
@@ -223,6 +212,20 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
       tmem_alloc(smem_u32(tmem_holder), kTmemCols);
       tmem_relinquish();
     }
+  }
+  // Barriers and TMEM are set up while the previous kernel may still be finishing; the group
+  // tables (written by the grouping kernels) are read only after the dependency wait.
+  pdl_enter<true>();
+  if (p.offsets != nullptr) {
+    for (int i = threadIdx.x; i <= groups; i += blockDim.x) {
+      s_off[i] = p.offsets[i];
+      s_blk[i] = p.blk_prefix[i];
+    }
+  } else if (threadIdx.x == 0) {
+    s_off[0] = 0;
+    s_off[1] = p.n_static;
+    s_blk[0] = 0;
+    s_blk[1] = (p.n_static + p.TB - 1) / p.TB;
   }
   tc_fence_before();
   __syncthreads();
@@ -731,25 +734,8 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  if constexpr (PAIR) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-    cfg.blockDim = dim3(threads_of<BMODE>(), 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kernel, a0, a1, b, p);
-    if (e != cudaSuccess) return e;
-  } else {
-    kernel<<<static_cast<unsigned>(grid), threads_of<BMODE>(), smem, stream>>>(a0, a1, b, p);
-  }
-  return cudaGetLastError();
+  return launch_kernel(kernel, dim3(static_cast<unsigned>(grid)), dim3(threads_of<BMODE>()), smem,
+                       stream, PAIR ? 2 : 1, a0, a1, b, p);
 }
 
 // CTA pairs (cta_group::2) for the expert GEMMs unless the build opts out.

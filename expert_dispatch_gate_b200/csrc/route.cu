@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     topk_kernel(const float* __restrict__ partials, int ksplit, int64_t split_stride,
                 const float* __restrict__ bias, float* __restrict__ logits_out, int64_t T, int E,
                 int k, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  pdl_enter<false>();
   const int lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -160,6 +161,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                       const float* __restrict__ bias, int64_t T, int H, int E, int k,
                       float* __restrict__ logits_out, int32_t* __restrict__ topk_idx,
                       float* __restrict__ topk_w) {
+  pdl_enter<false>();
   constexpr int VN = Vec16<Tin>::N;
   const int lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -227,29 +229,25 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 }
 
 template <typename Tin, int EMAX>
-void route_simt_launch(const Tin* x, const Tin* wr, const float* bias, int64_t T, int H, int E,
+cudaError_t route_simt_launch(const Tin* x, const Tin* wr, const float* bias, int64_t T, int H, int E,
                        int k, float* logits_out, int32_t* idx, float* w, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
   const unsigned block = kWarpsPerBlock * 32;
   if ((E * sizeof(Tin)) % 16 == 0)
-    route_simt_kernel<Tin, EMAX, true><<<grid, block, 0, st>>>(x, wr, bias, T, H, E, k, logits_out, idx, w);
-  else
-    route_simt_kernel<Tin, EMAX, false><<<grid, block, 0, st>>>(x, wr, bias, T, H, E, k, logits_out, idx, w);
+    return launch_kernel(route_simt_kernel<Tin, EMAX, true>, dim3(grid), dim3(block), 0, st, 1, x,
+                         wr, bias, T, H, E, k, logits_out, idx, w);
+  return launch_kernel(route_simt_kernel<Tin, EMAX, false>, dim3(grid), dim3(block), 0, st, 1, x,
+                       wr, bias, T, H, E, k, logits_out, idx, w);
 }
 
 template <typename Tin>
 cudaError_t route_simt_dispatch(const Tin* x, const Tin* wr, const float* bias, int64_t T, int H,
                                 int E, int k, float* logits_out, int32_t* idx, float* w,
                                 cudaStream_t st) {
-  if (E <= 8)
-    route_simt_launch<Tin, 8>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
-  else if (E <= 16)
-    route_simt_launch<Tin, 16>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
-  else if (E <= 32)
-    route_simt_launch<Tin, 32>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
-  else
-    route_simt_launch<Tin, 64>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
-  return cudaGetLastError();
+  if (E <= 8) return route_simt_launch<Tin, 8>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
+  if (E <= 16) return route_simt_launch<Tin, 16>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
+  if (E <= 32) return route_simt_launch<Tin, 32>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
+  return route_simt_launch<Tin, 64>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
 }
 
 }  // namespace
@@ -273,15 +271,12 @@ cudaError_t launch_topk(const float* partials, int ksplit, int64_t split_stride,
   if (T == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
   const unsigned block = kWarpsPerBlock * 32;
-  if (E <= 32)
-    topk_kernel<1><<<grid, block, 0, stream>>>(partials, ksplit, split_stride, bias, logits_out, T, E, k, topk_idx, topk_w);
-  else if (E <= 64)
-    topk_kernel<2><<<grid, block, 0, stream>>>(partials, ksplit, split_stride, bias, logits_out, T, E, k, topk_idx, topk_w);
-  else if (E <= 128)
-    topk_kernel<4><<<grid, block, 0, stream>>>(partials, ksplit, split_stride, bias, logits_out, T, E, k, topk_idx, topk_w);
-  else
-    topk_kernel<8><<<grid, block, 0, stream>>>(partials, ksplit, split_stride, bias, logits_out, T, E, k, topk_idx, topk_w);
-  return cudaGetLastError();
+  auto kernel = topk_kernel<8>;
+  if (E <= 32) kernel = topk_kernel<1>;
+  else if (E <= 64) kernel = topk_kernel<2>;
+  else if (E <= 128) kernel = topk_kernel<4>;
+  return launch_kernel(kernel, dim3(grid), dim3(block), 0, stream, 1, partials, ksplit,
+                       split_stride, bias, logits_out, T, E, k, topk_idx, topk_w);
 }
 
 }  // namespace moe
