@@ -44,8 +44,7 @@ constexpr int kCtrlBytes = 2560;    // barriers + group tables
 //   kEpiBF16:   one A operand, 128 features; y stored as bf16.
 //   kEpiBF16x2: two A operands = features [m0, m0+128) and [m0+128, m0+256) of one weight; both
 //               accumulators share the B tile, halving B traffic per weight byte; bf16 out.
-//   kEpiF32:    one A operand, fp32 out plus an optional per-feature bias (router logits).
-enum EpiMode { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2, kEpiBF16x2 = 3 };
+enum EpiMode { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiBF16x2 = 3 };
 template <int MODE>
 constexpr bool dual_a() { return MODE == kEpiSwiGLU || MODE == kEpiBF16x2; }
 template <int MODE>
@@ -76,19 +75,15 @@ struct TcParams {
   int m_rows_a;   // extent of A along M (a 64-wide chunk starting past it is not loaded)
   int m_valid;    // features stored by the epilogue
   int TB;         // max tokens per tile, multiple of 32, <= 256
-  int groups;     // experts (ignored when offsets == nullptr)
+  int groups;     // experts
   int k_top;      // GEMM1: B row = sorted_ids[slot] / k_top
   int rows_b;     // rows of the B tensor
   const __nv_bfloat16* b_ptr;  // B tensor [rows_b, K] (cp.async gather)
   const int32_t* sorted_ids;
-  const int32_t* offsets;     // [groups+1] slot offsets, or nullptr: one group of n_static rows
+  const int32_t* offsets;     // [groups+1] slot offsets
   const int32_t* blk_prefix;  // [groups+1] token blocks before each group
-  int n_static;
-  int ksplit;            // K split into ksplit equal ranges (router only; partial sums)
-  int64_t split_stride;  // elements between the partial-sum slabs of consecutive K ranges
   void* out;
   int64_t ldo;
-  const float* bias;
   int* err;
   int stages;
   int nbuf;       // TMEM accumulator buffers (1 or 2, 256 columns apart)
@@ -97,15 +92,12 @@ struct TcParams {
 };
 
 struct Tile {
-  int group, fb, n, row0, ks, kb0, kb1;
+  int group, fb, n, row0, kb0, kb1;
 };
 
 // Tile order: K range fastest, then token block, then feature block, then group (expert).
 __device__ __forceinline__ Tile decode_tile(int tile, int num_fb, int groups, int TB,
-                                            const int* s_off, const int* s_blk, int ksplit,
-                                            int kblocks) {
-  const int ks = tile % ksplit;
-  tile /= ksplit;
+                                            const int* s_off, const int* s_blk, int kblocks) {
   int lo = 0, hi = groups;  // largest lo with num_fb * s_blk[lo] <= tile
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -123,10 +115,8 @@ __device__ __forceinline__ Tile decode_tile(int tile, int num_fb, int groups, in
   const int bs = (cnt + nb - 1) / nb;
   t.n = min(bs, cnt - b * bs);
   t.row0 = s_off[lo] + b * bs;
-  const int per = kblocks / ksplit;
-  t.ks = ks;
-  t.kb0 = ks * per;
-  t.kb1 = t.kb0 + per;
+  t.kb0 = 0;
+  t.kb1 = kblocks;
   return t;
 }
 
@@ -187,7 +177,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int groups = (p.offsets != nullptr) ? p.groups : 1;
+  const int groups = p.groups;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const bool leader = (rank == 0);
 
@@ -216,23 +206,16 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
   // Barriers and TMEM are set up while the previous kernel may still be finishing; the group
   // tables (written by the grouping kernels) are read only after the dependency wait.
   pdl_enter<true>();
-  if (p.offsets != nullptr) {
-    for (int i = threadIdx.x; i <= groups; i += blockDim.x) {
-      s_off[i] = p.offsets[i];
-      s_blk[i] = p.blk_prefix[i];
-    }
-  } else if (threadIdx.x == 0) {
-    s_off[0] = 0;
-    s_off[1] = p.n_static;
-    s_blk[0] = 0;
-    s_blk[1] = (p.n_static + p.TB - 1) / p.TB;
+  for (int i = threadIdx.x; i <= groups; i += blockDim.x) {
+    s_off[i] = p.offsets[i];
+    s_blk[i] = p.blk_prefix[i];
   }
   tc_fence_before();
   __syncthreads();
   if constexpr (PAIR) cluster_sync_all();  // barriers of both CTAs are initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int num_tiles = p.num_fb * s_blk[groups] * p.ksplit;
+  const int num_tiles = p.num_fb * s_blk[groups];
   const int kblocks = p.K / kBK;
   const int tile0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int tstep = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
@@ -245,7 +228,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
     int it = 0;
     bool ok = true;
     for (int tile = tile0; ok && tile < num_tiles; tile += tstep) {
-      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
+      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, kblocks);
       const int npad = (t.n + 15) & ~15;
       const int bn = b_rows(npad);
       const int nbox = p.a_wide ? 1 : (bn + kRowBox - 1) / kRowBox;
@@ -373,7 +356,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
       int tc = 0;
       bool ok = true;
       for (int tile = tile0; ok && tile < num_tiles; tile += tstep) {
-        const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
+        const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, kblocks);
         const int npad = (t.n + 15) & ~15;
         const int buf = tc % p.nbuf;
         const uint32_t use = static_cast<uint32_t>(tc / p.nbuf);
@@ -445,7 +428,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
     int it = 0;
     bool ok = true;
     for (int tile = tile0; ok && tile < num_tiles; tile += tstep) {
-      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
+      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, kblocks);
       const int npad = (t.n + 15) & ~15;
       const int bn = b_rows(npad);
       const int first = b_first(npad);
@@ -490,7 +473,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
     int tc = 0;
     bool ok = true;
     for (int tile = tile0; tile < num_tiles; tile += tstep) {
-      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, p.ksplit, kblocks);
+      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, kblocks);
       const int buf = tc % p.nbuf;
       const uint32_t use = static_cast<uint32_t>(tc / p.nbuf);
       int got = 1;
@@ -504,89 +487,67 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
       const int m = t.fb * kTileFeatures + static_cast<int>(rank) * kCtaFeatures + q * 32 + lane;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(buf * 256);
-      if constexpr (MODE == kEpiF32) {
-        // router partial logits: fp32 stores straight from TMEM (token blocks of <= 64 rows)
-        for (int c0 = 32 * half; c0 < t.n; c0 += 64) {
+      // Read every accumulator chunk this warp owns into registers, already rounded to bf16
+      // (two values per word), hand the TMEM buffer back to the MMA issuer, and only then
+      // write the rows out: the next tile's MMAs run under these stores.
+      constexpr int kW = (MODE == kEpiBF16x2) ? 32 : 16;  // words held per 32-column chunk
+      uint32_t pk[kEpiChunks][kW];
+#pragma unroll
+      for (int i = 0; i < kEpiChunks; ++i) {
+        const int c0 = 32 * half + 64 * i;
+        if (c0 < t.n) {
           uint32_t v[32];
           tmem_ld32(tb + static_cast<uint32_t>(c0), v);
-          tmem_wait_ld();
-          const int cmax = min(32, t.n - c0);
-          if (m < p.m_valid) {
-            float* o = reinterpret_cast<float*>(p.out) + t.ks * p.split_stride +
-                       static_cast<size_t>(t.row0 + c0) * p.ldo + m;
+          if constexpr (kSwiGLU) {
+            uint32_t u[32];
+            tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), u);
+            tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < cmax) o[static_cast<size_t>(j) * p.ldo] = __uint_as_float(v[j]);
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
-          else mbar_arrive(smem_u32(&tempty[buf]));
-        }
-      } else {
-        // Read every accumulator chunk this warp owns into registers, already rounded to bf16
-        // (two values per word), hand the TMEM buffer back to the MMA issuer, and only then
-        // write the rows out: the next tile's MMAs run under these stores.
-        constexpr int kW = (MODE == kEpiBF16x2) ? 32 : 16;  // words held per 32-column chunk
-        uint32_t pk[kEpiChunks][kW];
+            for (int j = 0; j < 16; ++j)
+              pk[i][j] = pack_bf16x2(
+                  silu_f32(__uint_as_float(v[2 * j])) * __uint_as_float(u[2 * j]),
+                  silu_f32(__uint_as_float(v[2 * j + 1])) * __uint_as_float(u[2 * j + 1]));
+          } else {
+            tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < kEpiChunks; ++i) {
-          const int c0 = 32 * half + 64 * i;
-          if (c0 < t.n) {
-            uint32_t v[32];
-            tmem_ld32(tb + static_cast<uint32_t>(c0), v);
-            if constexpr (kSwiGLU) {
-              uint32_t u[32];
-              tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), u);
+            for (int j = 0; j < 16; ++j)
+              pk[i][j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+            if constexpr (kDual) {
+              tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), v);
               tmem_wait_ld();
 #pragma unroll
               for (int j = 0; j < 16; ++j)
-                pk[i][j] = pack_bf16x2(
-                    silu_f32(__uint_as_float(v[2 * j])) * __uint_as_float(u[2 * j]),
-                    silu_f32(__uint_as_float(v[2 * j + 1])) * __uint_as_float(u[2 * j + 1]));
-            } else {
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 16; ++j)
-                pk[i][j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-              if constexpr (kDual) {
-                tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                  pk[i][16 + j] =
-                      pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-              }
+                pk[i][16 + j] =
+                    pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
-          else mbar_arrive(smem_u32(&tempty[buf]));
-        }
-        // The last tile of a CTA pair may reach past the weight's feature extent (the second
-        // CTA's rows were loaded as zeros): those feature rows have no output.
-        const bool keep0 = m < p.m_valid;
-        const bool keep1 = (MODE == kEpiBF16x2) && (m + 128 < p.m_valid);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
+        else mbar_arrive(smem_u32(&tempty[buf]));
+      }
+      // The last tile of a CTA pair may reach past the weight's feature extent (the second
+      // CTA's rows were loaded as zeros): those feature rows have no output.
+      const bool keep0 = m < p.m_valid;
+      const bool keep1 = (MODE == kEpiBF16x2) && (m + 128 < p.m_valid);
 #pragma unroll
-        for (int i = 0; i < kEpiChunks; ++i) {
-          const int c0 = 32 * half + 64 * i;
-          if (c0 < t.n && keep0) {
-            const int cmax = min(32, t.n - c0);
-            uint16_t* o = reinterpret_cast<uint16_t*>(p.out) +
-                          static_cast<size_t>(t.row0 + c0) * p.ldo + m;
+      for (int i = 0; i < kEpiChunks; ++i) {
+        const int c0 = 32 * half + 64 * i;
+        if (c0 < t.n && keep0) {
+          const int cmax = min(32, t.n - c0);
+          uint16_t* o = reinterpret_cast<uint16_t*>(p.out) +
+                        static_cast<size_t>(t.row0 + c0) * p.ldo + m;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j < cmax) {
-                o[static_cast<size_t>(j) * p.ldo] = bf16_half(pk[i][j >> 1], j & 1);
-                if constexpr (MODE == kEpiBF16x2)
-                  if (keep1)
-                    o[static_cast<size_t>(j) * p.ldo + 128] = bf16_half(pk[i][16 + (j >> 1)], j & 1);
-              }
+          for (int j = 0; j < 32; ++j) {
+            if (j < cmax) {
+              o[static_cast<size_t>(j) * p.ldo] = bf16_half(pk[i][j >> 1], j & 1);
+              if constexpr (MODE == kEpiBF16x2)
+                if (keep1)
+                  o[static_cast<size_t>(j) * p.ldo + 128] =
+                      bf16_half(pk[i][16 + (j >> 1)], j & 1);
             }
           }
         }
@@ -750,50 +711,6 @@ constexpr bool kUsePairs =
 
 bool gemm1_uses_row_copy(int /*I*/) { return kUsePairs; }
 
-int route_token_block(int64_t T) { return T >= 64 ? 64 : static_cast<int>(((T + 31) / 32) * 32); }
-
-int route_ksplit(int64_t T, int H, int E) {
-  const int64_t kb_total = H / kBK;
-  const int64_t base = ((E + kBM - 1) / kBM) * ((T + route_token_block(T) - 1) / route_token_block(T));
-  int ks = 1;
-  // at most 8 ranges: the top-k kernel sums the partials of a token in one warp
-  while (ks * 2 <= 8 && ks * 2 <= kb_total && kb_total % (ks * 2) == 0 && base * ks * 2 <= 128)
-    ks *= 2;
-  return ks;
-}
-
-cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int H, int E,
-                                 float* partials, int ksplit, int* err, int num_sms,
-                                 cudaStream_t stream, std::string* detail) {
-  CUtensorMap a0, b;
-  if (!map_weights(&a0, w_router, static_cast<uint64_t>(E), static_cast<uint64_t>(H), 1, detail) ||
-      !map_row_boxes(&b, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), detail))
-    return cudaErrorInvalidValue;
-  TcParams p{};
-  p.K = H;
-  p.num_fb = (E + kBM - 1) / kBM;
-  p.m_rows_a = E;
-  p.m_valid = E;
-  p.TB = route_token_block(T);
-  p.groups = 1;
-  p.k_top = 1;
-  p.rows_b = T;
-  p.sorted_ids = nullptr;
-  p.offsets = nullptr;
-  p.blk_prefix = nullptr;
-  p.n_static = T;
-  p.ksplit = ksplit;
-  p.split_stride = static_cast<int64_t>(T) * E;
-  p.out = partials;
-  p.ldo = E;
-  p.bias = nullptr;
-  p.err = err;
-  p.a_wide = 0;
-  p.b_box_rows = kRowBox;
-  const int64_t tiles = static_cast<int64_t>(p.num_fb) * ((T + p.TB - 1) / p.TB) * ksplit;
-  return launch_mode<kEpiF32, kBTiled, false>(a0, a0, b, p, tiles, num_sms, stream, detail);
-}
-
 cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t* sorted_ids,
                             const int32_t* offsets, const int32_t* blk_prefix, const void* w_gate,
                             const void* w_up, void* hbuf, int64_t hbuf_rows, int H, int E, int k,
@@ -830,10 +747,8 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
     p.blk_prefix = blk_prefix;
     p.out = hbuf;
     p.ldo = I;
-    p.bias = nullptr;
     p.err = err;
     p.b_ptr = nullptr;
-    p.ksplit = 1;
     const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
     if (pair)
       return launch_mode<kEpiSwiGLU, kBTiled, true>(a0, a1, b, p, tiles, num_sms, stream, detail);
@@ -862,10 +777,8 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
   p.blk_prefix = blk_prefix;
   p.out = hbuf;
   p.ldo = I;
-  p.bias = nullptr;
   p.err = err;
   p.b_ptr = static_cast<const __nv_bfloat16*>(x);
-  p.ksplit = 1;
   const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
   if (use_gather4)
     return launch_mode<kEpiSwiGLU, kBGather4, false>(a0, a1, b, p, tiles, num_sms, stream, detail);
@@ -888,7 +801,6 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
   TcParams p{};
   p.a_wide = 1;
   p.b_box_rows = box_rows;
-  p.ksplit = 1;
   p.K = I;
   p.num_fb = pair ? (H + 511) / 512 : (dual ? H / 256 : H / kBM);
   p.m_rows_a = H;
@@ -902,7 +814,6 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
   p.blk_prefix = blk_prefix;
   p.out = y;
   p.ldo = H;
-  p.bias = nullptr;
   p.err = err;
   const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
   if (pair)

@@ -21,17 +21,19 @@ cudaError_t launch_topk(const float* partials, int ksplit, int64_t split_stride,
                         const float* bias, float* logits_out, int64_t T, int E, int k,
                         int32_t* topk_idx, float* topk_w, cudaStream_t stream);
 
-// ---- ffn_tc.cu (tcgen05 / TMEM / TMA, bf16)
-// Gate logits on the tensor cores (swap-AB: experts on MMA M), K split into `ksplit` ranges:
+// ---- route_tc.cu (tcgen05 / TMEM / TMA, bf16)
+// Gate logits on the tensor cores (tokens on the MMA's M side, experts on N, E in [16, 256],
+// E % 8 == 0), K split into `ksplit` ranges:
 // partials[ks][t][e] = sum over h in range ks of x[t,h] * w_router[h,e].
-int route_token_block(int64_t T);
 int route_ksplit(int64_t T, int H, int E);
 cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int H, int E,
                                  float* partials, int ksplit, int* err, int num_sms,
                                  cudaStream_t stream, std::string* detail);
+
+// ---- ffn_tc.cu (tcgen05 / TMEM / TMA, bf16)
 // Expert GEMM1: h[s, :] = silu(x[t] Wg[e]) * (x[t] Wu[e]) for kept slots; h rows = hbuf_rows.
 // With xs != nullptr the token rows come from the expert-major copy xs (contiguous per expert,
-// streamed by TMA, CTA pairs when I % 256 == 0); otherwise they are gathered from x through
+// streamed by TMA, CTA pairs); otherwise they are gathered from x through
 // sorted_ids by cp.async (single CTAs).
 bool gemm1_uses_row_copy(int I);
 cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t* sorted_ids,

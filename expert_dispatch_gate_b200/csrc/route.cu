@@ -62,8 +62,19 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   for (int i = 0; i < VPL; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
-      float acc = partials[t * E + e];
-      for (int ks = 1; ks < ksplit; ++ks) acc += partials[ks * split_stride + t * E + e];
+      // partial sums in ascending K-range order; loads issued four at a time
+      const float* src = partials + t * E + e;
+      float acc = src[0];
+      int ks = 1;
+      for (; ks + 4 <= ksplit; ks += 4) {
+        const float a0 = src[(ks + 0) * split_stride], a1 = src[(ks + 1) * split_stride];
+        const float a2 = src[(ks + 2) * split_stride], a3 = src[(ks + 3) * split_stride];
+        acc += a0;
+        acc += a1;
+        acc += a2;
+        acc += a3;
+      }
+      for (; ks < ksplit; ++ks) acc += src[ks * split_stride];
       if (bias != nullptr) acc += bias[e];
       v[i] = acc;
       if (logits_out != nullptr) logits_out[t * E + e] = acc;
