@@ -12,38 +12,12 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "select.cuh"
 
 namespace moe {
 namespace {
 
 constexpr int kWarpsPerBlock = 8;
-
-// Winner of (value desc, index asc) across the warp; every lane ends with the same pair.
-__device__ __forceinline__ void warp_argmax(float& bv, int& bi) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-    if (ov > bv || (ov == bv && oi < bi)) {
-      bv = ov;
-      bi = oi;
-    }
-  }
-}
-
-// Lane j < k holds the j-th selected (value, index); `top` is the largest logit. Writes
-// topk_idx and the weights exp(l_j - top) / sum_i exp(l_i - top).
-__device__ __forceinline__ void write_selection(int lane, int k, float my_v, int my_i, float top,
-                                                int32_t* idx_row, float* w_row) {
-  const float ex = (lane < k) ? expf(my_v - top) : 0.0f;
-  float s = ex;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane < k) {
-    idx_row[lane] = my_i;
-    w_row[lane] = ex / s;
-  }
-}
 
 // Logits distributed over lanes: lane holds experts lane, lane+32, ... (VPL per lane). Each
 // logit is the sum of the K-range partials in ascending order plus the optional bias.
@@ -83,28 +57,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
       taken |= 1u << i;
     }
   }
-  float my_v = 0.f, top = 0.f;
-  int my_i = 0;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int e = lane + 32 * i;
-      if (!((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < bi))) {
-        bv = v[i];
-        bi = e;
-      }
-    }
-    warp_argmax(bv, bi);
-    if ((bi & 31) == lane) taken |= 1u << ((bi >> 5) & 31);
-    if (lane == j) {
-      my_v = bv;
-      my_i = bi;
-    }
-    if (j == 0) top = bv;
-  }
-  write_selection(lane, k, my_v, my_i, top, topk_idx + t * k, topk_w + t * k);
+  warp_select_topk<VPL>(v, taken, k, lane, topk_idx + t * k, topk_w + t * k);
 }
 
 template <typename Tin>

@@ -27,6 +27,12 @@ SMALL = {
     "e16_nocap": W.Workload("e16n", 14, 97, 256, 16, 4, 256, "bf16", 0.0),
     "dense_e1": W.Workload("e1", 15, 130, 128, 1, 1, 128, "bf16", 1.25),
     "e64_k16_f32": W.Workload("e64f", 16, 77, 64, 64, 16, 96, "f32", 1.0),
+    # E = 96: the router's second 64-expert chunk is half zero-filled (N = 96, two
+    # accumulators); I = 640 leaves the last GEMM1 pair tile half outside the weight; H = 384
+    # runs GEMM2 with one feature block per tile
+    "e96_partial_tiles": W.Workload("e96", 17, 333, 384, 96, 4, 640, "bf16", 1.25),
+    # T = 50, H = 1024: one token tile, the router's K split into 4 ranges
+    "e128_router_ksplit": W.Workload("e128", 18, 50, 1024, 128, 6, 256, "bf16", 1.25),
 }
 
 
