@@ -23,7 +23,10 @@ Sources, cited by page title and section:
     C are dropped and take the residual path (contribute nothing to the MoE output).
 * [P5] "大模型推理加速200%+？这套国产融合算子库把CUDA/Triton全替换了" (csdn.net)
   - section "3.1 Moe Fuse Gate & Softmax TopK": exp only over the selected k, which equals the
-    renormalised full softmax in exact arithmetic.
+    renormalised full softmax in exact arithmetic; the gate selects expert groups first
+    ("优先选组") and keeps each group's top-1 / top-2.
+  - section "3.2 Fuse RMS RoPE & MoE Align & MoE Sum": the MoE sum also adds the shared expert's
+    output with a factor, and a bias.
 
 Readings taken where the pages are silent or disagree (each also listed in the design notes):
 
@@ -35,6 +38,14 @@ Readings taken where the pages are silent or disagree (each also listed in the d
 * Top-k ranks float32 logits (softmax is monotone); equal logits (including -0 vs +0) go to the
   lower expert index; the k indices are listed by descending logit, then ascending index.
 * SwiGLU expert: y = (silu(x Wg) * (x Wu)) Wd, silu(z) = z / (1 + exp(-z)); experts have no bias.
+* Group-limited routing (the pages name it, give no formula): the E experts form n_group equal
+  contiguous groups; a group's score is the float32 sum of its two largest logits (its only
+  logit when a group holds one expert); the topk_group groups with the highest scores are kept
+  (ties to the lower group index); the k largest logits among the kept groups' experts are
+  selected with the plain top-k rule; weights are renormalised over the k as before.
+* Shared expert and bias in the combine: out[t] = sum_j w[t,j] y[slot] + factor * shared[t] + b,
+  with shared[t] the shared expert's output row (computed by the caller) and b a per-feature
+  bias; both terms apply to every token, including a fully dropped one.
 
 Every function below is pinned by tests that do not re-run its own formula (brute force,
 closed forms, hand-worked fixtures under tests/golden, special cases reducing to a dense FFN).
@@ -49,8 +60,11 @@ import numpy as np
 __all__ = [
     "router_logits",
     "select_topk",
+    "group_scores",
+    "select_topk_grouped",
     "route_weights",
     "route",
+    "route_grouped",
     "capacity",
     "align",
     "swiglu_expert",
@@ -107,6 +121,59 @@ def route(x, w_router, k, logit_bias=None, logits=None):
     if logits is None:
         logits = router_logits(x, w_router, logit_bias)
     idx = select_topk(logits, k)
+    return np.asarray(logits, dtype=np.float32), idx, route_weights(logits, idx)
+
+
+def group_scores(logits, n_group):
+    """Score of each expert group per row: the float32 sum of the group's two largest float32
+    logits (the single logit when a group holds one expert). Shape [T, n_group], float32.
+
+    [P5] "3.1 Moe Fuse Gate & Softmax TopK" (select groups first, keep each group's top-1 and
+    top-2). The sum is one float32 addition, the same rounding the kernel performs.
+    """
+    l32 = np.asarray(logits, dtype=np.float32)
+    T, E = l32.shape
+    if n_group < 1 or E % n_group != 0:
+        raise ValueError("n_group must divide E")
+    gs = E // n_group
+    g = np.sort(l32.reshape(T, n_group, gs), axis=2)[:, :, ::-1]
+    if gs == 1:
+        return g[:, :, 0].astype(np.float32)
+    return (g[:, :, 0] + g[:, :, 1]).astype(np.float32)
+
+
+def select_topk_grouped(logits, k, n_group, topk_group):
+    """Group-limited top-k: keep the topk_group best-scoring groups (scores from group_scores,
+    ties to the lower group index), then the k largest logits among their experts, ordered and
+    tie-broken exactly as select_topk.
+
+    [P5] "3.1 Moe Fuse Gate & Softmax TopK" ("优先选组"). With topk_group == n_group (or
+    n_group == 1) this is select_topk.
+    """
+    l32 = np.asarray(logits, dtype=np.float32)
+    T, E = l32.shape
+    if not (1 <= topk_group <= n_group):
+        raise ValueError("need 1 <= topk_group <= n_group")
+    gs = E // n_group
+    if k < 1 or k > topk_group * gs:
+        raise ValueError("need 1 <= k <= topk_group * (E / n_group)")
+    sc = group_scores(l32, n_group)
+    gorder = np.argsort(-sc, axis=1, kind="stable")[:, :topk_group]
+    keep = np.zeros((T, n_group), dtype=bool)
+    np.put_along_axis(keep, gorder, True, axis=1)
+    order = np.argsort(-l32, axis=1, kind="stable")
+    out = np.empty((T, k), dtype=np.int32)
+    for t in range(T):
+        cand = [int(e) for e in order[t] if keep[t, int(e) // gs]]
+        out[t] = cand[:k]
+    return out
+
+
+def route_grouped(x, w_router, k, n_group, topk_group, logit_bias=None, logits=None):
+    """Router step with group-limited selection: (logits f32, topk_idx i32, topk_w f64)."""
+    if logits is None:
+        logits = router_logits(x, w_router, logit_bias)
+    idx = select_topk_grouped(logits, k, n_group, topk_group)
     return np.asarray(logits, dtype=np.float32), idx, route_weights(logits, idx)
 
 
@@ -219,12 +286,16 @@ def grouped_ffn_slots(x, sorted_ids, offsets, k, w_gate, w_up, w_down, slots=Non
     return out
 
 
-def combine(y_slots, slot_of, topk_w, tokens=None):
-    """Weighted merge back to token order: out[t] = sum_{kept j} w[t,j] * y[slot_of[t*k+j]].
+def combine(y_slots, slot_of, topk_w, tokens=None, shared=None, shared_factor=0.0,
+            out_bias=None):
+    """Weighted merge back to token order: out[t] = sum_{kept j} w[t,j] * y[slot_of[t*k+j]]
+    (+ shared_factor * shared[t] + out_bias when given).
 
-    [P1] "融合二：expert 计算的输出 + 合并结果" (accum += route_weight * expert_output).
-    A dropped assignment (slot -1) contributes nothing; a fully dropped token gives 0.
-    ``y_slots`` may be an array or a dict slot -> row.
+    [P1] "融合二：expert 计算的输出 + 合并结果" (accum += route_weight * expert_output);
+    [P5] "3.2 ... MoE Sum" (shared expert factor and bias added in the sum).
+    A dropped assignment (slot -1) contributes nothing; a fully dropped token gives 0 plus the
+    shared and bias terms. ``y_slots`` may be an array or a dict slot -> row; ``shared`` is
+    indexed by token.
     """
     w = np.asarray(topk_w, dtype=np.float64)
     T, k = w.shape
@@ -244,25 +315,40 @@ def combine(y_slots, slot_of, topk_w, tokens=None):
         rows[t] = acc
     if H is None:
         H = np.asarray(y_slots[0]).shape[-1] if len(y_slots) else 0
+    if H is None and shared is not None:
+        H = np.asarray(shared).shape[-1]
+    if H is None and out_bias is not None:
+        H = np.asarray(out_bias).shape[-1]
     out = np.zeros((len(rows), H), dtype=np.float64)
     for i, t in enumerate(toks):
         if rows[t] is not None:
             out[i] = rows[t]
+        if shared is not None:
+            out[i] += float(shared_factor) * np.asarray(shared[t], dtype=np.float64)
+        if out_bias is not None:
+            out[i] += np.asarray(out_bias, dtype=np.float64)
     return out
 
 
 def layer_forward(x, w_router, w_gate, w_up, w_down, k, capacity_factor,
-                  logit_bias=None, logits=None, tokens=None):
+                  logit_bias=None, logits=None, tokens=None, n_group=1, topk_group=1,
+                  shared=None, shared_factor=0.0, out_bias=None):
     """Whole MoE layer: route -> align -> experts -> combine, float64 throughout.
 
     [P1] "FlashAttention 在 MoE 模型里的位置" steps 2-5. ``logits`` (float32) may be supplied
     to route from given gate logits. ``tokens`` restricts the expert FFN and the combine to a
     subset of tokens (routing and capacity still see every token, since ranks depend on all).
+    ``n_group``/``topk_group`` select group-limited routing; ``shared``/``shared_factor``/
+    ``out_bias`` add the shared-expert and bias terms of the combine.
     Returns dict with out [len(tokens) or T, H] and all routing intermediates.
     """
     x = np.asarray(x)
     T = x.shape[0]
-    logits, idx, w = route(x, w_router, k, logit_bias=logit_bias, logits=logits)
+    if n_group > 1:
+        logits, idx, w = route_grouped(x, w_router, k, n_group, topk_group,
+                                       logit_bias=logit_bias, logits=logits)
+    else:
+        logits, idx, w = route(x, w_router, k, logit_bias=logit_bias, logits=logits)
     E = logits.shape[1]
     C = capacity(T, k, E, capacity_factor)
     al = align(idx, E, C)
@@ -275,7 +361,8 @@ def layer_forward(x, w_router, w_gate, w_up, w_down, k, capacity_factor,
                 need.add(s)
     y = grouped_ffn_slots(x, al["sorted_ids"], al["offsets"], k, w_gate, w_up, w_down,
                           slots=sorted(need))
-    out = combine(y, al["slot_of"], w, tokens=tok_list)
+    out = combine(y, al["slot_of"], w, tokens=tok_list, shared=shared,
+                  shared_factor=shared_factor, out_bias=out_bias)
     res = dict(al)
     res.update({"logits": logits, "topk_idx": idx, "topk_w": w, "C": C, "out": out,
                 "tokens": tok_list})

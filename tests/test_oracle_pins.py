@@ -306,3 +306,92 @@ def test_page_sizes(golden_dir):
     assert (fine.T, fine.k, fine.H, fine.E) == (d["T"], d["k"], d["H"], r["E"])
     mix = wlm.WORKLOADS["mixtral"]
     assert (mix.E, mix.k) == (g["mixtral_active"]["E"], g["mixtral_active"]["k"])
+
+
+# ---------------------------------------------------------------- group-limited routing
+
+
+def test_grouped_topk_hand_worked(golden_dir):
+    for c in _load(golden_dir, "grouped_routing.json")["cases"]:
+        l = np.asarray([c["logits"]], dtype=np.float32)
+        got = orc.select_topk_grouped(l, c["k"], c["n_group"], c["topk_group"])
+        assert got[0].tolist() == c["expected"], c["note"]
+        assert orc.select_topk(l, c["k"])[0].tolist() == c["plain"], c["note"]
+
+
+def test_grouped_topk_reduces_to_plain():
+    rng = np.random.default_rng(5)
+    l = np.round(rng.standard_normal((200, 32)) * 2).astype(np.float32) / 2  # many ties
+    for k in (1, 3, 8):
+        plain = orc.select_topk(l, k)
+        assert np.array_equal(orc.select_topk_grouped(l, k, 1, 1), plain)
+        assert np.array_equal(orc.select_topk_grouped(l, k, 4, 4), plain)
+        assert np.array_equal(orc.select_topk_grouped(l, k, 32, 32), plain)
+
+
+def test_grouped_topk_order_invariants():
+    """Kept groups beat every other group under (score desc, index asc); the selection beats
+    every other candidate of the kept groups under (logit desc, index asc)."""
+    rng = np.random.default_rng(6)
+    E, G, g, k = 64, 8, 3, 6
+    gs = E // G
+    l = np.round(rng.standard_normal((300, E)) * 3).astype(np.float32) / 4
+    idx = orc.select_topk_grouped(l, k, G, g)
+    for t in range(l.shape[0]):
+        row = l[t]
+        # group scores by brute force: best pair sum over distinct members
+        sc = []
+        for gi in range(G):
+            m = row[gi * gs:(gi + 1) * gs]
+            sc.append(max(np.float32(m[a]) + np.float32(m[b])
+                          for a in range(gs) for b in range(gs) if a != b))
+        sel = [int(e) for e in idx[t]]
+        kept = {e // gs for e in sel}
+        assert len(kept) <= g
+        # the kept set is exactly the g best groups
+        best = sorted(range(G), key=lambda gi: (-sc[gi], gi))[:g]
+        assert kept <= set(best)
+        cand = [e for e in range(E) if e // gs in best]
+        for s in sel:
+            for c in cand:
+                if c not in sel:
+                    assert row[s] > row[c] or (row[s] == row[c] and s < c)
+        # listed by (logit desc, index asc)
+        for a, b in zip(sel, sel[1:]):
+            assert row[a] > row[b] or (row[a] == row[b] and a < b)
+
+
+def test_group_scores_single_member_groups_are_the_logits():
+    l = np.asarray([[0.5, -1.0, 2.0, 0.0]], dtype=np.float32)
+    assert np.array_equal(orc.group_scores(l, 4), l)
+
+
+# ---------------------------------------------------------------- shared expert + bias in the combine
+
+
+def test_combine_shared_and_bias_hand_worked():
+    # T=2, k=2, H=2; token 0 keeps both slots, token 1 is fully dropped
+    y = np.asarray([[1.0, 2.0], [3.0, -1.0]])
+    slot_of = np.asarray([0, 1, -1, -1])
+    w = np.asarray([[0.75, 0.25], [0.5, 0.5]])
+    shared = np.asarray([[4.0, 8.0], [-2.0, 6.0]])
+    bias = np.asarray([0.5, -0.5])
+    out = orc.combine(y, slot_of, w, shared=shared, shared_factor=0.5, out_bias=bias)
+    # token 0: 0.75*[1,2] + 0.25*[3,-1] = [1.5, 1.25]; + 0.5*[4,8] = [3.5, 5.25]; + bias
+    # token 1: dropped -> 0.5*[-2,6] + bias = [-0.5, 2.5]
+    assert np.array_equal(out, np.asarray([[4.0, 4.75], [-0.5, 2.5]]))
+
+
+def test_combine_shared_terms_are_additive():
+    rng = np.random.default_rng(7)
+    T, k, H = 9, 3, 16
+    y = rng.standard_normal((T * k, H))
+    slot_of = rng.permutation(T * k)
+    slot_of[::4] = -1
+    w = rng.random((T, k))
+    shared = rng.standard_normal((T, H))
+    bias = rng.standard_normal(H)
+    base = orc.combine(y, slot_of, w)
+    assert np.array_equal(orc.combine(y, slot_of, w, shared=shared, shared_factor=0.0), base)
+    with_terms = orc.combine(y, slot_of, w, shared=shared, shared_factor=1.5, out_bias=bias)
+    assert np.allclose(with_terms - base, 1.5 * shared + bias, rtol=0, atol=1e-12)
