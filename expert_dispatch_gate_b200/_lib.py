@@ -38,12 +38,24 @@ class MoeShape(ctypes.Structure):
     ]
 
 
+class MoeLayerOpts(ctypes.Structure):
+    """moe_layer_opts: group-limited routing and the combine's shared-expert / bias terms."""
+    _fields_ = [
+        ("n_group", ctypes.c_int32),
+        ("topk_group", ctypes.c_int32),
+        ("shared_out", ctypes.c_void_p),
+        ("shared_factor", ctypes.c_float),
+        ("out_bias", ctypes.c_void_p),
+    ]
+
+
 _lib = None
 _P = ctypes.c_void_p
 
 
 def _signatures(lib):
     S = ctypes.POINTER(MoeShape)
+    O = ctypes.POINTER(MoeLayerOpts)
     st = ctypes.c_int
     sz = ctypes.c_size_t
     table = {
@@ -60,6 +72,11 @@ def _signatures(lib):
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_last_error_detail": (ctypes.c_char_p, []),
         "moe_set_stage_events": (st, [ctypes.POINTER(_P), ctypes.c_int32]),
+        "moe_route_ex": (st, [S, O, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
+        "moe_route_from_logits_ex": (st, [S, O, _P, _P, _P, _P]),
+        "moe_combine_ex": (st, [S, O, _P, _P, _P, _P, _P]),
+        "moe_layer_forward_ex": (st, [S, O, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, sz,
+                                      _P]),
     }
     for name, (res, args) in table.items():
         f = getattr(lib, name)
@@ -185,6 +202,46 @@ def moe_layer_forward(shape, x, w_router, logit_bias, w_gate, w_up, w_down, out,
                                 ptr(w_gate), ptr(w_up), ptr(w_down), ptr(out), ptr(logits_out),
                                 ptr(topk_idx), ptr(topk_w), ptr(counts), ptr(drop_mask), ptr(ws),
                                 int(ws_bytes), _stream(stream))
+    return _check(s) if check else s
+
+
+def make_opts(n_group=1, topk_group=1, shared_out=None, shared_factor=0.0, out_bias=None):
+    """A moe_layer_opts; the tensors must stay alive while the call is in flight."""
+    return MoeLayerOpts(int(n_group), int(topk_group), ptr(shared_out), float(shared_factor),
+                        ptr(out_bias))
+
+
+def _opts(opts):
+    return None if opts is None else ctypes.byref(opts)
+
+
+def moe_route_ex(shape, opts, x, w_router, logit_bias, logits_out, topk_idx, topk_w, ws,
+                 ws_bytes, stream=None, check=True):
+    s = lib().moe_route_ex(ctypes.byref(shape), _opts(opts), ptr(x), ptr(w_router),
+                           ptr(logit_bias), ptr(logits_out), ptr(topk_idx), ptr(topk_w), ptr(ws),
+                           int(ws_bytes), _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_route_from_logits_ex(shape, opts, logits, topk_idx, topk_w, stream=None, check=True):
+    s = lib().moe_route_from_logits_ex(ctypes.byref(shape), _opts(opts), ptr(logits),
+                                       ptr(topk_idx), ptr(topk_w), _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_combine_ex(shape, opts, y_slots, slot_of, topk_w, out, stream=None, check=True):
+    s = lib().moe_combine_ex(ctypes.byref(shape), _opts(opts), ptr(y_slots), ptr(slot_of),
+                             ptr(topk_w), ptr(out), _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_layer_forward_ex(shape, opts, x, w_router, logit_bias, w_gate, w_up, w_down, out,
+                         logits_out, topk_idx, topk_w, counts, drop_mask, ws, ws_bytes,
+                         stream=None, check=True):
+    s = lib().moe_layer_forward_ex(ctypes.byref(shape), _opts(opts), ptr(x), ptr(w_router),
+                                   ptr(logit_bias), ptr(w_gate), ptr(w_up), ptr(w_down), ptr(out),
+                                   ptr(logits_out), ptr(topk_idx), ptr(topk_w), ptr(counts),
+                                   ptr(drop_mask), ptr(ws), int(ws_bytes), _stream(stream))
     return _check(s) if check else s
 
 

@@ -4,8 +4,10 @@
 // accum += route_weight * expert_output; [P5] "大模型推理加速200%+？…", section "3.2 Fuse RMS RoPE &
 // MoE Align & MoE Sum" (128-bit vector reads/writes).
 //
-// out[t,:] = sum over kept j of topk_w[t,j] * y_slots[slot_of[t*k+j],:], fp32 accumulation in
-// ascending j, rounded once.
+// out[t,:] = sum over kept j of topk_w[t,j] * y_slots[slot_of[t*k+j],:]
+//            (+ shared_factor * shared[t,:]) (+ out_bias[:]),
+// fp32 accumulation in ascending j, then the shared-expert term, then the bias, rounded once
+// ([P5] section 3.2: the MoE sum fuses the shared expert's factor and the bias add).
 #include "common.cuh"
 #include "internal.h"
 
@@ -59,8 +61,9 @@ constexpr int kG = 4;
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 2)
     combine_kernel(const T* __restrict__ y, const int32_t* __restrict__ slot_of,
-                   const float* __restrict__ topk_w, T* __restrict__ out, int64_t Ttok, int H,
-                   int k, int segs) {
+                   const float* __restrict__ topk_w, const T* __restrict__ shared,
+                   float shared_factor, const float* __restrict__ out_bias, T* __restrict__ out,
+                   int64_t Ttok, int H, int k, int segs) {
   pdl_enter<false>();
   constexpr int N = Vec<T>::N;
   const int lane = threadIdx.x & 31;
@@ -107,6 +110,29 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
     }
+    if (shared != nullptr) {
+      const T* srow = shared + static_cast<size_t>(t) * H;
+#pragma unroll
+      for (int g = 0; g < kG; ++g) {
+        const int c = c0 + 32 * g;
+        if (c < nchunk) {
+          float v[N];
+          Vec<T>::widen(__ldg(reinterpret_cast<const uint4*>(srow) + c), v);
+#pragma unroll
+          for (int i = 0; i < N; ++i) acc[g][i] = fmaf(shared_factor, v[i], acc[g][i]);
+        }
+      }
+    }
+    if (out_bias != nullptr) {
+#pragma unroll
+      for (int g = 0; g < kG; ++g) {
+        const int c = c0 + 32 * g;
+        if (c < nchunk) {
+#pragma unroll
+          for (int i = 0; i < N; ++i) acc[g][i] += __ldg(out_bias + static_cast<size_t>(c) * N + i);
+        }
+      }
+    }
 #pragma unroll
     for (int g = 0; g < kG; ++g) {
       const int c = c0 + 32 * g;
@@ -150,7 +176,8 @@ cudaError_t launch_dispatch_rows(int dtype, const void* x, const int32_t* sorted
 }
 
 cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_of,
-                           const float* topk_w, void* out, int64_t T, int H, int k,
+                           const float* topk_w, const void* shared, float shared_factor,
+                           const float* out_bias, void* out, int64_t T, int H, int k,
                            cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const int n = (dtype == 0) ? 4 : 8;  // elements per 16-byte chunk
@@ -160,9 +187,11 @@ cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_o
   if (dtype == 0)
     return launch_kernel(combine_kernel<float>, grid, dim3(kThreads), 0, stream, 1,
                          static_cast<const float*>(y_slots), slot_of, topk_w,
+                         static_cast<const float*>(shared), shared_factor, out_bias,
                          static_cast<float*>(out), T, H, k, segs);
   return launch_kernel(combine_kernel<__nv_bfloat16>, grid, dim3(kThreads), 0, stream, 1,
                        static_cast<const __nv_bfloat16*>(y_slots), slot_of, topk_w,
+                       static_cast<const __nv_bfloat16*>(shared), shared_factor, out_bias,
                        static_cast<__nv_bfloat16*>(out), T, H, k, segs);
 }
 

@@ -17,9 +17,11 @@ cudaError_t launch_route_simt(int dtype, const void* x, const void* w_router, co
 // Top-k + renormalise, one warp per token, E <= 256: logits[t,e] = sum over ks of
 // partials[ks * split_stride + t*E + e] (ascending ks) + bias[e] (bias optional); the logits
 // are written to logits_out when it is non-null.
+// With n_group > 1 the selection is group-limited (n_group <= 32 groups, topk_group kept).
 cudaError_t launch_topk(const float* partials, int ksplit, int64_t split_stride,
                         const float* bias, float* logits_out, int64_t T, int E, int k,
-                        int32_t* topk_idx, float* topk_w, cudaStream_t stream);
+                        int n_group, int topk_group, int32_t* topk_idx, float* topk_w,
+                        cudaStream_t stream);
 
 // ---- route_tc.cu (tcgen05 / TMEM / TMA, bf16)
 // Gate logits on the tensor cores (tokens on the MMA's M side, experts on N, E in [16, 256],
@@ -76,7 +78,8 @@ cudaError_t launch_dispatch_rows(int dtype, const void* x, const int32_t* sorted
                                  const int32_t* offsets, int E, int k, int H, int64_t rows,
                                  void* xs, cudaStream_t stream);
 cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_of,
-                           const float* topk_w, void* out, int64_t T, int H, int k,
+                           const float* topk_w, const void* shared, float shared_factor,
+                           const float* out_bias, void* out, int64_t T, int H, int k,
                            cudaStream_t stream);
 
 }  // namespace moe

@@ -187,11 +187,41 @@ void record_stage(int i, cudaStream_t st) {
     cudaEventRecord(static_cast<cudaEvent_t>(g_events[i]), st);
 }
 
+// ---- routing / combine options (moe_layer_opts), validated once per call
+
+struct Opts {
+  int n_group = 1, topk_group = 1;
+  const void* shared = nullptr;
+  float shared_factor = 0.f;
+  const float* out_bias = nullptr;
+};
+
+moe_status read_opts(const moe_shape& s, const moe_layer_opts* o, Opts* out) {
+  *out = Opts{};
+  if (o == nullptr) return MOE_OK;
+  if (o->n_group < 1 || o->n_group > 32 || s.E % o->n_group != 0)
+    return fail(MOE_ERR_INVALID_ARG, "n_group must be in [1, 32] and divide E");
+  if (o->topk_group < 1 || o->topk_group > o->n_group)
+    return fail(MOE_ERR_INVALID_ARG, "topk_group must be in [1, n_group]");
+  if (o->n_group > 1 && s.k > o->topk_group * (s.E / o->n_group))
+    return fail(MOE_ERR_INVALID_ARG, "k exceeds the experts of the kept groups");
+  if (!std::isfinite(o->shared_factor))
+    return fail(MOE_ERR_INVALID_ARG, "shared_factor is not finite");
+  OPT_PTR(o->shared_out, "shared_out");
+  OPT_PTR(o->out_bias, "out_bias");
+  out->n_group = o->n_group;
+  out->topk_group = o->n_group > 1 ? o->topk_group : 1;
+  out->shared = o->shared_out;
+  out->shared_factor = o->shared_factor;
+  out->out_bias = o->out_bias;
+  return MOE_OK;
+}
+
 // ---- stage bodies (arguments already validated)
 
-moe_status do_route(const moe_shape& s, const Layout& L, const void* x, const void* w_router,
-                    const float* bias, float* logits_out, int32_t* topk_idx, float* topk_w,
-                    void* ws, cudaStream_t st) {
+moe_status do_route(const moe_shape& s, const Layout& L, const Opts& o, const void* x,
+                    const void* w_router, const float* bias, float* logits_out, int32_t* topk_idx,
+                    float* topk_w, void* ws, cudaStream_t st) {
   cudaError_t e;
   if (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0) {
     float* partials = at<float>(ws, L.logits);
@@ -200,12 +230,21 @@ moe_status do_route(const moe_shape& s, const Layout& L, const void* x, const vo
                                   L.ksplit, at<int>(ws, L.err), num_sms(), st, &d);
     if (e != cudaSuccess) return cuda_fail(e, "router gate GEMM (tcgen05)", d);
     e = moe::launch_topk(partials, L.ksplit, s.T * s.E, bias, logits_out, s.T, s.E, s.k,
-                         topk_idx, topk_w, st);
+                         o.n_group, o.topk_group, topk_idx, topk_w, st);
     if (e != cudaSuccess) return cuda_fail(e, "router top-k");
   } else {
-    e = moe::launch_route_simt(s.dtype, x, w_router, bias, s.T, s.H, s.E, s.k, logits_out,
-                               topk_idx, topk_w, st);
+    // the fused CUDA-core router selects plain top-k; with groups its logits (bias included)
+    // go through the group-limited top-k kernel
+    float* lg = logits_out;
+    if (o.n_group > 1 && lg == nullptr) lg = at<float>(ws, L.logits);
+    e = moe::launch_route_simt(s.dtype, x, w_router, bias, s.T, s.H, s.E, s.k, lg, topk_idx,
+                               topk_w, st);
     if (e != cudaSuccess) return cuda_fail(e, "router (CUDA cores)");
+    if (o.n_group > 1) {
+      e = moe::launch_topk(lg, 1, 0, nullptr, nullptr, s.T, s.E, s.k, o.n_group, o.topk_group,
+                           topk_idx, topk_w, st);
+      if (e != cudaSuccess) return cuda_fail(e, "router group-limited top-k");
+    }
   }
   return MOE_OK;
 }
@@ -261,10 +300,14 @@ int32_t moe_capacity(const moe_shape* shape) {
   return capacity_of(*shape);
 }
 
-moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router,
-                     const float* logit_bias, float* logits_out, int32_t* topk_idx,
-                     float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+moe_status moe_route_ex(const moe_shape* shape, const moe_layer_opts* opts, const void* x,
+                        const void* w_router, const float* logit_bias, float* logits_out,
+                        int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                        void* stream) {
   moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  Opts o;
+  st = read_opts(*shape, opts, &o);
   if (st != MOE_OK) return st;
   if (shape->T == 0) return MOE_OK;
   REQUIRE_PTR(x, "x");
@@ -276,22 +319,39 @@ moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router
   const Layout L = layout_of(*shape);
   st = check_ws(ws, ws_bytes, L.logits + static_cast<size_t>(shape->T) * shape->E * 4 * L.ksplit);
   if (st != MOE_OK) return st;
-  return do_route(*shape, L, x, w_router, logit_bias, logits_out, topk_idx, topk_w, ws,
+  return do_route(*shape, L, o, x, w_router, logit_bias, logits_out, topk_idx, topk_w, ws,
                   static_cast<cudaStream_t>(stream));
 }
 
-moe_status moe_route_from_logits(const moe_shape* shape, const float* logits, int32_t* topk_idx,
-                                 float* topk_w, void* stream) {
+moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router,
+                     const float* logit_bias, float* logits_out, int32_t* topk_idx,
+                     float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+  return moe_route_ex(shape, nullptr, x, w_router, logit_bias, logits_out, topk_idx, topk_w, ws,
+                      ws_bytes, stream);
+}
+
+moe_status moe_route_from_logits_ex(const moe_shape* shape, const moe_layer_opts* opts,
+                                    const float* logits, int32_t* topk_idx, float* topk_w,
+                                    void* stream) {
   moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  Opts o;
+  st = read_opts(*shape, opts, &o);
   if (st != MOE_OK) return st;
   if (shape->T == 0) return MOE_OK;
   REQUIRE_PTR(logits, "logits");
   REQUIRE_PTR(topk_idx, "topk_idx");
   REQUIRE_PTR(topk_w, "topk_w");
   cudaError_t e = moe::launch_topk(logits, 1, 0, nullptr, nullptr, shape->T, shape->E, shape->k,
-                                   topk_idx, topk_w, static_cast<cudaStream_t>(stream));
+                                   o.n_group, o.topk_group, topk_idx, topk_w,
+                                   static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "router top-k");
   return MOE_OK;
+}
+
+moe_status moe_route_from_logits(const moe_shape* shape, const float* logits, int32_t* topk_idx,
+                                 float* topk_w, void* stream) {
+  return moe_route_from_logits_ex(shape, nullptr, logits, topk_idx, topk_w, stream);
 }
 
 moe_status moe_align(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts,
@@ -379,29 +439,43 @@ moe_status moe_grouped_ffn(const moe_shape* shape, const void* x, const int32_t*
   return do_ffn(*shape, L, x, sorted_ids, offsets, w_gate, w_up, w_down, y_slots, ws, cs, false);
 }
 
-moe_status moe_combine(const moe_shape* shape, const void* y_slots, const int32_t* slot_of,
-                       const float* topk_w, void* out, void* stream) {
+moe_status moe_combine_ex(const moe_shape* shape, const moe_layer_opts* opts,
+                          const void* y_slots, const int32_t* slot_of, const float* topk_w,
+                          void* out, void* stream) {
   moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  Opts o;
+  st = read_opts(*shape, opts, &o);
   if (st != MOE_OK) return st;
   if (shape->T == 0) return MOE_OK;
   REQUIRE_PTR(y_slots, "y_slots");
   REQUIRE_PTR(slot_of, "slot_of");
   REQUIRE_PTR(topk_w, "topk_w");
   REQUIRE_PTR(out, "out");
-  cudaError_t e = moe::launch_combine(shape->dtype, y_slots, slot_of, topk_w, out, shape->T,
-                                      shape->H, shape->k, static_cast<cudaStream_t>(stream));
+  cudaError_t e = moe::launch_combine(shape->dtype, y_slots, slot_of, topk_w, o.shared,
+                                      o.shared_factor, o.out_bias, out, shape->T, shape->H,
+                                      shape->k, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "combine");
   return MOE_OK;
 }
 
-moe_status moe_layer_forward(const moe_shape* shape, const void* x, const void* w_router,
-                             const float* logit_bias, const void* w_gate, const void* w_up,
-                             const void* w_down, void* out, float* logits_out, int32_t* topk_idx,
-                             float* topk_w, int32_t* counts, uint8_t* drop_mask, void* ws,
-                             size_t ws_bytes, void* stream) {
+moe_status moe_combine(const moe_shape* shape, const void* y_slots, const int32_t* slot_of,
+                       const float* topk_w, void* out, void* stream) {
+  return moe_combine_ex(shape, nullptr, y_slots, slot_of, topk_w, out, stream);
+}
+
+moe_status moe_layer_forward_ex(const moe_shape* shape, const moe_layer_opts* opts,
+                                const void* x, const void* w_router, const float* logit_bias,
+                                const void* w_gate, const void* w_up, const void* w_down,
+                                void* out, float* logits_out, int32_t* topk_idx, float* topk_w,
+                                int32_t* counts, uint8_t* drop_mask, void* ws, size_t ws_bytes,
+                                void* stream) {
   moe_status st = check_shape(shape);
   if (st != MOE_OK) return st;
   const moe_shape& s = *shape;
+  Opts o;
+  st = read_opts(s, opts, &o);
+  if (st != MOE_OK) return st;
   REQUIRE_PTR(counts, "counts");
   const Layout L = layout_of(s);
   st = check_ws(ws, ws_bytes, L.total);
@@ -424,7 +498,7 @@ moe_status moe_layer_forward(const moe_shape* shape, const void* x, const void* 
   OPT_PTR(logit_bias, "logit_bias");
   OPT_PTR(logits_out, "logits_out");
 
-  st = do_route(s, L, x, w_router, logit_bias, logits_out, topk_idx, topk_w, ws, cs);
+  st = do_route(s, L, o, x, w_router, logit_bias, logits_out, topk_idx, topk_w, ws, cs);
   if (st != MOE_OK) return st;
   record_stage(0, cs);
   int32_t* offsets = at<int32_t>(ws, L.offsets);
@@ -438,10 +512,21 @@ moe_status moe_layer_forward(const moe_shape* shape, const void* x, const void* 
   void* y = at<void>(ws, L.yslots);
   st = do_ffn(s, L, x, sorted_ids, offsets, w_gate, w_up, w_down, y, ws, cs, true);
   if (st != MOE_OK) return st;
-  e = moe::launch_combine(s.dtype, y, slot_of, topk_w, out, s.T, s.H, s.k, cs);
+  e = moe::launch_combine(s.dtype, y, slot_of, topk_w, o.shared, o.shared_factor, o.out_bias, out,
+                          s.T, s.H, s.k, cs);
   if (e != cudaSuccess) return cuda_fail(e, "combine");
   record_stage(4, cs);
   return MOE_OK;
+}
+
+moe_status moe_layer_forward(const moe_shape* shape, const void* x, const void* w_router,
+                             const float* logit_bias, const void* w_gate, const void* w_up,
+                             const void* w_down, void* out, float* logits_out, int32_t* topk_idx,
+                             float* topk_w, int32_t* counts, uint8_t* drop_mask, void* ws,
+                             size_t ws_bytes, void* stream) {
+  return moe_layer_forward_ex(shape, nullptr, x, w_router, logit_bias, w_gate, w_up, w_down, out,
+                              logits_out, topk_idx, topk_w, counts, drop_mask, ws, ws_bytes,
+                              stream);
 }
 
 moe_status moe_check_error(void* ws, void* stream) {

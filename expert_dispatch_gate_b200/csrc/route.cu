@@ -20,12 +20,14 @@ namespace {
 constexpr int kWarpsPerBlock = 8;
 
 // Logits distributed over lanes: lane holds experts lane, lane+32, ... (VPL per lane). Each
-// logit is the sum of the K-range partials in ascending order plus the optional bias.
+// logit is the sum of the K-range partials in ascending order plus the optional bias. With
+// n_group > 1 the selection is group-limited (select.cuh).
 template <int VPL>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     topk_kernel(const float* __restrict__ partials, int ksplit, int64_t split_stride,
                 const float* __restrict__ bias, float* __restrict__ logits_out, int64_t T, int E,
-                int k, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+                int k, int n_group, int topk_group, int32_t* __restrict__ topk_idx,
+                float* __restrict__ topk_w) {
   pdl_enter<false>();
   const int lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -57,6 +59,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
       taken |= 1u << i;
     }
   }
+  if (n_group > 1) taken |= warp_group_exclude<VPL>(v, E, n_group, topk_group, lane);
   warp_select_topk<VPL>(v, taken, k, lane, topk_idx + t * k, topk_w + t * k);
 }
 
@@ -231,7 +234,8 @@ cudaError_t launch_route_simt(int dtype, const void* x, const void* w_router, co
 
 cudaError_t launch_topk(const float* partials, int ksplit, int64_t split_stride,
                         const float* bias, float* logits_out, int64_t T, int E, int k,
-                        int32_t* topk_idx, float* topk_w, cudaStream_t stream) {
+                        int n_group, int topk_group, int32_t* topk_idx, float* topk_w,
+                        cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
   const unsigned block = kWarpsPerBlock * 32;
@@ -240,7 +244,8 @@ cudaError_t launch_topk(const float* partials, int ksplit, int64_t split_stride,
   else if (E <= 64) kernel = topk_kernel<2>;
   else if (E <= 128) kernel = topk_kernel<4>;
   return launch_kernel(kernel, dim3(grid), dim3(block), 0, stream, 1, partials, ksplit,
-                       split_stride, bias, logits_out, T, E, k, topk_idx, topk_w);
+                       split_stride, bias, logits_out, T, E, k, n_group, topk_group, topk_idx,
+                       topk_w);
 }
 
 }  // namespace moe

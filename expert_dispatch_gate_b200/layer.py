@@ -30,7 +30,8 @@ class Workspace:
         return L.moe_check_error(self.buf, stream)
 
 
-def route(x, w_router, k, logit_bias=None, logits_out=True, ws=None, stream=None):
+def route(x, w_router, k, logit_bias=None, logits_out=True, ws=None, stream=None, n_group=1,
+          topk_group=1):
     T, H = x.shape
     E = w_router.shape[1]
     shape = shape_of(T, H, E, k, 128, 0.0, _dtype_code(x))
@@ -38,16 +39,26 @@ def route(x, w_router, k, logit_bias=None, logits_out=True, ws=None, stream=None
     idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
     w = torch.empty((T, k), dtype=torch.float32, device=x.device)
     logits = torch.empty((T, E), dtype=torch.float32, device=x.device) if logits_out else None
-    L.moe_route(shape, x, w_router, logit_bias, logits, idx, w, ws.buf, ws.nbytes, stream)
+    if n_group > 1:
+        L.moe_route_ex(shape, L.make_opts(n_group, topk_group), x, w_router, logit_bias, logits,
+                       idx, w, ws.buf, ws.nbytes, stream)
+    else:
+        L.moe_route(shape, x, w_router, logit_bias, logits, idx, w, ws.buf, ws.nbytes, stream)
     return idx, w, logits
 
 
-def route_from_logits(logits, k, stream=None):
+def route_from_logits(logits, k, stream=None, n_group=1, topk_group=1):
+    """Top-k selection and weights from given float32 logits; n_group > 1 makes the selection
+    group-limited (keep the topk_group best of n_group expert groups first)."""
     T, E = logits.shape
     shape = shape_of(T, 128, E, k, 128, 0.0, L.MOE_BF16 if E <= 64 or E % 8 == 0 else L.MOE_F32)
     idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
     w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
-    L.moe_route_from_logits(shape, logits, idx, w, stream)
+    if n_group > 1:
+        L.moe_route_from_logits_ex(shape, L.make_opts(n_group, topk_group), logits, idx, w,
+                                   stream)
+    else:
+        L.moe_route_from_logits(shape, logits, idx, w, stream)
     return idx, w
 
 
@@ -79,12 +90,18 @@ def grouped_ffn(x, sorted_ids, offsets, w_gate, w_up, w_down, k, capacity_factor
     return y
 
 
-def combine(y_slots, slot_of, topk_w, E, stream=None):
+def combine(y_slots, slot_of, topk_w, E, stream=None, shared=None, shared_factor=0.0,
+            out_bias=None):
+    """Weighted merge to token order; optionally + shared_factor * shared + out_bias."""
     T, k = topk_w.shape
     H = y_slots.shape[1]
     shape = shape_of(T, H, E, k, 128, 0.0, _dtype_code(y_slots))
     out = torch.empty((T, H), dtype=y_slots.dtype, device=y_slots.device)
-    L.moe_combine(shape, y_slots, slot_of, topk_w, out, stream)
+    if shared is not None or out_bias is not None:
+        opts = L.make_opts(shared_out=shared, shared_factor=shared_factor, out_bias=out_bias)
+        L.moe_combine_ex(shape, opts, y_slots, slot_of, topk_w, out, stream)
+    else:
+        L.moe_combine(shape, y_slots, slot_of, topk_w, out, stream)
     return out
 
 
@@ -93,9 +110,11 @@ class MoELayerOutputs(dict):
 
 
 def layer_forward(x, w_router, w_gate, w_up, w_down, k, capacity_factor, logit_bias=None,
-                  logits_out=True, ws=None, out=None, stream=None):
-    """Whole layer through moe_layer_forward. Returns out, topk_idx, topk_w, counts, drop_mask
-    (and logits when requested)."""
+                  logits_out=True, ws=None, out=None, stream=None, n_group=1, topk_group=1,
+                  shared=None, shared_factor=0.0, out_bias=None):
+    """Whole layer through moe_layer_forward (moe_layer_forward_ex when group-limited routing
+    or a shared-expert / bias term is asked for). Returns out, topk_idx, topk_w, counts,
+    drop_mask (and logits when requested)."""
     T, H = x.shape
     E, _, I = w_gate.shape
     dev = x.device
@@ -108,9 +127,15 @@ def layer_forward(x, w_router, w_gate, w_up, w_down, k, capacity_factor, logit_b
     res["counts"] = torch.empty(E, dtype=torch.int32, device=dev)
     res["drop_mask"] = torch.empty(T * k, dtype=torch.uint8, device=dev)
     res["logits"] = torch.empty((T, E), dtype=torch.float32, device=dev) if logits_out else None
-    L.moe_layer_forward(shape, x, w_router, logit_bias, w_gate, w_up, w_down, res["out"],
-                        res["logits"], res["topk_idx"], res["topk_w"], res["counts"],
-                        res["drop_mask"], ws.buf, ws.nbytes, stream)
+    if n_group > 1 or shared is not None or out_bias is not None:
+        opts = L.make_opts(n_group, topk_group, shared, shared_factor, out_bias)
+        L.moe_layer_forward_ex(shape, opts, x, w_router, logit_bias, w_gate, w_up, w_down,
+                               res["out"], res["logits"], res["topk_idx"], res["topk_w"],
+                               res["counts"], res["drop_mask"], ws.buf, ws.nbytes, stream)
+    else:
+        L.moe_layer_forward(shape, x, w_router, logit_bias, w_gate, w_up, w_down, res["out"],
+                            res["logits"], res["topk_idx"], res["topk_w"], res["counts"],
+                            res["drop_mask"], ws.buf, ws.nbytes, stream)
     res["ws"] = ws
     res["C"] = L.moe_capacity(shape)
     return res

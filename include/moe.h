@@ -158,6 +158,50 @@ moe_status moe_layer_forward(const moe_shape* shape, const void* x, const void* 
                              int32_t* topk_idx, float* topk_w, int32_t* counts,
                              uint8_t* drop_mask, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- Extensions of the routing and the combine.
+ *
+ * Group-limited routing, [P5] "大模型推理加速200%+？…", section "3.1 Moe Fuse Gate & Softmax
+ * TopK" (the gate selects expert groups first and keeps each group's top-1/top-2; the page
+ * gives no formula, this is the reading taken): the E experts form n_group equal contiguous
+ * groups; a group's score is the float32 sum of its two largest logits (its only logit when a
+ * group holds one expert); the topk_group best groups are kept (ties to the lower group
+ * index); the k largest logits among their experts are selected with the plain rule; weights
+ * are renormalised over the k as in moe_route.
+ *
+ * Shared expert and bias in the combine, [P5] section "3.2 Fuse RMS RoPE & MoE Align & MoE
+ * Sum" (the MoE sum fuses the shared expert's factor and a bias add):
+ *   out[t,:] = sum_j w[t,j] y[slot,:] + shared_factor * shared_out[t,:] + out_bias[:]
+ * accumulated in float32 in that order and rounded once; shared_out is the shared expert's
+ * output computed by the caller, [T,H] in the layer dtype, 16-byte aligned. Both terms apply
+ * to every token, a fully dropped one included. */
+typedef struct {
+  int32_t n_group;        /* >= 1, divides E, <= 32; 1 = plain top-k */
+  int32_t topk_group;     /* groups kept per token, 1..n_group; k <= topk_group * E / n_group */
+  const void* shared_out; /* [T,H] (dtype of the layer) or NULL */
+  float shared_factor;    /* multiplies shared_out */
+  const float* out_bias;  /* [H] float32 or NULL */
+} moe_layer_opts;
+
+/* moe_route / moe_route_from_logits / moe_combine / moe_layer_forward with `opts` (NULL or all
+ * defaults: identical to the plain call). Invalid options return MOE_ERR_INVALID_ARG before any
+ * launch. */
+moe_status moe_route_ex(const moe_shape* shape, const moe_layer_opts* opts, const void* x,
+                        const void* w_router, const float* logit_bias, float* logits_out,
+                        int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                        void* stream);
+moe_status moe_route_from_logits_ex(const moe_shape* shape, const moe_layer_opts* opts,
+                                    const float* logits, int32_t* topk_idx, float* topk_w,
+                                    void* stream);
+moe_status moe_combine_ex(const moe_shape* shape, const moe_layer_opts* opts,
+                          const void* y_slots, const int32_t* slot_of, const float* topk_w,
+                          void* out, void* stream);
+moe_status moe_layer_forward_ex(const moe_shape* shape, const moe_layer_opts* opts,
+                                const void* x, const void* w_router, const float* logit_bias,
+                                const void* w_gate, const void* w_up, const void* w_down,
+                                void* out, float* logits_out, int32_t* topk_idx, float* topk_w,
+                                int32_t* counts, uint8_t* drop_mask, void* ws, size_t ws_bytes,
+                                void* stream);
+
 /* Synchronises `stream`, reads and clears the device error word at the start of `ws`.
  * Returns MOE_OK, MOE_ERR_DEVICE (a kernel flagged a fault; see moe_last_error_detail) or
  * MOE_ERR_CUDA. */

@@ -74,6 +74,33 @@ def decided_tokens(logits_ref, k, delta):
     return np.all(gaps > 2.0 * delta, axis=1)
 
 
+def decided_tokens_grouped(logits_ref, k, n_group, topk_group, delta):
+    """Tokens whose group-limited selection cannot change under a perturbation of every logit
+    by at most delta: the topk_group+1 best group scores (each a sum of two logits, so it moves
+    by at most 2*delta) are more than 4*delta apart, and the k+1 best logits among the kept
+    groups' experts are more than 2*delta apart."""
+    l32 = np.asarray(logits_ref, dtype=np.float32)
+    T, E = l32.shape
+    gs = E // n_group
+    sc = orc.group_scores(l32, n_group).astype(np.float64)
+    margin = 1e-6 * max(1.0, float(np.abs(sc).max()))
+    dec = np.ones(T, dtype=bool)
+    order = np.argsort(-sc, axis=1, kind="stable")
+    if topk_group < n_group:
+        top = np.take_along_axis(sc, order[:, :topk_group + 1], axis=1)
+        dec &= np.all(top[:, :-1] - top[:, 1:] > 4.0 * delta + margin, axis=1)
+    l64 = l32.astype(np.float64)
+    for t in range(T):
+        if not dec[t]:
+            continue
+        kept = order[t, :topk_group]
+        cand = np.concatenate([l64[t, g * gs:(g + 1) * gs] for g in kept])
+        top = -np.sort(-cand)[:min(k + 1, cand.size)]
+        if top.size >= 2 and not np.all(top[:-1] - top[1:] > 2.0 * delta):
+            dec[t] = False
+    return dec
+
+
 def check_topk_valid(logits_ref, idx_gpu, k, delta, rows):
     """Fragile tokens: the GPU's set must be a top-k of some perturbation within delta."""
     l = np.asarray(logits_ref, dtype=np.float64)

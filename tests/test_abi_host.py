@@ -136,3 +136,33 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(L, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="no fallback"):
         L.lib()
+
+
+def test_layer_opts_struct_layout():
+    assert ctypes.sizeof(L.MoeLayerOpts) == 32
+    o = L.MoeLayerOpts
+    assert (o.n_group.offset, o.topk_group.offset, o.shared_out.offset, o.shared_factor.offset,
+            o.out_bias.offset) == (0, 4, 8, 16, 24)
+
+
+@pytest.mark.parametrize("opts,why", [
+    (dict(n_group=7, topk_group=1), "n_group must divide E"),
+    (dict(n_group=8, topk_group=9), "topk_group above n_group"),
+    (dict(n_group=8, topk_group=0), "topk_group below 1"),
+    (dict(n_group=64, topk_group=2), "more than 32 groups"),
+    (dict(n_group=16, topk_group=1), "k = 6 exceeds the 4 experts of one group"),
+    (dict(shared_factor=float("inf")), "non-finite factor"),
+    (dict(shared_out=ODD), "misaligned shared output"),
+    (dict(out_bias=ODD), "misaligned bias"),
+])
+def test_invalid_layer_opts_rejected_before_launch(lib, opts, why):
+    s = L.make_shape(64, 128, 64, 6, 128, 1.25, "bf16")
+    o = L.make_opts(**opts)
+    ws = L.moe_workspace_bytes(s)
+    got = L.moe_layer_forward_ex(s, o, *([BAD] * 12), BAD, ws, stream=0, check=False)
+    assert got == L.MOE_ERR_INVALID_ARG, why
+    assert L.moe_route_from_logits_ex(s, o, BAD, BAD, BAD, stream=0, check=False) == \
+        L.MOE_ERR_INVALID_ARG, why
+    assert L.moe_combine_ex(s, o, BAD, BAD, BAD, BAD, stream=0, check=False) == \
+        L.MOE_ERR_INVALID_ARG, why
+    assert L.last_error_detail()

@@ -13,6 +13,7 @@ from expert_dispatch_gate_b200 import layer as M
 from expert_dispatch_gate_b200 import workloads as W
 from oracle import moe_oracle as orc
 from tests.parity import (TOL_LOGITS, TOL_OUT, TOL_W, ExpertWeights, assert_close_rel,
+                          decided_tokens_grouped,
                           check_topk_valid, decided_tokens, inputs_np, np32, npi, to_dev)
 
 pytestmark = pytest.mark.gpu
@@ -30,9 +31,9 @@ SMALL = {
     # E = 96: the router's second 64-expert chunk is half zero-filled (N = 96, two
     # accumulators); I = 640 leaves the last GEMM1 pair tile half outside the weight; H = 384
     # runs GEMM2 with one feature block per tile
-    "e96_partial_tiles": W.Workload("e96", 17, 333, 384, 96, 4, 640, "bf16", 1.25),
+    "e96_partial_tiles": W.Workload("e96", 19, 333, 384, 96, 4, 640, "bf16", 1.25),
     # T = 50, H = 1024: one token tile, the router's K split into 4 ranges
-    "e128_router_ksplit": W.Workload("e128", 18, 50, 1024, 128, 6, 256, "bf16", 1.25),
+    "e128_router_ksplit": W.Workload("e128", 20, 50, 1024, 128, 6, 256, "bf16", 1.25),
 }
 
 
@@ -192,8 +193,11 @@ def test_combine(name):
 
 # ----------------------------------------------------------------- whole layer
 
-def compare_layer(wl, cpu_or_dev, dev, res, sample=None, seed=0):
-    """Compare moe_layer_forward's outputs with the oracle (see module docstring of parity)."""
+def compare_layer(wl, cpu_or_dev, dev, res, sample=None, seed=0, n_group=1, topk_group=1,
+                  shared=None, shared_factor=0.0, out_bias=None):
+    """Compare moe_layer_forward's outputs with the oracle (see module docstring of parity).
+    With n_group > 1 the routing is group-limited; shared / out_bias (host numpy) add the
+    combine's shared-expert and bias terms."""
     host = inputs_np(cpu_or_dev)
     T, E, k = wl.T, wl.E, wl.k
     L_o = orc.router_logits(host["x"], host["w_router"], host["logit_bias"])
@@ -201,12 +205,17 @@ def compare_layer(wl, cpu_or_dev, dev, res, sample=None, seed=0):
     tol = TOL_LOGITS[wl.dtype] * max(1.0, float(np.abs(L_o).max()))
     delta = float(np.abs(L_g - L_o).max())
     assert delta <= tol, (delta, tol)
-    idx_o = orc.select_topk(L_o, k)
+    if n_group > 1:
+        idx_o = orc.select_topk_grouped(L_o, k, n_group, topk_group)
+        dec = decided_tokens_grouped(L_o, k, n_group, topk_group, delta)
+    else:
+        idx_o = orc.select_topk(L_o, k)
+        dec = decided_tokens(L_o, k, delta)
     w_o = orc.route_weights(L_o, idx_o)
     idx_g, w_g = npi(res["topk_idx"]), npi(res["topk_w"])
-    dec = decided_tokens(L_o, k, delta)
     assert np.array_equal(idx_g[dec], idx_o[dec])
-    check_topk_valid(L_o, idx_g, k, delta, np.nonzero(~dec)[0])
+    if n_group == 1:
+        check_topk_valid(L_o, idx_g, k, delta, np.nonzero(~dec)[0])
     np.testing.assert_allclose(w_g[dec], w_o[dec], atol=TOL_W + k * delta, rtol=0)
     C = orc.capacity(T, k, E, wl.capacity_factor)
     assert res["C"] == C
@@ -244,7 +253,9 @@ def compare_layer(wl, cpu_or_dev, dev, res, sample=None, seed=0):
         comparable = sorted(rng.choice(comparable, size=sample, replace=False).tolist())
     ref = orc.layer_forward(host["x"], host["w_router"], ExpertWeights(dev["w_gate"]),
                             ExpertWeights(dev["w_up"]), ExpertWeights(dev["w_down"]), k,
-                            wl.capacity_factor, logit_bias=host["logit_bias"], tokens=comparable)
+                            wl.capacity_factor, logit_bias=host["logit_bias"], tokens=comparable,
+                            n_group=n_group, topk_group=topk_group, shared=shared,
+                            shared_factor=shared_factor, out_bias=out_bias)
     got = np32(res["out"])[comparable]
     r = assert_close_rel(got, ref["out"], TOL_OUT[wl.dtype], "layer output")
     return {"delta_logits": delta, "fragile": int((~dec).sum()), "compared": len(comparable),
