@@ -43,6 +43,12 @@ Readings taken where the pages are silent or disagree (each also listed in the d
   logit when a group holds one expert); the topk_group groups with the highest scores are kept
   (ties to the lower group index); the k largest logits among the kept groups' experts are
   selected with the plain top-k rule; weights are renormalised over the k as before.
+* FP8 expert weights (SURVEY's "next" row on FP8 experts; [P5] "3.4 ... MoE GEMM" lists W8A8 /
+  W4A16 quantised expert GEMMs without a scheme): weights only, e4m3 (OCP FP8: 1 sign, 4
+  exponent bits with bias 7, 3 mantissa bits, subnormals, no infinities, 448 the largest
+  finite value); one float32 scale per output channel, scale = max_k |W[k, m]| / 448 (1 when
+  the column is all zero); code = e4m3(W / scale) rounded to nearest, ties to even, saturating
+  at +-448; the GEMM uses decode(code) * scale. Activations stay bf16 (W8A16).
 * Shared expert and bias in the combine: out[t] = sum_j w[t,j] y[slot] + factor * shared[t] + b,
   with shared[t] the shared expert's output row (computed by the caller) and b a per-feature
   bias; both terms apply to every token, including a fully dropped one.
@@ -66,6 +72,10 @@ __all__ = [
     "route",
     "route_grouped",
     "capacity",
+    "e4m3_decode",
+    "e4m3_encode",
+    "quantize_weights_fp8",
+    "dequantize_weights_fp8",
     "align",
     "swiglu_expert",
     "grouped_ffn_slots",
@@ -175,6 +185,62 @@ def route_grouped(x, w_router, k, n_group, topk_group, logit_bias=None, logits=N
         logits = router_logits(x, w_router, logit_bias)
     idx = select_topk_grouped(logits, k, n_group, topk_group)
     return np.asarray(logits, dtype=np.float32), idx, route_weights(logits, idx)
+
+
+def e4m3_decode(codes):
+    """Value of each FP8 e4m3 code (uint8), float64, from the format's definition:
+    sign s, exponent field e (4 bits, bias 7), mantissa field m (3 bits);
+    e > 0: (-1)^s * 2^(e-7) * (1 + m/8); e == 0: (-1)^s * 2^-6 * (m/8); e == 15 and m == 7: NaN.
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    s = (c >> 7) & 1
+    e = (c >> 3) & 15
+    m = c & 7
+    mag = np.where(e > 0, np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64)),
+                   np.ldexp(m / 8.0, -6))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return np.where(s == 1, -mag, mag)
+
+
+def e4m3_encode(values):
+    """Nearest e4m3 code of each float32 value, ties to the even code (even mantissa field),
+    saturating to +-448 (the largest finite magnitude); -0 keeps its sign. Finite inputs only.
+
+    Chosen among the 127 finite non-negative codes by exact float64 comparison: the nearest
+    magnitude wins; at an exact midpoint the code with an even mantissa field wins.
+    """
+    v = np.asarray(values, dtype=np.float32).astype(np.float64)
+    if not np.all(np.isfinite(v)):
+        raise ValueError("e4m3_encode takes finite values")
+    mags = e4m3_decode(np.arange(127, dtype=np.uint8))      # codes 0..126: 0 .. 448, ascending
+    a = np.minimum(np.abs(v), 448.0)
+    hi = np.searchsorted(mags, a, side="left")               # first magnitude >= a
+    hi = np.minimum(hi, 126)
+    lo = np.maximum(hi - 1, 0)
+    d_lo = a - mags[lo]
+    d_hi = mags[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(a == mags[hi], hi, np.where(pick_hi, hi, lo)).astype(np.int64)
+    sign = np.signbit(v).astype(np.int64)
+    return (code | (sign << 7)).astype(np.uint8)
+
+
+def quantize_weights_fp8(w):
+    """Per-output-channel e4m3 quantisation of expert weights w [E, K, M] (reduction dim K,
+    output channels M): scale[e, m] = float32(max_k |w[e, k, m]| / 448) (1 when the column is
+    all zero), code[e, k, m] = e4m3(float32(w / scale)). Returns (codes uint8, scale float32).
+    Both divisions are single float32 operations, the rounding the GPU performs."""
+    w32 = np.asarray(w, dtype=np.float32)
+    amax = np.max(np.abs(w32), axis=1)                       # [E, M], exact
+    scale = np.where(amax > 0, (amax / np.float32(448.0)).astype(np.float32), np.float32(1.0))
+    scale = scale.astype(np.float32)
+    q = e4m3_encode((w32 / scale[:, None, :]).astype(np.float32))
+    return q, scale
+
+
+def dequantize_weights_fp8(codes, scale):
+    """decode(code) * scale, float64 [E, K, M]: the weights the FP8 expert GEMMs apply."""
+    return e4m3_decode(codes) * np.asarray(scale, dtype=np.float64)[:, None, :]
 
 
 def capacity(T, k, E, capacity_factor):

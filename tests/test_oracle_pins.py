@@ -395,3 +395,69 @@ def test_combine_shared_terms_are_additive():
     assert np.array_equal(orc.combine(y, slot_of, w, shared=shared, shared_factor=0.0), base)
     with_terms = orc.combine(y, slot_of, w, shared=shared, shared_factor=1.5, out_bias=bias)
     assert np.allclose(with_terms - base, 1.5 * shared + bias, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- FP8 (e4m3) weights
+
+
+def test_e4m3_decode_landmarks():
+    d = orc.e4m3_decode(np.arange(256, dtype=np.uint8))
+    # format landmarks: zero, smallest subnormal 2^-9, largest subnormal 7*2^-9, smallest
+    # normal 2^-6, one, largest finite 448; NaN only at S.1111.111
+    assert d[0x00] == 0.0 and d[0x01] == 2.0 ** -9 and d[0x07] == 7 * 2.0 ** -9
+    assert d[0x08] == 2.0 ** -6 and d[0x38] == 1.0 and d[0x7E] == 448.0
+    assert np.isnan(d[0x7F]) and np.isnan(d[0xFF]) and np.sum(np.isnan(d)) == 2
+    assert np.array_equal(d[0x80:0xFF], -d[0x00:0x7F])
+    # the 127 non-negative finite codes are strictly increasing
+    assert np.all(np.diff(d[:0x7F]) > 0)
+    # within a binade the step is 2^(e-7)/8
+    for e in range(1, 16):
+        codes = [(e << 3) | m for m in range(8) if (e << 3) | m < 0x7F]
+        steps = np.diff(d[codes])
+        assert np.all(steps == 2.0 ** (e - 7) / 8)
+
+
+def test_e4m3_roundtrip_and_ties():
+    codes = np.asarray([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    vals = orc.e4m3_decode(codes)
+    assert np.array_equal(orc.e4m3_encode(vals.astype(np.float32)), codes)
+    mags = orc.e4m3_decode(np.arange(127, dtype=np.uint8))
+    mids = (mags[:-1] + mags[1:]) / 2          # exact in float32 (4 significant bits)
+    assert np.array_equal(mids.astype(np.float32).astype(np.float64), mids)
+    got = orc.e4m3_encode(mids.astype(np.float32)).astype(np.int64)
+    lo = np.arange(126)
+    assert np.array_equal(got, np.where(lo % 2 == 0, lo, lo + 1))  # ties to the even code
+    assert np.array_equal(orc.e4m3_encode((mids * (1 - 2.0 ** -12)).astype(np.float32)), lo)
+    assert np.array_equal(orc.e4m3_encode((mids * (1 + 2.0 ** -12)).astype(np.float32)), lo + 1)
+    # saturation
+    assert orc.e4m3_encode(np.float32([1e6, -1e6, 480.0, 449.0]))[:4].tolist() == [0x7E, 0xFE, 0x7E, 0x7E]
+
+
+def test_e4m3_encode_matches_torch_conversion_in_range():
+    rng = np.random.default_rng(8)
+    v = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 0.1, 1.0, 30.0)])
+    v = np.clip(v, -463.0, 463.0).astype(np.float32)   # torch does not saturate above that
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(orc.e4m3_encode(v), ref)
+
+
+def test_quantize_weights_fp8_per_channel():
+    rng = np.random.default_rng(9)
+    E, K, M = 3, 64, 48
+    w = (rng.standard_normal((E, K, M)) * rng.uniform(1e-3, 5, size=(1, 1, M))).astype(np.float32)
+    w[1, :, 7] = 0.0                                     # an all-zero column
+    q, scale = orc.quantize_weights_fp8(w)
+    assert q.dtype == np.uint8 and scale.dtype == np.float32 and scale.shape == (E, M)
+    assert scale[1, 7] == 1.0 and np.all(q[1, :, 7] == 0)
+    deq = orc.dequantize_weights_fp8(q, scale)
+    amax = np.abs(w).max(axis=1)
+    # each column's largest element lands on +-448 (code 0x7E) and stays within rounding of itself
+    for e in range(E):
+        for m in range(M):
+            if amax[e, m] > 0:
+                assert np.abs(orc.e4m3_decode(q[e, :, m])).max() == 448.0
+    # error bound: half an e4m3 step at the element's magnitude (relative 2^-4 for normals,
+    # 2^-10 * scale below the normal range), plus the float32 division's rounding
+    a = np.abs(w.astype(np.float64))
+    bound = np.maximum(a * 2.0 ** -4, 2.0 ** -10 * scale[:, None, :]) * (1 + 1e-6)
+    assert np.all(np.abs(deq - w) <= bound)
