@@ -56,6 +56,7 @@ _P = ctypes.c_void_p
 def _signatures(lib):
     S = ctypes.POINTER(MoeShape)
     O = ctypes.POINTER(MoeLayerOpts)
+    i64 = ctypes.c_int64
     st = ctypes.c_int
     sz = ctypes.c_size_t
     table = {
@@ -77,6 +78,9 @@ def _signatures(lib):
         "moe_combine_ex": (st, [S, O, _P, _P, _P, _P, _P]),
         "moe_layer_forward_ex": (st, [S, O, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, sz,
                                       _P]),
+        "moe_quantize_weights_fp8": (st, [_P, i64, i64, i64, _P, _P, _P]),
+        "moe_grouped_ffn_w8": (st, [S] + [_P] * 11 + [sz, _P]),
+        "moe_layer_forward_w8": (st, [S, O] + [_P] * 16 + [sz, _P]),
     }
     for name, (res, args) in table.items():
         f = getattr(lib, name)
@@ -242,6 +246,32 @@ def moe_layer_forward_ex(shape, opts, x, w_router, logit_bias, w_gate, w_up, w_d
                                    ptr(logit_bias), ptr(w_gate), ptr(w_up), ptr(w_down), ptr(out),
                                    ptr(logits_out), ptr(topk_idx), ptr(topk_w), ptr(counts),
                                    ptr(drop_mask), ptr(ws), int(ws_bytes), _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_quantize_weights_fp8(w, E, K, M, codes, scale, stream=None, check=True):
+    s = lib().moe_quantize_weights_fp8(ptr(w), int(E), int(K), int(M), ptr(codes), ptr(scale),
+                                       _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_grouped_ffn_w8(shape, x, sorted_ids, offsets, q_gate, q_up, q_down, s_gate, s_up, s_down,
+                       y_slots, ws, ws_bytes, stream=None, check=True):
+    s = lib().moe_grouped_ffn_w8(ctypes.byref(shape), ptr(x), ptr(sorted_ids), ptr(offsets),
+                                 ptr(q_gate), ptr(q_up), ptr(q_down), ptr(s_gate), ptr(s_up),
+                                 ptr(s_down), ptr(y_slots), ptr(ws), int(ws_bytes),
+                                 _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_layer_forward_w8(shape, opts, x, w_router, logit_bias, q_gate, q_up, q_down, s_gate,
+                         s_up, s_down, out, logits_out, topk_idx, topk_w, counts, drop_mask, ws,
+                         ws_bytes, stream=None, check=True):
+    s = lib().moe_layer_forward_w8(ctypes.byref(shape), _opts(opts), ptr(x), ptr(w_router),
+                                   ptr(logit_bias), ptr(q_gate), ptr(q_up), ptr(q_down),
+                                   ptr(s_gate), ptr(s_up), ptr(s_down), ptr(out), ptr(logits_out),
+                                   ptr(topk_idx), ptr(topk_w), ptr(counts), ptr(drop_mask),
+                                   ptr(ws), int(ws_bytes), _stream(stream))
     return _check(s) if check else s
 
 

@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmoe.so")
 SOURCES = ["moe_api.cu", "route.cu", "route_tc.cu", "align.cu", "combine.cu", "ffn_simt.cu",
-           "ffn_tc.cu"]
+           "ffn_tc.cu", "quant.cu"]
 HEADERS = ["common.cuh", "internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -24,6 +24,9 @@
 //   * Every mbarrier wait is bounded; on timeout the CTA raises an error word and winds down.
 #include <mutex>
 
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -60,8 +63,10 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiChunks = 4;
 constexpr int kMaxTokenBlock = 256;
 constexpr int kGatherWarp0 = 2 + kEpiWarps;
-template <int BMODE>
-constexpr int threads_of() { return 32 * (kGatherWarp0 + (BMODE == kBCpAsync ? 4 : 0)); }
+// W8: FP8 (e4m3) weights, converted to bf16 in shared memory by four converter warps
+// (warps 10-13) before the bf16 MMA; the per-channel scale is applied in the epilogue.
+template <int BMODE, bool W8 = false>
+constexpr int threads_of() { return 32 * (kGatherWarp0 + ((BMODE == kBCpAsync || W8) ? 4 : 0)); }
 
 // Token rows of B one CTA keeps per stage: all TB, or the half it holds in a CTA pair (rounded
 // up to whole 32-row TMA boxes).
@@ -89,6 +94,9 @@ struct TcParams {
   int nbuf;       // TMEM accumulator buffers (1 or 2, 256 columns apart)
   int a_wide;     // A maps are 4-D: one box = all 64-feature chunks of a CTA's feature rows
   int b_box_rows; // rows per B box (contiguous-rows mode)
+  const float* scale0;  // W8: per-channel scales [groups][scale_ld] of A0 (gate, or down)
+  const float* scale1;  // W8: of A1 (up)
+  int scale_ld;
 };
 
 struct Tile {
@@ -127,6 +135,17 @@ __device__ __forceinline__ Tile decode_tile(int tile, int num_fb, int groups, in
 // SiLU itself is below 1e-35 in magnitude.
 __device__ __forceinline__ float silu_f32(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
+// Two e4m3 codes (first in the low byte) as two bf16 (first in the low half). The hardware
+// e4m3 -> f16 conversion is exact, and so is f16 -> f32 -> bf16 for these values (at most 4
+// significant bits, exponents within bf16's range).
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t codes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes),
+                                                    __NV_E4M3);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
 // Round two floats to bf16 (nearest-even) and pack them, the first in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -142,8 +161,14 @@ __device__ __forceinline__ uint16_t bf16_half(uint32_t w, int hi) {
 // rows. B traffic per weight byte halves. Stage bookkeeping lives in the even CTA: its full[s]
 // counts both CTAs' A bytes (TMA completes there), and its tempty[b] counts both epilogues;
 // MMA completions are signalled to both CTAs at once (commit with a two-CTA mask).
-template <int MODE, int BMODE, bool PAIR>
-__global__ void __launch_bounds__(threads_of<BMODE>(), 1)
+//
+// W8: A arrives as e4m3 boxes (128 features x 64 K, one byte each) in the stage ring; the
+// converter warps rewrite each stage's A as bf16 into a two-slot ring in the layout the bf16
+// TMA boxes have (MN-major, 128-byte swizzle), and the MMA reads A from there. Every e4m3 value
+// is exactly a bf16 value, so the MMA sees decode(code) exactly; the channel scale multiplies
+// the fp32 accumulator in the epilogue.
+template <int MODE, int BMODE, bool PAIR, bool W8 = false>
+__global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
     tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0,
                     const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB, const TcParams p) {
@@ -153,6 +178,7 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
   // full[s] arrivals: the producer's expect_tx (+ one completion-tracked arrival per cp.async
   // gatherer thread). Pairs stream B by TMA only.
   static_assert(!(PAIR && BMODE != kBTiled), "CTA pairs take the B operand by TMA boxes");
+  static_assert(!(W8 && (PAIR || BMODE != kBTiled)), "FP8 weights: single CTAs, TMA-streamed B");
   constexpr uint32_t kFullCount = 1u + (kCp ? 128u : 0u);
   // one arrival per epilogue warp (both CTAs' warps in PAIR mode)
   constexpr uint32_t kTemptyCount = PAIR ? 2u * kEpiWarps : kEpiWarps;
@@ -161,10 +187,12 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int a_bytes = kDual ? 32768 : 16384;
-  const int stage_bytes = a_bytes + b_rows_smem(PAIR, p.TB) * 128;
+  const int a_bytes = kDual ? 32768 : 16384;         // bf16 A of one k-block, as the MMA reads it
+  constexpr int a8_bytes = kDual ? 16384 : 8192;     // W8: the same A as e4m3 codes
+  const int stage_bytes = (W8 ? a8_bytes : a_bytes) + b_rows_smem(PAIR, p.TB) * 128;
   const int S = p.stages;
-  uint8_t* ctrl = smem + static_cast<size_t>(S) * stage_bytes;
+  uint8_t* a16 = smem + static_cast<size_t>(S) * stage_bytes;  // W8: two bf16 A slots
+  uint8_t* ctrl = a16 + (W8 ? 2 * a_bytes : 0);
   uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
   uint64_t* empty = full + kMaxStages;
   uint64_t* tfull = empty + kMaxStages;
@@ -172,6 +200,8 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  uint64_t* cfull = reinterpret_cast<uint64_t*>(ctrl + 176);  // W8: bf16 slot written
+  uint64_t* cempty = cfull + 2;                                // W8: bf16 slot consumed
   int* s_off = reinterpret_cast<int*>(ctrl + 256);
   int* s_blk = s_off + (kMaxGroups + 1);
 
@@ -191,6 +221,12 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
       mbar_init(smem_u32(&tempty[b]), kTemptyCount);
     }
     mbar_init(smem_u32(drain), 1);
+    if constexpr (W8) {
+      for (int j = 0; j < 2; ++j) {
+        mbar_init(smem_u32(&cfull[j]), 4);  // one arrival per converter warp
+        mbar_init(smem_u32(&cempty[j]), 1);
+      }
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -247,7 +283,8 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
       }
       const int m0 = t.fb * kTileFeatures + static_cast<int>(rank) * kCtaFeatures;
       const bool hi_chunk = p.a_wide || (m0 + 64) < p.m_rows_a;
-      uint32_t tx = (hi_chunk ? 16384u : 8192u) * (kDual ? 2u : 1u);
+      uint32_t tx = W8 ? static_cast<uint32_t>(a8_bytes)
+                       : (hi_chunk ? 16384u : 8192u) * (kDual ? 2u : 1u);
       if constexpr (BMODE == kBGather4) tx += static_cast<uint32_t>(npad) * 128u;
       if constexpr (BMODE == kBTiled)
         tx += static_cast<uint32_t>(nbox) * static_cast<uint32_t>(p.b_box_rows) * 128u;
@@ -264,8 +301,19 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
           break;
         }
         const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
-        const uint32_t sb = sa + a_bytes;
-        if constexpr (PAIR) {
+        const uint32_t sb = sa + (W8 ? a8_bytes : a_bytes);
+        if constexpr (W8) {
+          // e4m3 boxes of 128 features x 64 K per weight operand, then the token rows
+          const uint32_t fbar = smem_u32(&full[s]);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(fbar, tx);
+            tma_load_3d(sa, &tmA0, m0, kb * kBK, t.group, fbar);
+            if constexpr (kSwiGLU) tma_load_3d(sa + 8192, &tmA1, m0, kb * kBK, t.group, fbar);
+            else if constexpr (kDual) tma_load_3d(sa + 8192, &tmA0, m0 + 128, kb * kBK, t.group, fbar);
+            tma_load_2d(sb, &tmB, kb * kBK, brow0, fbar);
+          }
+          __syncwarp();
+        } else if constexpr (PAIR) {
           const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
           if (lane == 0 && p.a_wide) {
             // one box per weight operand: all feature chunks of this CTA's rows
@@ -350,9 +398,11 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
       constexpr uint32_t kFull = 0xffffffffu;
       const uint32_t S = static_cast<uint32_t>(p.stages);
       const uint32_t sbase = smem_u32(smem);
-      const uint64_t adesc0 = smem_desc_sw128(sbase, 8192, 1024);
-      const uint64_t bdesc0 = smem_desc_sw128(sbase + a_bytes, 16, 1024);
+      // W8: A comes from the bf16 slots; the stage ring holds the e4m3 codes and B
+      const uint64_t adesc0 = smem_desc_sw128(W8 ? smem_u32(a16) : sbase, 8192, 1024);
+      const uint64_t bdesc0 = smem_desc_sw128(sbase + (W8 ? a8_bytes : a_bytes), 16, 1024);
       uint32_t s = 0, ph = 0, soff = 0;
+      uint32_t kbi = 0;  // W8: k-blocks issued (bf16 slot kbi & 1, its use count kbi >> 1)
       int tc = 0;
       bool ok = true;
       for (int tile = tile0; ok && tile < num_tiles; tile += tstep) {
@@ -377,8 +427,16 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
             ok = false;
             break;
           }
+          if constexpr (W8) {
+            if (!__all_sync(kFull, mbar_wait(smem_u32(&cfull[kbi & 1]), (kbi >> 1) & 1u,
+                                             abort_flag))) {
+              ok = false;
+              break;
+            }
+          }
           tc_fence_after();
-          const uint64_t ad = adesc0 + (soff >> 4);
+          const uint64_t ad =
+              W8 ? adesc0 + (kbi & 1) * static_cast<uint32_t>(a_bytes >> 4) : adesc0 + (soff >> 4);
           const uint64_t bd = bdesc0 + (soff >> 4);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
@@ -396,6 +454,8 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
           }
           if constexpr (PAIR) tc_commit_pair_mc_elect(smem_u32(&empty[s]), 0x3);
           else tc_commit_elect(smem_u32(&empty[s]));
+          if constexpr (W8) tc_commit_elect(smem_u32(&cempty[kbi & 1]));
+          ++kbi;
           if (++s == S) {
             s = 0;
             ph ^= 1u;
@@ -466,6 +526,69 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
       if (lane == 0) flag_error(p.err, kDevWaitTimeout);
     }
     cp_async_wait_all();
+  } else if (W8 && warp >= kGatherWarp0) {
+    // ------------------------------------------------------------ e4m3 -> bf16 converters
+    // Thread g (0..127) takes 16-byte units g, g+128, ... of the stage's e4m3 A: unit u is
+    // operand u / 512, K row (u % 512) / 8 and features 16 * (u % 8) .. +15 of that row. Each
+    // unit becomes two 16-byte bf16 units at the same K row of the 64-feature chunk holding
+    // those features, with the 128-byte swizzle (16-byte unit index XOR K row % 8) of both
+    // layouts.
+    constexpr uint32_t kFull = 0xffffffffu;
+    constexpr int kUnits = a8_bytes / 16;
+    const int g = threadIdx.x - kGatherWarp0 * 32;
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t a16base = smem_u32(a16);
+    uint32_t s = 0, ph = 0, kbi = 0;
+    bool ok = true;
+    for (int tile = tile0; ok && tile < num_tiles; tile += tstep) {
+      const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, kblocks);
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        const uint32_t j = kbi & 1u;
+        const bool got = mbar_wait(smem_u32(&full[s]), ph, abort_flag) &&
+                         mbar_wait(smem_u32(&cempty[j]), ((kbi >> 1) & 1u) ^ 1u, abort_flag);
+        if (!__all_sync(kFull, got)) {
+          ok = false;
+          break;
+        }
+        const uint32_t src0 = sbase + s * static_cast<uint32_t>(stage_bytes);
+        const uint32_t dst0 = a16base + j * static_cast<uint32_t>(a_bytes);
+#pragma unroll 2
+        for (int u = g; u < kUnits; u += 128) {
+          const int o = u >> 9, k = (u >> 3) & 63, v = u & 7;
+          uint32_t w[4];
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                       : "r"(src0 + o * 8192 + k * 128 + ((v ^ (k & 7)) << 4)));
+          uint32_t b[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            b[2 * i] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w[i] & 0xffffu));
+            b[2 * i + 1] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w[i] >> 16));
+          }
+          const uint32_t d = dst0 + o * 16384 + (v >> 2) * 8192 + k * 128;
+          const int u0 = (v & 3) * 2;
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(d + ((u0 ^ (k & 7)) << 4)),
+                       "r"(b[0]), "r"(b[1]), "r"(b[2]), "r"(b[3])
+                       : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           d + (((u0 + 1) ^ (k & 7)) << 4)),
+                       "r"(b[4]), "r"(b[5]), "r"(b[6]), "r"(b[7])
+                       : "memory");
+        }
+        fence_proxy_async_smem();  // generic-proxy writes, read next by the tensor core
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&cfull[j]));
+        ++kbi;
+        if (++s == static_cast<uint32_t>(S)) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) flag_error(p.err, kDevWaitTimeout);
+    }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..9)
     const int q = warp & 3;               // TMEM lane quadrant this warp may read
@@ -492,6 +615,16 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
       // write the rows out: the next tile's MMAs run under these stores.
       constexpr int kW = (MODE == kEpiBF16x2) ? 32 : 16;  // words held per 32-column chunk
       uint32_t pk[kEpiChunks][kW];
+      // W8: channel scales of this lane's feature rows (1 otherwise, and then unused)
+      float sc0 = 1.0f, sc1 = 1.0f;
+      if constexpr (W8) {
+        const size_t so = static_cast<size_t>(t.group) * p.scale_ld + m;
+        sc0 = p.scale0[so];
+        if constexpr (kSwiGLU) sc1 = p.scale1[so];
+        else if constexpr (kDual) sc1 = p.scale0[so + 128];
+      }
+      auto scl0 = [&](uint32_t a) { return W8 ? __uint_as_float(a) * sc0 : __uint_as_float(a); };
+      auto scl1 = [&](uint32_t a) { return W8 ? __uint_as_float(a) * sc1 : __uint_as_float(a); };
 #pragma unroll
       for (int i = 0; i < kEpiChunks; ++i) {
         const int c0 = 32 * half + 64 * i;
@@ -504,21 +637,19 @@ __global__ void __launch_bounds__(threads_of<BMODE>(), 1)
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              pk[i][j] = pack_bf16x2(
-                  silu_f32(__uint_as_float(v[2 * j])) * __uint_as_float(u[2 * j]),
-                  silu_f32(__uint_as_float(v[2 * j + 1])) * __uint_as_float(u[2 * j + 1]));
+              pk[i][j] = pack_bf16x2(silu_f32(scl0(v[2 * j])) * scl1(u[2 * j]),
+                                     silu_f32(scl0(v[2 * j + 1])) * scl1(u[2 * j + 1]));
           } else {
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              pk[i][j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+              pk[i][j] = pack_bf16x2(scl0(v[2 * j]), scl0(v[2 * j + 1]));
             if constexpr (kDual) {
               tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), v);
               tmem_wait_ld();
 #pragma unroll
               for (int j = 0; j < 16; ++j)
-                pk[i][16 + j] =
-                    pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+                pk[i][16 + j] = pack_bf16x2(scl1(v[2 * j]), scl1(v[2 * j + 1]));
             }
           }
         }
@@ -668,13 +799,36 @@ bool map_weights(CUtensorMap* m, const void* base, uint64_t mdim, uint64_t kdim,
   return r == CUDA_SUCCESS;
 }
 
-template <int MODE, int BMODE, bool PAIR>
+// e4m3 weights [G][K][M] (one byte each): box {128 features, 64 K, 1 group}, 128-byte
+// swizzle (a box row is one K index: 128 bytes).
+bool map_weights_fp8(CUtensorMap* m, const void* base, uint64_t mdim, uint64_t kdim,
+                     uint64_t groups, std::string* d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) {
+    if (d) *d = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  cuuint64_t dims[3] = {mdim, kdim, groups};
+  cuuint64_t strides[2] = {mdim, mdim * kdim};
+  cuuint32_t box[3] = {128, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && d)
+    *d = "cuTensorMapEncodeTiled(e4m3 weights) failed with code " + std::to_string(r);
+  return r == CUDA_SUCCESS;
+}
+
+template <int MODE, int BMODE, bool PAIR, bool W8 = false>
 cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                         TcParams p, int64_t tiles_ub, int num_sms, cudaStream_t stream,
                         std::string* d) {
   const int a_bytes = dual_a<MODE>() ? 32768 : 16384;
-  const int stage_bytes = a_bytes + b_rows_smem(PAIR, p.TB) * 128;
-  int stages = (kSmemLimit - 1024 - kCtrlBytes) / stage_bytes;
+  const int a8_bytes = dual_a<MODE>() ? 16384 : 8192;
+  const int stage_bytes = (W8 ? a8_bytes : a_bytes) + b_rows_smem(PAIR, p.TB) * 128;
+  const int extra = W8 ? 2 * a_bytes : 0;  // the two bf16 A slots
+  int stages = (kSmemLimit - 1024 - kCtrlBytes - extra) / stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) {
     if (d) *d = "tile too large for shared memory";
@@ -686,17 +840,17 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   }
   p.stages = stages;
   p.nbuf = ((dual_a<MODE>() ? 2 : 1) * p.TB <= 256) ? 2 : 1;
-  const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + kCtrlBytes;
+  const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + extra + kCtrlBytes;
   const int64_t units = PAIR ? num_sms / 2 : num_sms;  // CTA pairs or CTAs, one per SM
   int64_t grid = tiles_ub < units ? tiles_ub : units;
   if (grid < 1) grid = 1;
   if (PAIR) grid *= 2;
-  auto kernel = tc_grouped_gemm<MODE, BMODE, PAIR>;
+  auto kernel = tc_grouped_gemm<MODE, BMODE, PAIR, W8>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return launch_kernel(kernel, dim3(static_cast<unsigned>(grid)), dim3(threads_of<BMODE>()), smem,
-                       stream, PAIR ? 2 : 1, a0, a1, b, p);
+  return launch_kernel(kernel, dim3(static_cast<unsigned>(grid)), dim3(threads_of<BMODE, W8>()),
+                       smem, stream, PAIR ? 2 : 1, a0, a1, b, p);
 }
 
 // CTA pairs (cta_group::2) for the expert GEMMs unless the build opts out.
@@ -821,6 +975,83 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
   if (dual)
     return launch_mode<kEpiBF16x2, kBTiled, false>(a0, a0, b, p, tiles, num_sms, stream, detail);
   return launch_mode<kEpiBF16, kBTiled, false>(a0, a0, b, p, tiles, num_sms, stream, detail);
+}
+
+// ---- FP8 (e4m3) expert weights: single CTAs, B streamed by TMA from contiguous rows.
+
+cudaError_t launch_gemm1_w8(const void* xs, const int32_t* offsets, const int32_t* blk_prefix,
+                            const uint8_t* q_gate, const uint8_t* q_up, const float* s_gate,
+                            const float* s_up, void* hbuf, int64_t hbuf_rows, int H, int E,
+                            int I, int TB, int64_t ub_blocks, int* err, int num_sms,
+                            cudaStream_t stream, std::string* detail) {
+  CUtensorMap a0, a1, b;
+  if (!map_weights_fp8(&a0, q_gate, I, H, E, detail) ||
+      !map_weights_fp8(&a1, q_up, I, H, E, detail) ||
+      !map_row_boxes(&b, xs, static_cast<uint64_t>(H), static_cast<uint64_t>(hbuf_rows), detail,
+                     static_cast<uint32_t>(TB)))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.a_wide = 1;
+  p.b_box_rows = TB;
+  p.K = H;
+  p.num_fb = I / kBM;
+  p.m_rows_a = I;
+  p.m_valid = I;
+  p.TB = TB;
+  p.groups = E;
+  p.k_top = 1;
+  p.rows_b = static_cast<int>(hbuf_rows);
+  p.sorted_ids = nullptr;
+  p.offsets = offsets;
+  p.blk_prefix = blk_prefix;
+  p.out = hbuf;
+  p.ldo = I;
+  p.err = err;
+  p.b_ptr = nullptr;
+  p.scale0 = s_gate;
+  p.scale1 = s_up;
+  p.scale_ld = I;
+  const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
+  return launch_mode<kEpiSwiGLU, kBTiled, false, true>(a0, a1, b, p, tiles, num_sms, stream,
+                                                       detail);
+}
+
+cudaError_t launch_gemm2_w8(const void* hbuf, int64_t hbuf_rows, const int32_t* offsets,
+                            const int32_t* blk_prefix, const uint8_t* q_down, const float* s_down,
+                            void* y, int H, int E, int I, int TB, int64_t ub_blocks, int* err,
+                            int num_sms, cudaStream_t stream, std::string* detail) {
+  CUtensorMap a0, b;
+  const bool dual = (H % 256) == 0;
+  if (!map_weights_fp8(&a0, q_down, H, I, E, detail) ||
+      !map_row_boxes(&b, hbuf, static_cast<uint64_t>(I), static_cast<uint64_t>(hbuf_rows), detail,
+                     static_cast<uint32_t>(TB)))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.a_wide = 1;
+  p.b_box_rows = TB;
+  p.K = I;
+  p.num_fb = dual ? H / 256 : H / kBM;
+  p.m_rows_a = H;
+  p.m_valid = H;
+  p.TB = TB;
+  p.groups = E;
+  p.k_top = 1;
+  p.rows_b = static_cast<int>(hbuf_rows);
+  p.sorted_ids = nullptr;
+  p.offsets = offsets;
+  p.blk_prefix = blk_prefix;
+  p.out = y;
+  p.ldo = H;
+  p.err = err;
+  p.scale0 = s_down;
+  p.scale1 = nullptr;
+  p.scale_ld = H;
+  const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
+  if (dual)
+    return launch_mode<kEpiBF16x2, kBTiled, false, true>(a0, a0, b, p, tiles, num_sms, stream,
+                                                         detail);
+  return launch_mode<kEpiBF16, kBTiled, false, true>(a0, a0, b, p, tiles, num_sms, stream,
+                                                     detail);
 }
 
 }  // namespace moe

@@ -82,4 +82,19 @@ cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_o
                            const float* out_bias, void* out, int64_t T, int H, int k,
                            cudaStream_t stream);
 
+// ---- FP8 (e4m3) expert weights (quant.cu, ffn_tc.cu)
+// codes[e][k][m] = e4m3(w / scale[e][m]), scale[e][m] = max_k |w[e][k][m]| / 448 (w bf16 [E][K][M]).
+cudaError_t launch_quantize_fp8(const void* w, int64_t E, int K, int M, uint8_t* codes,
+                                float* scale, int num_sms, cudaStream_t stream);
+// The expert GEMMs with e4m3 weights and their per-channel scales (xs: expert-major rows).
+cudaError_t launch_gemm1_w8(const void* xs, const int32_t* offsets, const int32_t* blk_prefix,
+                            const uint8_t* q_gate, const uint8_t* q_up, const float* s_gate,
+                            const float* s_up, void* hbuf, int64_t hbuf_rows, int H, int E,
+                            int I, int TB, int64_t ub_blocks, int* err, int num_sms,
+                            cudaStream_t stream, std::string* detail);
+cudaError_t launch_gemm2_w8(const void* hbuf, int64_t hbuf_rows, const int32_t* offsets,
+                            const int32_t* blk_prefix, const uint8_t* q_down, const float* s_down,
+                            void* y, int H, int E, int I, int TB, int64_t ub_blocks, int* err,
+                            int num_sms, cudaStream_t stream, std::string* detail);
+
 }  // namespace moe

@@ -142,7 +142,7 @@ Layout layout_of(const moe_shape& s) {
   L.slot_of = take(static_cast<size_t>(L.A) * 4);
   L.hbuf = take(static_cast<size_t>(L.a_cap) * s.I * es);
   L.yslots = take(static_cast<size_t>(L.a_cap) * s.H * es);
-  L.xs = gemm1_from_copy(s) ? take(static_cast<size_t>(L.a_cap) * s.H * es) : 0;
+  L.xs = s.dtype == MOE_BF16 ? take(static_cast<size_t>(L.a_cap) * s.H * es) : 0;
   L.total = off;
   return L;
 }
@@ -249,11 +249,43 @@ moe_status do_route(const moe_shape& s, const Layout& L, const Opts& o, const vo
   return MOE_OK;
 }
 
+// Expert weights: bf16 / f32 tensors, or e4m3 codes with per-channel scales (w8).
+struct FfnWeights {
+  const void* w_gate = nullptr;
+  const void* w_up = nullptr;
+  const void* w_down = nullptr;
+  const uint8_t* q_gate = nullptr;
+  const uint8_t* q_up = nullptr;
+  const uint8_t* q_down = nullptr;
+  const float* s_gate = nullptr;
+  const float* s_up = nullptr;
+  const float* s_down = nullptr;
+  bool w8 = false;
+};
+
 moe_status do_ffn(const moe_shape& s, const Layout& L, const void* x, const int32_t* sorted_ids,
-                  const int32_t* offsets, const void* w_gate, const void* w_up, const void* w_down,
-                  void* y, void* ws, cudaStream_t st, bool stage_events) {
+                  const int32_t* offsets, const FfnWeights& fw, void* y, void* ws, cudaStream_t st,
+                  bool stage_events) {
+  const void* w_gate = fw.w_gate;
+  const void* w_up = fw.w_up;
+  const void* w_down = fw.w_down;
   cudaError_t e;
-  if (s.dtype == MOE_BF16) {
+  if (fw.w8) {
+    const int64_t ub_blocks = (s.E < L.a_cap ? s.E : L.a_cap) + L.a_cap / L.TB;
+    std::string d;
+    void* xs = at<void>(ws, L.xs);
+    e = moe::launch_dispatch_rows(s.dtype, x, sorted_ids, offsets, s.E, s.k, s.H, L.a_cap, xs, st);
+    if (e != cudaSuccess) return cuda_fail(e, "expert-major row copy");
+    e = moe::launch_gemm1_w8(xs, offsets, at<int32_t>(ws, L.blk_prefix), fw.q_gate, fw.q_up,
+                             fw.s_gate, fw.s_up, at<void>(ws, L.hbuf), L.a_cap, s.H, s.E, s.I,
+                             L.TB, ub_blocks, at<int>(ws, L.err), num_sms(), st, &d);
+    if (e != cudaSuccess) return cuda_fail(e, "expert GEMM1 (tcgen05, e4m3 weights)", d);
+    if (stage_events) record_stage(2, st);
+    e = moe::launch_gemm2_w8(at<void>(ws, L.hbuf), L.a_cap, offsets, at<int32_t>(ws, L.blk_prefix),
+                             fw.q_down, fw.s_down, y, s.H, s.E, s.I, L.TB, ub_blocks,
+                             at<int>(ws, L.err), num_sms(), st, &d);
+    if (e != cudaSuccess) return cuda_fail(e, "expert GEMM2 (tcgen05, e4m3 weights)", d);
+  } else if (s.dtype == MOE_BF16) {
     const int64_t ub_blocks = (s.E < L.a_cap ? s.E : L.a_cap) + L.a_cap / L.TB;
     std::string d;
     void* xs = nullptr;
@@ -436,7 +468,11 @@ moe_status moe_grouped_ffn(const moe_shape* shape, const void* x, const int32_t*
                                                   at<int32_t>(ws, L.blk_prefix), cs);
     if (e != cudaSuccess) return cuda_fail(e, "expert GEMM tile plan");
   }
-  return do_ffn(*shape, L, x, sorted_ids, offsets, w_gate, w_up, w_down, y_slots, ws, cs, false);
+  FfnWeights fw;
+  fw.w_gate = w_gate;
+  fw.w_up = w_up;
+  fw.w_down = w_down;
+  return do_ffn(*shape, L, x, sorted_ids, offsets, fw, y_slots, ws, cs, false);
 }
 
 moe_status moe_combine_ex(const moe_shape* shape, const moe_layer_opts* opts,
@@ -464,12 +500,15 @@ moe_status moe_combine(const moe_shape* shape, const void* y_slots, const int32_
   return moe_combine_ex(shape, nullptr, y_slots, slot_of, topk_w, out, stream);
 }
 
-moe_status moe_layer_forward_ex(const moe_shape* shape, const moe_layer_opts* opts,
-                                const void* x, const void* w_router, const float* logit_bias,
-                                const void* w_gate, const void* w_up, const void* w_down,
-                                void* out, float* logits_out, int32_t* topk_idx, float* topk_w,
-                                int32_t* counts, uint8_t* drop_mask, void* ws, size_t ws_bytes,
-                                void* stream) {
+}  // extern "C"
+
+namespace {
+
+moe_status layer_impl(const moe_shape* shape, const moe_layer_opts* opts, const void* x,
+                      const void* w_router, const float* logit_bias, const FfnWeights& fw,
+                      void* out, float* logits_out, int32_t* topk_idx, float* topk_w,
+                      int32_t* counts, uint8_t* drop_mask, void* ws, size_t ws_bytes,
+                      void* stream) {
   moe_status st = check_shape(shape);
   if (st != MOE_OK) return st;
   const moe_shape& s = *shape;
@@ -488,9 +527,19 @@ moe_status moe_layer_forward_ex(const moe_shape* shape, const moe_layer_opts* op
   }
   REQUIRE_PTR(x, "x");
   REQUIRE_PTR(w_router, "w_router");
-  REQUIRE_PTR(w_gate, "w_gate");
-  REQUIRE_PTR(w_up, "w_up");
-  REQUIRE_PTR(w_down, "w_down");
+  if (fw.w8) {
+    if (s.dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "e4m3 expert weights need bf16");
+    REQUIRE_PTR(fw.q_gate, "q_gate");
+    REQUIRE_PTR(fw.q_up, "q_up");
+    REQUIRE_PTR(fw.q_down, "q_down");
+    REQUIRE_PTR(fw.s_gate, "s_gate");
+    REQUIRE_PTR(fw.s_up, "s_up");
+    REQUIRE_PTR(fw.s_down, "s_down");
+  } else {
+    REQUIRE_PTR(fw.w_gate, "w_gate");
+    REQUIRE_PTR(fw.w_up, "w_up");
+    REQUIRE_PTR(fw.w_down, "w_down");
+  }
   REQUIRE_PTR(out, "out");
   REQUIRE_PTR(topk_idx, "topk_idx");
   REQUIRE_PTR(topk_w, "topk_w");
@@ -510,12 +559,100 @@ moe_status moe_layer_forward_ex(const moe_shape* shape, const moe_layer_opts* op
   if (e != cudaSuccess) return cuda_fail(e, "align");
   record_stage(1, cs);
   void* y = at<void>(ws, L.yslots);
-  st = do_ffn(s, L, x, sorted_ids, offsets, w_gate, w_up, w_down, y, ws, cs, true);
+  st = do_ffn(s, L, x, sorted_ids, offsets, fw, y, ws, cs, true);
   if (st != MOE_OK) return st;
   e = moe::launch_combine(s.dtype, y, slot_of, topk_w, o.shared, o.shared_factor, o.out_bias, out,
                           s.T, s.H, s.k, cs);
   if (e != cudaSuccess) return cuda_fail(e, "combine");
   record_stage(4, cs);
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_layer_forward_ex(const moe_shape* shape, const moe_layer_opts* opts,
+                                const void* x, const void* w_router, const float* logit_bias,
+                                const void* w_gate, const void* w_up, const void* w_down,
+                                void* out, float* logits_out, int32_t* topk_idx, float* topk_w,
+                                int32_t* counts, uint8_t* drop_mask, void* ws, size_t ws_bytes,
+                                void* stream) {
+  FfnWeights fw;
+  fw.w_gate = w_gate;
+  fw.w_up = w_up;
+  fw.w_down = w_down;
+  return layer_impl(shape, opts, x, w_router, logit_bias, fw, out, logits_out, topk_idx, topk_w,
+                    counts, drop_mask, ws, ws_bytes, stream);
+}
+
+moe_status moe_layer_forward_w8(const moe_shape* shape, const moe_layer_opts* opts,
+                                const void* x, const void* w_router, const float* logit_bias,
+                                const uint8_t* q_gate, const uint8_t* q_up, const uint8_t* q_down,
+                                const float* s_gate, const float* s_up, const float* s_down,
+                                void* out, float* logits_out, int32_t* topk_idx, float* topk_w,
+                                int32_t* counts, uint8_t* drop_mask, void* ws, size_t ws_bytes,
+                                void* stream) {
+  FfnWeights fw;
+  fw.q_gate = q_gate;
+  fw.q_up = q_up;
+  fw.q_down = q_down;
+  fw.s_gate = s_gate;
+  fw.s_up = s_up;
+  fw.s_down = s_down;
+  fw.w8 = true;
+  return layer_impl(shape, opts, x, w_router, logit_bias, fw, out, logits_out, topk_idx, topk_w,
+                    counts, drop_mask, ws, ws_bytes, stream);
+}
+
+moe_status moe_grouped_ffn_w8(const moe_shape* shape, const void* x, const int32_t* sorted_ids,
+                              const int32_t* offsets, const uint8_t* q_gate, const uint8_t* q_up,
+                              const uint8_t* q_down, const float* s_gate, const float* s_up,
+                              const float* s_down, void* y_slots, void* ws, size_t ws_bytes,
+                              void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "e4m3 expert weights need bf16");
+  if (shape->T == 0) return MOE_OK;
+  REQUIRE_PTR(x, "x");
+  REQUIRE_PTR(sorted_ids, "sorted_ids");
+  REQUIRE_PTR(offsets, "offsets");
+  REQUIRE_PTR(q_gate, "q_gate");
+  REQUIRE_PTR(q_up, "q_up");
+  REQUIRE_PTR(q_down, "q_down");
+  REQUIRE_PTR(s_gate, "s_gate");
+  REQUIRE_PTR(s_up, "s_up");
+  REQUIRE_PTR(s_down, "s_down");
+  REQUIRE_PTR(y_slots, "y_slots");
+  const Layout L = layout_of(*shape);
+  st = check_ws(ws, ws_bytes, L.total);
+  if (st != MOE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = moe::launch_plan_from_offsets(offsets, shape->E, L.TB,
+                                                at<int32_t>(ws, L.blk_prefix), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "expert GEMM tile plan");
+  FfnWeights fw;
+  fw.q_gate = q_gate;
+  fw.q_up = q_up;
+  fw.q_down = q_down;
+  fw.s_gate = s_gate;
+  fw.s_up = s_up;
+  fw.s_down = s_down;
+  fw.w8 = true;
+  return do_ffn(*shape, L, x, sorted_ids, offsets, fw, y_slots, ws, cs, false);
+}
+
+moe_status moe_quantize_weights_fp8(const void* w, int64_t E, int64_t K, int64_t M,
+                                    uint8_t* codes, float* scale, void* stream) {
+  if (E < 0 || K < 1 || M < 2 || M % 2 != 0 || K > (1 << 30) || M > (1 << 30))
+    return fail(MOE_ERR_INVALID_ARG, "need E >= 0, K >= 1 and an even M >= 2");
+  if (E == 0) return MOE_OK;
+  REQUIRE_PTR(w, "w");
+  REQUIRE_PTR(codes, "codes");
+  REQUIRE_PTR(scale, "scale");
+  cudaError_t e = moe::launch_quantize_fp8(w, E, static_cast<int>(K), static_cast<int>(M), codes,
+                                           scale, num_sms(), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "e4m3 weight quantisation");
   return MOE_OK;
 }
 

@@ -139,3 +139,57 @@ def layer_forward(x, w_router, w_gate, w_up, w_down, k, capacity_factor, logit_b
     res["ws"] = ws
     res["C"] = L.moe_capacity(shape)
     return res
+
+
+def quantize_fp8(w, stream=None):
+    """e4m3 codes [E,K,M] (uint8) and per-channel float32 scales [E,M] of bf16 weights [E,K,M]."""
+    E, K, M = w.shape
+    codes = torch.empty((E, K, M), dtype=torch.uint8, device=w.device)
+    scale = torch.empty((E, M), dtype=torch.float32, device=w.device)
+    L.moe_quantize_weights_fp8(w, E, K, M, codes, scale, stream)
+    return codes, scale
+
+
+class Fp8Weights:
+    """The three expert weights as e4m3 codes + scales (quantised on the device)."""
+
+    def __init__(self, w_gate, w_up, w_down, stream=None):
+        self.q_gate, self.s_gate = quantize_fp8(w_gate, stream)
+        self.q_up, self.s_up = quantize_fp8(w_up, stream)
+        self.q_down, self.s_down = quantize_fp8(w_down, stream)
+        self.E, self.H, self.I = w_gate.shape
+
+    def args(self):
+        return (self.q_gate, self.q_up, self.q_down, self.s_gate, self.s_up, self.s_down)
+
+
+def grouped_ffn_w8(x, sorted_ids, offsets, fp8, k, capacity_factor, ws=None, stream=None):
+    T, H = x.shape
+    shape = shape_of(T, H, fp8.E, k, fp8.I, capacity_factor, L.MOE_BF16)
+    ws = ws or Workspace(shape, x.device)
+    y = torch.empty((T * k, H), dtype=x.dtype, device=x.device)
+    L.moe_grouped_ffn_w8(shape, x, sorted_ids, offsets, *fp8.args(), y, ws.buf, ws.nbytes, stream)
+    return y
+
+
+def layer_forward_w8(x, w_router, fp8, k, capacity_factor, logit_bias=None, logits_out=True,
+                     ws=None, out=None, stream=None, opts=None):
+    """Whole layer with e4m3 expert weights (moe_layer_forward_w8)."""
+    T, H = x.shape
+    E = w_router.shape[1]
+    dev = x.device
+    shape = shape_of(T, H, E, k, fp8.I, capacity_factor, _dtype_code(x))
+    ws = ws or Workspace(shape, dev)
+    res = MoELayerOutputs()
+    res["out"] = out if out is not None else torch.empty((T, H), dtype=x.dtype, device=dev)
+    res["topk_idx"] = torch.empty((T, k), dtype=torch.int32, device=dev)
+    res["topk_w"] = torch.empty((T, k), dtype=torch.float32, device=dev)
+    res["counts"] = torch.empty(E, dtype=torch.int32, device=dev)
+    res["drop_mask"] = torch.empty(T * k, dtype=torch.uint8, device=dev)
+    res["logits"] = torch.empty((T, E), dtype=torch.float32, device=dev) if logits_out else None
+    L.moe_layer_forward_w8(shape, opts, x, w_router, logit_bias, *fp8.args(), res["out"],
+                           res["logits"], res["topk_idx"], res["topk_w"], res["counts"],
+                           res["drop_mask"], ws.buf, ws.nbytes, stream)
+    res["ws"] = ws
+    res["C"] = L.moe_capacity(shape)
+    return res

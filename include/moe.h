@@ -202,6 +202,39 @@ moe_status moe_layer_forward_ex(const moe_shape* shape, const moe_layer_opts* op
                                 int32_t* counts, uint8_t* drop_mask, void* ws, size_t ws_bytes,
                                 void* stream);
 
+/* ---- FP8 (e4m3) expert weights, weight-only (W8A16).
+ *
+ * [P5] section "4.3 MOE量化方案矩阵" lists W16A16, W8A8 (INT8/FP8), W4A8 and W4A16 expert GEMMs
+ * with offline weight repacking, without a numeric scheme. The reading taken: the FP8 weights
+ * of W8A8 with the 16-bit activations of W4A16. For one weight tensor w [E][K][M] (K the
+ * reduction dimension, M the output channels: K = H, M = I for gate/up; K = I, M = H for down)
+ *   scale[e][m] = max_k |w[e][k][m]| / 448 (1 for an all-zero column), float32
+ *   codes[e][k][m] = e4m3(w[e][k][m] / scale[e][m]): OCP FP8 E4M3 (bias 7, subnormals, 448 the
+ *                    largest finite value), nearest-even, saturating
+ * The expert GEMMs apply decode(codes) * scale: every e4m3 value is exactly a bf16 value, so
+ * the tensor cores see decode(codes) exactly and the scale multiplies the float32 accumulator.
+ * Halves the expert-weight bytes the layer streams. */
+
+/* Quantises bf16 weights w [E][K][M] (M even) into codes [E][K][M] (uint8, 16-byte aligned)
+ * and scale [E][M] (float32). Asynchronous on `stream`. */
+moe_status moe_quantize_weights_fp8(const void* w, int64_t E, int64_t K, int64_t M,
+                                    uint8_t* codes, float* scale, void* stream);
+
+/* moe_grouped_ffn / moe_layer_forward_ex with e4m3 expert weights (bf16 shapes only):
+ * q_gate, q_up [E][H][I] and s_gate, s_up [E][I]; q_down [E][I][H] and s_down [E][H]. */
+moe_status moe_grouped_ffn_w8(const moe_shape* shape, const void* x, const int32_t* sorted_ids,
+                              const int32_t* offsets, const uint8_t* q_gate, const uint8_t* q_up,
+                              const uint8_t* q_down, const float* s_gate, const float* s_up,
+                              const float* s_down, void* y_slots, void* ws, size_t ws_bytes,
+                              void* stream);
+moe_status moe_layer_forward_w8(const moe_shape* shape, const moe_layer_opts* opts,
+                                const void* x, const void* w_router, const float* logit_bias,
+                                const uint8_t* q_gate, const uint8_t* q_up, const uint8_t* q_down,
+                                const float* s_gate, const float* s_up, const float* s_down,
+                                void* out, float* logits_out, int32_t* topk_idx, float* topk_w,
+                                int32_t* counts, uint8_t* drop_mask, void* ws, size_t ws_bytes,
+                                void* stream);
+
 /* Synchronises `stream`, reads and clears the device error word at the start of `ws`.
  * Returns MOE_OK, MOE_ERR_DEVICE (a kernel flagged a fault; see moe_last_error_detail) or
  * MOE_ERR_CUDA. */

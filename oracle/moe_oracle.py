@@ -43,8 +43,9 @@ Readings taken where the pages are silent or disagree (each also listed in the d
   logit when a group holds one expert); the topk_group groups with the highest scores are kept
   (ties to the lower group index); the k largest logits among the kept groups' experts are
   selected with the plain top-k rule; weights are renormalised over the k as before.
-* FP8 expert weights (SURVEY's "next" row on FP8 experts; [P5] "3.4 ... MoE GEMM" lists W8A8 /
-  W4A16 quantised expert GEMMs without a scheme): weights only, e4m3 (OCP FP8: 1 sign, 4
+* FP8 expert weights ([P5] section "4.3 MOE量化方案矩阵" lists W16A16, W8A8 (INT8/FP8), W4A8
+  and W4A16 expert GEMMs with offline weight repacking, without a numeric scheme; the reading
+  taken is the FP8 weight format of W8A8 with the 16-bit activations of W4A16): weights only, e4m3 (OCP FP8: 1 sign, 4
   exponent bits with bias 7, 3 mantissa bits, subnormals, no infinities, 448 the largest
   finite value); one float32 scale per output channel, scale = max_k |W[k, m]| / 448 (1 when
   the column is all zero); code = e4m3(W / scale) rounded to nearest, ties to even, saturating

@@ -43,6 +43,22 @@ class ExpertWeights:
         return self.w.shape[0]
 
 
+class DequantExpertWeights:
+    """Expert e's matrix after the oracle's FP8 quantisation (decode(code) * scale, float64),
+    computed on demand from the seeded bf16 weights of a (device) [E, K, M] tensor."""
+
+    def __init__(self, w):
+        self.w = w
+
+    def __getitem__(self, e):
+        w = self.w[int(e)].detach().float().cpu().numpy()[None]
+        q, sc = orc.quantize_weights_fp8(w)
+        return orc.dequantize_weights_fp8(q, sc)[0]
+
+    def __len__(self):
+        return self.w.shape[0]
+
+
 def rel_err(got, ref):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)

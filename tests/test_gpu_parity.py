@@ -194,7 +194,7 @@ def test_combine(name):
 # ----------------------------------------------------------------- whole layer
 
 def compare_layer(wl, cpu_or_dev, dev, res, sample=None, seed=0, n_group=1, topk_group=1,
-                  shared=None, shared_factor=0.0, out_bias=None):
+                  shared=None, shared_factor=0.0, out_bias=None, weights=None):
     """Compare moe_layer_forward's outputs with the oracle (see module docstring of parity).
     With n_group > 1 the routing is group-limited; shared / out_bias (host numpy) add the
     combine's shared-expert and bias terms."""
@@ -251,8 +251,10 @@ def compare_layer(wl, cpu_or_dev, dev, res, sample=None, seed=0, n_group=1, topk
     if sample is not None and len(comparable) > sample:
         rng = np.random.default_rng(seed)
         comparable = sorted(rng.choice(comparable, size=sample, replace=False).tolist())
-    ref = orc.layer_forward(host["x"], host["w_router"], ExpertWeights(dev["w_gate"]),
-                            ExpertWeights(dev["w_up"]), ExpertWeights(dev["w_down"]), k,
+    if weights is None:
+        weights = (ExpertWeights(dev["w_gate"]), ExpertWeights(dev["w_up"]),
+                   ExpertWeights(dev["w_down"]))
+    ref = orc.layer_forward(host["x"], host["w_router"], weights[0], weights[1], weights[2], k,
                             wl.capacity_factor, logit_bias=host["logit_bias"], tokens=comparable,
                             n_group=n_group, topk_group=topk_group, shared=shared,
                             shared_factor=shared_factor, out_bias=out_bias)
