@@ -136,20 +136,23 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ algorithmic cost model
 
-def stage_costs(wl, counts, hbm_peak, tc_peak):
-    """Algorithmic bytes/flops per stage for one step, from the step's routing counts."""
+def stage_costs(wl, counts, hbm_peak, tc_peak, fp8_weights=False):
+    """Algorithmic bytes/flops per stage for one step, from the step's routing counts. With
+    e4m3 expert weights a weight element is 1 byte, plus a float32 scale per output channel."""
     es = 2 if wl.dtype == "bf16" else 4
     T, H, E, k, I = wl.T, wl.H, wl.E, wl.k, wl.I
     A = T * k
     a_kept = int(counts.sum())
     used = int((counts > 0).sum())
     bias = E * 4 if wl.zipf_s > 0 else 0
+    wes, ws_ = (1, 4) if fp8_weights else (es, 0)  # weight element bytes, scale bytes
     c = {
         "route": {"bytes": T * H * es + H * E * es + bias + T * k * 8, "flops": 2 * T * H * E},
         "align": {"bytes": T * k * 4 * 3 + A * (4 + 4 + 1) + E * 8, "flops": 0},
-        "gemm1": {"bytes": used * 2 * H * I * es + a_kept * H * es + a_kept * I * es,
+        "gemm1": {"bytes": used * 2 * H * I * wes + used * 2 * I * ws_ + a_kept * H * es
+                           + a_kept * I * es,
                   "flops": 4 * a_kept * H * I},
-        "gemm2": {"bytes": used * I * H * es + a_kept * I * es + a_kept * H * es,
+        "gemm2": {"bytes": used * I * H * wes + used * H * ws_ + a_kept * I * es + a_kept * H * es,
                   "flops": 2 * a_kept * I * H},
         "combine": {"bytes": a_kept * H * es + T * k * 8 + T * H * es, "flops": 2 * a_kept * H},
     }
@@ -292,10 +295,23 @@ def run_ours(args, world, rank, local):
     drop = torch.empty(wl.T * wl.k, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    fp8 = None
+    if args.weights == "fp8":
+        # e4m3 expert weights, quantised once on the device before anything is timed
+        fp8 = M.Fp8Weights(inp["w_gate"], inp["w_up"], inp["w_down"])
+        torch.cuda.synchronize()
+
+    def forward(x, o):
+        if fp8 is not None:
+            L.moe_layer_forward_w8(shape, None, x, inp["w_router"], inp["logit_bias"], *fp8.args(),
+                                   o[0], None, o[1], o[2], o[3], o[4], ws.buf, ws.nbytes, stream)
+        else:
+            L.moe_layer_forward(shape, x, inp["w_router"], inp["logit_bias"], inp["w_gate"],
+                                inp["w_up"], inp["w_down"], o[0], None, o[1], o[2], o[3], o[4],
+                                ws.buf, ws.nbytes, stream)
+
     def step(x=inp["x"]):
-        L.moe_layer_forward(shape, x, inp["w_router"], inp["logit_bias"], inp["w_gate"],
-                            inp["w_up"], inp["w_down"], out, None, idx, wts, counts, drop, ws.buf,
-                            ws.nbytes, stream)
+        forward(x, (out, idx, wts, counts, drop))
 
     for _ in range(args.warmup):
         step()
@@ -340,7 +356,8 @@ def run_ours(args, world, rank, local):
             st_ms[s] += prev.elapsed_time(ev[i][j]) / args.steps
             prev = ev[i][j]
     cnt = counts.cpu().numpy()
-    cost = stage_costs(wl, cnt, peaks["hbm_gbs"], peaks["bf16_tflops_sustained"])
+    cost = stage_costs(wl, cnt, peaks["hbm_gbs"], peaks["bf16_tflops_sustained"],
+                       fp8_weights=fp8 is not None)
     kernels = {}
     for s in STAGES:
         t = st_ms[s] * 1e-3
@@ -370,9 +387,7 @@ def run_ours(args, world, rank, local):
     outs_devs = [outs_dev, [torch.empty_like(t) for t in outs_dev]]
 
     def fwd(x, o):
-        L.moe_layer_forward(shape, x, inp["w_router"], inp["logit_bias"], inp["w_gate"],
-                            inp["w_up"], inp["w_down"], o[0], None, o[1], o[2], o[3], o[4], ws.buf,
-                            ws.nbytes, stream)
+        forward(x, o)
 
     def e2e_serial(n):
         for _ in range(n):
@@ -446,12 +461,16 @@ def run_ours(args, world, rank, local):
                    "I": wl.I, "capacity": int(L.moe_capacity(shape)),
                    "kept_assignments": int(cnt.sum()), "experts_used": int((cnt > 0).sum()),
                    "parallelism": "replicas" if world > 1 else "single-gpu",
+                   "expert_weights": ("e4m3 codes + float32 per-channel scales (W8A16)"
+                                      if fp8 is not None else wl.dtype),
                    "l2": "inputs larger than L2: %.1f GB of expert weights streamed per step"
-                         % (3 * wl.E * wl.H * wl.I * (2 if wl.dtype == "bf16" else 4) / 1e9)},
+                         % (3 * wl.E * wl.H * wl.I * (1 if fp8 is not None else
+                                                      (2 if wl.dtype == "bf16" else 4)) / 1e9)},
         "roofline": {"kernel": dom, "bound": bound, "achieved": round(ach, 1),
                      "peak": peak, "unit": unit, "frac": round(ach / peak, 3),
                      "peak_source": f"{peaks_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
-                     "traffic": recorded_traffic(dom, args.workload),
+                     "traffic": recorded_traffic(dom + ("_w8" if fp8 is not None else ""),
+                                                 args.workload),
                      "algorithmic_bytes": cost[dom]["bytes"],
                      "tensor_frac": round(cost[dom]["flops"] / t_dom / 1e12 / peaks["bf16_tflops_sustained"], 3)},
         "route_align_combine_gbs": round(rac_bytes / rac_t / 1e9, 1),
@@ -522,6 +541,8 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=0, help="override T (decode sweep)")
     ap.add_argument("--cpu-sample-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
+                    help="expert weights: the layer dtype (default) or e4m3 + per-channel scales")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
