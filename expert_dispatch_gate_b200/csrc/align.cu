@@ -26,18 +26,18 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kPerWarp = kAlignChunk / kWarps;  // 256 assignments per warp, 8 steps of 32
+constexpr int kSinglePerWarp = kAlignSingle / kWarps;  // one-block path: 256 per warp
 constexpr int kMaxE = 256;
 
 __global__ void __launch_bounds__(kThreads)
-    align_hist_kernel(const int32_t* __restrict__ idx, int64_t A, int E,
+    align_hist_kernel(const int32_t* __restrict__ idx, int64_t A, int E, int chunk,
                       int32_t* __restrict__ blk_hist, int* err) {
   pdl_enter<false>();
   __shared__ int h[kMaxE];
   for (int e = threadIdx.x; e < E; e += kThreads) h[e] = 0;
   __syncthreads();
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kAlignChunk;
-  const int64_t end = min(A, base + kAlignChunk);
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * chunk;
+  const int64_t end = min(A, base + chunk);
   for (int64_t a = base + threadIdx.x; a < end; a += kThreads) {
     const int e = idx[a];
     if (e >= 0 && e < E) atomicAdd(&h[e], 1);
@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 __global__ void __launch_bounds__(kThreads)
-    align_scatter_kernel(const int32_t* __restrict__ idx, int64_t A, int E, int C,
+    align_scatter_kernel(const int32_t* __restrict__ idx, int64_t A, int E, int C, int chunk,
                          const int32_t* __restrict__ blk_base, const int32_t* __restrict__ offsets,
                          int32_t* __restrict__ sorted_ids, int32_t* __restrict__ slot_of,
                          uint8_t* __restrict__ drop_mask) {
@@ -125,10 +125,11 @@ __global__ void __launch_bounds__(kThreads)
   for (int i = threadIdx.x; i < kWarps * kMaxE; i += kThreads) (&wrun[0][0])[i] = 0;
   for (int e = threadIdx.x; e < E; e += kThreads) s_off[e] = offsets[e];
   __syncthreads();
-  const int64_t wbase = static_cast<int64_t>(blockIdx.x) * kAlignChunk + warp * kPerWarp;
+  const int per_warp = chunk / kWarps;  // a multiple of 32
+  const int64_t wbase = static_cast<int64_t>(blockIdx.x) * chunk + warp * per_warp;
 
-  // pass 1: per-warp per-expert counts of this warp's 256 assignments
-  for (int step = 0; step < kPerWarp / 32; ++step) {
+  // pass 1: per-warp per-expert counts of this warp's assignments
+  for (int step = 0; step < per_warp / 32; ++step) {
     const int64_t a = wbase + step * 32 + lane;
     const int e = (a < A) ? idx[a] : -1;
     const bool ok = (e >= 0 && e < E);
@@ -149,7 +150,7 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
   // pass 2: stable ranks in assignment order
-  for (int step = 0; step < kPerWarp / 32; ++step) {
+  for (int step = 0; step < per_warp / 32; ++step) {
     const int64_t a = wbase + step * 32 + lane;
     const bool in = a < A;
     const int e = in ? idx[a] : -1;
@@ -179,7 +180,7 @@ __global__ void __launch_bounds__(kThreads)
     sorted_ids[s] = -1;
 }
 
-// Whole grouping in one block when every assignment fits one chunk (A <= kAlignChunk): the
+// Whole grouping in one block when every assignment fits one chunk (A <= kAlignSingle): the
 // histogram, scan and stable scatter of the three kernels above, without two launches.
 __global__ void __launch_bounds__(kThreads)
     align_single_chunk_kernel(const int32_t* __restrict__ idx, int64_t A, int E, int C, int TB,
@@ -194,9 +195,9 @@ __global__ void __launch_bounds__(kThreads)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kWarps * kMaxE; i += kThreads) (&wrun[0][0])[i] = 0;
   __syncthreads();
-  const int64_t wbase = static_cast<int64_t>(warp) * kPerWarp;
+  const int64_t wbase = static_cast<int64_t>(warp) * kSinglePerWarp;
   // per-warp per-expert counts
-  for (int step = 0; step < kPerWarp / 32; ++step) {
+  for (int step = 0; step < kSinglePerWarp / 32; ++step) {
     const int64_t a = wbase + step * 32 + lane;
     const int e = (a < A) ? idx[a] : -1;
     const bool ok = (e >= 0 && e < E);
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
   // stable ranks in assignment order, then the scatter
-  for (int step = 0; step < kPerWarp / 32; ++step) {
+  for (int step = 0; step < kSinglePerWarp / 32; ++step) {
     const int64_t a = wbase + step * 32 + lane;
     const bool in = a < A;
     const int ea = in ? idx[a] : -1;
@@ -281,19 +282,20 @@ cudaError_t launch_align(const int32_t* topk_idx, int64_t A, int E, int C, int T
                          int32_t* blk_prefix, int32_t* sorted_ids, int32_t* slot_of,
                          uint8_t* drop_mask, int* err, cudaStream_t stream) {
   if (A == 0) return cudaSuccess;
-  const int nblk = static_cast<int>((A + kAlignChunk - 1) / kAlignChunk);
-  if (nblk == 1)
+  if (A <= kAlignSingle)
     return launch_kernel(align_single_chunk_kernel, dim3(1), dim3(kThreads), 0, stream, 1,
                          topk_idx, A, E, C, TB, counts, offsets, blk_prefix, sorted_ids, slot_of,
                          drop_mask, err);
+  const int chunk = align_chunk(A);
+  const int nblk = static_cast<int>((A + chunk - 1) / chunk);
   cudaError_t e = launch_kernel(align_hist_kernel, dim3(nblk), dim3(kThreads), 0, stream, 1,
-                                topk_idx, A, E, blk_hist, err);
+                                topk_idx, A, E, chunk, blk_hist, err);
   if (e == cudaSuccess)
     e = launch_kernel(align_scan_kernel, dim3(1), dim3(kThreads), 0, stream, 1, blk_hist, nblk, E,
                       C, TB, counts, offsets, blk_prefix);
   if (e == cudaSuccess)
     e = launch_kernel(align_scatter_kernel, dim3(nblk), dim3(kThreads), 0, stream, 1, topk_idx, A,
-                      E, C, blk_hist, offsets, sorted_ids, slot_of, drop_mask);
+                      E, C, chunk, blk_hist, offsets, sorted_ids, slot_of, drop_mask);
   return e;
 }
 
@@ -309,7 +311,7 @@ namespace {
 struct NoAllocScratch {
   int err[64];
   int blk_prefix[320];
-  int blk_hist[(kNoAllocMaxAssignments / kAlignChunk) * 256];
+  int blk_hist[kNoAllocMaxBlocks * 256];
 };
 static __device__ __align__(256) NoAllocScratch g_noalloc_scratch;
 
@@ -321,6 +323,8 @@ cudaError_t launch_align_noalloc(const int32_t* topk_idx, int64_t A, int E, int 
                                  int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
                                  int32_t* slot_of, uint8_t* drop_mask, cudaStream_t stream) {
   if (A > kNoAllocMaxAssignments || E > 256) return cudaErrorInvalidValue;
+  if (A > kAlignSingle && (A + align_chunk(A) - 1) / align_chunk(A) > kNoAllocMaxBlocks)
+    return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

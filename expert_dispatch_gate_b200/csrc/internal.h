@@ -57,7 +57,19 @@ cudaError_t launch_gemm2_simt(const float* hbuf, const int32_t* offsets, const f
                               float* y, int64_t A, int H, int E, int I, cudaStream_t stream);
 
 // ---- align.cu
-constexpr int kAlignChunk = 2048;  // assignments per align block
+// Grouping: one block does everything up to kAlignSingle assignments; above that the
+// histogram / scatter blocks take align_chunk(A) assignments each (a multiple of 256 between
+// kAlignChunkMin and kAlignChunkMax, aiming at about 128 blocks).
+constexpr int kAlignSingle = 2048;
+constexpr int kAlignChunkMin = 512;
+constexpr int kAlignChunkMax = 2048;
+inline int align_chunk(int64_t A) {
+  int64_t c = (A + 127) / 128;
+  c = (c + 255) / 256 * 256;
+  if (c < kAlignChunkMin) c = kAlignChunkMin;
+  if (c > kAlignChunkMax) c = kAlignChunkMax;
+  return static_cast<int>(c);
+}
 cudaError_t launch_align(const int32_t* topk_idx, int64_t A, int E, int C, int TB,
                          int32_t* blk_hist, int32_t* counts, int32_t* offsets,
                          int32_t* blk_prefix, int32_t* sorted_ids, int32_t* slot_of,
@@ -65,6 +77,11 @@ cudaError_t launch_align(const int32_t* topk_idx, int64_t A, int E, int C, int T
 // Same grouping with its scratch in a file-scope device array instead of a workspace;
 // at most kNoAllocMaxAssignments assignments and 256 experts.
 constexpr int64_t kNoAllocMaxAssignments = 262144;
+// align_chunk(A) >= ceil(A / 128) up to 128 * kAlignChunkMax = 262144 assignments, so the
+// grouping of at most kNoAllocMaxAssignments uses at most 128 chunk histograms.
+constexpr int kNoAllocMaxBlocks = 128;
+static_assert(kNoAllocMaxAssignments <= int64_t{kNoAllocMaxBlocks} * kAlignChunkMax,
+              "the no-allocation scratch holds 128 chunk histograms");
 cudaError_t launch_align_noalloc(const int32_t* topk_idx, int64_t A, int E, int C, int TB,
                                  int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
                                  int32_t* slot_of, uint8_t* drop_mask, cudaStream_t stream);

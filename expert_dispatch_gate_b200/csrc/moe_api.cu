@@ -123,7 +123,7 @@ Layout layout_of(const moe_shape& s) {
   L.A = s.T * s.k;
   const int64_t ec = static_cast<int64_t>(s.E) * L.C;
   L.a_cap = L.A < ec ? L.A : ec;
-  L.nblk = static_cast<int>((L.A + moe::kAlignChunk - 1) / moe::kAlignChunk);
+  L.nblk = static_cast<int>((L.A + moe::align_chunk(L.A) - 1) / moe::align_chunk(L.A));
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
