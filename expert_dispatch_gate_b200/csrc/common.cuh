@@ -147,13 +147,6 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // Row gather: four rows (r0..r3) of a 2-D tensor whose box is {box_cols, 1}, starting at
 // column `col`, written as four consecutive box rows at dst.
@@ -298,16 +291,6 @@ __device__ __forceinline__ void cluster_sync_all() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// 3-D tiled load into this CTA's shared memory whose completion is counted on an mbarrier of
-// either CTA of the pair (`bar` is a shared::cluster address).
-__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, int c0,
-                                                 int c1, int c2, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
-      : "memory");
-}
 __device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap* map, int c0,
                                                  int c1, int c2, int c3, uint32_t bar) {
   asm volatile(
@@ -360,9 +343,6 @@ __device__ __forceinline__ void tc_commit_pair_mc_elect(uint32_t bar, uint16_t c
 
 // ------------------------------------------------------------------ misc
 
-__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
-  return __uint_as_float(static_cast<uint32_t>(b) << 16);
-}
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;

@@ -35,7 +35,6 @@ namespace {
 
 constexpr int kBM = 128;        // MMA M: output features per tile
 constexpr int kBK = 64;         // K per pipeline stage: one 128-byte swizzle row of bf16
-constexpr int kRowBox = 32;     // rows per 2-D TMA box of B in the contiguous-rows mode
 constexpr int kMaxStages = 8;
 constexpr int kMaxGroups = 256;
 constexpr int kTmemCols = 512;
@@ -77,7 +76,6 @@ __host__ __device__ constexpr int b_rows_smem(bool pair, int TB) {
 struct TcParams {
   int K;          // reduction length (multiple of 64)
   int num_fb;     // feature blocks of 128
-  int m_rows_a;   // extent of A along M (a 64-wide chunk starting past it is not loaded)
   int m_valid;    // features stored by the epilogue
   int TB;         // max tokens per tile, multiple of 32, <= 256
   int groups;     // experts
@@ -92,7 +90,6 @@ struct TcParams {
   int* err;
   int stages;
   int nbuf;       // TMEM accumulator buffers (1 or 2, 256 columns apart)
-  int a_wide;     // A maps are 4-D: one box = all 64-feature chunks of a CTA's feature rows
   int b_box_rows; // rows per B box (contiguous-rows mode)
   const float* scale0;  // W8: per-channel scales [groups][scale_ld] of A0 (gate, or down)
   const float* scale1;  // W8: of A1 (up)
@@ -266,8 +263,6 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
     for (int tile = tile0; ok && tile < num_tiles; tile += tstep) {
       const Tile t = decode_tile(tile, p.num_fb, groups, p.TB, s_off, s_blk, kblocks);
       const int npad = (t.n + 15) & ~15;
-      const int bn = b_rows(npad);
-      const int nbox = p.a_wide ? 1 : (bn + kRowBox - 1) / kRowBox;
       int rows[8];
       if constexpr (BMODE == kBGather4) {
 #pragma unroll
@@ -282,12 +277,11 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
         }
       }
       const int m0 = t.fb * kTileFeatures + static_cast<int>(rank) * kCtaFeatures;
-      const bool hi_chunk = p.a_wide || (m0 + 64) < p.m_rows_a;
-      uint32_t tx = W8 ? static_cast<uint32_t>(a8_bytes)
-                       : (hi_chunk ? 16384u : 8192u) * (kDual ? 2u : 1u);
+      // A: one box per weight operand (all feature chunks of this CTA's rows); B: one box of
+      // b_box_rows token rows, or npad gathered rows
+      uint32_t tx = static_cast<uint32_t>(W8 ? a8_bytes : a_bytes);
       if constexpr (BMODE == kBGather4) tx += static_cast<uint32_t>(npad) * 128u;
-      if constexpr (BMODE == kBTiled)
-        tx += static_cast<uint32_t>(nbox) * static_cast<uint32_t>(p.b_box_rows) * 128u;
+      if constexpr (BMODE == kBTiled) tx += static_cast<uint32_t>(p.b_box_rows) * 128u;
       if constexpr (PAIR) tx *= 2u;  // both CTAs' loads complete on the even CTA's barrier
       const int brow0 = t.row0 + b_first(npad);
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
@@ -315,53 +309,20 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
           __syncwarp();
         } else if constexpr (PAIR) {
           const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
-          if (lane == 0 && p.a_wide) {
-            // one box per weight operand: all feature chunks of this CTA's rows
+          if (lane == 0) {
             if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), tx);
             tma_load_4d_pair(sa, &tmA0, 0, kb * kBK, m0 >> 6, t.group, fbar);
             if constexpr (kSwiGLU) tma_load_4d_pair(sa + 16384, &tmA1, 0, kb * kBK, m0 >> 6, t.group, fbar);
-            if constexpr (BMODE == kBTiled)
-              tma_load_2d_pair(sb, &tmB, kb * kBK, brow0, fbar);
-          } else if (lane == 0) {
-            if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), tx);
-            tma_load_3d_pair(sa, &tmA0, m0, kb * kBK, t.group, fbar);
-            if (hi_chunk) tma_load_3d_pair(sa + 8192, &tmA0, m0 + 64, kb * kBK, t.group, fbar);
-            if constexpr (kSwiGLU) {
-              tma_load_3d_pair(sa + 16384, &tmA1, m0, kb * kBK, t.group, fbar);
-              if (hi_chunk)
-                tma_load_3d_pair(sa + 16384 + 8192, &tmA1, m0 + 64, kb * kBK, t.group, fbar);
-            } else if constexpr (kDual) {
-              tma_load_3d_pair(sa + 16384, &tmA0, m0 + 128, kb * kBK, t.group, fbar);
-              tma_load_3d_pair(sa + 16384 + 8192, &tmA0, m0 + 192, kb * kBK, t.group, fbar);
-            }
-            if constexpr (BMODE == kBTiled)
-              for (int j = 0; j < nbox; ++j)
-                tma_load_2d_pair(sb + j * (kRowBox * 128), &tmB, kb * kBK, brow0 + j * kRowBox,
-                                 fbar);
+            tma_load_2d_pair(sb, &tmB, kb * kBK, brow0, fbar);
           }
           __syncwarp();
         } else {
           const uint32_t fbar = smem_u32(&full[s]);
-          if (lane == 0 && p.a_wide) {
+          if (lane == 0) {
             mbar_arrive_expect_tx(fbar, tx);
             tma_load_4d(sa, &tmA0, 0, kb * kBK, m0 >> 6, t.group, fbar);
             if constexpr (kSwiGLU) tma_load_4d(sa + 16384, &tmA1, 0, kb * kBK, m0 >> 6, t.group, fbar);
             if constexpr (BMODE == kBTiled) tma_load_2d(sb, &tmB, kb * kBK, brow0, fbar);
-          } else if (lane == 0) {
-            mbar_arrive_expect_tx(fbar, tx);
-            tma_load_3d(sa, &tmA0, m0, kb * kBK, t.group, fbar);
-            if (hi_chunk) tma_load_3d(sa + 8192, &tmA0, m0 + 64, kb * kBK, t.group, fbar);
-            if constexpr (kSwiGLU) {
-              tma_load_3d(sa + 16384, &tmA1, m0, kb * kBK, t.group, fbar);
-              if (hi_chunk)
-                tma_load_3d(sa + 16384 + 8192, &tmA1, m0 + 64, kb * kBK, t.group, fbar);
-            } else if constexpr (kDual) {
-              tma_load_3d(sa + 16384, &tmA0, m0 + 128, kb * kBK, t.group, fbar);
-              tma_load_3d(sa + 16384 + 8192, &tmA0, m0 + 192, kb * kBK, t.group, fbar);
-            }
-            if constexpr (BMODE == kBTiled)
-              for (int j = 0; j < nbox; ++j)
-                tma_load_2d(sb + j * (kRowBox * 128), &tmB, kb * kBK, brow0 + j * kRowBox, fbar);
           }
           __syncwarp();
           if constexpr (BMODE == kBGather4) {
@@ -740,9 +701,9 @@ bool map_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, st
   return r == CUDA_SUCCESS;
 }
 
-// bf16 [rows, cols] row-major, box = {64 columns, 32 rows}, 128-byte swizzle: contiguous rows.
+// bf16 [rows, cols] row-major, box = {64 columns, box_rows rows}, 128-byte swizzle: contiguous rows.
 bool map_row_boxes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, std::string* d,
-                   uint32_t box_rows = kRowBox) {
+                   uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) {
     if (d) *d = "cuTensorMapEncodeTiled is not available from the driver";
@@ -780,24 +741,6 @@ bool map_weights_wide(CUtensorMap* m, const void* base, uint64_t mdim, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
-// bf16 [groups, kdim, mdim] (mdim contiguous), box = {64, 64, 1}, 128-byte swizzle.
-bool map_weights(CUtensorMap* m, const void* base, uint64_t mdim, uint64_t kdim, uint64_t groups,
-                 std::string* d) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) {
-    if (d) *d = "cuTensorMapEncodeTiled is not available from the driver";
-    return false;
-  }
-  cuuint64_t dims[3] = {mdim, kdim, groups};
-  cuuint64_t strides[2] = {mdim * 2, mdim * kdim * 2};
-  cuuint32_t box[3] = {64, 64, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS && d) *d = "cuTensorMapEncodeTiled(weights) failed with code " + std::to_string(r);
-  return r == CUDA_SUCCESS;
-}
 
 // e4m3 weights [G][K][M] (one byte each): box {128 features, 64 K, 1 group}, 128-byte
 // swizzle (a box row is one K index: 128 bytes).
@@ -886,11 +829,9 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
                        static_cast<uint32_t>(box_rows)))
       return cudaErrorInvalidValue;
     TcParams p{};
-    p.a_wide = 1;
     p.b_box_rows = box_rows;
     p.K = H;
     p.num_fb = pair ? (I + 255) / 256 : I / kBM;
-    p.m_rows_a = I;
     p.m_valid = I;
     p.TB = TB;
     p.groups = E;
@@ -916,11 +857,9 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
   const bool use_gather4 = false;  // cp.async row gather
 #endif
   TcParams p{};
-  p.a_wide = 1;
   p.b_box_rows = 0;
   p.K = H;
   p.num_fb = I / kBM;
-  p.m_rows_a = I;
   p.m_valid = I;
   p.TB = TB;
   p.groups = E;
@@ -953,11 +892,9 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
                      static_cast<uint32_t>(box_rows)))
     return cudaErrorInvalidValue;
   TcParams p{};
-  p.a_wide = 1;
   p.b_box_rows = box_rows;
   p.K = I;
   p.num_fb = pair ? (H + 511) / 512 : (dual ? H / 256 : H / kBM);
-  p.m_rows_a = H;
   p.m_valid = H;
   p.TB = TB;
   p.groups = E;
@@ -991,11 +928,9 @@ cudaError_t launch_gemm1_w8(const void* xs, const int32_t* offsets, const int32_
                      static_cast<uint32_t>(TB)))
     return cudaErrorInvalidValue;
   TcParams p{};
-  p.a_wide = 1;
   p.b_box_rows = TB;
   p.K = H;
   p.num_fb = I / kBM;
-  p.m_rows_a = I;
   p.m_valid = I;
   p.TB = TB;
   p.groups = E;
@@ -1027,11 +962,9 @@ cudaError_t launch_gemm2_w8(const void* hbuf, int64_t hbuf_rows, const int32_t* 
                      static_cast<uint32_t>(TB)))
     return cudaErrorInvalidValue;
   TcParams p{};
-  p.a_wide = 1;
   p.b_box_rows = TB;
   p.K = I;
   p.num_fb = dual ? H / 256 : H / kBM;
-  p.m_rows_a = H;
   p.m_valid = H;
   p.TB = TB;
   p.groups = E;
