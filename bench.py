@@ -8,6 +8,11 @@ moe_layer_forward (route -> align -> GEMM1 -> GEMM2 -> combine) over the whole b
 
 N > 1 runs under torchrun as independent replicas (one process per GPU, no data-path
 collective); timing is the max over ranks. Rank 0 prints one JSON line.
+
+    python bench.py --sweep route-align-combine --workload skewed [--sweep-tokens 4096,...]
+
+times the router, the grouping and the combine alone over a range of T (one GPU) and prints
+one JSON line with each stage's HBM GB/s.
 """
 from __future__ import annotations
 
@@ -267,10 +272,10 @@ def oracle_baseline(wl, dev, n_tokens, reps=1):
 
 def launches_per_step(wl):
     """Kernels one moe_layer_forward launches: router (tensor-core GEMM + top-k, or one fused
-    CUDA-core kernel), align (one kernel up to 2048 assignments, else three), two expert
+    CUDA-core kernel), align (one launch up to 65536 assignments, else three), two expert
     GEMMs, combine."""
     route = 2 if (wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0) else 1
-    align = 1 if wl.T * wl.k <= 2048 else 3
+    align = 1 if wl.T * wl.k <= 65536 else 3
     # expert-major copy of the token rows before GEMM1 (when CTA pairs run GEMM1)
     copy = 1 if (wl.dtype == "bf16" and wl.I % 256 == 0) else 0
     return route + align + copy + 2 + 1
@@ -490,6 +495,91 @@ def run_ours(args, world, rank, local):
     return line
 
 
+RAC_SWEEP_TOKENS = (4096, 8192, 16384, 32768, 65536, 131072)
+
+
+def run_rac_sweep(args, local):
+    """route -> align -> combine alone, through the C ABI, on one workload's shape with T swept:
+    each stage's CUDA-event time and algorithmic HBM GB/s against the measured copy bandwidth.
+    The combine reads seeded synthetic expert outputs (one row per assignment slot). Before
+    every step a 256 MB buffer is written so that no stage starts from a warm L2."""
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peaks_src = load_peaks()
+    base = W.WORKLOADS[args.workload]
+    tokens = [int(t) for t in args.sweep_tokens.split(",")] if args.sweep_tokens else \
+        list(RAC_SWEEP_TOKENS)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stages = ("route", "align", "combine")
+    points = []
+    with ClockSampler(local) as clk:
+        for T in tokens:
+            wl = base.with_tokens(T)
+            inp = W.make_inputs(wl, dev, weights=False)
+            y = W.make_y_slots(wl, dev)
+            shape = M.shape_of(wl.T, wl.H, wl.E, wl.k, wl.I, wl.capacity_factor, wl.dtype)
+            ws = M.Workspace(shape, dev)
+            A = wl.T * wl.k
+            idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+            wts = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
+            counts = torch.empty(wl.E, dtype=torch.int32, device=dev)
+            offsets = torch.empty(wl.E + 1, dtype=torch.int32, device=dev)
+            sorted_ids = torch.empty(A, dtype=torch.int32, device=dev)
+            slot_of = torch.empty(A, dtype=torch.int32, device=dev)
+            drop = torch.empty(A, dtype=torch.uint8, device=dev)
+            out = torch.empty((wl.T, wl.H), dtype=wl.torch_dtype, device=dev)
+
+            def step(ev=None):
+                flush.fill_(1)
+                if ev is not None:
+                    ev[0].record(stream)
+                L.moe_route(shape, inp["x"], inp["w_router"], inp["logit_bias"], None, idx, wts,
+                            ws.buf, ws.nbytes, stream)
+                if ev is not None:
+                    ev[1].record(stream)
+                L.moe_align(shape, idx, counts, offsets, sorted_ids, slot_of, drop, ws.buf,
+                            ws.nbytes, stream)
+                if ev is not None:
+                    ev[2].record(stream)
+                L.moe_combine(shape, y, slot_of, wts, out, stream)
+                if ev is not None:
+                    ev[3].record(stream)
+
+            for _ in range(args.warmup):
+                step()
+            torch.cuda.synchronize()
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                   for _ in range(args.steps)]
+            for ev in evs:
+                step(ev)
+            torch.cuda.synchronize()
+            ws.check()
+            us = {s_: statistics.median(ev[j].elapsed_time(ev[j + 1]) for ev in evs) * 1e3
+                  for j, s_ in enumerate(stages)}
+            cost = stage_costs(wl, counts.cpu().numpy(), peaks["hbm_gbs"],
+                               peaks["bf16_tflops_sustained"])
+            pt = {"T": T, "assignments": A, "kept": int(counts.sum().item())}
+            for s_ in stages:
+                gbs = cost[s_]["bytes"] / (us[s_] * 1e-6) / 1e9
+                pt[s_] = {"us": round(us[s_], 2), "bytes": cost[s_]["bytes"],
+                          "gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 3)}
+            tot_b = sum(cost[s_]["bytes"] for s_ in stages)
+            tot_us = sum(us[s_] for s_ in stages)
+            pt["total"] = {"us": round(tot_us, 2), "bytes": tot_b,
+                           "gbs": round(tot_b / (tot_us * 1e-6) / 1e9, 1),
+                           "frac": round(tot_b / (tot_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3)}
+            points.append(pt)
+            del inp, y, ws, out
+            torch.cuda.empty_cache()
+    return {"sweep": "route_align_combine", "unit": "GB/s",
+            "workload": base.describe().split(": ", 1)[1].replace(f"T={base.T} ", ""),
+            "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": peaks_src,
+            "timing": f"median of {args.steps} steps after {args.warmup} warm-up, CUDA events "
+                      "around each stage, L2 overwritten (256 MB) before every step",
+            "points": points, "clocks": clk.summary()}
+
+
 def run_reference(args, world, rank, local):
     """The reference arm: the CPU oracle itself, on the same workload, bounded samples."""
     if rank != 0:
@@ -543,12 +633,21 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
                     help="expert weights: the layer dtype (default) or e4m3 + per-channel scales")
+    ap.add_argument("--sweep", choices=["route-align-combine"], default=None,
+                    help="time route -> align -> combine alone over a range of T (HBM GB/s per "
+                         "stage; one GPU) instead of the layer")
+    ap.add_argument("--sweep-tokens", default="",
+                    help="comma-separated T values for --sweep (default 4096 ... 131072)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_setup()
     try:
-        if args.impl == "reference":
+        if args.sweep:
+            if world > 1:
+                ap.error("--sweep runs on one GPU")
+            line = run_rac_sweep(args, local)
+        elif args.impl == "reference":
             line = run_reference(args, world, rank, local)
         else:
             line = run_ours(args, world, rank, local)

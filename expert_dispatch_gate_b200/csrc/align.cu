@@ -9,12 +9,14 @@
 //
 // Rank of assignment a = t*k + j inside expert e = idx[t,j]: number of earlier assignments (in
 // a order, i.e. token order) routed to e. Kept iff rank < C. The result is deterministic and
-// identical to the sequential definition:
-//   1. hist:    per 2048-assignment chunk, per-expert counts (shared-memory atomics).
+// identical to the sequential definition. Up to kAlignCluster assignments one launch does all
+// of it (one block up to kAlignSingle, one cluster of CTAs above); beyond that three kernels:
+//   1. hist:    per chunk of align_chunk(A) assignments, per-expert counts (shared-memory
+//               atomics).
 //   2. scan:    one block; per expert, exclusive prefix over chunks (chunk bases), raw totals,
 //               counts = min(raw, C), offsets = exclusive scan of counts, and the token-block
 //               plan blk_prefix used by the expert GEMMs.
-//   3. scatter: per chunk, stable in-chunk ranks (warp __match_any_sync + per-warp prefix),
+//   3. scatter: per chunk, stable in-chunk ranks (warp_peers + per-warp prefix),
 //               then slot = offsets[e] + rank for kept assignments; fills the -1 tail.
 #include <mutex>
 
@@ -26,8 +28,40 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSinglePerWarp = kAlignSingle / kWarps;  // one-block path: 256 per warp
+constexpr int kBlockThreads = 1024;  // threads of each CTA of the one-launch cluster grouping
 constexpr int kMaxE = 256;
+constexpr int kClusterCtas = 8;       // CTAs of the one-launch grouping's cluster (portable size)
+
+// Lanes of the warp whose key equals this lane's, for keys below 2^nbits (nbits <= 8); lanes
+// with ok == false belong to no group and get 0. Warp-level multisplit by ballots over the
+// key's bits (S. Ashkiani et al., "GPU Multisplit", PPoPP 2016): a lane's peers are the
+// intersection, over the bits, of the lanes that agree with it on that bit.
+__device__ __forceinline__ uint32_t warp_peers(uint32_t key, bool ok, int nbits) {
+  uint32_t peers = __ballot_sync(0xffffffffu, ok);
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    if (b < nbits) {  // uniform across the warp
+      const bool bit = (key >> b) & 1u;
+      const uint32_t m = __ballot_sync(0xffffffffu, bit);
+      peers &= bit ? m : ~m;
+    }
+  }
+  return ok ? peers : 0u;
+}
+
+// The two halves of a cluster-wide barrier, for work between arriving and waiting.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 32-bit load from another CTA's shared memory (a shared::cluster address from mapa_shared).
+__device__ __forceinline__ int ld_shared_cluster_s32(uint32_t cluster_addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
 
 __global__ void __launch_bounds__(kThreads)
     align_hist_kernel(const int32_t* __restrict__ idx, int64_t A, int E, int chunk,
@@ -48,7 +82,8 @@ __global__ void __launch_bounds__(kThreads)
     blk_hist[static_cast<size_t>(blockIdx.x) * E + e] = h[e];
 }
 
-// Exclusive block-wide scan of one int per thread (kThreads threads).
+// Exclusive block-wide scan of one int per thread (NW warps, NW <= 32; sh holds NW ints).
+template <int NW = kWarps>
 __device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int inc = v;
@@ -60,17 +95,17 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int& total) 
   if (lane == 31) sh[warp] = inc;
   __syncthreads();
   if (warp == 0) {
-    int w = (lane < kWarps) ? sh[lane] : 0;
+    int w = (lane < NW) ? sh[lane] : 0;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int o = __shfl_up_sync(0xffffffffu, w, off);
       if (lane >= off) w += o;
     }
-    if (lane < kWarps) sh[lane] = w;  // inclusive warp totals
+    if (lane < NW) sh[lane] = w;  // inclusive warp totals
   }
   __syncthreads();
   const int warp_base = (warp > 0) ? sh[warp - 1] : 0;
-  total = sh[kWarps - 1];
+  total = sh[NW - 1];
   __syncthreads();
   return warp_base + inc - v;
 }
@@ -128,14 +163,12 @@ __global__ void __launch_bounds__(kThreads)
   const int per_warp = chunk / kWarps;  // a multiple of 32
   const int64_t wbase = static_cast<int64_t>(blockIdx.x) * chunk + warp * per_warp;
 
+  const int nbits = (E > 1) ? 32 - __clz(E - 1) : 0;
   // pass 1: per-warp per-expert counts of this warp's assignments
   for (int step = 0; step < per_warp / 32; ++step) {
     const int64_t a = wbase + step * 32 + lane;
     const int e = (a < A) ? idx[a] : -1;
-    const bool ok = (e >= 0 && e < E);
-    const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : (E + lane));
-    if (ok && lane == __ffs(peers) - 1) wrun[warp][e] += __popc(peers);
-    __syncwarp();
+    if (e >= 0 && e < E) atomicAdd(&wrun[warp][e], 1);
   }
   __syncthreads();
   // per expert: exclusive prefix across the warps, seeded with this chunk's base
@@ -155,7 +188,7 @@ __global__ void __launch_bounds__(kThreads)
     const bool in = a < A;
     const int e = in ? idx[a] : -1;
     const bool ok = (e >= 0 && e < E);
-    const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : (E + lane));
+    const uint32_t peers = warp_peers(static_cast<uint32_t>(e), ok, nbits);
     int rank = 0;
     if (ok) rank = wrun[warp][e] + __popc(peers & lanemask_lt());
     __syncwarp();
@@ -180,67 +213,127 @@ __global__ void __launch_bounds__(kThreads)
     sorted_ids[s] = -1;
 }
 
-// Whole grouping in one block when every assignment fits one chunk (A <= kAlignSingle): the
-// histogram, scan and stable scatter of the three kernels above, without two launches.
-__global__ void __launch_bounds__(kThreads)
-    align_single_chunk_kernel(const int32_t* __restrict__ idx, int64_t A, int E, int C, int TB,
-                              int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                              int32_t* __restrict__ blk_prefix, int32_t* __restrict__ sorted_ids,
-                              int32_t* __restrict__ slot_of, uint8_t* __restrict__ drop_mask,
-                              int* err) {
+// Whole grouping in one launch of one cluster of CS CTAs of NT threads (CS = 1: a single
+// block), for A <= CS * NT * MAXS. CTA r of the cluster owns a contiguous slice of the
+// assignments and warp w of it a contiguous segment of `steps` rounds of 32. idx is read once,
+// 8 loads of a lane in flight together, into 16-bit codes in dynamic shared memory
+// (code_sm[round * NT + thread], NT * MAXS * 2 bytes; 0xFFFF: no assignment or an invalid id).
+//   1. per-warp per-expert counts (shared-memory atomics: counting needs no order);
+//   2. per expert, the exclusive prefix over this CTA's warps and the CTA's total;
+//   3. cluster barrier; every CTA reads all CTAs' totals through distributed shared memory,
+//      giving its own base (CTAs of lower rank) and the raw totals; each derives counts,
+//      offsets and the token-block plan (CTA 0 writes them);
+//   4. stable ranks in assignment order (warp_peers) and the scatter.
+// A second cluster barrier, arrived on after the remote reads and waited on at exit, keeps
+// every CTA's totals alive until no CTA reads them any more.
+template <int NT, int CS, int MAXS>
+__global__ void __launch_bounds__(NT, 1)
+    align_cluster_kernel(const int32_t* __restrict__ idx, int64_t A, int E, int C, int TB,
+                         int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                         int32_t* __restrict__ blk_prefix, int32_t* __restrict__ sorted_ids,
+                         int32_t* __restrict__ slot_of, uint8_t* __restrict__ drop_mask,
+                         int* err) {
+  constexpr int NW = NT / 32;
+  static_assert(MAXS % 8 == 0, "ids are loaded 8 rounds at a time");
+  constexpr int kBatch = 8;
   pdl_enter<false>();
-  __shared__ int wrun[kWarps][kMaxE];
-  __shared__ int s_off[kMaxE + 1];
-  __shared__ int sh[kWarps];
+  __shared__ int wrun[NW][kMaxE];
+  __shared__ int cta_tot[kMaxE];
+  __shared__ int s_off[kMaxE];
+  __shared__ int sh[NW];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < kWarps * kMaxE; i += kThreads) (&wrun[0][0])[i] = 0;
-  __syncthreads();
-  const int64_t wbase = static_cast<int64_t>(warp) * kSinglePerWarp;
-  // per-warp per-expert counts
-  for (int step = 0; step < kSinglePerWarp / 32; ++step) {
-    const int64_t a = wbase + step * 32 + lane;
-    const int e = (a < A) ? idx[a] : -1;
-    const bool ok = (e >= 0 && e < E);
-    if (a < A && !ok) flag_error(err, kDevBadExpert);
-    const uint32_t peers = __match_any_sync(0xffffffffu, ok ? e : (E + lane));
-    if (ok && lane == __ffs(peers) - 1) wrun[warp][e] += __popc(peers);
-    __syncwarp();
-  }
-  __syncthreads();
-  // per expert: exclusive prefix across warps and the raw total
-  const int e = threadIdx.x;
-  int raw = 0;
-  if (e < E) {
+  const int r = (CS > 1) ? static_cast<int>(cluster_ctarank()) : 0;
+  for (int i = threadIdx.x; i < NW * kMaxE; i += NT) (&wrun[0][0])[i] = 0;
+  // rounds per warp: ceil(ceil(A / (CS * NW)) / 32) <= MAXS; A <= CS * NT * MAXS (checked by
+  // the launcher), so 32-bit indices suffice
+  const int An = static_cast<int>(A);
+  const int steps = ((An + CS * NW - 1) / (CS * NW) + 31) / 32;
+  const int wbase = (r * NW + warp) * steps * 32;
+  const int nbits = (E > 1) ? 32 - __clz(E - 1) : 0;
+  extern __shared__ uint16_t code_sm[];
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const int c = wrun[w][e];
-      wrun[w][e] = raw;
-      raw += c;
+  for (int s0 = 0; s0 < MAXS; s0 += kBatch) {
+    if (s0 >= steps) break;  // uniform across the block
+    int raw[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int a = wbase + (s0 + j) * 32 + lane;
+      raw[j] = (s0 + j < steps && a < An) ? __ldg(idx + a) : -1;
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int s = s0 + j;
+      const int a = wbase + s * 32 + lane;
+      const bool ok = (raw[j] >= 0 && raw[j] < E);
+      if (s < steps && a < An && !ok) flag_error(err, kDevBadExpert);
+      code_sm[s * NT + threadIdx.x] = ok ? static_cast<uint16_t>(raw[j]) : uint16_t{0xFFFF};
     }
   }
-  const int cnt = (e < E) ? min(raw, C) : 0;
+  __syncthreads();
+  // 1. per-warp per-expert counts
+  for (int s = 0; s < steps; ++s) {
+    const uint32_t c = code_sm[s * NT + threadIdx.x];
+    if (c != 0xFFFFu) atomicAdd(&wrun[warp][c], 1);
+  }
+  __syncthreads();
+  // 2. per expert: exclusive prefix across this CTA's warps, and the CTA's total
+  const int e = threadIdx.x;
+  int mine = 0;
+  if (e < E) {
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const int c = wrun[w][e];
+      wrun[w][e] = mine;
+      mine += c;
+    }
+    cta_tot[e] = mine;
+  }
+  // 3. this CTA's base and the raw totals over the cluster, in CTA-rank order
+  int before = 0, raw_tot = mine;
+  if constexpr (CS > 1) {
+    cluster_sync_all();
+    if (e < E) {
+      const uint32_t loc = smem_u32(&cta_tot[e]);
+      raw_tot = 0;
+#pragma unroll
+      for (int q = 0; q < CS; ++q) {
+        const int v = ld_shared_cluster_s32(mapa_shared(loc, q));
+        if (q < r) before += v;
+        raw_tot += v;
+      }
+    }
+    cluster_arrive();
+  }
+  const int cnt = (e < E) ? min(raw_tot, C) : 0;
   const int nb = (cnt + TB - 1) / TB;
   int tot_cnt, tot_nb;
-  const int off = block_exclusive_scan(cnt, sh, tot_cnt);
-  const int bp = block_exclusive_scan(nb, sh, tot_nb);
+  const int off = block_exclusive_scan<NW>(cnt, sh, tot_cnt);
+  const int bp = block_exclusive_scan<NW>(nb, sh, tot_nb);
   if (e < E) {
-    counts[e] = cnt;
-    offsets[e] = off;
     s_off[e] = off;
-    if (blk_prefix != nullptr) blk_prefix[e] = bp;
+    if (r == 0) {
+      counts[e] = cnt;
+      offsets[e] = off;
+      if (blk_prefix != nullptr) blk_prefix[e] = bp;
+    }
+    if (before != 0) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) wrun[w][e] += before;
+    }
   }
-  if (e == 0) {
+  if (e == 0 && r == 0) {
     offsets[E] = tot_cnt;
     if (blk_prefix != nullptr) blk_prefix[E] = tot_nb;
   }
   __syncthreads();
-  // stable ranks in assignment order, then the scatter
-  for (int step = 0; step < kSinglePerWarp / 32; ++step) {
-    const int64_t a = wbase + step * 32 + lane;
-    const bool in = a < A;
-    const int ea = in ? idx[a] : -1;
-    const bool ok = (ea >= 0 && ea < E);
-    const uint32_t peers = __match_any_sync(0xffffffffu, ok ? ea : (E + lane));
+  // 4. stable ranks in assignment order, then the scatter
+  for (int s = 0; s < steps; ++s) {  // uniform across the block
+    const int a = wbase + s * 32 + lane;
+    const bool in = a < An;
+    const uint32_t c = code_sm[s * NT + threadIdx.x];
+    const bool ok = c != 0xFFFFu;
+    const int ea = static_cast<int>(c);
+    const uint32_t peers = warp_peers(c, ok, nbits);
     int rank = 0;
     if (ok) rank = wrun[warp][ea] + __popc(peers & lanemask_lt());
     __syncwarp();
@@ -249,7 +342,7 @@ __global__ void __launch_bounds__(kThreads)
     if (in) {
       if (ok && rank < C) {
         const int slot = s_off[ea] + rank;
-        sorted_ids[slot] = static_cast<int32_t>(a);
+        sorted_ids[slot] = a;
         slot_of[a] = slot;
         drop_mask[a] = 0;
       } else {
@@ -258,7 +351,8 @@ __global__ void __launch_bounds__(kThreads)
       }
     }
   }
-  for (int64_t sl = tot_cnt + threadIdx.x; sl < A; sl += kThreads) sorted_ids[sl] = -1;
+  for (int sl = tot_cnt + r * NT + threadIdx.x; sl < An; sl += CS * NT) sorted_ids[sl] = -1;
+  if constexpr (CS > 1) cluster_wait();
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -282,10 +376,24 @@ cudaError_t launch_align(const int32_t* topk_idx, int64_t A, int E, int C, int T
                          int32_t* blk_prefix, int32_t* sorted_ids, int32_t* slot_of,
                          uint8_t* drop_mask, int* err, cudaStream_t stream) {
   if (A == 0) return cudaSuccess;
-  if (A <= kAlignSingle)
-    return launch_kernel(align_single_chunk_kernel, dim3(1), dim3(kThreads), 0, stream, 1,
-                         topk_idx, A, E, C, TB, counts, offsets, blk_prefix, sorted_ids, slot_of,
-                         drop_mask, err);
+  if (A <= kAlignSingle) {
+    constexpr int kMaxs = kAlignSingle / kThreads;
+    return launch_kernel(align_cluster_kernel<kThreads, 1, kMaxs>, dim3(1), dim3(kThreads),
+                         size_t{kThreads} * kMaxs * 2, stream, 1, topk_idx, A, E, C, TB, counts,
+                         offsets, blk_prefix, sorted_ids, slot_of, drop_mask, err);
+  }
+  if (A <= kAlignCluster) {
+    constexpr int kMaxs = kAlignCluster / (kClusterCtas * kBlockThreads);
+    static_assert(kMaxs * kClusterCtas * kBlockThreads == kAlignCluster, "cluster capacity");
+    auto kernel = align_cluster_kernel<kBlockThreads, kClusterCtas, kMaxs>;
+    constexpr size_t kCodeBytes = size_t{kBlockThreads} * kMaxs * 2;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kCodeBytes));
+    if (e != cudaSuccess) return e;
+    return launch_kernel(kernel, dim3(kClusterCtas), dim3(kBlockThreads), kCodeBytes, stream,
+                         kClusterCtas, topk_idx, A, E, C, TB, counts, offsets, blk_prefix,
+                         sorted_ids, slot_of, drop_mask, err);
+  }
   const int chunk = align_chunk(A);
   const int nblk = static_cast<int>((A + chunk - 1) / chunk);
   cudaError_t e = launch_kernel(align_hist_kernel, dim3(nblk), dim3(kThreads), 0, stream, 1,
@@ -323,7 +431,7 @@ cudaError_t launch_align_noalloc(const int32_t* topk_idx, int64_t A, int E, int 
                                  int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
                                  int32_t* slot_of, uint8_t* drop_mask, cudaStream_t stream) {
   if (A > kNoAllocMaxAssignments || E > 256) return cudaErrorInvalidValue;
-  if (A > kAlignSingle && (A + align_chunk(A) - 1) / align_chunk(A) > kNoAllocMaxBlocks)
+  if (A > kAlignCluster && (A + align_chunk(A) - 1) / align_chunk(A) > kNoAllocMaxBlocks)
     return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

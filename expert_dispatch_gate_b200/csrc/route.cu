@@ -19,11 +19,39 @@ namespace {
 
 constexpr int kWarpsPerBlock = 8;
 
-// Logits distributed over lanes: lane holds experts lane, lane+32, ... (VPL per lane). Each
-// logit is the sum of the K-range partials in ascending order plus the optional bias. With
-// n_group > 1 the selection is group-limited (select.cuh).
+// Logits distributed over lanes: lane l holds experts VPL*l ... VPL*l + VPL - 1. Each logit is
+// the sum of the K-range partials in ascending order plus the optional bias. With n_group > 1
+// the selection is group-limited (select.cuh).
 template <int VPL>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+__device__ __forceinline__ void load_run(const float* p, bool vec, bool in, float (&o)[VPL]) {
+  if (!in) {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) o[i] = 0.f;
+  } else if (VPL >= 4 && vec) {
+#pragma unroll
+    for (int i = 0; i < VPL; i += 4) {
+      const float4 q = __ldg(reinterpret_cast<const float4*>(p + i));
+      o[i] = q.x;
+      o[i + 1] = q.y;
+      o[i + 2] = q.z;
+      o[i + 3] = q.w;
+    }
+  } else if (VPL == 2 && vec) {
+    const float2 q = __ldg(reinterpret_cast<const float2*>(p));
+    o[0] = q.x;
+    o[VPL - 1] = q.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) o[i] = __ldg(p + i);
+  }
+}
+
+// Partial sums in ascending K-range order. Four K ranges are loaded per group with no branch
+// between the loads, so one group costs one memory latency. vec: E % VPL == 0, so a lane's run
+// of VPL logits is one or two aligned vector loads (rows start on 16-byte boundaries then);
+// otherwise a lane with experts past E reads only those below E.
+template <int VPL>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
     topk_kernel(const float* __restrict__ partials, int ksplit, int64_t split_stride,
                 const float* __restrict__ bias, float* __restrict__ logits_out, int64_t T, int E,
                 int k, int n_group, int topk_group, int32_t* __restrict__ topk_idx,
@@ -32,31 +60,46 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   const int lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
   if (t >= T) return;
+  const int e0 = VPL * lane;
+  const bool vec = (E % VPL) == 0;
+  const bool full = e0 + VPL <= E;  // every expert of this lane exists
+  const float* row = partials + t * E + e0;
   float v[VPL];
   uint32_t taken = 0;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
-    const int e = lane + 32 * i;
-    if (e < E) {
-      // partial sums in ascending K-range order; loads issued four at a time
-      const float* src = partials + t * E + e;
-      float acc = src[0];
-      int ks = 1;
-      for (; ks + 4 <= ksplit; ks += 4) {
-        const float a0 = src[(ks + 0) * split_stride], a1 = src[(ks + 1) * split_stride];
-        const float a2 = src[(ks + 2) * split_stride], a3 = src[(ks + 3) * split_stride];
-        acc += a0;
-        acc += a1;
-        acc += a2;
-        acc += a3;
+    v[i] = 0.f;
+    if (e0 + i >= E) taken |= 1u << i;
+  }
+  for (int ks0 = 0; ks0 < ksplit; ks0 += 4) {
+    float p[4][VPL];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool in = ks0 + j < ksplit;
+      if (full) {
+        load_run<VPL>(row + (ks0 + j) * split_stride, vec, in, p[j]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < VPL; ++i)
+          p[j][i] = (in && e0 + i < E) ? __ldg(row + (ks0 + j) * split_stride + i) : 0.f;
       }
-      for (; ks < ksplit; ++ks) acc += src[ks * split_stride];
-      if (bias != nullptr) acc += bias[e];
-      v[i] = acc;
-      if (logits_out != nullptr) logits_out[t * E + e] = acc;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (ks0 + j < ksplit) {
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) v[i] = (ks0 + j == 0) ? p[j][i] : v[i] + p[j][i];
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = e0 + i;
+    if (e < E) {
+      if (bias != nullptr) v[i] += __ldg(bias + e);
+      if (logits_out != nullptr) logits_out[t * E + e] = v[i];
     } else {
       v[i] = -INFINITY;
-      taken |= 1u << i;
     }
   }
   if (n_group > 1) taken |= warp_group_exclude<VPL>(v, E, n_group, topk_group, lane);

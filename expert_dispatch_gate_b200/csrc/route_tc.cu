@@ -12,6 +12,8 @@
 // alternate between two accumulators (even / odd K steps), which keeps two independent
 // accumulate chains in flight; the epilogue adds the two.
 //
+// When E % 128 == 0, two CTAs of a cluster share each 256-token tile (cta_group::2, below).
+//
 // Warps: 0 TMA producer, 1 MMA issuer (converged warp, elected lane), 2-5 epilogue (one TMEM
 // lane quadrant each).
 #include <cuda.h>
@@ -36,7 +38,7 @@ constexpr int kRtCtrl = 256;
 struct RtParams {
   int T, H, E;
   int npad;            // N of the MMA: E rounded up to 16
-  int nch;             // 64-expert chunks of B per stage
+  int nch;             // 64-expert chunks of B loaded per stage by this CTA
   int kb_per_split;    // k-blocks of one K range
   int two_acc;         // 1: alternate two accumulators over K steps
   int stages;
@@ -45,6 +47,14 @@ struct RtParams {
   int* err;
 };
 
+// PAIR: two CTAs of a cluster share one 256-token tile with tcgen05.mma.cta_group::2 (M = 256):
+// each CTA loads its own 128 token rows (A) and half of the expert chunks of Wr (B, so E % 128
+// == 0); both CTAs' loads complete on the even CTA's `full` barrier, the even CTA issues the
+// MMAs, and its commits arrive on both CTAs' `empty` and `done` barriers. Each CTA's TMEM holds
+// its own 128 tokens x N experts, drained by its own epilogue. Per CTA and k-block that is
+// 16 KB of x and 16 KB of Wr instead of 16 + 32 KB: a third less L2-to-SM traffic, and more
+// k-blocks in flight in the same shared memory.
+template <bool PAIR>
 __global__ void __launch_bounds__(kRtThreads, 1)
     route_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
                       const __grid_constant__ CUtensorMap tmW, const RtParams p) {
@@ -62,6 +72,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = (rank == 0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
@@ -72,15 +84,22 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), kRtTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_holder), kRtTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_holder), kRtTmemCols);
+      tmem_relinquish();
+    }
   }
   pdl_enter<false>();
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // both CTAs' barriers are initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int row0 = static_cast<int>(blockIdx.x) * kRtM;
+  const int row0 = PAIR ? static_cast<int>(blockIdx.x >> 1) * (2 * kRtM) + static_cast<int>(rank) * kRtM
+                        : static_cast<int>(blockIdx.x) * kRtM;
   const int ks = static_cast<int>(blockIdx.y);
   const int kb0 = ks * p.kb_per_split;
   const int nkb = p.kb_per_split;
@@ -89,7 +108,9 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t s = 0, ph = 0;
-      const uint32_t tx = static_cast<uint32_t>(stage_bytes);
+      // in PAIR mode the even CTA's barrier expects both CTAs' bytes
+      const uint32_t tx = static_cast<uint32_t>(stage_bytes) * (PAIR ? 2u : 1u);
+      const int c0 = static_cast<int>(rank) * p.nch;  // first expert chunk this CTA loads
       bool ok = true;
       int issued = 0;
       for (int i = 0; i < nkb; ++i) {
@@ -98,11 +119,19 @@ __global__ void __launch_bounds__(kRtThreads, 1)
           break;
         }
         const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
-        const uint32_t fb = smem_u32(&full[s]);
         const int kc = (kb0 + i) * kRtBK;
-        mbar_arrive_expect_tx(fb, tx);
-        tma_load_2d(sa, &tmX, kc, row0, fb);
-        for (int c = 0; c < p.nch; ++c) tma_load_2d(sa + 16384 + c * 8192, &tmW, c * 64, kc, fb);
+        if constexpr (PAIR) {
+          const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), tx);
+          tma_load_2d_pair(sa, &tmX, kc, row0, fb);
+          for (int c = 0; c < p.nch; ++c)
+            tma_load_2d_pair(sa + 16384 + c * 8192, &tmW, (c0 + c) * 64, kc, fb);
+        } else {
+          const uint32_t fb = smem_u32(&full[s]);
+          mbar_arrive_expect_tx(fb, tx);
+          tma_load_2d(sa, &tmX, kc, row0, fb);
+          for (int c = 0; c < p.nch; ++c) tma_load_2d(sa + 16384 + c * 8192, &tmW, c * 64, kc, fb);
+        }
         ++issued;
         if (++s == static_cast<uint32_t>(S)) {
           s = 0;
@@ -113,63 +142,71 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         *abort_flag = 1;
         flag_error(p.err, kDevWaitTimeout);
       }
-      // every load issued lands before the CTA may exit
-      for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
-        mbar_wait(smem_u32(&full[i % S]), static_cast<uint32_t>(i / S) & 1u, nullptr);
+      // Every load issued lands before the CTA may exit. In PAIR mode the loads complete on the
+      // even CTA's barriers; the cluster barrier at the end keeps the odd CTA alive until then.
+      if (!PAIR || leader) {
+        for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
+          mbar_wait_cluster(smem_u32(&full[i % S]), static_cast<uint32_t>(i / S) & 1u, nullptr);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (whole warp)
-    constexpr uint32_t kFull = 0xffffffffu;
-    const uint32_t sbase = smem_u32(smem);
-    const uint64_t adesc0 = smem_desc_sw128(sbase, 16, 1024);            // x rows, K-major
-    const uint64_t bdesc0 = smem_desc_sw128(sbase + 16384, 8192, 1024);  // Wr, MN-major
-    const uint32_t idesc = idesc_bf16(kRtM, p.npad, /*a_mn_major=*/false, /*b_mn_major=*/true);
-    const uint32_t d1 = tmem_base + (p.two_acc ? static_cast<uint32_t>(p.npad) : 0u);
-    uint32_t s = 0, ph = 0, soff = 0;
-    uint32_t acc0 = 0, acc1 = 0;
-    bool ok = true;
-    for (int i = 0; i < nkb; ++i) {
-      if (!__all_sync(kFull, mbar_wait(smem_u32(&full[s]), ph, abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint64_t ad = adesc0 + (soff >> 4);
-      const uint64_t bd = bdesc0 + (soff >> 4);
+    if (leader) {
+      constexpr uint32_t kFull = 0xffffffffu;
+      const uint32_t sbase = smem_u32(smem);
+      const uint64_t adesc0 = smem_desc_sw128(sbase, 16, 1024);            // x rows, K-major
+      const uint64_t bdesc0 = smem_desc_sw128(sbase + 16384, 8192, 1024);  // Wr, MN-major
+      const uint32_t idesc = idesc_bf16(PAIR ? 2 * kRtM : kRtM, p.npad, /*a_mn_major=*/false,
+                                        /*b_mn_major=*/true);
+      const uint32_t d1 = tmem_base + (p.two_acc ? static_cast<uint32_t>(p.npad) : 0u);
+      uint32_t s = 0, ph = 0, soff = 0;
+      uint32_t acc0 = 0, acc1 = 0;
+      bool ok = true;
+      for (int i = 0; i < nkb; ++i) {
+        if (!__all_sync(kFull, mbar_wait_cluster(smem_u32(&full[s]), ph, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t ad = adesc0 + (soff >> 4);
+        const uint64_t bd = bdesc0 + (soff >> 4);
 #pragma unroll
-      for (int kk = 0; kk < kRtBK / 16; ++kk) {
-        // A advances 16 K-columns (32 B) per step, B 16 K-rows (2 KB)
-        if ((kk & 1) == 0 || !p.two_acc) {
-          tc_mma_bf16_elect(tmem_base, ad + kk * 2, bd + kk * 128, idesc, acc0);
-          acc0 = 1u;
+        for (int kk = 0; kk < kRtBK / 16; ++kk) {
+          // A advances 16 K-columns (32 B) per step, B 16 K-rows (2 KB)
+          const bool second = p.two_acc && (kk & 1);
+          const uint32_t d = second ? d1 : tmem_base;
+          const uint32_t acc = second ? acc1 : acc0;
+          if constexpr (PAIR) tc_mma_bf16_pair_elect(d, ad + kk * 2, bd + kk * 128, idesc, acc);
+          else tc_mma_bf16_elect(d, ad + kk * 2, bd + kk * 128, idesc, acc);
+          if (second) acc1 = 1u;
+          else acc0 = 1u;
+        }
+        if constexpr (PAIR) tc_commit_pair_mc_elect(smem_u32(&empty[s]), 0x3);
+        else tc_commit_elect(smem_u32(&empty[s]));
+        if (++s == static_cast<uint32_t>(S)) {
+          s = 0;
+          ph ^= 1u;
+          soff = 0;
         } else {
-          tc_mma_bf16_elect(d1, ad + kk * 2, bd + kk * 128, idesc, acc1);
-          acc1 = 1u;
+          soff += static_cast<uint32_t>(stage_bytes);
         }
       }
-      tc_commit_elect(smem_u32(&empty[s]));
-      if (++s == static_cast<uint32_t>(S)) {
-        s = 0;
-        ph ^= 1u;
-        soff = 0;
-      } else {
-        soff += static_cast<uint32_t>(stage_bytes);
+      if (!ok && lane == 0) {
+        *abort_flag = 1;
+        flag_error(p.err, kDevWaitTimeout);
       }
+      // completes once every MMA issued has finished (also when the loop stopped early)
+      if constexpr (PAIR) tc_commit_pair_mc_elect(smem_u32(done), 0x3);
+      else tc_commit_elect(smem_u32(done));
     }
-    if (!ok && lane == 0) {
-      *abort_flag = 1;
-      flag_error(p.err, kDevWaitTimeout);
-    }
-    // completes once every MMA issued has finished (also when the loop stopped early)
-    tc_commit_elect(smem_u32(done));
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;
     const int t = row0 + q * 32 + lane;
     int got = 1;
-    if (lane == 0) got = mbar_wait(smem_u32(done), 0u, abort_flag) ? 1 : 0;
+    if (lane == 0) got = mbar_wait_cluster(smem_u32(done), 0u, abort_flag) ? 1 : 0;
     got = __shfl_sync(0xffffffffu, got, 0);
     if (!got) {
       if (lane == 0) {
@@ -210,12 +247,14 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   }
 
   // The MMA completion barrier also guards TMEM release when the epilogue gave up early.
-  if (warp == 1 && lane == 0) mbar_wait(smem_u32(done), 0u, nullptr);
+  if (warp == 1 && lane == 0) mbar_wait_cluster(smem_u32(done), 0u, nullptr);
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // no CTA leaves while its peer may still signal it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kRtTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, kRtTmemCols);
+    else tmem_dealloc(tmem_base, kRtTmemCols);
   }
 }
 
@@ -261,14 +300,18 @@ bool map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint
 
 }  // namespace
 
+// CTA pairs need whole 64-expert chunks in each half of B.
+bool route_uses_pairs(int E) { return E % 128 == 0; }
+
 int route_ksplit(int64_t T, int H, int E) {
-  (void)E;
   const int64_t kb_total = H / kRtBK;
-  const int64_t tiles = (T + kRtM - 1) / kRtM;
+  // CTAs per K range: one per 128 tokens, rounded up to whole pairs when pairs are used
+  int64_t ctas = (T + kRtM - 1) / kRtM;
+  if (route_uses_pairs(E)) ctas = 2 * ((T + 2 * kRtM - 1) / (2 * kRtM));
   int ks = 1;
   // split K while the grid stays within about 128 CTAs and each range keeps >= 4 k-blocks
   while (ks * 2 <= 16 && kb_total % (ks * 2) == 0 && kb_total / (ks * 2) >= 4 &&
-         tiles * ks * 2 <= 128)
+         ctas * ks * 2 <= 128)
     ks *= 2;
   return ks;
 }
@@ -282,6 +325,7 @@ cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int
     if (detail) *detail = "router GEMM shape outside the tensor-core path";
     return cudaErrorInvalidValue;
   }
+  const bool pair = route_uses_pairs(E);
   CUtensorMap mx, mw;
   if (!map_2d(&mx, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), kRtM, detail) ||
       !map_2d(&mw, w_router, static_cast<uint64_t>(E), static_cast<uint64_t>(H), kRtBK, detail))
@@ -291,7 +335,7 @@ cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int
   p.H = H;
   p.E = E;
   p.npad = (E + 15) & ~15;
-  p.nch = (E + 63) / 64;
+  p.nch = pair ? E / 128 : (E + 63) / 64;
   p.kb_per_split = H / kRtBK / ksplit;
   p.two_acc = (2 * p.npad <= kRtTmemCols) ? 1 : 0;
   p.split_stride = static_cast<int64_t>(T) * E;
@@ -304,12 +348,14 @@ cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int
   if (stages < 2) stages = 2;
   p.stages = stages;
   const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + kRtCtrl;
-  cudaError_t e = cudaFuncSetAttribute(route_gemm_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kernel = pair ? route_gemm_kernel<true> : route_gemm_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>((T + kRtM - 1) / kRtM), static_cast<unsigned>(ksplit));
-  return launch_kernel(route_gemm_kernel, grid, dim3(kRtThreads), smem, stream, 1, mx, mw, p);
+  const unsigned tiles = pair ? 2u * static_cast<unsigned>((T + 2 * kRtM - 1) / (2 * kRtM))
+                              : static_cast<unsigned>((T + kRtM - 1) / kRtM);
+  const dim3 grid(tiles, static_cast<unsigned>(ksplit));
+  return launch_kernel(kernel, grid, dim3(kRtThreads), smem, stream, pair ? 2 : 1, mx, mw, p);
 }
 
 }  // namespace moe

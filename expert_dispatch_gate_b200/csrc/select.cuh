@@ -45,8 +45,9 @@ __device__ __forceinline__ void write_selection(int lane, int k, float my_v, int
 // Group-limited selection ([P5] section 3.1, "select groups first"): the E experts form
 // n_group equal contiguous groups (n_group <= 32); a group's score is the float32 sum of its
 // two largest logits (its only logit when a group holds one expert); the topk_group groups
-// with the highest scores (ties to the lower group index) stay selectable. Returns the bit
-// mask of v[] entries of this lane to exclude (experts outside the kept groups).
+// with the highest scores (ties to the lower group index) stay selectable. Lane l holds
+// experts VPL*l ... VPL*l + VPL - 1 in v[]. Returns the bit mask of v[] entries of this lane to
+// exclude (experts outside the kept groups).
 template <int VPL>
 __device__ __forceinline__ uint32_t warp_group_exclude(const float (&v)[VPL], int E, int n_group,
                                                        int topk_group, int lane) {
@@ -57,7 +58,7 @@ __device__ __forceinline__ uint32_t warp_group_exclude(const float (&v)[VPL], in
     float a1 = -INFINITY, a2 = -INFINITY;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      const int e = lane + 32 * i;
+      const int e = VPL * lane + i;
       if (e < E && e / gs == g) {
         const float x = v[i];
         if (x > a1) {
@@ -93,38 +94,71 @@ __device__ __forceinline__ uint32_t warp_group_exclude(const float (&v)[VPL], in
   uint32_t excl = 0;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
-    const int e = lane + 32 * i;
+    const int e = VPL * lane + i;
     if (e < E && !((keep >> (e / gs)) & 1u)) excl |= 1u << i;
   }
   return excl;
 }
 
-// One token's logits spread over the warp: lane holds experts lane, lane + 32, ... in v[]
-// (VPL per lane); bit i of `taken` marks v[i] as absent (expert id >= E). Selects the top k
-// and writes idx_row[0..k) and w_row[0..k).
+// Order-preserving 32-bit key of a finite float: key(a) < key(b) iff a < b, with -0 mapped to
+// +0 so that the two zeros rank equal. key 0 belongs to no finite float.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  uint32_t u = __float_as_uint(v);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// This lane's best entry not yet taken: the largest key, the lower index on equal keys (entries
+// are scanned in ascending index order, and only a strictly larger key replaces the best).
+// Lane l holds experts VPL*l + i.
+template <int VPL>
+__device__ __forceinline__ void lane_best(const uint32_t (&key)[VPL], uint32_t taken, int lane,
+                                          uint32_t& bk, int& bi) {
+  bk = 0u;
+  bi = 0x7fffffff;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    if (!((taken >> i) & 1u) && key[i] > bk) {
+      bk = key[i];
+      bi = VPL * lane + i;
+    }
+  }
+}
+
+// One token's logits spread over the warp: lane l holds experts VPL*l ... VPL*l + VPL - 1 in
+// v[]; bit i of `taken` marks v[i] as absent (expert id >= E, or excluded). Selects the top k
+// and writes idx_row[0..k) and w_row[0..k). Each round takes the warp's largest key with one
+// max-reduction (redux.sync). Lanes hold disjoint ascending index ranges, so among the lanes
+// holding that key the lowest lane has the lowest expert index (ballot + find-first); one
+// shuffle broadcasts it, and only the winning lane rescans its own entries.
 template <int VPL>
 __device__ __forceinline__ void warp_select_topk(const float (&v)[VPL], uint32_t taken, int k,
                                                  int lane, int32_t* idx_row, float* w_row) {
+  uint32_t key[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) key[i] = order_key(v[i]);
+  uint32_t bk;
+  int bi;
+  lane_best<VPL>(key, taken, lane, bk, bi);
   float my_v = 0.f, top = 0.f;
   int my_i = 0;
   for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int e = lane + 32 * i;
-      if (!((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < bi))) {
-        bv = v[i];
-        bi = e;
-      }
-    }
-    warp_argmax(bv, bi);
-    if ((bi & 31) == lane) taken |= 1u << ((bi >> 5) & 31);
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const int wl = __ffs(__ballot_sync(0xffffffffu, bk == m)) - 1;
+    const int win = __shfl_sync(0xffffffffu, bi, wl);
+    const float val = key_value(m);
     if (lane == j) {
-      my_v = bv;
-      my_i = bi;
+      my_v = val;
+      my_i = win;
     }
-    if (j == 0) top = bv;
+    if (j == 0) top = val;
+    if (lane == wl) {
+      taken |= 1u << (win - VPL * lane);
+      lane_best<VPL>(key, taken, lane, bk, bi);
+    }
   }
   write_selection(lane, k, my_v, my_i, top, idx_row, w_row);
 }

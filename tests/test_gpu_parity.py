@@ -69,6 +69,8 @@ def oracle_routing(wl, cpu):
 @pytest.mark.parametrize("T,E,k,ties", [
     (1, 8, 2, False), (300, 8, 1, True), (300, 64, 6, True), (1000, 256, 8, True),
     (257, 256, 16, False), (33, 16, 16, True), (4096, 256, 8, False), (129, 128, 4, True),
+    # experts not a multiple of the per-lane run (scalar loads, lanes past E)
+    (50, 37, 3, True), (64, 5, 2, True), (100, 200, 8, True), (77, 104, 7, True),
 ])
 def test_route_from_logits_bitexact(T, E, k, ties):
     logits = W.random_logits(T, E, seed=T * 7 + E + k, ties=ties)
@@ -84,9 +86,26 @@ def test_route_from_logits_bitexact(T, E, k, ties):
 
 # ----------------------------------------------------------------- route (gate GEMM + selection)
 
-@pytest.mark.parametrize("name", list(SMALL))
+# Router-only shapes for the tensor-core gate GEMM: CTA pairs (E % 128 == 0) over several
+# 256-token tiles with a ragged tail, a pair whose second CTA has one token, the longest K split
+# (T = 2, H = 4096), and a single-CTA shape with E = 192.
+ROUTER = {
+    "pairs_ragged": W.Workload("r1", 21, 1000, 512, 256, 8, 128, "bf16", 1.25),
+    "pairs_e128_k6": W.Workload("r2", 22, 257, 2048, 128, 6, 128, "bf16", 1.25),
+    "pairs_short_peer": W.Workload("r3", 23, 129, 256, 256, 8, 128, "bf16", 1.25),
+    "pairs_t2_ksplit16": W.Workload("r4", 24, 2, 4096, 256, 8, 128, "bf16", 1.25),
+    "single_e192": W.Workload("r5", 25, 513, 4096, 192, 8, 128, "bf16", 1.25),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL) + list(ROUTER))
 def test_router(name):
-    wl, cpu, dev = small_inputs(name)
+    if name in ROUTER:
+        wl = ROUTER[name]
+        cpu = W.make_inputs(wl, "cpu", weights=False)
+        dev = {k: (None if v is None else v.cuda()) for k, v in cpu.items()}
+    else:
+        wl, cpu, dev = small_inputs(name)
     idx_g, w_g, logits_g = M.route(dev["x"], dev["w_router"], wl.k, dev["logit_bias"])
     torch.cuda.synchronize()
     L_o, idx_o, w_o, _, _ = oracle_routing(wl, cpu)
@@ -112,6 +131,12 @@ def test_router(name):
     (4096, 256, 8, 1.25, "uniform"), (4096, 256, 8, 1.25, "zipf"), (3000, 64, 6, 1.25, "zipf"),
     (2500, 16, 4, 1.0, "one"), (777, 32, 3, 0.5, "uniform"), (2049, 1, 1, 1.25, "one"),
     (20000, 64, 6, 1.25, "zipf"),
+    # the grouping's three launch forms and their edges: one 256-thread block up to 2048
+    # assignments, one cluster of 8 CTAs up to 65536, chunked kernels beyond
+    (256, 16, 8, 1.25, "zipf"), (1024, 128, 2, 1.0, "uniform"), (1025, 128, 2, 1.0, "uniform"),
+    (4097, 256, 8, 1.25, "zipf"), (8192, 256, 8, 1.25, "zipf"), (5462, 96, 6, 0.75, "uniform"),
+    (8193, 256, 8, 1.25, "uniform"), (10923, 64, 6, 1.25, "zipf"),
+    (32768, 256, 8, 1.25, "zipf"), (40000, 64, 8, 1.25, "zipf"), (43691, 64, 6, 0.0, "uniform"),
 ])
 def test_align_bitexact(T, E, k, cf, mode):
     idx = W.random_topk_idx(T, E, k, seed=T + 31 * E + k, mode=mode)
@@ -135,16 +160,24 @@ def test_align_every_expert_exactly_at_capacity():
         assert np.array_equal(npi(res[key]), al[key]), key
 
 
-def test_align_flags_out_of_range_expert_ids():
-    idx = W.random_topk_idx(100, 16, 2, seed=3)
+@pytest.mark.parametrize("T", [100, 3000, 140000])  # each launch form of the grouping
+def test_align_flags_out_of_range_expert_ids(T):
+    idx = W.random_topk_idx(T, 16, 2, seed=3)
     idx[7, 1] = 16
     idx[50, 0] = -3
+    idx[T - 1, 1] = 1 << 20
     res = M.align(idx.cuda(), 16, 0.0)
     with pytest.raises(L.MoeError) as ei:
         res["ws"].check()
     assert ei.value.status == L.MOE_ERR_DEVICE
     drop = npi(res["drop_mask"])
-    assert drop[7 * 2 + 1] == 1 and drop[50 * 2] == 1
+    assert drop[7 * 2 + 1] == 1 and drop[50 * 2] == 1 and drop[2 * T - 1] == 1
+    slot_of = npi(res["slot_of"])
+    assert slot_of[7 * 2 + 1] == -1 and slot_of[50 * 2] == -1 and slot_of[2 * T - 1] == -1
+    # every valid assignment is kept (no capacity limit) and grouped by the oracle's rule
+    valid = idx.numpy().copy()
+    bad = (valid < 0) | (valid >= 16)
+    assert int(npi(res["counts"]).sum()) == int((~bad).sum())
     assert res["ws"].check() == L.MOE_OK  # the error word was cleared
 
 
