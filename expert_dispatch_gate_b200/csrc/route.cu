@@ -3,8 +3,10 @@
 // [P4] "MoE Router" (2048ai.net), section "Router 就是一个小型网络": logits = x Wr (bias-free
 // Linear), softmax, top-k, divide the k selected weights by their sum.
 // [P5] "大模型推理加速200%+？…", section "3.1 Moe Fuse Gate & Softmax TopK": gate + softmax + top-k
-// in one kernel, warp-shuffle arg-max with the winner erased each round, exp evaluated only for
+// in one kernel, a warp-level arg-max with the winner erased each round, exp evaluated only for
 // the k selected logits (exp(l - m) / sum over the selection equals the renormalised softmax).
+// With E >= 64 in bf16 the gate GEMM runs on the tensor cores (route_tc.cu) and topk_kernel
+// below does the selection; the CUDA-core kernel further down fuses both for small E.
 //
 // Selection rule: the k largest float32 logits, ties to the lower expert index (-0 == +0);
 // listed by descending logit then ascending index. Logits must be finite.

@@ -2,9 +2,11 @@
 //
 // [P4] "MoE Router" (2048ai.net), section "Router 就是一个小型网络": softmax over the logits, keep
 // the top k, divide the k kept weights by their sum.
-// [P5] "大模型推理加速200%+？…", section "3.1 Moe Fuse Gate & Softmax TopK": warp-shuffle arg-max
-// with the winner erased each round; exp only for the k selected logits
-// (exp(l - m) / sum over the selection equals the renormalised softmax).
+// [P5] "大模型推理加速200%+？…", section "3.1 Moe Fuse Gate & Softmax TopK": a warp-level arg-max
+// per round with the winner erased, and exp only for the k selected logits
+// (exp(l - m) / sum over the selection equals the renormalised softmax). Here each round's
+// arg-max is one redux.sync max-reduction over order-preserving integer keys plus a ballot,
+// instead of a shuffle tree (warp_select_topk).
 //
 // Selection rule: the k largest float32 logits, ties to the lower expert index (-0 == +0);
 // listed by descending logit then ascending index. Logits must be finite.
