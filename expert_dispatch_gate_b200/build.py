@@ -21,7 +21,8 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmoe.so")
 SOURCES = ["moe_api.cu", "route.cu", "route_tc.cu", "align.cu", "combine.cu", "ffn_simt.cu",
            "ffn_tc.cu", "quant.cu"]
-HEADERS = ["common.cuh", "internal.h"]
+# every header under csrc/: a change to any of them rebuilds every object
+HEADERS = sorted(f for f in os.listdir(CSRC) if f.endswith((".cuh", ".h")))
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3",
