@@ -98,7 +98,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   if constexpr (PAIR) cluster_sync_all();  // both CTAs' barriers are initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int row0 = PAIR ? static_cast<int>(blockIdx.x >> 1) * (2 * kRtM) + static_cast<int>(rank) * kRtM
+  const int row0 = PAIR ? static_cast<int>(blockIdx.x >> 1) * (2 * kRtM) +
+                               static_cast<int>(rank) * kRtM
                         : static_cast<int>(blockIdx.x) * kRtM;
   const int ks = static_cast<int>(blockIdx.y);
   const int kb0 = ks * p.kb_per_split;
