@@ -19,9 +19,12 @@ def lib():
 
 def test_library_exports_every_header_function(lib):
     names = L.header_functions()
-    assert len(names) >= 12
+    assert len(names) >= 20
+    assert "moe_layer_forward_w8" in names  # names with digits are parsed too
     for n in names:
         assert hasattr(lib, n), n
+        # the binding declares every header function's argument types
+        assert getattr(lib, n).argtypes is not None, n
 
 
 def test_shape_struct_layout():
