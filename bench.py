@@ -153,7 +153,8 @@ def stage_costs(wl, counts, hbm_peak, tc_peak, fp8_weights=False):
     wes, ws_ = (1, 4) if fp8_weights else (es, 0)  # weight element bytes, scale bytes
     c = {
         "route": {"bytes": T * H * es + H * E * es + bias + T * k * 8, "flops": 2 * T * H * E},
-        "align": {"bytes": T * k * 4 * 3 + A * (4 + 4 + 1) + E * 8, "flops": 0},
+        # read the expert ids once; write sorted_ids, slot_of and the drop mask; counts, offsets
+        "align": {"bytes": A * 4 + A * (4 + 4 + 1) + E * 8, "flops": 0},
         "gemm1": {"bytes": used * 2 * H * I * wes + used * 2 * I * ws_ + a_kept * H * es
                            + a_kept * I * es,
                   "flops": 4 * a_kept * H * I},
