@@ -81,6 +81,7 @@ def _signatures(lib):
         "moe_quantize_weights_fp8": (st, [_P, i64, i64, i64, _P, _P, _P]),
         "moe_grouped_ffn_w8": (st, [S] + [_P] * 11 + [sz, _P]),
         "moe_layer_forward_w8": (st, [S, O] + [_P] * 16 + [sz, _P]),
+        "moe_probe_stalled_wait": (st, [_P, sz, _P]),
     }
     for name, (res, args) in table.items():
         f = getattr(lib, name)
@@ -289,3 +290,8 @@ def moe_set_stage_events(events):
             e.record()
     arr = (_P * len(events))(*[e.cuda_event for e in events])
     return _check(lib().moe_set_stage_events(arr, len(events)))
+
+
+def moe_probe_stalled_wait(ws, ws_bytes, stream=None, check=True):
+    s = lib().moe_probe_stalled_wait(ptr(ws), int(ws_bytes), _stream(stream))
+    return _check(s) if check else s

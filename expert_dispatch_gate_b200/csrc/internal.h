@@ -93,6 +93,9 @@ cudaError_t launch_align_noalloc(const int32_t* topk_idx, int64_t A, int E, int 
 cudaError_t launch_plan_from_offsets(const int32_t* offsets, int E, int TB, int32_t* blk_prefix,
                                      cudaStream_t stream);
 
+// ---- probe.cu: one bounded wait that nothing satisfies (failure-detection test)
+cudaError_t launch_stalled_wait(int* err, cudaStream_t stream);
+
 // ---- combine.cu
 // Expert-major copy of the token rows: xs[s,:] = x[sorted_ids[s]/k,:] for kept slots.
 cudaError_t launch_dispatch_rows(int dtype, const void* x, const int32_t* sorted_ids,

@@ -666,6 +666,14 @@ moe_status moe_layer_forward(const moe_shape* shape, const void* x, const void* 
                               stream);
 }
 
+moe_status moe_probe_stalled_wait(void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_ws(ws, ws_bytes, 256);
+  if (st != MOE_OK) return st;
+  cudaError_t e = moe::launch_stalled_wait(at<int>(ws, 0), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stalled-wait probe");
+  return MOE_OK;
+}
+
 moe_status moe_check_error(void* ws, void* stream) {
   if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -678,7 +686,7 @@ moe_status moe_check_error(void* ws, void* stream) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
     if (e != cudaSuccess) return cuda_fail(e, "moe_check_error (clear)");
     const char* what = word == 1 ? "an expert id outside [0, E) in topk_idx"
-                       : word == 2 ? "a bounded pipeline wait ran out in an expert GEMM"
+                       : word == 2 ? "a bounded wait ran out in a pipelined kernel (stalled pipeline)"
                                    : "unknown device error";
     return fail(MOE_ERR_DEVICE, std::string("device error ") + std::to_string(word) + ": " + what);
   }

@@ -240,6 +240,14 @@ moe_status moe_layer_forward_w8(const moe_shape* shape, const moe_layer_opts* op
  * MOE_ERR_CUDA. */
 moe_status moe_check_error(void* ws, void* stream);
 
+/* Failure-detection check: launches one kernel whose single wait (the bounded mbarrier wait
+ * every pipelined kernel of the library uses) is never satisfied. After the wait limit (2 s)
+ * the kernel records device error 2 in the error word at the start of `ws` (ws_bytes >= 256)
+ * and returns, so moe_check_error then reports MOE_ERR_DEVICE and clears the word; the
+ * context stays usable. Returns MOE_ERR_WORKSPACE without launching when ws is NULL or too
+ * small. */
+moe_status moe_probe_stalled_wait(void* ws, size_t ws_bytes, void* stream);
+
 /* Static description of a status code. */
 const char* moe_status_string(moe_status status);
 

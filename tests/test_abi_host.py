@@ -169,3 +169,11 @@ def test_invalid_layer_opts_rejected_before_launch(lib, opts, why):
     assert L.moe_combine_ex(s, o, BAD, BAD, BAD, BAD, stream=0, check=False) == \
         L.MOE_ERR_INVALID_ARG, why
     assert L.last_error_detail()
+
+
+def test_stalled_wait_probe_refuses_a_missing_or_small_workspace(lib):
+    # validation happens on the host: nothing is launched, so no GPU is needed
+    assert L.moe_probe_stalled_wait(None, 0, check=False) == L.MOE_ERR_WORKSPACE
+    buf = ctypes.create_string_buffer(512)
+    addr = (ctypes.addressof(buf) + 15) & ~15
+    assert L.moe_probe_stalled_wait(addr, 128, check=False) == L.MOE_ERR_WORKSPACE
