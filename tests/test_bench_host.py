@@ -55,3 +55,5 @@ def test_launches_per_step():
     assert bench.launches_per_step(W.WORKLOADS["skewed"]) == 2 + 3 + 0 + 2 + 1
     # tiny f32: one fused CUDA-core router kernel
     assert bench.launches_per_step(W.WORKLOADS["tiny"]) == 1 + 1 + 0 + 2 + 1
+    # e4m3 expert weights always make the row copy
+    assert bench.launches_per_step(W.WORKLOADS["skewed"], fp8_weights=True) == 2 + 3 + 1 + 2 + 1
