@@ -271,15 +271,15 @@ def oracle_baseline(wl, dev, n_tokens, reps=1):
 
 # ------------------------------------------------------------------ the GPU arm
 
-def launches_per_step(wl, fp8_weights=False):
+def launches_per_step(wl):
     """Kernels one moe_layer_forward launches: router (tensor-core GEMM + top-k, or one fused
     CUDA-core kernel), align (one launch up to 65536 assignments, else three), two expert
     GEMMs, combine."""
     route = 2 if (wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0) else 1
     align = 1 if wl.T * wl.k <= 65536 else 3
-    # expert-major copy of the token rows before GEMM1: when CTA pairs run GEMM1, and always
-    # with e4m3 expert weights
-    copy = 1 if (wl.dtype == "bf16" and (wl.I % 256 == 0 or fp8_weights)) else 0
+    # expert-major copy of the token rows before GEMM1: every bf16 layer (GEMM1 runs on CTA
+    # pairs, and the e4m3-weight GEMM1 reads the copy too)
+    copy = 1 if wl.dtype == "bf16" else 0
     return route + align + copy + 2 + 1
 
 
@@ -450,7 +450,7 @@ def run_ours(args, world, rank, local):
     h2d = x_host.numel() * x_host.element_size()
     d2h = sum(t.numel() * t.element_size() for t in outs_host)
 
-    per_step = launches_per_step(wl, fp8_weights=fp8 is not None)
+    per_step = launches_per_step(wl)
     line = {
         "metric": METRIC,
         "value": round(value, 1),

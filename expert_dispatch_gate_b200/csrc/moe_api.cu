@@ -100,9 +100,9 @@ int token_block(const moe_shape& s, int32_t C) {
   return static_cast<int>(tb);
 }
 
-// GEMM1 reads the token rows from an expert-major copy made right after the grouping when
-// CTA pairs can share it (I % 256 == 0): the copy is streamed by TMA, half per CTA. Otherwise
-// GEMM1 gathers the rows straight from x.
+// GEMM1 reads the token rows from an expert-major copy made right after the grouping when it
+// runs on CTA pairs (every bf16 layer unless the build opts out of pairs): the copy is
+// streamed by TMA, half per CTA. Otherwise GEMM1 gathers the rows straight from x.
 bool gemm1_from_copy(const moe_shape& s) {
   return s.dtype == MOE_BF16 && moe::gemm1_uses_row_copy(s.I);
 }
