@@ -461,3 +461,90 @@ def test_quantize_weights_fp8_per_channel():
     a = np.abs(w.astype(np.float64))
     bound = np.maximum(a * 2.0 ** -4, 2.0 ** -10 * scale[:, None, :]) * (1 + 1e-6)
     assert np.all(np.abs(deq - w) <= bound)
+
+
+# ---------------------------------------------------------------- grouped routing through the whole layer
+
+
+def _grouped_fixture(golden_dir):
+    g = _load(golden_dir, "layer_grouped.json")
+    arr = {k_: np.asarray(g[k_], dtype=np.float64)
+           for k_ in ("x", "w_router", "w_gate", "w_up", "w_down", "shared", "out_bias")}
+    return g, arr
+
+
+def _grouped_layer(g, arr, n_group=None, topk_group=None):
+    return orc.layer_forward(arr["x"], arr["w_router"], arr["w_gate"], arr["w_up"], arr["w_down"],
+                             g["k"], g["capacity_factor"],
+                             n_group=g["n_group"] if n_group is None else n_group,
+                             topk_group=g["topk_group"] if topk_group is None else topk_group,
+                             shared=arr["shared"], shared_factor=g["shared_factor"],
+                             out_bias=arr["out_bias"])
+
+
+def _matches(res, g):
+    return (res["topk_idx"].tolist() == g["topk_idx"]
+            and np.allclose(res["topk_w"], np.asarray(g["topk_w"]), rtol=0, atol=g["tolerance"])
+            and np.allclose(res["out"], np.asarray(g["out"]), rtol=0, atol=g["tolerance"]))
+
+
+def test_route_grouped_hand_worked(golden_dir):
+    g, arr = _grouped_fixture(golden_dir)
+    logits, idx, w = orc.route_grouped(arr["x"], arr["w_router"], g["k"], g["n_group"],
+                                       g["topk_group"])
+    assert np.array_equal(logits, arr["x"].astype(np.float32))
+    assert idx.tolist() == g["topk_idx"]
+    np.testing.assert_allclose(w, np.asarray(g["topk_w"]), rtol=0, atol=g["tolerance"])
+    # the fixture's tokens all select differently without the group step
+    _, plain, _ = orc.route(arr["x"], arr["w_router"], g["k"])
+    assert plain.tolist() == g["plain_topk_idx"]
+    assert all(a != b for a, b in zip(plain.tolist(), g["topk_idx"]))
+
+
+def test_layer_grouped_hand_worked(golden_dir):
+    g, arr = _grouped_fixture(golden_dir)
+    res = _grouped_layer(g, arr)
+    assert res["C"] == g["C"]
+    assert res["topk_idx"].tolist() == g["topk_idx"]
+    np.testing.assert_allclose(res["topk_w"], np.asarray(g["topk_w"]), rtol=0, atol=g["tolerance"])
+    assert res["counts"].tolist() == g["counts"]
+    assert res["slot_of"].tolist() == g["slot_of"]
+    np.testing.assert_allclose(res["out"], np.asarray(g["out"]), rtol=0, atol=g["tolerance"])
+
+
+def test_layer_grouped_fixture_rejects_planted_mistakes(golden_dir, monkeypatch):
+    """The fixture fails for the plausible mistakes in the grouped layer path."""
+    g, arr = _grouped_fixture(golden_dir)
+    assert _matches(_grouped_layer(g, arr), g)
+    # n_group and topk_group swapped: one group means plain routing
+    assert not _matches(_grouped_layer(g, arr, n_group=g["topk_group"], topk_group=g["n_group"]), g)
+    with pytest.raises(ValueError):
+        orc.select_topk_grouped(arr["x"], g["k"], g["topk_group"], g["n_group"])
+
+    real = orc.route_grouped
+
+    def weights_from_plain_selection(x, w_router, k, n_group, topk_group, logit_bias=None,
+                                     logits=None):
+        lg, idx, _ = real(x, w_router, k, n_group, topk_group, logit_bias=logit_bias,
+                          logits=logits)
+        return lg, idx, orc.route_weights(lg, orc.select_topk(lg, k))
+
+    monkeypatch.setattr(orc, "route_grouped", weights_from_plain_selection)
+    assert not _matches(_grouped_layer(g, arr), g)
+
+    def groups_scored_by_top1(x, w_router, k, n_group, topk_group, logit_bias=None, logits=None):
+        lg = orc.router_logits(x, w_router, logit_bias) if logits is None else logits
+        l32 = np.asarray(lg, dtype=np.float32)
+        T, E = l32.shape
+        gs = E // n_group
+        sc = l32.reshape(T, n_group, gs).max(axis=2)
+        keep = np.argsort(-sc, axis=1, kind="stable")[:, :topk_group]
+        masked = np.full_like(l32, -np.inf)
+        for t in range(T):
+            for grp in keep[t]:
+                masked[t, grp * gs:(grp + 1) * gs] = l32[t, grp * gs:(grp + 1) * gs]
+        idx = orc.select_topk(masked, k)
+        return l32, idx, orc.route_weights(l32, idx)
+
+    monkeypatch.setattr(orc, "route_grouped", groups_scored_by_top1)
+    assert not _matches(_grouped_layer(g, arr), g)
