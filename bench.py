@@ -39,6 +39,7 @@ from expert_dispatch_gate_b200 import workloads as W  # noqa: E402
 METRIC = "MoE-layer tokens/s (E=256,k=8,T=4096,1 GPU); route+align+combine HBM GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 STAGES = ["route", "align", "gemm1", "gemm2", "combine"]
+L2_BYTES = 126 << 20  # B200 L2
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -288,113 +289,181 @@ def workload_of(args):
     return wl.with_tokens(args.tokens) if args.tokens else wl
 
 
+def layer_config(wl, capacity, world, fp8):
+    """The `config` object of a layer line; the reference arm prints the same keys."""
+    wes = 1 if fp8 else (2 if wl.dtype == "bf16" else 4)
+    wb = 3 * wl.E * wl.H * wl.I * wes
+    return {"workload": wl.describe(), "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
+            "capacity": int(capacity),
+            "parallelism": "replicas" if world > 1 else "single-gpu",
+            "expert_weights": ("e4m3 codes + float32 per-channel scales (W8A16)"
+                               if fp8 else wl.dtype),
+            "l2": (("inputs larger than L2: %.1f GB of expert weights streamed per step"
+                    % (wb / 1e9)) if wb > L2_BYTES else
+                   "inputs fit in L2 (%.1f MB of expert weights); L2 not flushed" % (wb / 1e6))}
+
+
+class LayerRun:
+    """One workload's layer on the device: inputs, outputs, workspace and the forward call."""
+
+    def __init__(self, wl, dev, fp8=False):
+        self.wl, self.dev = wl, dev
+        self.inp = W.make_inputs(wl, dev)
+        self.shape = M.shape_of(wl.T, wl.H, wl.E, wl.k, wl.I, wl.capacity_factor, wl.dtype)
+        self.ws = M.Workspace(self.shape, dev)
+        self.outs = [torch.empty((wl.T, wl.H), dtype=wl.torch_dtype, device=dev),
+                     torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev),
+                     torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev),
+                     torch.empty(wl.E, dtype=torch.int32, device=dev),
+                     torch.empty(wl.T * wl.k, dtype=torch.uint8, device=dev)]
+        self.stream = torch.cuda.current_stream(dev)
+        self.fp8 = None
+        if fp8:
+            # e4m3 expert weights, quantised once on the device before anything is timed
+            self.fp8 = M.Fp8Weights(self.inp["w_gate"], self.inp["w_up"], self.inp["w_down"])
+            torch.cuda.synchronize()
+
+    def forward(self, x, o):
+        inp, ws = self.inp, self.ws
+        if self.fp8 is not None:
+            L.moe_layer_forward_w8(self.shape, None, x, inp["w_router"], inp["logit_bias"],
+                                   *self.fp8.args(), o[0], None, o[1], o[2], o[3], o[4], ws.buf,
+                                   ws.nbytes, self.stream)
+        else:
+            L.moe_layer_forward(self.shape, x, inp["w_router"], inp["logit_bias"], inp["w_gate"],
+                                inp["w_up"], inp["w_down"], o[0], None, o[1], o[2], o[3], o[4],
+                                ws.buf, ws.nbytes, self.stream)
+
+    def step(self):
+        self.forward(self.inp["x"], self.outs)
+
+    def time_stages(self, steps, warmup, world, local, peaks):
+        """Device-resident timing: total CUDA-event time over `steps` layer calls (max over
+        ranks) and the per-stage times the library records on its stream; returns the layer
+        line's timing keys."""
+        wl, stream = self.wl, self.stream
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+        self.ws.check()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in STAGES] for _ in range(steps)]
+        for e in ev:
+            for x in e:
+                x.record(stream)
+        for s in starts:
+            s.record(stream)
+        torch.cuda.synchronize()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clk:
+            t_start.record(stream)
+            for i in range(steps):
+                starts[i].record(stream)
+                L.moe_set_stage_events(ev[i])
+                self.step()
+            t_end.record(stream)
+            torch.cuda.synchronize()
+        L.moe_set_stage_events(None)
+        barrier(world)
+        ms = t_start.elapsed_time(t_end)
+        self.ws.check()
+        ms_max = max_over_ranks(ms, world, "cuda")
+        value = aggregate_throughput(wl.T * steps, world, ms_max / 1e3)
+        st_ms = {s: 0.0 for s in STAGES}
+        for i in range(steps):
+            prev = starts[i]
+            for j, s in enumerate(STAGES):
+                st_ms[s] += prev.elapsed_time(ev[i][j]) / steps
+                prev = ev[i][j]
+        cnt = self.outs[3].cpu().numpy()
+        fp8 = self.fp8 is not None
+        cost = stage_costs(wl, cnt, peaks["hbm_gbs"], peaks["bf16_tflops_sustained"],
+                           fp8_weights=fp8)
+        kernels = {}
+        for s in STAGES:
+            t = st_ms[s] * 1e-3
+            kernels[s] = {"us": round(st_ms[s] * 1e3, 2),
+                          "gbs": round(cost[s]["bytes"] / t / 1e9, 1),
+                          "tflops": round(cost[s]["flops"] / t / 1e12, 1),
+                          "bytes": cost[s]["bytes"], "flops": cost[s]["flops"],
+                          "frac_hbm": round(cost[s]["bytes"] / t / 1e9 / peaks["hbm_gbs"], 3)}
+        dom = max(["gemm1", "gemm2"], key=lambda s: st_ms[s])
+        t_dom = st_ms[dom] * 1e-3
+        bound = "hbm" if cost[dom]["t_hbm_us"] >= cost[dom]["t_tc_us"] else "tensor"
+        if bound == "hbm":
+            ach, peak, unit = cost[dom]["bytes"] / t_dom / 1e9, peaks["hbm_gbs"], "GB/s"
+        else:
+            ach, peak, unit = (cost[dom]["flops"] / t_dom / 1e12, peaks["bf16_tflops_sustained"],
+                               "TFLOP/s")
+        tflops_dom = cost[dom]["flops"] / t_dom / 1e12
+        rac_bytes = sum(cost[s]["bytes"] for s in ("route", "align", "combine"))
+        rac_t = sum(st_ms[s] for s in ("route", "align", "combine")) * 1e-3
+        return {
+            "value": value, "ms_max": ms_max, "cnt": cnt, "kernels": kernels, "clocks": clk.summary(),
+            "roofline": {"kernel": dom, "bound": bound, "achieved": round(ach, 1), "peak": peak,
+                         "unit": unit, "frac": round(ach / peak, 3),
+                         "peak_source": "%s (%s)" % (peaks.get("_source", "measured"),
+                                                     "hbm_gbs" if bound == "hbm"
+                                                     else "bf16_tflops_sustained"),
+                         "algorithmic_bytes": cost[dom]["bytes"],
+                         "tensor_frac": round(tflops_dom / peaks["bf16_tflops_sustained"], 3),
+                         "tensor_frac_burst": round(tflops_dom / peaks["bf16_tflops"], 3)},
+            "route_align_combine_gbs": round(rac_bytes / rac_t / 1e9, 1),
+            "route_align_combine_frac": round(rac_bytes / rac_t / 1e9 / peaks["hbm_gbs"], 3),
+        }
+
+    def release(self):
+        del self.inp, self.ws, self.outs, self.fp8
+        torch.cuda.empty_cache()
+
+
+def other_workloads(args, dev, world, local, peaks):
+    """The other layer configurations, timed the same way as the headline (device-resident
+    inputs, stage events): Mixtral-shaped, skewed-load, and the decode sweep."""
+    res = {}
+    cases = [("mixtral", W.WORKLOADS["mixtral"]), ("skewed", W.WORKLOADS["skewed"])]
+    cases += [(f"decode_T{t}", W.WORKLOADS["decode"].with_tokens(t)) for t in W.DECODE_TOKENS]
+    for key, wl in cases:
+        run = LayerRun(wl, dev)
+        t = run.time_stages(args.steps, args.warmup, world, local, peaks)
+        res[key] = {"workload": wl.describe(), "value": round(t["value"], 1), "unit": "tokens/s",
+                    "ms_per_step": round(t["ms_max"] / args.steps, 4),
+                    "stage_us": {s: t["kernels"][s]["us"] for s in STAGES},
+                    "roofline": t["roofline"],
+                    "route_align_combine_gbs": t["route_align_combine_gbs"],
+                    "kept_assignments": int(t["cnt"].sum()),
+                    "experts_used": int((t["cnt"] > 0).sum()),
+                    "gpu_launches": launches_per_step(wl) * args.steps}
+        run.release()
+    return res
+
+
 def run_ours(args, world, rank, local):
     wl = workload_of(args)
     dev = torch.device("cuda", local)
-    inp = W.make_inputs(wl, dev)
     peaks, peaks_src = load_peaks()
-    shape = M.shape_of(wl.T, wl.H, wl.E, wl.k, wl.I, wl.capacity_factor, wl.dtype)
-    ws = M.Workspace(shape, dev)
-    out = torch.empty((wl.T, wl.H), dtype=wl.torch_dtype, device=dev)
-    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
-    wts = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
-    counts = torch.empty(wl.E, dtype=torch.int32, device=dev)
-    drop = torch.empty(wl.T * wl.k, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    fp8 = None
-    if args.weights == "fp8":
-        # e4m3 expert weights, quantised once on the device before anything is timed
-        fp8 = M.Fp8Weights(inp["w_gate"], inp["w_up"], inp["w_down"])
-        torch.cuda.synchronize()
-
-    def forward(x, o):
-        if fp8 is not None:
-            L.moe_layer_forward_w8(shape, None, x, inp["w_router"], inp["logit_bias"], *fp8.args(),
-                                   o[0], None, o[1], o[2], o[3], o[4], ws.buf, ws.nbytes, stream)
-        else:
-            L.moe_layer_forward(shape, x, inp["w_router"], inp["logit_bias"], inp["w_gate"],
-                                inp["w_up"], inp["w_down"], o[0], None, o[1], o[2], o[3], o[4],
-                                ws.buf, ws.nbytes, stream)
-
-    def step(x=inp["x"]):
-        forward(x, (out, idx, wts, counts, drop))
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    ws.check()
-
-    # per-stage events: one set per timed step
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in STAGES] for _ in range(args.steps)]
-    for e in ev:
-        for x in e:
-            x.record(stream)
-    for s in starts:
-        s.record(stream)
-    torch.cuda.synchronize()
-
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t_start.record(stream)
-        for i in range(args.steps):
-            starts[i].record(stream)
-            L.moe_set_stage_events(ev[i])
-            step()
-        t_end.record(stream)
-        torch.cuda.synchronize()
-    L.moe_set_stage_events(None)
-    barrier(world)
-    ms = t_start.elapsed_time(t_end)
-    ws.check()
-    ms_max = max_over_ranks(ms, world, "cuda")
-    secs = ms_max / 1e3
-    value = aggregate_throughput(wl.T * args.steps, world, secs)
-
-    # per-stage durations (ms), averaged over the timed steps
-    st_ms = {s: 0.0 for s in STAGES}
-    for i in range(args.steps):
-        prev = starts[i]
-        for j, s in enumerate(STAGES):
-            st_ms[s] += prev.elapsed_time(ev[i][j]) / args.steps
-            prev = ev[i][j]
-    cnt = counts.cpu().numpy()
-    cost = stage_costs(wl, cnt, peaks["hbm_gbs"], peaks["bf16_tflops_sustained"],
-                       fp8_weights=fp8 is not None)
-    kernels = {}
-    for s in STAGES:
-        t = st_ms[s] * 1e-3
-        kernels[s] = {"us": round(st_ms[s] * 1e3, 2),
-                      "gbs": round(cost[s]["bytes"] / t / 1e9, 1),
-                      "tflops": round(cost[s]["flops"] / t / 1e12, 1),
-                      "bytes": cost[s]["bytes"], "flops": cost[s]["flops"],
-                      "frac_hbm": round(cost[s]["bytes"] / t / 1e9 / peaks["hbm_gbs"], 3)}
-    dom = max(["gemm1", "gemm2"], key=lambda s: st_ms[s])
-    t_dom = st_ms[dom] * 1e-3
-    bound = "hbm" if cost[dom]["t_hbm_us"] >= cost[dom]["t_tc_us"] else "tensor"
-    if bound == "hbm":
-        ach, peak, unit = cost[dom]["bytes"] / t_dom / 1e9, peaks["hbm_gbs"], "GB/s"
-    else:
-        ach, peak, unit = cost[dom]["flops"] / t_dom / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
-    rac_bytes = sum(cost[s]["bytes"] for s in ("route", "align", "combine"))
-    rac_t = sum(st_ms[s] for s in ("route", "align", "combine")) * 1e-3
+    peaks["_source"] = peaks_src
+    run = LayerRun(wl, dev, fp8=args.weights == "fp8")
+    inp, stream = run.inp, run.stream
+    t = run.time_stages(args.steps, args.warmup, world, local, peaks)
+    cnt = t["cnt"]
+    dom = t["roofline"]["kernel"]
+    t["roofline"]["traffic"] = recorded_traffic(dom + ("_w8" if run.fp8 is not None else ""),
+                                                args.workload)
 
     # End to end through the C ABI with host buffers: every step copies its x in from pinned host
     # memory and its outputs back out. Measured twice: serially (copy in, forward, copy out on one
     # stream) and as a throughput pipeline, where step i+1's copy in and step i-1's copy out run
     # on two copy streams while step i computes (x and the outputs double-buffered on the device).
     x_host = inp["x"].cpu().pin_memory()
-    outs_dev = [out, idx, wts, counts, drop]
-    outs_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs_dev]
+    outs_dev = run.outs
+    outs_host = [torch.empty(t_.shape, dtype=t_.dtype, pin_memory=True) for t_ in outs_dev]
     x_devs = [torch.empty_like(inp["x"]) for _ in range(2)]
-    outs_devs = [outs_dev, [torch.empty_like(t) for t in outs_dev]]
-
-    def fwd(x, o):
-        forward(x, o)
+    outs_devs = [outs_dev, [torch.empty_like(t_) for t_ in outs_dev]]
+    fwd = run.forward
 
     def e2e_serial(n):
         for _ in range(n):
@@ -446,43 +515,30 @@ def run_ours(args, world, rank, local):
 
     e2e_serial_ms = timed(e2e_serial)
     e2e_ms = timed(e2e_pipelined)
-    ws.check()
+    run.ws.check()
     h2d = x_host.numel() * x_host.element_size()
-    d2h = sum(t.numel() * t.element_size() for t in outs_host)
+    d2h = sum(t_.numel() * t_.element_size() for t_ in outs_host)
 
     per_step = launches_per_step(wl)
     line = {
         "metric": METRIC,
-        "value": round(value, 1),
+        "value": round(t["value"], 1),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms_max / args.steps, 4),
+        "ms_per_step": round(t["ms_max"] / args.steps, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": wl.dtype,
         "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights; no dataset)",
-        "config": {"workload": wl.describe(), "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k,
-                   "I": wl.I, "capacity": int(L.moe_capacity(shape)),
-                   "kept_assignments": int(cnt.sum()), "experts_used": int((cnt > 0).sum()),
-                   "parallelism": "replicas" if world > 1 else "single-gpu",
-                   "expert_weights": ("e4m3 codes + float32 per-channel scales (W8A16)"
-                                      if fp8 is not None else wl.dtype),
-                   "l2": "inputs larger than L2: %.1f GB of expert weights streamed per step"
-                         % (3 * wl.E * wl.H * wl.I * (1 if fp8 is not None else
-                                                      (2 if wl.dtype == "bf16" else 4)) / 1e9)},
-        "roofline": {"kernel": dom, "bound": bound, "achieved": round(ach, 1),
-                     "peak": peak, "unit": unit, "frac": round(ach / peak, 3),
-                     "peak_source": f"{peaks_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
-                     "traffic": recorded_traffic(dom + ("_w8" if fp8 is not None else ""),
-                                                 args.workload),
-                     "algorithmic_bytes": cost[dom]["bytes"],
-                     "tensor_frac": round(cost[dom]["flops"] / t_dom / 1e12 / peaks["bf16_tflops_sustained"], 3)},
-        "route_align_combine_gbs": round(rac_bytes / rac_t / 1e9, 1),
-        "route_align_combine_frac": round(rac_bytes / rac_t / 1e9 / peaks["hbm_gbs"], 3),
-        "kernels": kernels,
+        "config": layer_config(wl, L.moe_capacity(run.shape), world, run.fp8 is not None),
+        "routing": {"kept_assignments": int(cnt.sum()), "experts_used": int((cnt > 0).sum())},
+        "roofline": t["roofline"],
+        "route_align_combine_gbs": t["route_align_combine_gbs"],
+        "route_align_combine_frac": t["route_align_combine_frac"],
+        "kernels": t["kernels"],
         "e2e": {"value": round(aggregate_throughput(wl.T * args.steps, world, e2e_ms / 1e3), 1),
                 "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "copies": "each step's copies overlap the neighbouring steps' forward passes "
@@ -490,10 +546,15 @@ def run_ours(args, world, rank, local):
                 "serial_value": round(aggregate_throughput(wl.T * args.steps, world,
                                                            e2e_serial_ms / 1e3), 1)},
         "gpu_launches": per_step * args.steps,
-        "clocks": clk.summary(),
+        "clocks": t["clocks"],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_baseline(wl, inp, args.cpu_sample_tokens)
+    run.release()
+    del x_devs, outs_devs, outs_dev, inp
+    if (world == 1 and args.workload == "fine" and not args.no_other_workloads
+            and args.weights == "bf16" and not args.tokens):
+        line["other_workloads"] = other_workloads(args, dev, world, local, peaks)
     return line
 
 
@@ -583,40 +644,52 @@ def run_rac_sweep(args, local):
 
 
 def run_reference(args, world, rank, local):
-    """The reference arm: the CPU oracle itself, on the same workload, bounded samples."""
+    """The reference arm: the CPU oracle itself on the host cores, on the same workload and
+    config. Each step is one bounded sample: routing and grouping over all T tokens (capacity
+    ranks depend on every token), the expert FFN and combine on `--cpu-sample-tokens` sampled
+    tokens (the same sample size as the GPU arm's cpu_baseline). `ms_per_step` is the measured
+    wall time of one such sample; `value` extrapolates the sample to tokens/s over the whole
+    batch. Under torchrun only rank 0 runs it."""
     if rank != 0:
         return None
     wl = workload_of(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = W.make_inputs(wl, dev)
-    n_tok = max(1, args.cpu_sample_tokens // 4)
+    n_tok = max(1, args.cpu_sample_tokens)
     from oracle import moe_oracle as orc
     host = {"x": inp["x"].float().cpu().numpy(), "w_router": inp["w_router"].float().cpu().numpy(),
             "logit_bias": None if inp["logit_bias"] is None else inp["logit_bias"].cpu().numpy()}
     logits = orc.router_logits(host["x"], host["w_router"], host["logit_bias"])
     idx = orc.select_topk(logits, wl.k)
+    C = orc.capacity(wl.T, wl.k, wl.E, wl.capacity_factor)
     rng = np.random.default_rng(0)
     toks = rng.choice(wl.T, size=min(n_tok, wl.T), replace=False)
     experts = sorted(set(idx[toks].reshape(-1).tolist()))
     weights = [HostExperts(inp[n], experts) for n in ("w_gate", "w_up", "w_down")]
+    del inp
     for _ in range(args.warmup):
         oracle_sample_time(wl, host, weights, n_tok)
-    per = []
+    per, wall = [], []
     for _ in range(args.steps):
+        w0 = time.perf_counter()
         t_ra, t_ffn, s = oracle_sample_time(wl, host, weights, n_tok)
+        wall.append(time.perf_counter() - w0)
         per.append(t_ra / wl.T + t_ffn / s)
     per_token = sum(per) / len(per)
     value = 1.0 / per_token
+    sample = (f"per step: float64 NumPy oracle, routing + capacity grouping over all {wl.T} "
+              f"tokens, expert SwiGLU FFN + combine on {s} sampled tokens; tokens/s = "
+              f"1 / (t_route_align/T + t_ffn/{s})")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(per_token * wl.T * 1e3, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.describe(), "T": wl.T},
+        "ms_per_step": round(sum(wall) / len(wall) * 1e3, 3),
+        "ms_per_step_extrapolated_to_T": round(per_token * wl.T * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights; no dataset)",
+        "config": layer_config(wl, C, world, False),
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cpu_threads(),
-                         "kind": "oracle",
-                         "sample": f"per step: routing + grouping over all {wl.T} tokens, FFN + "
-                                   f"combine on {n_tok} sampled tokens, extrapolated to T"},
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -633,6 +706,9 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=0, help="override T (decode sweep)")
     ap.add_argument("--cpu-sample-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="time only the selected workload (by default a one-GPU run also times "
+                         "the Mixtral-shaped, skewed and decode layers under other_workloads)")
     ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
                     help="expert weights: the layer dtype (default) or e4m3 + per-channel scales")
     ap.add_argument("--sweep", choices=["route-align-combine"], default=None,

@@ -56,3 +56,22 @@ def test_launches_per_step():
     assert bench.launches_per_step(W.WORKLOADS["skewed"]) == 2 + 3 + 1 + 2 + 1
     # tiny f32: one fused CUDA-core router kernel
     assert bench.launches_per_step(W.WORKLOADS["tiny"]) == 1 + 1 + 0 + 2 + 1
+
+
+def test_reference_arm_line_matches_our_config_and_reports_its_own_wall_time():
+    """The reference arm (the oracle on the host) prints the same config keys as the GPU arm,
+    the measured wall time of its sample as ms_per_step, and the extrapolation separately."""
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                        "--steps", "3", "--warmup", "3"], capture_output=True, text=True,
+                       cwd=bench.ROOT, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    wl = W.WORKLOADS["tiny"]
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["config"] == bench.layer_config(wl, 64, 1, False)
+    assert line["ms_per_step"] <= line["ms_per_step_extrapolated_to_T"] * 10
+    assert line["cpu_baseline"]["value"] == line["value"] == line["e2e"]["value"]
+    assert "8 sampled tokens" in line["cpu_baseline"]["sample"]
