@@ -82,6 +82,9 @@ def _signatures(lib):
         "moe_grouped_ffn_w8": (st, [S] + [_P] * 11 + [sz, _P]),
         "moe_layer_forward_w8": (st, [S, O] + [_P] * 16 + [sz, _P]),
         "moe_probe_stalled_wait": (st, [_P, sz, _P]),
+        "moe_ep_plan": (st, [S, ctypes.c_int32, ctypes.c_int32, i64] + [_P] * 7 + [_P, sz, _P]),
+        "moe_ep_dispatch": (st, [S, ctypes.c_int32, _P, _P, _P, _P, _P]),
+        "moe_ep_combine": (st, [S, ctypes.c_int32, _P, _P, _P, _P, _P, _P]),
     }
     for name, (res, args) in table.items():
         f = getattr(lib, name)
@@ -198,6 +201,26 @@ def moe_grouped_ffn(shape, x, sorted_ids, offsets, w_gate, w_up, w_down, y_slots
 def moe_combine(shape, y_slots, slot_of, topk_w, out, stream=None, check=True):
     s = lib().moe_combine(ctypes.byref(shape), ptr(y_slots), ptr(slot_of), ptr(topk_w), ptr(out),
                           _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_ep_plan(shape, R, rank, T_total, topk_idx, slot_of_local, offsets_local, counts_all,
+                owner, slot, own_offsets, ws, ws_bytes, stream=None, check=True):
+    s = lib().moe_ep_plan(ctypes.byref(shape), int(R), int(rank), int(T_total), ptr(topk_idx),
+                          ptr(slot_of_local), ptr(offsets_local), ptr(counts_all), ptr(owner),
+                          ptr(slot), ptr(own_offsets), ptr(ws), int(ws_bytes), _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_ep_dispatch(shape, R, x, owner, slot, peer_xs, stream=None, check=True):
+    s = lib().moe_ep_dispatch(ctypes.byref(shape), int(R), ptr(x), ptr(owner), ptr(slot),
+                              ptr(peer_xs), _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_ep_combine(shape, R, peer_y, owner, slot, topk_w, out, stream=None, check=True):
+    s = lib().moe_ep_combine(ctypes.byref(shape), int(R), ptr(peer_y), ptr(owner), ptr(slot),
+                             ptr(topk_w), ptr(out), _stream(stream))
     return _check(s) if check else s
 
 

@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmoe.so")
 SOURCES = ["moe_api.cu", "route.cu", "route_tc.cu", "align.cu", "combine.cu", "ffn_simt.cu",
-           "ffn_tc.cu", "quant.cu", "probe.cu"]
+           "ffn_tc.cu", "quant.cu", "probe.cu", "ep.cu"]
 # every header under csrc/: a change to any of them rebuilds every object
 HEADERS = sorted(f for f in os.listdir(CSRC) if f.endswith((".cuh", ".h")))
 

@@ -96,6 +96,17 @@ cudaError_t launch_plan_from_offsets(const int32_t* offsets, int E, int TB, int3
 // ---- probe.cu: one bounded wait that nothing satisfies (failure-detection test)
 cudaError_t launch_stalled_wait(int* err, cudaStream_t stream);
 
+// ---- ep.cu (expert parallelism over R ranks; see the entry points in moe.h)
+cudaError_t launch_ep_plan(const int32_t* topk_idx, const int32_t* slot_of_local,
+                           const int32_t* offsets_local, const int32_t* counts_all, int64_t A,
+                           int E, int R, int rank, int C, int32_t* owner, int32_t* slot,
+                           int32_t* own_offsets, int* err, int num_sms, cudaStream_t stream);
+cudaError_t launch_ep_dispatch(int dtype, const void* x, const int32_t* owner, const int32_t* slot,
+                               void* const* peer_xs, int64_t A, int k, int H, cudaStream_t stream);
+cudaError_t launch_ep_combine(int dtype, const void* const* peer_y, const int32_t* owner,
+                              const int32_t* slot, const float* topk_w, void* out, int64_t T,
+                              int H, int k, cudaStream_t stream);
+
 // ---- combine.cu
 // Expert-major copy of the token rows: xs[s,:] = x[sorted_ids[s]/k,:] for kept slots.
 cudaError_t launch_dispatch_rows(int dtype, const void* x, const int32_t* sorted_ids,

@@ -500,6 +500,81 @@ moe_status moe_combine(const moe_shape* shape, const void* y_slots, const int32_
   return moe_combine_ex(shape, nullptr, y_slots, slot_of, topk_w, out, stream);
 }
 
+// ---- expert parallelism (ep.cu)
+
+static moe_status check_ep(const moe_shape* shape, int32_t R) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (R < 1 || R > shape->E || shape->E % R != 0)
+    return fail(MOE_ERR_INVALID_ARG, "the E experts must split evenly over R >= 1 ranks");
+  return MOE_OK;
+}
+
+moe_status moe_ep_plan(const moe_shape* shape, int32_t R, int32_t rank, int64_t T_total,
+                       const int32_t* topk_idx, const int32_t* slot_of_local,
+                       const int32_t* offsets_local, const int32_t* counts_all, int32_t* owner,
+                       int32_t* slot, int32_t* own_offsets, void* ws, size_t ws_bytes,
+                       void* stream) {
+  moe_status st = check_ep(shape, R);
+  if (st != MOE_OK) return st;
+  if (rank < 0 || rank >= R) return fail(MOE_ERR_INVALID_ARG, "rank outside [0, R)");
+  if (T_total < shape->T) return fail(MOE_ERR_INVALID_ARG, "T_total below this rank's T");
+  st = check_ws(ws, ws_bytes, 256);
+  if (st != MOE_OK) return st;
+  REQUIRE_PTR(counts_all, "counts_all");
+  REQUIRE_PTR(own_offsets, "own_offsets");
+  if (shape->T > 0) {
+    REQUIRE_PTR(topk_idx, "topk_idx");
+    REQUIRE_PTR(slot_of_local, "slot_of_local");
+    REQUIRE_PTR(offsets_local, "offsets_local");
+    REQUIRE_PTR(owner, "owner");
+    REQUIRE_PTR(slot, "slot");
+  }
+  moe_shape whole = *shape;
+  whole.T = T_total;
+  const int C = capacity_of(whole);
+  cudaError_t e = moe::launch_ep_plan(topk_idx, slot_of_local, offsets_local, counts_all,
+                                      shape->T * shape->k, shape->E, R, rank, C, owner, slot,
+                                      own_offsets, at<int>(ws, 0), num_sms(),
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "expert-parallel plan");
+  return MOE_OK;
+}
+
+moe_status moe_ep_dispatch(const moe_shape* shape, int32_t R, const void* x,
+                           const int32_t* owner, const int32_t* slot, void* const* peer_xs,
+                           void* stream) {
+  moe_status st = check_ep(shape, R);
+  if (st != MOE_OK) return st;
+  if (shape->T == 0) return MOE_OK;
+  REQUIRE_PTR(x, "x");
+  REQUIRE_PTR(owner, "owner");
+  REQUIRE_PTR(slot, "slot");
+  REQUIRE_PTR(peer_xs, "peer_xs");
+  cudaError_t e = moe::launch_ep_dispatch(shape->dtype, x, owner, slot, peer_xs,
+                                          shape->T * shape->k, shape->k, shape->H,
+                                          static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "expert-parallel dispatch");
+  return MOE_OK;
+}
+
+moe_status moe_ep_combine(const moe_shape* shape, int32_t R, const void* const* peer_y,
+                          const int32_t* owner, const int32_t* slot, const float* topk_w,
+                          void* out, void* stream) {
+  moe_status st = check_ep(shape, R);
+  if (st != MOE_OK) return st;
+  if (shape->T == 0) return MOE_OK;
+  REQUIRE_PTR(peer_y, "peer_y");
+  REQUIRE_PTR(owner, "owner");
+  REQUIRE_PTR(slot, "slot");
+  REQUIRE_PTR(topk_w, "topk_w");
+  REQUIRE_PTR(out, "out");
+  cudaError_t e = moe::launch_ep_combine(shape->dtype, peer_y, owner, slot, topk_w, out, shape->T,
+                                         shape->H, shape->k, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "expert-parallel combine");
+  return MOE_OK;
+}
+
 }  // extern "C"
 
 namespace {

@@ -113,19 +113,29 @@ __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// This lane's best entry not yet taken: the largest key, the lower index on equal keys (entries
-// are scanned in ascending index order, and only a strictly larger key replaces the best).
-// Lane l holds experts VPL*l + i.
+// This lane's two best entries not yet taken, in (key descending, index ascending) order:
+// entries are scanned in ascending index order and only a strictly larger key displaces one.
+// Lane l holds experts VPL*l + i. Key 0 (no finite float) marks "none".
 template <int VPL>
-__device__ __forceinline__ void lane_best(const uint32_t (&key)[VPL], uint32_t taken, int lane,
-                                          uint32_t& bk, int& bi) {
+__device__ __forceinline__ void lane_best2(const uint32_t (&key)[VPL], uint32_t taken, int lane,
+                                           uint32_t& bk, int& bi, uint32_t& sk, int& si) {
   bk = 0u;
   bi = 0x7fffffff;
+  sk = 0u;
+  si = 0x7fffffff;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
-    if (!((taken >> i) & 1u) && key[i] > bk) {
-      bk = key[i];
-      bi = VPL * lane + i;
+    if (!((taken >> i) & 1u)) {
+      const uint32_t kk = key[i];
+      if (kk > bk) {
+        sk = bk;
+        si = bi;
+        bk = kk;
+        bi = VPL * lane + i;
+      } else if (kk > sk) {
+        sk = kk;
+        si = VPL * lane + i;
+      }
     }
   }
 }
@@ -135,16 +145,18 @@ __device__ __forceinline__ void lane_best(const uint32_t (&key)[VPL], uint32_t t
 // and writes idx_row[0..k) and w_row[0..k). Each round takes the warp's largest key with one
 // max-reduction (redux.sync). Lanes hold disjoint ascending index ranges, so among the lanes
 // holding that key the lowest lane has the lowest expert index (ballot + find-first); one
-// shuffle broadcasts it, and only the winning lane rescans its own entries.
+// shuffle broadcasts it. Each lane keeps its two best remaining entries: the winning lane
+// promotes its second, and rescans only when it wins while holding no second (its second
+// was promoted on an earlier win), which with k picks spread over 32 lanes is rare.
 template <int VPL>
 __device__ __forceinline__ void warp_select_topk(const float (&v)[VPL], uint32_t taken, int k,
                                                  int lane, int32_t* idx_row, float* w_row) {
   uint32_t key[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) key[i] = order_key(v[i]);
-  uint32_t bk;
-  int bi;
-  lane_best<VPL>(key, taken, lane, bk, bi);
+  uint32_t bk, sk;
+  int bi, si;
+  lane_best2<VPL>(key, taken, lane, bk, bi, sk, si);
   float my_v = 0.f, top = 0.f;
   int my_i = 0;
   for (int j = 0; j < k; ++j) {
@@ -159,7 +171,14 @@ __device__ __forceinline__ void warp_select_topk(const float (&v)[VPL], uint32_t
     if (j == 0) top = val;
     if (lane == wl) {
       taken |= 1u << (win - VPL * lane);
-      lane_best<VPL>(key, taken, lane, bk, bi);
+      if (sk != 0u) {
+        bk = sk;
+        bi = si;
+        sk = 0u;
+        si = 0x7fffffff;
+      } else {
+        lane_best2<VPL>(key, taken, lane, bk, bi, sk, si);
+      }
     }
   }
   write_selection(lane, k, my_v, my_i, top, idx_row, w_row);

@@ -235,6 +235,47 @@ moe_status moe_layer_forward_w8(const moe_shape* shape, const moe_layer_opts* op
                                 int32_t* counts, uint8_t* drop_mask, void* ws, size_t ws_bytes,
                                 void* stream);
 
+/* Expert parallelism over R ranks, [P4] section "Token 分发的通信瓶颈" (rows go to the devices
+ * that own their experts and the outputs come back) with the capacity of section
+ * "昇腾NPU的通信计算重叠". Rank r holds its own T tokens (shape->T) and the experts
+ * [r*E/R, (r+1)*E/R); shape->E is the total E, which R must divide. The ranks compute what one
+ * device computes on the concatenated batch (rank 0's tokens first): capacity C from T_total,
+ * drops by the global token order, each expert's rows expert-major in that order at its owner.
+ * Steps on rank r: moe_route; moe_align with capacity_factor <= 0 (the local grouping);
+ * gather every rank's `counts` into counts_all [R,E] (a collective between devices);
+ * moe_ep_plan; moe_ep_dispatch on every rank; moe_grouped_ffn on the owner's rows (E/R
+ * experts, k = 1, identity sorted_ids, own_offsets); moe_ep_combine on every rank.
+ *
+ * moe_ep_plan: owner [T*k] (rank owning the expert, -1 if dropped) and slot [T*k] (row in the
+ * owner's slot-major buffer, -1 if dropped) of this rank's assignments, and own_offsets
+ * [E/R + 1], the first slot of each of this rank's experts and the total. topk_idx [T,k],
+ * slot_of_local [T*k], offsets_local [E+1] are moe_align's outputs for this rank's tokens
+ * without a capacity limit; counts_all [R,E] int32 holds every rank's local counts. An expert
+ * id outside [0, E) sets the error word at the start of `ws` (ws_bytes >= 256) and that
+ * assignment is dropped. */
+moe_status moe_ep_plan(const moe_shape* shape, int32_t R, int32_t rank, int64_t T_total,
+                       const int32_t* topk_idx, const int32_t* slot_of_local,
+                       const int32_t* offsets_local, const int32_t* counts_all, int32_t* owner,
+                       int32_t* slot, int32_t* own_offsets, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Stores the token row x[a/k,:] of every kept assignment a into peer_xs[owner[a]] at row
+ * slot[a]. peer_xs is a device array of R device pointers to the ranks' slot-major row buffers
+ * ([rows, H] dtype, 16-byte aligned; the other ranks' buffers mapped into this device's address
+ * space, or other buffers of the same device when ranks are emulated on one device). The
+ * stores are plain global stores; the caller orders them before the owners read. */
+moe_status moe_ep_dispatch(const moe_shape* shape, int32_t R, const void* x,
+                           const int32_t* owner, const int32_t* slot, void* const* peer_xs,
+                           void* stream);
+
+/* out[t,:] = sum over kept j, ascending, of topk_w[t,j] * peer_y[owner][slot,:], accumulated in
+ * float32 and rounded once (a fully dropped token gives a zero row): moe_combine with each
+ * expert output row read from its owner. peer_y is a device array of R device pointers to the
+ * ranks' expert outputs ([rows, H] dtype, slot-major, as moe_grouped_ffn writes them). */
+moe_status moe_ep_combine(const moe_shape* shape, int32_t R, const void* const* peer_y,
+                          const int32_t* owner, const int32_t* slot, const float* topk_w,
+                          void* out, void* stream);
+
 /* Synchronises `stream`, reads and clears the device error word at the start of `ws`.
  * Returns MOE_OK, MOE_ERR_DEVICE (a kernel flagged a fault; see moe_last_error_detail) or
  * MOE_ERR_CUDA. */

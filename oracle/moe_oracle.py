@@ -50,6 +50,13 @@ Readings taken where the pages are silent or disagree (each also listed in the d
   finite value); one float32 scale per output channel, scale = max_k |W[k, m]| / 448 (1 when
   the column is all zero); code = e4m3(W / scale) rounded to nearest, ties to even, saturating
   at +-448; the GEMM uses decode(code) * scale. Activations stay bf16 (W8A16).
+* FP8 weights and activations (W8A8, the same [P5] section): the weights as above; the
+  activations entering each expert GEMM quantised per row to e4m3 the same way (one float32 scale
+  per token row of x, one per slot row of h: scale = max |row| / 448, code = e4m3(v / scale)).
+  The SwiGLU intermediate h is rounded to bfloat16 before its quantisation, since the GPU keeps h
+  in bf16 between the two GEMMs and a quantised code is decided in the kernel's precision. Both
+  scales of a product are applied to the accumulated sum: y[m] = s_act * s_w[m] * sum_k
+  decode(q_act[k]) * decode(q_w[k, m]).
 * Shared expert and bias in the combine: out[t] = sum_j w[t,j] y[slot] + factor * shared[t] + b,
   with shared[t] the shared expert's output row (computed by the caller) and b a per-feature
   bias; both terms apply to every token, including a fully dropped one.
@@ -77,6 +84,9 @@ __all__ = [
     "e4m3_encode",
     "quantize_weights_fp8",
     "dequantize_weights_fp8",
+    "bf16_round",
+    "quantize_rows_fp8",
+    "swiglu_expert_w8a8",
     "align",
     "swiglu_expert",
     "grouped_ffn_slots",
@@ -244,6 +254,54 @@ def dequantize_weights_fp8(codes, scale):
     return e4m3_decode(codes) * np.asarray(scale, dtype=np.float64)[:, None, :]
 
 
+def bf16_round(values):
+    """Nearest bfloat16 of each value, as float32: rounded to float32 first (the precision the
+    GPU computes h in), then to the 8 significant bits of bfloat16, ties to the even pattern."""
+    f = np.ascontiguousarray(np.asarray(values, dtype=np.float64).astype(np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).reshape(f.shape)
+
+
+def quantize_rows_fp8(a):
+    """Per-row e4m3 quantisation of activations a [N, K]: scale[n] = float32(max_k |a[n, k]| /
+    448) (1 for an all-zero row), code[n, k] = e4m3(float32(a[n, k] / scale[n])), nearest-even,
+    saturating. Returns (codes uint8 [N, K], scale float32 [N]); both divisions are single
+    float32 operations, as on the GPU."""
+    a32 = np.asarray(a, dtype=np.float32)
+    if a32.shape[0] == 0:
+        return np.zeros(a32.shape, dtype=np.uint8), np.zeros(0, dtype=np.float32)
+    amax = np.max(np.abs(a32), axis=1)
+    scale = np.where(amax > 0, (amax / np.float32(448.0)).astype(np.float32),
+                     np.float32(1.0)).astype(np.float32)
+    return e4m3_encode((a32 / scale[:, None]).astype(np.float32)), scale
+
+
+def swiglu_expert_w8a8(x_rows, wg, wu, wd):
+    """One expert's SwiGLU FFN with e4m3 weights and e4m3 activations (W8A8), float64 sums.
+
+    wg, wu, wd are (codes, scale) pairs of the expert's weights as quantize_weights_fp8 makes
+    them ([K, M] codes, [M] scales). x rows are quantised per row; the intermediate
+    h = silu(g) * u is rounded to bfloat16 and quantised per row before the down projection:
+      g[m] = s_x * s_g[m] * sum_k dec(q_x[k]) dec(q_g[k, m])   (u likewise)
+      y[m] = s_h * s_d[m] * sum_i dec(q_h[i]) dec(q_d[i, m])
+    """
+    qx, sx = quantize_rows_fp8(x_rows)
+    xd = e4m3_decode(qx) * sx.astype(np.float64)[:, None]
+
+    def deq(w):
+        q, sc = w
+        return e4m3_decode(q) * np.asarray(sc, dtype=np.float64)[None, :]
+
+    g = xd @ deq(wg)
+    u = xd @ deq(wu)
+    with np.errstate(over="ignore"):
+        h = g * u / (1.0 + np.exp(-g))
+    qh, sh = quantize_rows_fp8(bf16_round(h))
+    hd = e4m3_decode(qh) * sh.astype(np.float64)[:, None]
+    return hd @ deq(wd)
+
+
 def capacity(T, k, E, capacity_factor):
     """Per-expert capacity C = ceil(cf * T * k / E), exact rational arithmetic, capped at T.
 
@@ -321,13 +379,17 @@ def swiglu_expert(x_rows, w_gate_e, w_up_e, w_down_e):
     return h @ np.asarray(w_down_e, dtype=np.float64)
 
 
-def grouped_ffn_slots(x, sorted_ids, offsets, k, w_gate, w_up, w_down, slots=None):
+def grouped_ffn_slots(x, sorted_ids, offsets, k, w_gate, w_up, w_down, slots=None,
+                      expert_fn=None):
     """Expert output per kept slot: y[s] = expert_e(x[sorted_ids[s] // k]) for s in expert e's range.
 
     [P1] "FlashAttention 在 MoE 模型里的位置" step 4. ``w_*`` may be arrays or any object whose
-    ``[e]`` returns expert e's matrix. ``slots`` restricts the evaluation to a subset (returned
-    as a dict slot -> row); by default every kept slot is evaluated into a [A_kept, H] array.
+    ``[e]`` returns expert e's matrix (or what ``expert_fn`` takes for it). ``slots`` restricts
+    the evaluation to a subset (returned as a dict slot -> row); by default every kept slot is
+    evaluated into a [A_kept, H] array. ``expert_fn`` (default swiglu_expert) evaluates one
+    expert on a block of rows: swiglu_expert_w8a8 for FP8 weights and activations.
     """
+    expert_fn = swiglu_expert if expert_fn is None else expert_fn
     offsets = np.asarray(offsets, dtype=np.int64)
     E = len(offsets) - 1
     sorted_ids = np.asarray(sorted_ids, dtype=np.int64)
@@ -340,13 +402,13 @@ def grouped_ffn_slots(x, sorted_ids, offsets, k, w_gate, w_up, w_down, slots=Non
         if not sl:
             continue
         toks = sorted_ids[sl] // k
-        y = swiglu_expert(x[toks], w_gate[e], w_up[e], w_down[e])
+        y = expert_fn(x[toks], w_gate[e], w_up[e], w_down[e])
         for i, s in enumerate(sl):
             result[s] = y[i]
     if slots is not None:
         return result
     a_kept = int(offsets[-1])
-    H = np.asarray(w_down[0]).shape[1] if a_kept else 0
+    H = (len(next(iter(result.values()))) if result else 0) if a_kept else 0
     out = np.zeros((a_kept, H), dtype=np.float64)
     for s, row in result.items():
         out[s] = row
@@ -399,14 +461,16 @@ def combine(y_slots, slot_of, topk_w, tokens=None, shared=None, shared_factor=0.
 
 def layer_forward(x, w_router, w_gate, w_up, w_down, k, capacity_factor,
                   logit_bias=None, logits=None, tokens=None, n_group=1, topk_group=1,
-                  shared=None, shared_factor=0.0, out_bias=None):
+                  shared=None, shared_factor=0.0, out_bias=None, expert_fn=None):
     """Whole MoE layer: route -> align -> experts -> combine, float64 throughout.
 
     [P1] "FlashAttention 在 MoE 模型里的位置" steps 2-5. ``logits`` (float32) may be supplied
     to route from given gate logits. ``tokens`` restricts the expert FFN and the combine to a
     subset of tokens (routing and capacity still see every token, since ranks depend on all).
     ``n_group``/``topk_group`` select group-limited routing; ``shared``/``shared_factor``/
-    ``out_bias`` add the shared-expert and bias terms of the combine.
+    ``out_bias`` add the shared-expert and bias terms of the combine. ``expert_fn`` replaces the
+    expert FFN (swiglu_expert_w8a8 for FP8 weights and activations, with ``w_*[e]`` the
+    (codes, scale) pairs).
     Returns dict with out [len(tokens) or T, H] and all routing intermediates.
     """
     x = np.asarray(x)
@@ -427,7 +491,7 @@ def layer_forward(x, w_router, w_gate, w_up, w_down, k, capacity_factor,
             if s >= 0:
                 need.add(s)
     y = grouped_ffn_slots(x, al["sorted_ids"], al["offsets"], k, w_gate, w_up, w_down,
-                          slots=sorted(need))
+                          slots=sorted(need), expert_fn=expert_fn)
     out = combine(y, al["slot_of"], w, tokens=tok_list, shared=shared,
                   shared_factor=shared_factor, out_bias=out_bias)
     res = dict(al)

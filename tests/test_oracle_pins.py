@@ -548,3 +548,109 @@ def test_layer_grouped_fixture_rejects_planted_mistakes(golden_dir, monkeypatch)
 
     monkeypatch.setattr(orc, "route_grouped", groups_scored_by_top1)
     assert not _matches(_grouped_layer(g, arr), g)
+
+
+# ---------------------------------------------------------------- FP8 weights and activations (W8A8)
+
+
+def test_bf16_round_matches_torch_including_ties():
+    rng = np.random.default_rng(21)
+    v = np.concatenate([rng.standard_normal(50000) * s for s in (1e-30, 1e-3, 1.0, 1e20)])
+    v = v.astype(np.float32)
+    # exact ties: float32 patterns whose low 16 bits are 0x8000, both parities of bit 16
+    ties = (rng.integers(0x00800000, 0x7f000000, size=4000, dtype=np.uint32) & ~np.uint32(0xffff)) \
+        | np.uint32(0x8000)
+    v = np.concatenate([v, ties.view(np.float32), -ties.view(np.float32)])
+    ref = torch.from_numpy(v).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(orc.bf16_round(v), ref)
+    # float64 input: rounded to float32 first, then to bfloat16
+    d = rng.standard_normal(20000) * 3.0
+    assert np.array_equal(orc.bf16_round(d),
+                          torch.from_numpy(d.astype(np.float32)).to(torch.bfloat16).float().numpy())
+
+
+def test_quantize_rows_fp8_matches_torch_and_landmarks():
+    rng = np.random.default_rng(22)
+    a = (rng.standard_normal((40, 96)) * rng.uniform(1e-3, 50, size=(40, 1))).astype(np.float32)
+    a[5] = 0.0
+    q, sc = orc.quantize_rows_fp8(a)
+    assert q.shape == a.shape and q.dtype == np.uint8 and sc.shape == (40,)
+    t = torch.from_numpy(a)
+    sc_t = t.abs().amax(dim=1) / 448.0
+    sc_t = torch.where(sc_t > 0, sc_t, torch.ones_like(sc_t))
+    q_t = (t / sc_t[:, None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(sc, sc_t.numpy()) and np.array_equal(q, q_t)
+    assert sc[5] == 1.0 and np.all(q[5] == 0)
+    dec = orc.e4m3_decode(q)
+    assert np.all(np.abs(np.delete(dec, 5, axis=0)).max(axis=1) == 448.0)
+    # a row already on the e4m3 grid with max 448 * 2^-8 is reproduced exactly
+    grid = orc.e4m3_decode(np.arange(0, 127, 3, dtype=np.uint8)) * 2.0 ** -8
+    row = np.concatenate([grid, -grid[::-1], [448.0 * 2.0 ** -8]]).astype(np.float32)[None]
+    q2, s2 = orc.quantize_rows_fp8(row)
+    assert s2[0] == 2.0 ** -8 and np.array_equal(orc.e4m3_decode(q2) * s2[0], row.astype(np.float64))
+    # no rows
+    q0, s0 = orc.quantize_rows_fp8(np.zeros((0, 8), dtype=np.float32))
+    assert q0.shape == (0, 8) and s0.shape == (0,)
+
+
+def _w8a8_expert_torch(x, wg, wu, wd):
+    """The W8A8 expert written independently with torch ops: per-row e4m3 of the activations by
+    torch's float8 conversion, float64 matmuls, torch's silu, torch's bfloat16 rounding of h."""
+    def q_rows(a):
+        a = torch.as_tensor(a, dtype=torch.float32)
+        sc = a.abs().amax(dim=1) / 448.0
+        sc = torch.where(sc > 0, sc, torch.ones_like(sc))
+        return (a / sc[:, None]).to(torch.float8_e4m3fn).to(torch.float64) * sc.double()[:, None]
+
+    def deq(w):
+        q, sc = w
+        return (torch.from_numpy(q).view(torch.float8_e4m3fn).to(torch.float64)
+                * torch.from_numpy(sc).double()[None, :])
+
+    xd = q_rows(x)
+    g, u = xd @ deq(wg), xd @ deq(wu)
+    h = (torch.nn.functional.silu(g) * u).float().to(torch.bfloat16).float()
+    return (q_rows(h) @ deq(wd)).numpy()
+
+
+def test_swiglu_expert_w8a8_matches_an_independent_torch_composition(monkeypatch):
+    rng = np.random.default_rng(23)
+    H, I, n = 64, 48, 9
+    x = rng.standard_normal((n, H)).astype(np.float32)
+    ws = [orc.quantize_weights_fp8((rng.standard_normal((1, H, I)) / 8).astype(np.float32)),
+          orc.quantize_weights_fp8((rng.standard_normal((1, H, I)) / 8).astype(np.float32)),
+          orc.quantize_weights_fp8((rng.standard_normal((1, I, H)) / 7).astype(np.float32))]
+    wg, wu, wd = [(q[0], s[0]) for q, s in ws]
+    got = orc.swiglu_expert_w8a8(x, wg, wu, wd)
+    ref = _w8a8_expert_torch(x, wg, wu, wd)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    # planted mistakes fail: h not rounded to bf16 before its quantisation, or the activation
+    # scale of x dropped
+    real_round, real_rows = orc.bf16_round, orc.quantize_rows_fp8
+    monkeypatch.setattr(orc, "bf16_round", lambda v: np.asarray(v, dtype=np.float64))
+    bad = orc.swiglu_expert_w8a8(x, wg, wu, wd)
+    assert not np.allclose(bad, ref, rtol=1e-9, atol=1e-9 * np.abs(ref).max())
+    monkeypatch.setattr(orc, "bf16_round", real_round)
+
+    def rows_without_scale(a):
+        q, sc = real_rows(a)
+        return q, np.ones_like(sc)
+    monkeypatch.setattr(orc, "quantize_rows_fp8", rows_without_scale)
+    bad = orc.swiglu_expert_w8a8(x, wg, wu, wd)
+    assert not np.allclose(bad, ref, rtol=1e-3, atol=1e-3 * np.abs(ref).max())
+
+
+def test_layer_w8a8_close_to_the_exact_layer():
+    """The quantised layer stays within the e4m3 error scale of the exact float64 layer on the
+    same routing (each quantised operand is within 2^-4 relative; the output error is a few
+    percent of the output's scale)."""
+    wl = wlm.Workload("q", 0, 24, 64, 4, 2, 32, "f32", 0.0)
+    a = {k_: (v.numpy() if v is not None else None) for k_, v in wlm.make_inputs(wl).items()}
+    qs = [orc.quantize_weights_fp8(a[n]) for n in ("w_gate", "w_up", "w_down")]
+    pairs = [[(q[e], s[e]) for e in range(wl.E)] for q, s in qs]
+    exact = orc.layer_forward(a["x"], a["w_router"], a["w_gate"], a["w_up"], a["w_down"], wl.k, 0.0)
+    quant = orc.layer_forward(a["x"], a["w_router"], pairs[0], pairs[1], pairs[2], wl.k, 0.0,
+                              expert_fn=orc.swiglu_expert_w8a8)
+    assert np.array_equal(quant["topk_idx"], exact["topk_idx"])
+    err = np.abs(quant["out"] - exact["out"]).max() / np.abs(exact["out"]).max()
+    assert 1e-4 < err < 0.1
