@@ -142,9 +142,12 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ algorithmic cost model
 
-def stage_costs(wl, counts, hbm_peak, tc_peak, fp8_weights=False):
+def stage_costs(wl, counts, hbm_peak, tc_peak, fp8_weights=False, fp8_acts=False):
     """Algorithmic bytes/flops per stage for one step, from the step's routing counts. With
-    e4m3 expert weights a weight element is 1 byte, plus a float32 scale per output channel."""
+    e4m3 expert weights a weight element is 1 byte, plus a float32 scale per output channel.
+    With e4m3 activations too (W8A8), x is read once to be quantised, the GEMMs read e4m3 token
+    rows, and the SwiGLU intermediate is stored once and read once as e4m3 (its bf16 copy before
+    quantisation is implementation traffic)."""
     es = 2 if wl.dtype == "bf16" else 4
     T, H, E, k, I = wl.T, wl.H, wl.E, wl.k, wl.I
     A = T * k
@@ -163,6 +166,10 @@ def stage_costs(wl, counts, hbm_peak, tc_peak, fp8_weights=False):
                   "flops": 2 * a_kept * I * H},
         "combine": {"bytes": a_kept * H * es + T * k * 8 + T * H * es, "flops": 2 * a_kept * H},
     }
+    if fp8_acts:
+        c["gemm1"]["bytes"] = (used * 2 * H * I + used * 2 * I * 4 + T * H * es + a_kept * H
+                               + a_kept * I)
+        c["gemm2"]["bytes"] = used * I * H + used * H * 4 + a_kept * I + a_kept * H * es
     for v in c.values():
         v["t_hbm_us"] = v["bytes"] / (hbm_peak * 1e9) * 1e6
         v["t_tc_us"] = v["flops"] / (tc_peak * 1e12) * 1e6
@@ -272,16 +279,22 @@ def oracle_baseline(wl, dev, n_tokens, reps=1):
 
 # ------------------------------------------------------------------ the GPU arm
 
-def launches_per_step(wl):
-    """Kernels one moe_layer_forward launches: router (tensor-core GEMM + top-k, or one fused
-    CUDA-core kernel), align (one launch up to 65536 assignments, else three), two expert
-    GEMMs, combine."""
-    route = 2 if (wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0) else 1
+def launches_per_step(wl, weights="bf16"):
+    """Kernels one moe_layer_forward launches: router (one tensor-core kernel with the top-k
+    fused; for at most 64 tokens a CUDA-core GEMV + top-k; one fused CUDA-core kernel for E < 64
+    or f32), align (one launch up to 65536 assignments, else three), the expert-major row copy
+    (bf16), two expert GEMMs, combine."""
+    route = 1
+    if wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0:
+        gemv = (wl.T <= 64 and wl.E % 32 == 0 and wl.H % 128 == 0 and wl.H <= 16 * 512)
+        route = 2 if gemv else 1
     align = 1 if wl.T * wl.k <= 65536 else 3
     # expert-major copy of the token rows before GEMM1: every bf16 layer (GEMM1 runs on CTA
     # pairs, and the e4m3-weight GEMM1 reads the copy too)
     copy = 1 if wl.dtype == "bf16" else 0
-    return route + align + copy + 2 + 1
+    # W8A8: the token rows and the SwiGLU rows are quantised by one launch each
+    quant = 2 if weights == "w8a8" else 0
+    return route + align + copy + quant + 2 + 1
 
 
 def workload_of(args):
@@ -289,15 +302,18 @@ def workload_of(args):
     return wl.with_tokens(args.tokens) if args.tokens else wl
 
 
-def layer_config(wl, capacity, world, fp8):
+def layer_config(wl, capacity, world, weights="bf16"):
     """The `config` object of a layer line; the reference arm prints the same keys."""
+    fp8 = weights in ("fp8", "w8a8")
     wes = 1 if fp8 else (2 if wl.dtype == "bf16" else 4)
     wb = 3 * wl.E * wl.H * wl.I * wes
     return {"workload": wl.describe(), "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
             "capacity": int(capacity),
             "parallelism": "replicas" if world > 1 else "single-gpu",
-            "expert_weights": ("e4m3 codes + float32 per-channel scales (W8A16)"
-                               if fp8 else wl.dtype),
+            "expert_weights": {"fp8": "e4m3 codes + float32 per-channel scales (W8A16)",
+                               "w8a8": "e4m3 codes + float32 per-channel scales, e4m3 "
+                                       "activations with float32 per-row scales (W8A8)"}.get(
+                                           weights, wl.dtype),
             "l2": (("inputs larger than L2: %.1f GB of expert weights streamed per step"
                     % (wb / 1e9)) if wb > L2_BYTES else
                    "inputs fit in L2 (%.1f MB of expert weights); L2 not flushed" % (wb / 1e6))}
@@ -306,7 +322,7 @@ def layer_config(wl, capacity, world, fp8):
 class LayerRun:
     """One workload's layer on the device: inputs, outputs, workspace and the forward call."""
 
-    def __init__(self, wl, dev, fp8=False):
+    def __init__(self, wl, dev, fp8=False, w8a8=False):
         self.wl, self.dev = wl, dev
         self.inp = W.make_inputs(wl, dev)
         self.shape = M.shape_of(wl.T, wl.H, wl.E, wl.k, wl.I, wl.capacity_factor, wl.dtype)
@@ -318,14 +334,23 @@ class LayerRun:
                      torch.empty(wl.T * wl.k, dtype=torch.uint8, device=dev)]
         self.stream = torch.cuda.current_stream(dev)
         self.fp8 = None
+        self.w8a8 = None
         if fp8:
             # e4m3 expert weights, quantised once on the device before anything is timed
             self.fp8 = M.Fp8Weights(self.inp["w_gate"], self.inp["w_up"], self.inp["w_down"])
             torch.cuda.synchronize()
+        if w8a8:
+            # K-major e4m3 expert weights, packed once on the device before anything is timed
+            self.w8a8 = M.W8A8Weights(self.inp["w_gate"], self.inp["w_up"], self.inp["w_down"])
+            torch.cuda.synchronize()
 
     def forward(self, x, o):
         inp, ws = self.inp, self.ws
-        if self.fp8 is not None:
+        if self.w8a8 is not None:
+            L.moe_layer_forward_w8a8(self.shape, None, x, inp["w_router"], inp["logit_bias"],
+                                     *self.w8a8.args(), o[0], None, o[1], o[2], o[3], o[4],
+                                     ws.buf, ws.nbytes, self.stream)
+        elif self.fp8 is not None:
             L.moe_layer_forward_w8(self.shape, None, x, inp["w_router"], inp["logit_bias"],
                                    *self.fp8.args(), o[0], None, o[1], o[2], o[3], o[4], ws.buf,
                                    ws.nbytes, self.stream)
@@ -379,9 +404,9 @@ class LayerRun:
                 st_ms[s] += prev.elapsed_time(ev[i][j]) / steps
                 prev = ev[i][j]
         cnt = self.outs[3].cpu().numpy()
-        fp8 = self.fp8 is not None
+        fp8 = self.fp8 is not None or self.w8a8 is not None
         cost = stage_costs(wl, cnt, peaks["hbm_gbs"], peaks["bf16_tflops_sustained"],
-                           fp8_weights=fp8)
+                           fp8_weights=fp8, fp8_acts=self.w8a8 is not None)
         kernels = {}
         for s in STAGES:
             t = st_ms[s] * 1e-3
@@ -416,7 +441,7 @@ class LayerRun:
         }
 
     def release(self):
-        del self.inp, self.ws, self.outs, self.fp8
+        del self.inp, self.ws, self.outs, self.fp8, self.w8a8
         torch.cuda.empty_cache()
 
 
@@ -446,13 +471,14 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     peaks, peaks_src = load_peaks()
     peaks["_source"] = peaks_src
-    run = LayerRun(wl, dev, fp8=args.weights == "fp8")
+    run = LayerRun(wl, dev, fp8=args.weights == "fp8", w8a8=args.weights == "w8a8")
     inp, stream = run.inp, run.stream
     t = run.time_stages(args.steps, args.warmup, world, local, peaks)
     cnt = t["cnt"]
     dom = t["roofline"]["kernel"]
-    t["roofline"]["traffic"] = recorded_traffic(dom + ("_w8" if run.fp8 is not None else ""),
-                                                args.workload)
+    t["roofline"]["traffic"] = recorded_traffic(
+        dom + ("_w8" if run.fp8 is not None else "_w8a8" if run.w8a8 is not None else ""),
+        args.workload)
 
     # End to end through the C ABI with host buffers: every step copies its x in from pinned host
     # memory and its outputs back out. Measured twice: serially (copy in, forward, copy out on one
@@ -519,7 +545,7 @@ def run_ours(args, world, rank, local):
     h2d = x_host.numel() * x_host.element_size()
     d2h = sum(t_.numel() * t_.element_size() for t_ in outs_host)
 
-    per_step = launches_per_step(wl)
+    per_step = launches_per_step(wl, args.weights)
     line = {
         "metric": METRIC,
         "value": round(t["value"], 1),
@@ -533,7 +559,7 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": wl.dtype,
         "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights; no dataset)",
-        "config": layer_config(wl, L.moe_capacity(run.shape), world, run.fp8 is not None),
+        "config": layer_config(wl, L.moe_capacity(run.shape), world, args.weights),
         "routing": {"kept_assignments": int(cnt.sum()), "experts_used": int((cnt > 0).sum())},
         "roofline": t["roofline"],
         "route_align_combine_gbs": t["route_align_combine_gbs"],
@@ -687,7 +713,7 @@ def run_reference(args, world, rank, local):
         "ms_per_step_extrapolated_to_T": round(per_token * wl.T * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights; no dataset)",
-        "config": layer_config(wl, C, world, False),
+        "config": layer_config(wl, C, world),
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cpu_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -709,8 +735,9 @@ def main(argv=None):
     ap.add_argument("--no-other-workloads", action="store_true",
                     help="time only the selected workload (by default a one-GPU run also times "
                          "the Mixtral-shaped, skewed and decode layers under other_workloads)")
-    ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
-                    help="expert weights: the layer dtype (default) or e4m3 + per-channel scales")
+    ap.add_argument("--weights", choices=["bf16", "fp8", "w8a8"], default="bf16",
+                    help="expert weights: the layer dtype (default), e4m3 + per-channel scales "
+                         "(fp8, bf16 activations), or e4m3 weights and activations (w8a8)")
     ap.add_argument("--sweep", choices=["route-align-combine"], default=None,
                     help="time route -> align -> combine alone over a range of T (HBM GB/s per "
                          "stage; one GPU) instead of the layer")

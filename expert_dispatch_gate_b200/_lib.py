@@ -82,9 +82,15 @@ def _signatures(lib):
         "moe_grouped_ffn_w8": (st, [S] + [_P] * 11 + [sz, _P]),
         "moe_layer_forward_w8": (st, [S, O] + [_P] * 16 + [sz, _P]),
         "moe_probe_stalled_wait": (st, [_P, sz, _P]),
+        "moe_pack_weights_w8a8": (st, [_P, i64, i64, i64, _P, _P, _P]),
+        "moe_quantize_rows_fp8": (st, [_P, i64, i64, _P, _P, _P]),
+        "moe_grouped_ffn_w8a8": (st, [S] + [_P] * 11 + [sz, _P]),
+        "moe_layer_forward_w8a8": (st, [S, O] + [_P] * 16 + [sz, _P]),
         "moe_ep_plan": (st, [S, ctypes.c_int32, ctypes.c_int32, i64] + [_P] * 7 + [_P, sz, _P]),
         "moe_ep_dispatch": (st, [S, ctypes.c_int32, _P, _P, _P, _P, _P]),
         "moe_ep_combine": (st, [S, ctypes.c_int32, _P, _P, _P, _P, _P, _P]),
+        "moe_ep_signal": (st, [ctypes.c_int32, ctypes.c_int32, ctypes.c_uint32, _P, _P]),
+        "moe_ep_wait": (st, [ctypes.c_int32, ctypes.c_uint32, _P, _P, sz, _P]),
     }
     for name, (res, args) in table.items():
         f = getattr(lib, name)
@@ -218,6 +224,18 @@ def moe_ep_dispatch(shape, R, x, owner, slot, peer_xs, stream=None, check=True):
     return _check(s) if check else s
 
 
+def moe_ep_signal(R, rank, epoch, peer_flags, stream=None, check=True):
+    s = lib().moe_ep_signal(int(R), int(rank), int(epoch) & 0xffffffff, ptr(peer_flags),
+                            _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_ep_wait(R, epoch, flags, ws, ws_bytes, stream=None, check=True):
+    s = lib().moe_ep_wait(int(R), int(epoch) & 0xffffffff, ptr(flags), ptr(ws), int(ws_bytes),
+                          _stream(stream))
+    return _check(s) if check else s
+
+
 def moe_ep_combine(shape, R, peer_y, owner, slot, topk_w, out, stream=None, check=True):
     s = lib().moe_ep_combine(ctypes.byref(shape), int(R), ptr(peer_y), ptr(owner), ptr(slot),
                              ptr(topk_w), ptr(out), _stream(stream))
@@ -276,6 +294,38 @@ def moe_layer_forward_ex(shape, opts, x, w_router, logit_bias, w_gate, w_up, w_d
 def moe_quantize_weights_fp8(w, E, K, M, codes, scale, stream=None, check=True):
     s = lib().moe_quantize_weights_fp8(ptr(w), int(E), int(K), int(M), ptr(codes), ptr(scale),
                                        _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_pack_weights_w8a8(w, E, K, M, codes, scale, stream=None, check=True):
+    s = lib().moe_pack_weights_w8a8(ptr(w), int(E), int(K), int(M), ptr(codes), ptr(scale),
+                                    _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_quantize_rows_fp8(a, N, K, codes, scale, stream=None, check=True):
+    s = lib().moe_quantize_rows_fp8(ptr(a), int(N), int(K), ptr(codes), ptr(scale),
+                                    _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_grouped_ffn_w8a8(shape, x, sorted_ids, offsets, qk_gate, qk_up, qk_down, s_gate, s_up,
+                         s_down, y_slots, ws, ws_bytes, stream=None, check=True):
+    s = lib().moe_grouped_ffn_w8a8(ctypes.byref(shape), ptr(x), ptr(sorted_ids), ptr(offsets),
+                                   ptr(qk_gate), ptr(qk_up), ptr(qk_down), ptr(s_gate), ptr(s_up),
+                                   ptr(s_down), ptr(y_slots), ptr(ws), int(ws_bytes),
+                                   _stream(stream))
+    return _check(s) if check else s
+
+
+def moe_layer_forward_w8a8(shape, opts, x, w_router, logit_bias, qk_gate, qk_up, qk_down, s_gate,
+                           s_up, s_down, out, logits_out, topk_idx, topk_w, counts, drop_mask, ws,
+                           ws_bytes, stream=None, check=True):
+    s = lib().moe_layer_forward_w8a8(ctypes.byref(shape), _opts(opts), ptr(x), ptr(w_router),
+                                     ptr(logit_bias), ptr(qk_gate), ptr(qk_up), ptr(qk_down),
+                                     ptr(s_gate), ptr(s_up), ptr(s_down), ptr(out),
+                                     ptr(logits_out), ptr(topk_idx), ptr(topk_w), ptr(counts),
+                                     ptr(drop_mask), ptr(ws), int(ws_bytes), _stream(stream))
     return _check(s) if check else s
 
 

@@ -13,9 +13,10 @@
 // of it (one block up to kAlignSingle, one cluster of CTAs above); beyond that three kernels:
 //   1. hist:    per chunk of align_chunk(A) assignments, per-expert counts (shared-memory
 //               atomics).
-//   2. scan:    one block; per expert, exclusive prefix over chunks (chunk bases), raw totals,
-//               counts = min(raw, C), offsets = exclusive scan of counts, and the token-block
-//               plan blk_prefix used by the expert GEMMs.
+//   2. scan:    one block; per expert, exclusive prefix over chunks (chunk bases; the chunks
+//               of an expert split over several threads), raw totals, counts = min(raw, C),
+//               offsets = exclusive scan of counts, and the token-block plan blk_prefix used by
+//               the expert GEMMs.
 //   3. scatter: per chunk, stable in-chunk ranks (warp_peers + per-warp prefix),
 //               then slot = offsets[e] + rank for kept assignments; fills the -1 tail.
 #include <mutex>
@@ -110,39 +111,77 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int& total) 
   return warp_base + inc - v;
 }
 
-__global__ void __launch_bounds__(kThreads)
+// Chunk bases, counts, offsets and the token-block plan, one block of kScanThreads threads.
+// Thread (s, e), tid = s * Ep + e (Ep = E rounded up to a power of two, S = kScanThreads / Ep
+// splits capped at kScanMaxSplit), owns the chunks [s*per, (s+1)*per) of expert e: it sums them
+// (pass 1), takes the sums of the splits before it as its base, then rewrites each chunk's count
+// as the running base (pass 2). Every chain of dependent loads is per/8 batches long instead of
+// nblk/8 for one thread per expert.
+constexpr int kScanThreads = 1024;
+constexpr int kScanMaxSplit = 64;
+
+__global__ void __launch_bounds__(kScanThreads)
     align_scan_kernel(int32_t* __restrict__ blk_hist, int nblk, int E, int C, int TB,
                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                       int32_t* __restrict__ blk_prefix) {
   pdl_enter<false>();
-  __shared__ int sh[kWarps];
-  const int e = threadIdx.x;
-  int run = 0;
-  if (e < E) {
-    // chunk bases in place; loads batched so they overlap
-    for (int b0 = 0; b0 < nblk; b0 += 8) {
+  __shared__ int part[kScanThreads];
+  __shared__ int sh[kScanThreads / 32];
+  int Ep = 1;
+  while (Ep < E) Ep <<= 1;
+  int S = kScanThreads / Ep;
+  if (S > kScanMaxSplit) S = kScanMaxSplit;
+  const int tid = threadIdx.x;
+  const int e = tid % Ep, sp = tid / Ep;
+  const bool act = sp < S && e < E;
+  const int per = (nblk + S - 1) / S;
+  const int c0 = sp * per;
+  const int c1 = min(nblk, c0 + per);
+  int sum = 0;
+  if (act) {
+    for (int b0 = c0; b0 < c1; b0 += 8) {
       int c[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        c[i] = (b0 + i < nblk) ? blk_hist[static_cast<size_t>(b0 + i) * E + e] : 0;
+        c[i] = (b0 + i < c1) ? blk_hist[static_cast<size_t>(b0 + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum += c[i];
+    }
+  }
+  part[tid] = sum;
+  __syncthreads();
+  int base = 0, raw = 0;
+  if (act) {
+    for (int q = 0; q < S; ++q) {
+      const int v = part[q * Ep + e];
+      if (q < sp) base += v;
+      raw += v;
+    }
+    int run = base;
+    for (int b0 = c0; b0 < c1; b0 += 8) {
+      int c[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        c[i] = (b0 + i < c1) ? blk_hist[static_cast<size_t>(b0 + i) * E + e] : 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        if (b0 + i < nblk) blk_hist[static_cast<size_t>(b0 + i) * E + e] = run;
+        if (b0 + i < c1) blk_hist[static_cast<size_t>(b0 + i) * E + e] = run;
         run += c[i];
       }
     }
   }
-  const int cnt = (e < E) ? min(run, C) : 0;
+  // counts, offsets and the plan: threads tid < Ep hold experts e = tid (split 0)
+  const int cnt = (sp == 0 && e < E) ? min(raw, C) : 0;
   const int nb = (cnt + TB - 1) / TB;
   int tot_cnt, tot_nb;
-  const int off = block_exclusive_scan(cnt, sh, tot_cnt);
-  const int bp = block_exclusive_scan(nb, sh, tot_nb);
-  if (e < E) {
+  const int off = block_exclusive_scan<kScanThreads / 32>(cnt, sh, tot_cnt);
+  const int bp = block_exclusive_scan<kScanThreads / 32>(nb, sh, tot_nb);
+  if (sp == 0 && e < E) {
     counts[e] = cnt;
     offsets[e] = off;
     if (blk_prefix != nullptr) blk_prefix[e] = bp;
   }
-  if (e == 0) {
+  if (tid == 0) {
     offsets[E] = tot_cnt;
     if (blk_prefix != nullptr) blk_prefix[E] = tot_nb;
   }
@@ -399,8 +438,8 @@ cudaError_t launch_align(const int32_t* topk_idx, int64_t A, int E, int C, int T
   cudaError_t e = launch_kernel(align_hist_kernel, dim3(nblk), dim3(kThreads), 0, stream, 1,
                                 topk_idx, A, E, chunk, blk_hist, err);
   if (e == cudaSuccess)
-    e = launch_kernel(align_scan_kernel, dim3(1), dim3(kThreads), 0, stream, 1, blk_hist, nblk, E,
-                      C, TB, counts, offsets, blk_prefix);
+    e = launch_kernel(align_scan_kernel, dim3(1), dim3(kScanThreads), 0, stream, 1, blk_hist,
+                      nblk, E, C, TB, counts, offsets, blk_prefix);
   if (e == cudaSuccess)
     e = launch_kernel(align_scatter_kernel, dim3(nblk), dim3(kThreads), 0, stream, 1, topk_idx, A,
                       E, C, chunk, blk_hist, offsets, sorted_ids, slot_of, drop_mask);
@@ -425,6 +464,25 @@ static __device__ __align__(256) NoAllocScratch g_noalloc_scratch;
 
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[64] = {};
+void* g_noalloc_ctx[64] = {};  // the context each cached address belongs to
+
+// The current driver context (CUcontext as void*), through the runtime's driver entry point so
+// that the library does not link libcuda itself; nullptr if it cannot be queried.
+void* current_context() {
+  using CtxGetCurrentFn = int (*)(void**);
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+  });
+  void* ctx = nullptr;
+  if (fn == nullptr || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
 }  // namespace
 
 cudaError_t launch_align_noalloc(const int32_t* topk_idx, int64_t A, int E, int C, int TB,
@@ -440,13 +498,18 @@ cudaError_t launch_align_noalloc(const int32_t* topk_idx, int64_t A, int E, int 
   void* base = nullptr;
   {
     // In host code g_noalloc_scratch names a host-side stand-in, not device memory: the
-    // device address is looked up once per device, with that device current.
+    // device address is looked up once per device and context, with that device current. A
+    // new context on the device (after cudaDeviceReset, say) loads the module again, so the
+    // address is looked up again then; with no context query available it is looked up on
+    // every call.
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    void* ctx = current_context();
+    if (g_noalloc_ptr[dev] == nullptr || ctx == nullptr || g_noalloc_ctx[dev] != ctx) {
       void* p = nullptr;
       e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
       if (e != cudaSuccess) return e;
       g_noalloc_ptr[dev] = p;
+      g_noalloc_ctx[dev] = ctx;
     }
     base = g_noalloc_ptr[dev];
   }

@@ -16,6 +16,9 @@
 // Rows move by plain stores into, and plain loads from, the other ranks' buffers through the
 // pointers in peer_xs / peer_y (peer memory mapped into this device's address space, or, when R
 // ranks are emulated on one device, the other ranks' buffers there). No TMA touches peer memory.
+// Ordering between ranks uses one flag word per (announcing rank, receiving rank): the announcing
+// rank stores a step number (epoch) with a system-scope release after its stores, and the
+// receiving rank waits for it with a bounded system-scope acquire loop.
 #include "common.cuh"
 #include "internal.h"
 
@@ -92,6 +95,45 @@ __global__ void __launch_bounds__(kThreads)
   const uint4* src = x + (a / k) * row_chunks;
   uint4* dst = peer_xs[o] + static_cast<int64_t>(slot[a]) * row_chunks;
   for (int c = lane; c < row_chunks; c += 32) dst[c] = __ldg(src + c);
+  // the rows reach the owner's memory before any later signal of this stream
+  __threadfence_system();
+}
+
+// Step signal: stores `epoch` into slot `rank` of every rank's flag array (peer_flags[q] is rank
+// q's array of R words), with release semantics at system scope, after a system-scope fence.
+// Launched after the work it announces (the dispatch stores, or the owner's expert outputs), in
+// stream order, so that work is complete and visible before any rank can see the new epoch.
+__global__ void __launch_bounds__(32) ep_signal_kernel(uint32_t* const* __restrict__ peer_flags,
+                                                       int R, int rank, uint32_t epoch) {
+  pdl_enter<false>();
+  __threadfence_system();
+  for (int q = threadIdx.x; q < R; q += 32) {
+    uint32_t* f = peer_flags[q] + rank;
+    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(f), "r"(epoch) : "memory");
+  }
+}
+
+// Bounded wait until every rank q < R has signalled `epoch` in flags[q] (epochs compared modulo
+// 2^32). A rank that never signals ends the wait after kWaitLimitNs: the kernel records
+// kDevWaitTimeout in the error word and returns, so the host reads a status instead of a hang.
+__global__ void __launch_bounds__(32) ep_wait_kernel(const uint32_t* __restrict__ flags, int R,
+                                                     uint32_t epoch, int* err) {
+  pdl_enter<false>();
+  bool ok = true;
+  for (int q = threadIdx.x; q < R; q += 32) {
+    const unsigned long long t0 = global_ns();
+    for (uint32_t i = 0;; ++i) {
+      uint32_t v;
+      asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(flags + q) : "memory");
+      if (static_cast<int32_t>(v - epoch) >= 0) break;
+      if ((i & 15u) == 15u && global_ns() - t0 > kWaitLimitNs) {
+        ok = false;
+        break;
+      }
+      __nanosleep(256);
+    }
+  }
+  if (!ok) flag_error(err, kDevWaitTimeout);
 }
 
 template <typename T>
@@ -219,6 +261,17 @@ cudaError_t launch_ep_dispatch(int dtype, const void* x, const int32_t* owner, c
   return launch_kernel(ep_dispatch_kernel, dim3(grid), dim3(kThreads), 0, stream, 1,
                        static_cast<const uint4*>(x), owner, slot,
                        reinterpret_cast<uint4* const*>(peer_xs), A, k, row_chunks);
+}
+
+cudaError_t launch_ep_signal(uint32_t* const* peer_flags, int R, int rank, uint32_t epoch,
+                             cudaStream_t stream) {
+  return launch_kernel(ep_signal_kernel, dim3(1), dim3(32), 0, stream, 1, peer_flags, R, rank,
+                       epoch);
+}
+
+cudaError_t launch_ep_wait(const uint32_t* flags, int R, uint32_t epoch, int* err,
+                           cudaStream_t stream) {
+  return launch_kernel(ep_wait_kernel, dim3(1), dim3(32), 0, stream, 1, flags, R, epoch, err);
 }
 
 cudaError_t launch_ep_combine(int dtype, const void* const* peer_y, const int32_t* owner,

@@ -94,6 +94,7 @@ struct TcParams {
   const float* scale0;  // W8: per-channel scales [groups][scale_ld] of A0 (gate, or down)
   const float* scale1;  // W8: of A1 (up)
   int scale_ld;
+  const float* act_scale;  // F8: per-row scale of the B operand (token / slot rows), [rows_b]
 };
 
 struct Tile {
@@ -164,7 +165,13 @@ __device__ __forceinline__ uint16_t bf16_half(uint32_t w, int hi) {
 // TMA boxes have (MN-major, 128-byte swizzle), and the MMA reads A from there. Every e4m3 value
 // is exactly a bf16 value, so the MMA sees decode(code) exactly; the channel scale multiplies
 // the fp32 accumulator in the epilogue.
-template <int MODE, int BMODE, bool PAIR, bool W8 = false>
+//
+// F8: both operands e4m3 (weights and activations, W8A8) on the native kind::f8f6f4 MMA. The
+// weight codes are stored K-major ([E][M][K], the repacked layout), so A and B are both K-major
+// 128-byte-swizzled boxes of 128 K values; a stage covers K = 128 with the same bytes as a
+// bf16 stage of K = 64, and each of its four MMAs takes K = 32. The epilogue multiplies the fp32
+// accumulator by the channel scale of the weights and the row scale of the activations.
+template <int MODE, int BMODE, bool PAIR, bool W8 = false, bool F8 = false>
 __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
     tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0,
                     const __grid_constant__ CUtensorMap tmA1,
@@ -176,6 +183,8 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
   // gatherer thread). Pairs stream B by TMA only.
   static_assert(!(PAIR && BMODE != kBTiled), "CTA pairs take the B operand by TMA boxes");
   static_assert(!(W8 && (PAIR || BMODE != kBTiled)), "FP8 weights: single CTAs, TMA-streamed B");
+  static_assert(!(F8 && (W8 || BMODE != kBTiled)), "e4m3 operands: TMA-streamed B rows");
+  constexpr int kStageK = F8 ? 128 : kBK;  // K elements per stage (128 bytes of a row)
   constexpr uint32_t kFullCount = 1u + (kCp ? 128u : 0u);
   // one arrival per epilogue warp (both CTAs' warps in PAIR mode)
   constexpr uint32_t kTemptyCount = PAIR ? 2u * kEpiWarps : kEpiWarps;
@@ -249,7 +258,7 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int num_tiles = p.num_fb * s_blk[groups];
-  const int kblocks = p.K / kBK;
+  const int kblocks = p.K / kStageK;
   const int tile0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int tstep = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   // B rows of a tile held by this CTA: all npad rows, or half of them per CTA in PAIR mode
@@ -307,6 +316,28 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
             tma_load_2d(sb, &tmB, kb * kBK, brow0, fbar);
           }
           __syncwarp();
+        } else if constexpr (F8) {
+          // K-major e4m3 boxes: 128 K bytes x 128 feature rows per weight operand (256 rows in
+          // one box for the two feature blocks of kEpiBF16x2), then the token rows
+          const int kc = kb * kStageK;
+          if constexpr (PAIR) {
+            const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
+            if (lane == 0) {
+              if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), tx);
+              tma_load_3d_pair(sa, &tmA0, kc, m0, t.group, fbar);
+              if constexpr (kSwiGLU) tma_load_3d_pair(sa + 16384, &tmA1, kc, m0, t.group, fbar);
+              tma_load_2d_pair(sb, &tmB, kc, brow0, fbar);
+            }
+          } else {
+            const uint32_t fbar = smem_u32(&full[s]);
+            if (lane == 0) {
+              mbar_arrive_expect_tx(fbar, tx);
+              tma_load_3d(sa, &tmA0, kc, m0, t.group, fbar);
+              if constexpr (kSwiGLU) tma_load_3d(sa + 16384, &tmA1, kc, m0, t.group, fbar);
+              tma_load_2d(sb, &tmB, kc, brow0, fbar);
+            }
+          }
+          __syncwarp();
         } else if constexpr (PAIR) {
           const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
           if (lane == 0) {
@@ -360,7 +391,9 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
       const uint32_t S = static_cast<uint32_t>(p.stages);
       const uint32_t sbase = smem_u32(smem);
       // W8: A comes from the bf16 slots; the stage ring holds the e4m3 codes and B
-      const uint64_t adesc0 = smem_desc_sw128(W8 ? smem_u32(a16) : sbase, 8192, 1024);
+      // A: MN-major bf16 (weights [E][K][M]) or K-major e4m3 (F8: repacked [E][M][K])
+      const uint64_t adesc0 = F8 ? smem_desc_sw128(sbase, 16, 1024)
+                                 : smem_desc_sw128(W8 ? smem_u32(a16) : sbase, 8192, 1024);
       const uint64_t bdesc0 = smem_desc_sw128(sbase + (W8 ? a8_bytes : a_bytes), 16, 1024);
       uint32_t s = 0, ph = 0, soff = 0;
       uint32_t kbi = 0;  // W8: k-blocks issued (bf16 slot kbi & 1, its use count kbi >> 1)
@@ -380,7 +413,8 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * 256);
         const uint32_t d1 = d0 + static_cast<uint32_t>(p.TB);
         const uint32_t idesc =
-            idesc_bf16(PAIR ? 2 * kBM : kBM, npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
+            F8 ? idesc_e4m3(PAIR ? 2 * kBM : kBM, npad)
+               : idesc_bf16(PAIR ? 2 * kBM : kBM, npad, /*a_mn_major=*/true, /*b_mn_major=*/false);
         uint32_t acc = 0;
 #pragma unroll 2
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
@@ -400,16 +434,29 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
               W8 ? adesc0 + (kbi & 1) * static_cast<uint32_t>(a_bytes >> 4) : adesc0 + (soff >> 4);
           const uint64_t bd = bdesc0 + (soff >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            // A advances 16 K-rows (2 KB), B 16 K-columns (32 B) per step; the second A
-            // operand sits 16 KB after the first
-            if constexpr (PAIR) tc_mma_bf16_pair_elect(d0, ad + kk * 128, bd + kk * 2, idesc, acc);
-            else tc_mma_bf16_elect(d0, ad + kk * 128, bd + kk * 2, idesc, acc);
-            if constexpr (kDual) {
-              if constexpr (PAIR)
-                tc_mma_bf16_pair_elect(d1, ad + 1024 + kk * 128, bd + kk * 2, idesc, acc);
-              else
-                tc_mma_bf16_elect(d1, ad + 1024 + kk * 128, bd + kk * 2, idesc, acc);
+          for (int kk = 0; kk < 4; ++kk) {
+            // bf16: A advances 16 K-rows (2 KB), B 16 K-columns (32 B) per step; F8: both
+            // advance 32 K-columns (32 B) per step. The second A operand sits 16 KB after the
+            // first.
+            constexpr uint32_t kAStep = F8 ? 2u : 128u;
+            if constexpr (F8) {
+              if constexpr (PAIR) tc_mma_f8_pair_elect(d0, ad + kk * kAStep, bd + kk * 2, idesc, acc);
+              else tc_mma_f8_elect(d0, ad + kk * kAStep, bd + kk * 2, idesc, acc);
+              if constexpr (kDual) {
+                if constexpr (PAIR)
+                  tc_mma_f8_pair_elect(d1, ad + 1024 + kk * kAStep, bd + kk * 2, idesc, acc);
+                else
+                  tc_mma_f8_elect(d1, ad + 1024 + kk * kAStep, bd + kk * 2, idesc, acc);
+              }
+            } else {
+              if constexpr (PAIR) tc_mma_bf16_pair_elect(d0, ad + kk * kAStep, bd + kk * 2, idesc, acc);
+              else tc_mma_bf16_elect(d0, ad + kk * kAStep, bd + kk * 2, idesc, acc);
+              if constexpr (kDual) {
+                if constexpr (PAIR)
+                  tc_mma_bf16_pair_elect(d1, ad + 1024 + kk * kAStep, bd + kk * 2, idesc, acc);
+                else
+                  tc_mma_bf16_elect(d1, ad + 1024 + kk * kAStep, bd + kk * 2, idesc, acc);
+              }
             }
             acc = 1u;
           }
@@ -576,20 +623,28 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
       // write the rows out: the next tile's MMAs run under these stores.
       constexpr int kW = (MODE == kEpiBF16x2) ? 32 : 16;  // words held per 32-column chunk
       uint32_t pk[kEpiChunks][kW];
-      // W8: channel scales of this lane's feature rows (1 otherwise, and then unused)
+      // W8 / F8: channel scales of this lane's feature rows (1 otherwise, and then unused)
       float sc0 = 1.0f, sc1 = 1.0f;
-      if constexpr (W8) {
+      if constexpr (W8 || F8) {
         const size_t so = static_cast<size_t>(t.group) * p.scale_ld + m;
         sc0 = p.scale0[so];
         if constexpr (kSwiGLU) sc1 = p.scale1[so];
         else if constexpr (kDual) sc1 = p.scale0[so + 128];
       }
-      auto scl0 = [&](uint32_t a) { return W8 ? __uint_as_float(a) * sc0 : __uint_as_float(a); };
-      auto scl1 = [&](uint32_t a) { return W8 ? __uint_as_float(a) * sc1 : __uint_as_float(a); };
+      auto scl0 = [&](uint32_t a) {
+        return (W8 || F8) ? __uint_as_float(a) * sc0 : __uint_as_float(a);
+      };
+      auto scl1 = [&](uint32_t a) {
+        return (W8 || F8) ? __uint_as_float(a) * sc1 : __uint_as_float(a);
+      };
 #pragma unroll
       for (int i = 0; i < kEpiChunks; ++i) {
         const int c0 = 32 * half + 64 * i;
         if (c0 < t.n) {
+          // F8: the row scale of column (token row) c0 + lane, broadcast to the warp per column
+          float csv = 1.0f;
+          if constexpr (F8) csv = (c0 + lane < t.n) ? p.act_scale[t.row0 + c0 + lane] : 0.0f;
+          auto cs = [&](int col) { return F8 ? __shfl_sync(0xffffffffu, csv, col) : 1.0f; };
           uint32_t v[32];
           tmem_ld32(tb + static_cast<uint32_t>(c0), v);
           if constexpr (kSwiGLU) {
@@ -597,20 +652,23 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
             tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), u);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              pk[i][j] = pack_bf16x2(silu_f32(scl0(v[2 * j])) * scl1(u[2 * j]),
-                                     silu_f32(scl0(v[2 * j + 1])) * scl1(u[2 * j + 1]));
+            for (int j = 0; j < 16; ++j) {
+              const float ca = cs(2 * j), cb = cs(2 * j + 1);
+              pk[i][j] = pack_bf16x2(silu_f32(scl0(v[2 * j]) * ca) * (scl1(u[2 * j]) * ca),
+                                     silu_f32(scl0(v[2 * j + 1]) * cb) * (scl1(u[2 * j + 1]) * cb));
+            }
           } else {
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              pk[i][j] = pack_bf16x2(scl0(v[2 * j]), scl0(v[2 * j + 1]));
+              pk[i][j] = pack_bf16x2(scl0(v[2 * j]) * cs(2 * j), scl0(v[2 * j + 1]) * cs(2 * j + 1));
             if constexpr (kDual) {
               tmem_ld32(tb + static_cast<uint32_t>(p.TB + c0), v);
               tmem_wait_ld();
 #pragma unroll
               for (int j = 0; j < 16; ++j)
-                pk[i][16 + j] = pack_bf16x2(scl1(v[2 * j]), scl1(v[2 * j + 1]));
+                pk[i][16 + j] =
+                    pack_bf16x2(scl1(v[2 * j]) * cs(2 * j), scl1(v[2 * j + 1]) * cs(2 * j + 1));
             }
           }
         }
@@ -763,7 +821,48 @@ bool map_weights_fp8(CUtensorMap* m, const void* base, uint64_t mdim, uint64_t k
   return r == CUDA_SUCCESS;
 }
 
-template <int MODE, int BMODE, bool PAIR, bool W8 = false>
+// K-major e4m3 weight codes [groups][mdim][kdim] (K contiguous): box {128 K bytes, box_rows
+// feature rows, 1 group}, 128-byte swizzle.
+bool map_weights_kmajor_e4m3(CUtensorMap* m, const void* base, uint64_t kdim, uint64_t mdim,
+                             uint64_t groups, uint32_t box_rows, std::string* d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) {
+    if (d) *d = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  cuuint64_t dims[3] = {kdim, mdim, groups};
+  cuuint64_t strides[2] = {kdim, kdim * mdim};
+  cuuint32_t box[3] = {128, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && d)
+    *d = "cuTensorMapEncodeTiled(K-major e4m3 weights) failed with code " + std::to_string(r);
+  return r == CUDA_SUCCESS;
+}
+
+// e4m3 rows [rows][cols] (one byte each): box {128 columns, box_rows rows}, 128-byte swizzle.
+bool map_rows_e4m3(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                   uint32_t box_rows, std::string* d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) {
+    if (d) *d = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && d)
+    *d = "cuTensorMapEncodeTiled(e4m3 rows) failed with code " + std::to_string(r);
+  return r == CUDA_SUCCESS;
+}
+
+template <int MODE, int BMODE, bool PAIR, bool W8 = false, bool F8 = false>
 cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                         TcParams p, int64_t tiles_ub, int num_sms, cudaStream_t stream,
                         std::string* d) {
@@ -788,7 +887,7 @@ cudaError_t launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   int64_t grid = tiles_ub < units ? tiles_ub : units;
   if (grid < 1) grid = 1;
   if (PAIR) grid *= 2;
-  auto kernel = tc_grouped_gemm<MODE, BMODE, PAIR, W8>;
+  auto kernel = tc_grouped_gemm<MODE, BMODE, PAIR, W8, F8>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -985,6 +1084,92 @@ cudaError_t launch_gemm2_w8(const void* hbuf, int64_t hbuf_rows, const int32_t* 
                                                          detail);
   return launch_mode<kEpiBF16, kBTiled, false, true>(a0, a0, b, p, tiles, num_sms, stream,
                                                      detail);
+}
+
+// ---- FP8 weights and activations (W8A8): native e4m3 MMAs on CTA pairs, B streamed by TMA
+// from expert-major e4m3 rows.
+
+cudaError_t launch_gemm1_f8(const void* xs8, const float* sx, const int32_t* offsets,
+                            const int32_t* blk_prefix, const uint8_t* qk_gate,
+                            const uint8_t* qk_up, const float* s_gate, const float* s_up,
+                            void* hbuf, int64_t hbuf_rows, int H, int E, int I, int TB,
+                            int64_t ub_blocks, int* err, int num_sms, cudaStream_t stream,
+                            std::string* detail) {
+  CUtensorMap a0, a1, b;
+  const bool pair = kUsePairs;
+  const int box_rows = b_rows_smem(pair, TB);
+  if (!map_weights_kmajor_e4m3(&a0, qk_gate, H, I, E, 128, detail) ||
+      !map_weights_kmajor_e4m3(&a1, qk_up, H, I, E, 128, detail) ||
+      !map_rows_e4m3(&b, xs8, static_cast<uint64_t>(H), static_cast<uint64_t>(hbuf_rows),
+                     static_cast<uint32_t>(box_rows), detail))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.b_box_rows = box_rows;
+  p.K = H;
+  p.num_fb = pair ? (I + 255) / 256 : I / kBM;
+  p.m_valid = I;
+  p.TB = TB;
+  p.groups = E;
+  p.k_top = 1;
+  p.rows_b = static_cast<int>(hbuf_rows);
+  p.offsets = offsets;
+  p.blk_prefix = blk_prefix;
+  p.out = hbuf;
+  p.ldo = I;
+  p.err = err;
+  p.scale0 = s_gate;
+  p.scale1 = s_up;
+  p.scale_ld = I;
+  p.act_scale = sx;
+  const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
+  if (pair)
+    return launch_mode<kEpiSwiGLU, kBTiled, true, false, true>(a0, a1, b, p, tiles, num_sms,
+                                                               stream, detail);
+  return launch_mode<kEpiSwiGLU, kBTiled, false, false, true>(a0, a1, b, p, tiles, num_sms, stream,
+                                                              detail);
+}
+
+cudaError_t launch_gemm2_f8(const void* h8, const float* sh, int64_t hbuf_rows,
+                            const int32_t* offsets, const int32_t* blk_prefix,
+                            const uint8_t* qk_down, const float* s_down, void* y, int H, int E,
+                            int I, int TB, int64_t ub_blocks, int* err, int num_sms,
+                            cudaStream_t stream, std::string* detail) {
+  CUtensorMap a0, b;
+  const bool dual = (H % 256) == 0;
+  const bool pair = kUsePairs && dual;
+  const int box_rows = b_rows_smem(pair, TB);
+  // a CTA's 256 (dual) or 128 feature rows of the down projection as one box
+  if (!map_weights_kmajor_e4m3(&a0, qk_down, I, H, E, dual ? 256 : 128, detail) ||
+      !map_rows_e4m3(&b, h8, static_cast<uint64_t>(I), static_cast<uint64_t>(hbuf_rows),
+                     static_cast<uint32_t>(box_rows), detail))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.b_box_rows = box_rows;
+  p.K = I;
+  p.num_fb = pair ? (H + 511) / 512 : (dual ? H / 256 : H / kBM);
+  p.m_valid = H;
+  p.TB = TB;
+  p.groups = E;
+  p.k_top = 1;
+  p.rows_b = static_cast<int>(hbuf_rows);
+  p.offsets = offsets;
+  p.blk_prefix = blk_prefix;
+  p.out = y;
+  p.ldo = H;
+  p.err = err;
+  p.scale0 = s_down;
+  p.scale1 = nullptr;
+  p.scale_ld = H;
+  p.act_scale = sh;
+  const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
+  if (pair)
+    return launch_mode<kEpiBF16x2, kBTiled, true, false, true>(a0, a0, b, p, tiles, num_sms,
+                                                               stream, detail);
+  if (dual)
+    return launch_mode<kEpiBF16x2, kBTiled, false, false, true>(a0, a0, b, p, tiles, num_sms,
+                                                                stream, detail);
+  return launch_mode<kEpiBF16, kBTiled, false, false, true>(a0, a0, b, p, tiles, num_sms, stream,
+                                                            detail);
 }
 
 }  // namespace moe

@@ -23,14 +23,26 @@ cudaError_t launch_topk(const float* partials, int ksplit, int64_t split_stride,
                         int n_group, int topk_group, int32_t* topk_idx, float* topk_w,
                         cudaStream_t stream);
 
+// Gate logits for a few tokens (decode) on CUDA cores, bf16, E % 32 == 0, T <= kRouteGemvMaxT:
+// partials[ks][t][e] for kRouteGemvSplit K ranges of H / kRouteGemvSplit rows each (the layout
+// launch_topk sums).
+constexpr int kRouteGemvMaxT = 64;
+constexpr int kRouteGemvSplit = 16;
+bool route_uses_gemv(int64_t T, int H, int E);
+cudaError_t launch_route_gemv(const void* x, const void* w_router, int T, int H, int E,
+                              float* partials, cudaStream_t stream);
+
 // ---- route_tc.cu (tcgen05 / TMEM / TMA, bf16)
-// Gate logits on the tensor cores (tokens on the MMA's M side, experts on N, E in [16, 256],
-// E % 8 == 0), K split into `ksplit` ranges:
-// partials[ks][t][e] = sum over h in range ks of x[t,h] * w_router[h,e].
-int route_ksplit(int64_t T, int H, int E);
-cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int H, int E,
-                                 float* partials, int ksplit, int* err, int num_sms,
-                                 cudaStream_t stream, std::string* detail);
+// The whole router in one launch for E in [16, 256], E % 8 == 0: gate logits on the tensor
+// cores (tokens on the MMA's M side, experts on N), the K split into `ksplit` ranges whose
+// partial logits are summed (ascending range) inside a thread-block cluster through distributed
+// shared memory, then top-k + renormalised weights (select.cuh) and, when logits_out is non-null,
+// the logits (bias included). The launch layout (CTA pairs or single CTAs, the number of K
+// ranges) is chosen per T so that every cluster fits on the GPU at once when possible.
+cudaError_t launch_route_tc(const void* x, const void* w_router, const float* bias, int T, int H,
+                            int E, int k, int n_group, int topk_group, float* logits_out,
+                            int32_t* topk_idx, float* topk_w, int* err, cudaStream_t stream,
+                            std::string* detail);
 
 // ---- ffn_tc.cu (tcgen05 / TMEM / TMA, bf16)
 // Expert GEMM1: h[s, :] = silu(x[t] Wg[e]) * (x[t] Wu[e]) for kept slots; h rows = hbuf_rows.
@@ -46,6 +58,21 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
 // Expert GEMM2: y[s, :] = h[s] Wd[e].
 cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* offsets,
                             const int32_t* blk_prefix, const void* w_down, void* y, int H, int E,
+                            int I, int TB, int64_t ub_blocks, int* err, int num_sms,
+                            cudaStream_t stream, std::string* detail);
+
+// FP8 weights and activations (W8A8): GEMM1 from expert-major e4m3 rows xs8 [rows][H] with row
+// scales sx, K-major weight codes [E][I][H] and channel scales [E][I]; h written as bf16.
+// GEMM2 from e4m3 rows h8 [rows][I] with row scales sh, K-major codes [E][H][I], scales [E][H].
+cudaError_t launch_gemm1_f8(const void* xs8, const float* sx, const int32_t* offsets,
+                            const int32_t* blk_prefix, const uint8_t* qk_gate,
+                            const uint8_t* qk_up, const float* s_gate, const float* s_up,
+                            void* hbuf, int64_t hbuf_rows, int H, int E, int I, int TB,
+                            int64_t ub_blocks, int* err, int num_sms, cudaStream_t stream,
+                            std::string* detail);
+cudaError_t launch_gemm2_f8(const void* h8, const float* sh, int64_t hbuf_rows,
+                            const int32_t* offsets, const int32_t* blk_prefix,
+                            const uint8_t* qk_down, const float* s_down, void* y, int H, int E,
                             int I, int TB, int64_t ub_blocks, int* err, int num_sms,
                             cudaStream_t stream, std::string* detail);
 
@@ -93,6 +120,21 @@ cudaError_t launch_align_noalloc(const int32_t* topk_idx, int64_t A, int E, int 
 cudaError_t launch_plan_from_offsets(const int32_t* offsets, int E, int TB, int32_t* blk_prefix,
                                      cudaStream_t stream);
 
+// ---- quant.cu: FP8 weights and activations (W8A8)
+// Weights w [E][K][M] bf16 -> K-major e4m3 codes [E][M][K] and per-channel scales [E][M]
+// (K % 64 == 0, M % 64 == 0).
+cudaError_t launch_pack_w8a8(const void* w, int64_t E, int K, int M, uint8_t* codes, float* scale,
+                             cudaStream_t stream);
+// Per-row e4m3 codes [N][K] and scales [N] of bf16 rows a [N][K] (K % 8 == 0); rows at or past
+// *n_dev (a device count, when non-null) are skipped.
+cudaError_t launch_quantize_rows(const void* a, int64_t N, const int32_t* n_dev, int K,
+                                 uint8_t* codes, float* scale, cudaStream_t stream);
+// Expert-major copy of quantised token rows: xs8[s] = x8[sorted_ids[s] / k], sx[s] likewise, for
+// the kept slots s < offsets[E] (H % 16 == 0).
+cudaError_t launch_dispatch_rows_q8(const uint8_t* x8, const float* sxt, const int32_t* sorted_ids,
+                                    const int32_t* offsets, int E, int k, int H, int64_t rows,
+                                    uint8_t* xs8, float* sx, cudaStream_t stream);
+
 // ---- probe.cu: one bounded wait that nothing satisfies (failure-detection test)
 cudaError_t launch_stalled_wait(int* err, cudaStream_t stream);
 
@@ -103,6 +145,10 @@ cudaError_t launch_ep_plan(const int32_t* topk_idx, const int32_t* slot_of_local
                            int32_t* own_offsets, int* err, int num_sms, cudaStream_t stream);
 cudaError_t launch_ep_dispatch(int dtype, const void* x, const int32_t* owner, const int32_t* slot,
                                void* const* peer_xs, int64_t A, int k, int H, cudaStream_t stream);
+cudaError_t launch_ep_signal(uint32_t* const* peer_flags, int R, int rank, uint32_t epoch,
+                             cudaStream_t stream);
+cudaError_t launch_ep_wait(const uint32_t* flags, int R, uint32_t epoch, int* err,
+                           cudaStream_t stream);
 cudaError_t launch_ep_combine(int dtype, const void* const* peer_y, const int32_t* owner,
                               const int32_t* slot, const float* topk_w, void* out, int64_t T,
                               int H, int k, cudaStream_t stream);

@@ -109,11 +109,13 @@ bool gemm1_from_copy(const moe_shape& s) {
 
 struct Layout {
   size_t err, logits, blk_hist, offsets, blk_prefix, sorted_ids, slot_of, hbuf, yslots, xs, total;
+  size_t logits_bytes;
+  size_t x8, h8;  // W8A8 (bf16 shapes): e4m3 token rows + scales, e4m3 h rows + scales
   int64_t A, a_cap;
   int nblk;
   int32_t C;
   int TB;
-  int ksplit;  // router K split (tensor-core router only)
+  int ksplit;  // K ranges of the split-K GEMV router (1 otherwise)
 };
 
 Layout layout_of(const moe_shape& s) {
@@ -132,9 +134,14 @@ Layout layout_of(const moe_shape& s) {
   };
   const size_t es = elem_size(s.dtype);
   L.err = take(256);
-  L.ksplit = (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0 && s.T > 0)
-                 ? moe::route_ksplit(s.T, s.H, s.E) : 1;
-  L.logits = take(static_cast<size_t>(s.T) * s.E * 4 * L.ksplit);
+  L.ksplit = 1;  // K ranges of the split-K GEMV router (its partial logits live here)
+  if (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0 && moe::route_uses_gemv(s.T, s.H, s.E))
+    L.ksplit = moe::kRouteGemvSplit;
+  // partial logits of the split-K GEMV (a few tokens), or the logits of the CUDA-core router
+  // before a group-limited selection; the tensor-core router keeps its partials on chip
+  const bool gemv = L.ksplit > 1 && moe::route_uses_gemv(s.T, s.H, s.E);
+  L.logits_bytes = static_cast<size_t>(s.T) * s.E * 4 * (gemv ? L.ksplit : 1);
+  L.logits = take(L.logits_bytes);
   L.blk_hist = take(static_cast<size_t>(L.nblk) * s.E * 4);
   L.offsets = take(static_cast<size_t>(s.E + 1) * 4);
   L.blk_prefix = take(static_cast<size_t>(s.E + 1) * 4);
@@ -143,6 +150,13 @@ Layout layout_of(const moe_shape& s) {
   L.hbuf = take(static_cast<size_t>(L.a_cap) * s.I * es);
   L.yslots = take(static_cast<size_t>(L.a_cap) * s.H * es);
   L.xs = s.dtype == MOE_BF16 ? take(static_cast<size_t>(L.a_cap) * s.H * es) : 0;
+  // W8A8: x quantised per token ([T][H] codes, then T scales) and h per slot ([a_cap][I] codes,
+  // then a_cap scales); the expert-major e4m3 rows and their scales reuse the xs region
+  L.x8 = s.dtype == MOE_BF16 ? take(static_cast<size_t>(s.T) * s.H + static_cast<size_t>(s.T) * 4)
+                             : 0;
+  L.h8 = s.dtype == MOE_BF16
+             ? take(static_cast<size_t>(L.a_cap) * s.I + static_cast<size_t>(L.a_cap) * 4)
+             : 0;
   L.total = off;
   return L;
 }
@@ -224,14 +238,21 @@ moe_status do_route(const moe_shape& s, const Layout& L, const Opts& o, const vo
                     float* topk_w, void* ws, cudaStream_t st) {
   cudaError_t e;
   if (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0) {
-    float* partials = at<float>(ws, L.logits);
-    std::string d;
-    e = moe::launch_route_gemm_tc(x, w_router, static_cast<int>(s.T), s.H, s.E, partials,
-                                  L.ksplit, at<int>(ws, L.err), num_sms(), st, &d);
-    if (e != cudaSuccess) return cuda_fail(e, "router gate GEMM (tcgen05)", d);
-    e = moe::launch_topk(partials, L.ksplit, s.T * s.E, bias, logits_out, s.T, s.E, s.k,
-                         o.n_group, o.topk_group, topk_idx, topk_w, st);
-    if (e != cudaSuccess) return cuda_fail(e, "router top-k");
+    if (moe::route_uses_gemv(s.T, s.H, s.E)) {
+      // a few tokens: stream the router weight once on CUDA cores (split-K GEMV), then select
+      float* partials = at<float>(ws, L.logits);
+      e = moe::launch_route_gemv(x, w_router, static_cast<int>(s.T), s.H, s.E, partials, st);
+      if (e != cudaSuccess) return cuda_fail(e, "router gate GEMV (CUDA cores)");
+      e = moe::launch_topk(partials, L.ksplit, s.T * s.E, bias, logits_out, s.T, s.E, s.k,
+                           o.n_group, o.topk_group, topk_idx, topk_w, st);
+      if (e != cudaSuccess) return cuda_fail(e, "router top-k");
+    } else {
+      std::string d;
+      e = moe::launch_route_tc(x, w_router, bias, static_cast<int>(s.T), s.H, s.E, s.k,
+                               o.n_group, o.topk_group, logits_out, topk_idx, topk_w,
+                               at<int>(ws, L.err), st, &d);
+      if (e != cudaSuccess) return cuda_fail(e, "router (tcgen05 gate GEMM + top-k)", d);
+    }
   } else {
     // the fused CUDA-core router selects plain top-k; with groups its logits (bias included)
     // go through the group-limited top-k kernel
@@ -260,7 +281,8 @@ struct FfnWeights {
   const float* s_gate = nullptr;
   const float* s_up = nullptr;
   const float* s_down = nullptr;
-  bool w8 = false;
+  bool w8 = false;   // e4m3 weights [E][K][M], bf16 activations (W8A16)
+  bool a8 = false;   // K-major e4m3 weights [E][M][K] and e4m3 activations (W8A8)
 };
 
 moe_status do_ffn(const moe_shape& s, const Layout& L, const void* x, const int32_t* sorted_ids,
@@ -270,7 +292,34 @@ moe_status do_ffn(const moe_shape& s, const Layout& L, const void* x, const int3
   const void* w_up = fw.w_up;
   const void* w_down = fw.w_down;
   cudaError_t e;
-  if (fw.w8) {
+  if (fw.a8) {
+    // x quantised once per token, copied expert-major with its scales; GEMM1 on e4m3 rows; h
+    // (bf16) quantised per slot row; GEMM2 on e4m3 rows
+    const int64_t ub_blocks = (s.E < L.a_cap ? s.E : L.a_cap) + L.a_cap / L.TB;
+    std::string d;
+    uint8_t* x8 = at<uint8_t>(ws, L.x8);
+    float* sxt = reinterpret_cast<float*>(x8 + static_cast<size_t>(s.T) * s.H);
+    uint8_t* xs8 = at<uint8_t>(ws, L.xs);
+    float* sx = reinterpret_cast<float*>(xs8 + static_cast<size_t>(L.a_cap) * s.H);
+    uint8_t* h8 = at<uint8_t>(ws, L.h8);
+    float* sh = reinterpret_cast<float*>(h8 + static_cast<size_t>(L.a_cap) * s.I);
+    e = moe::launch_quantize_rows(x, s.T, nullptr, s.H, x8, sxt, st);
+    if (e != cudaSuccess) return cuda_fail(e, "e4m3 quantisation of the token rows");
+    e = moe::launch_dispatch_rows_q8(x8, sxt, sorted_ids, offsets, s.E, s.k, s.H, L.a_cap, xs8,
+                                     sx, st);
+    if (e != cudaSuccess) return cuda_fail(e, "expert-major copy of the e4m3 rows");
+    e = moe::launch_gemm1_f8(xs8, sx, offsets, at<int32_t>(ws, L.blk_prefix), fw.q_gate, fw.q_up,
+                             fw.s_gate, fw.s_up, at<void>(ws, L.hbuf), L.a_cap, s.H, s.E, s.I,
+                             L.TB, ub_blocks, at<int>(ws, L.err), num_sms(), st, &d);
+    if (e != cudaSuccess) return cuda_fail(e, "expert GEMM1 (tcgen05, e4m3 x e4m3)", d);
+    if (stage_events) record_stage(2, st);
+    e = moe::launch_quantize_rows(at<void>(ws, L.hbuf), L.a_cap, offsets + s.E, s.I, h8, sh, st);
+    if (e != cudaSuccess) return cuda_fail(e, "e4m3 quantisation of the SwiGLU rows");
+    e = moe::launch_gemm2_f8(h8, sh, L.a_cap, offsets, at<int32_t>(ws, L.blk_prefix), fw.q_down,
+                             fw.s_down, y, s.H, s.E, s.I, L.TB, ub_blocks, at<int>(ws, L.err),
+                             num_sms(), st, &d);
+    if (e != cudaSuccess) return cuda_fail(e, "expert GEMM2 (tcgen05, e4m3 x e4m3)", d);
+  } else if (fw.w8) {
     const int64_t ub_blocks = (s.E < L.a_cap ? s.E : L.a_cap) + L.a_cap / L.TB;
     std::string d;
     void* xs = at<void>(ws, L.xs);
@@ -349,7 +398,7 @@ moe_status moe_route_ex(const moe_shape* shape, const moe_layer_opts* opts, cons
   OPT_PTR(logit_bias, "logit_bias");
   OPT_PTR(logits_out, "logits_out");
   const Layout L = layout_of(*shape);
-  st = check_ws(ws, ws_bytes, L.logits + static_cast<size_t>(shape->T) * shape->E * 4 * L.ksplit);
+  st = check_ws(ws, ws_bytes, L.logits + L.logits_bytes);
   if (st != MOE_OK) return st;
   return do_route(*shape, L, o, x, w_router, logit_bias, logits_out, topk_idx, topk_w, ws,
                   static_cast<cudaStream_t>(stream));
@@ -558,6 +607,31 @@ moe_status moe_ep_dispatch(const moe_shape* shape, int32_t R, const void* x,
   return MOE_OK;
 }
 
+moe_status moe_ep_signal(int32_t R, int32_t rank, uint32_t epoch, uint32_t* const* peer_flags,
+                         void* stream) {
+  if (R < 1 || R > 256) return fail(MOE_ERR_INVALID_ARG, "R must be in [1, 256]");
+  if (rank < 0 || rank >= R) return fail(MOE_ERR_INVALID_ARG, "rank outside [0, R)");
+  REQUIRE_PTR(peer_flags, "peer_flags");
+  cudaError_t e = moe::launch_ep_signal(peer_flags, R, rank, epoch,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "expert-parallel signal");
+  return MOE_OK;
+}
+
+moe_status moe_ep_wait(int32_t R, uint32_t epoch, const uint32_t* flags, void* ws,
+                       size_t ws_bytes, void* stream) {
+  if (R < 1 || R > 256) return fail(MOE_ERR_INVALID_ARG, "R must be in [1, 256]");
+  if (flags == nullptr) return fail(MOE_ERR_INVALID_ARG, "flags is NULL");
+  if ((reinterpret_cast<uintptr_t>(flags) & 3u) != 0)
+    return fail(MOE_ERR_INVALID_ARG, "flags is not 4-byte aligned");
+  moe_status st = check_ws(ws, ws_bytes, 256);
+  if (st != MOE_OK) return st;
+  cudaError_t e = moe::launch_ep_wait(flags, R, epoch, at<int>(ws, 0),
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "expert-parallel wait");
+  return MOE_OK;
+}
+
 moe_status moe_ep_combine(const moe_shape* shape, int32_t R, const void* const* peer_y,
                           const int32_t* owner, const int32_t* slot, const float* topk_w,
                           void* out, void* stream) {
@@ -602,7 +676,7 @@ moe_status layer_impl(const moe_shape* shape, const moe_layer_opts* opts, const 
   }
   REQUIRE_PTR(x, "x");
   REQUIRE_PTR(w_router, "w_router");
-  if (fw.w8) {
+  if (fw.w8 || fw.a8) {
     if (s.dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "e4m3 expert weights need bf16");
     REQUIRE_PTR(fw.q_gate, "q_gate");
     REQUIRE_PTR(fw.q_up, "q_up");
@@ -729,6 +803,90 @@ moe_status moe_quantize_weights_fp8(const void* w, int64_t E, int64_t K, int64_t
                                            scale, num_sms(), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "e4m3 weight quantisation");
   return MOE_OK;
+}
+
+moe_status moe_pack_weights_w8a8(const void* w, int64_t E, int64_t K, int64_t M, uint8_t* codes,
+                                 float* scale, void* stream) {
+  if (E < 0 || K < 64 || M < 64 || K % 64 != 0 || M % 64 != 0 || K > (1 << 30) || M > (1 << 30))
+    return fail(MOE_ERR_INVALID_ARG, "need E >= 0 and K, M positive multiples of 64");
+  if (E == 0) return MOE_OK;
+  REQUIRE_PTR(w, "w");
+  REQUIRE_PTR(codes, "codes");
+  REQUIRE_PTR(scale, "scale");
+  cudaError_t e = moe::launch_pack_w8a8(w, E, static_cast<int>(K), static_cast<int>(M), codes,
+                                        scale, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "W8A8 weight packing");
+  return MOE_OK;
+}
+
+moe_status moe_quantize_rows_fp8(const void* a, int64_t N, int64_t K, uint8_t* codes,
+                                 float* scale, void* stream) {
+  if (N < 0 || K < 8 || K % 8 != 0 || K > (1 << 30))
+    return fail(MOE_ERR_INVALID_ARG, "need N >= 0 and K a positive multiple of 8");
+  if (N == 0) return MOE_OK;
+  REQUIRE_PTR(a, "a");
+  REQUIRE_PTR(codes, "codes");
+  REQUIRE_PTR(scale, "scale");
+  cudaError_t e = moe::launch_quantize_rows(a, N, nullptr, static_cast<int>(K), codes, scale,
+                                            static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "e4m3 row quantisation");
+  return MOE_OK;
+}
+
+moe_status moe_grouped_ffn_w8a8(const moe_shape* shape, const void* x, const int32_t* sorted_ids,
+                                const int32_t* offsets, const uint8_t* qk_gate,
+                                const uint8_t* qk_up, const uint8_t* qk_down, const float* s_gate,
+                                const float* s_up, const float* s_down, void* y_slots, void* ws,
+                                size_t ws_bytes, void* stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "e4m3 expert weights need bf16");
+  if (shape->T == 0) return MOE_OK;
+  REQUIRE_PTR(x, "x");
+  REQUIRE_PTR(sorted_ids, "sorted_ids");
+  REQUIRE_PTR(offsets, "offsets");
+  REQUIRE_PTR(qk_gate, "qk_gate");
+  REQUIRE_PTR(qk_up, "qk_up");
+  REQUIRE_PTR(qk_down, "qk_down");
+  REQUIRE_PTR(s_gate, "s_gate");
+  REQUIRE_PTR(s_up, "s_up");
+  REQUIRE_PTR(s_down, "s_down");
+  REQUIRE_PTR(y_slots, "y_slots");
+  const Layout L = layout_of(*shape);
+  st = check_ws(ws, ws_bytes, L.total);
+  if (st != MOE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = moe::launch_plan_from_offsets(offsets, shape->E, L.TB,
+                                                at<int32_t>(ws, L.blk_prefix), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "expert GEMM tile plan");
+  FfnWeights fw;
+  fw.q_gate = qk_gate;
+  fw.q_up = qk_up;
+  fw.q_down = qk_down;
+  fw.s_gate = s_gate;
+  fw.s_up = s_up;
+  fw.s_down = s_down;
+  fw.a8 = true;
+  return do_ffn(*shape, L, x, sorted_ids, offsets, fw, y_slots, ws, cs, false);
+}
+
+moe_status moe_layer_forward_w8a8(const moe_shape* shape, const moe_layer_opts* opts,
+                                  const void* x, const void* w_router, const float* logit_bias,
+                                  const uint8_t* qk_gate, const uint8_t* qk_up,
+                                  const uint8_t* qk_down, const float* s_gate, const float* s_up,
+                                  const float* s_down, void* out, float* logits_out,
+                                  int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                  uint8_t* drop_mask, void* ws, size_t ws_bytes, void* stream) {
+  FfnWeights fw;
+  fw.q_gate = qk_gate;
+  fw.q_up = qk_up;
+  fw.q_down = qk_down;
+  fw.s_gate = s_gate;
+  fw.s_up = s_up;
+  fw.s_down = s_down;
+  fw.a8 = true;
+  return layer_impl(shape, opts, x, w_router, logit_bias, fw, out, logits_out, topk_idx, topk_w,
+                    counts, drop_mask, ws, ws_bytes, stream);
 }
 
 moe_status moe_layer_forward(const moe_shape* shape, const void* x, const void* w_router,

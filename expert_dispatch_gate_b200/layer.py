@@ -193,3 +193,69 @@ def layer_forward_w8(x, w_router, fp8, k, capacity_factor, logit_bias=None, logi
     res["ws"] = ws
     res["C"] = L.moe_capacity(shape)
     return res
+
+
+# ---- FP8 weights and activations (W8A8)
+
+def pack_w8a8(w, stream=None):
+    """K-major e4m3 codes [E,M,K] (uint8) and per-channel float32 scales [E,M] of bf16 weights
+    [E,K,M] (moe_pack_weights_w8a8)."""
+    E, K, M = w.shape
+    codes = torch.empty((E, M, K), dtype=torch.uint8, device=w.device)
+    scale = torch.empty((E, M), dtype=torch.float32, device=w.device)
+    L.moe_pack_weights_w8a8(w, E, K, M, codes, scale, stream)
+    return codes, scale
+
+
+def quantize_rows_fp8(a, stream=None):
+    """Per-row e4m3 codes [N,K] (uint8) and float32 scales [N] of bf16 rows a [N,K]."""
+    N, K = a.shape
+    codes = torch.empty((N, K), dtype=torch.uint8, device=a.device)
+    scale = torch.empty(N, dtype=torch.float32, device=a.device)
+    L.moe_quantize_rows_fp8(a, N, K, codes, scale, stream)
+    return codes, scale
+
+
+class W8A8Weights:
+    """The three expert weights repacked as K-major e4m3 codes + scales (on the device)."""
+
+    def __init__(self, w_gate, w_up, w_down, stream=None):
+        self.q_gate, self.s_gate = pack_w8a8(w_gate, stream)
+        self.q_up, self.s_up = pack_w8a8(w_up, stream)
+        self.q_down, self.s_down = pack_w8a8(w_down, stream)
+        self.E, self.H, self.I = w_gate.shape
+
+    def args(self):
+        return (self.q_gate, self.q_up, self.q_down, self.s_gate, self.s_up, self.s_down)
+
+
+def grouped_ffn_w8a8(x, sorted_ids, offsets, wq, k, capacity_factor, ws=None, stream=None):
+    T, H = x.shape
+    shape = shape_of(T, H, wq.E, k, wq.I, capacity_factor, L.MOE_BF16)
+    ws = ws or Workspace(shape, x.device)
+    y = torch.empty((T * k, H), dtype=x.dtype, device=x.device)
+    L.moe_grouped_ffn_w8a8(shape, x, sorted_ids, offsets, *wq.args(), y, ws.buf, ws.nbytes, stream)
+    return y
+
+
+def layer_forward_w8a8(x, w_router, wq, k, capacity_factor, logit_bias=None, logits_out=True,
+                       ws=None, out=None, stream=None, opts=None):
+    """Whole layer with W8A8 expert GEMMs (moe_layer_forward_w8a8)."""
+    T, H = x.shape
+    E = w_router.shape[1]
+    dev = x.device
+    shape = shape_of(T, H, E, k, wq.I, capacity_factor, _dtype_code(x))
+    ws = ws or Workspace(shape, dev)
+    res = MoELayerOutputs()
+    res["out"] = out if out is not None else torch.empty((T, H), dtype=x.dtype, device=dev)
+    res["topk_idx"] = torch.empty((T, k), dtype=torch.int32, device=dev)
+    res["topk_w"] = torch.empty((T, k), dtype=torch.float32, device=dev)
+    res["counts"] = torch.empty(E, dtype=torch.int32, device=dev)
+    res["drop_mask"] = torch.empty(T * k, dtype=torch.uint8, device=dev)
+    res["logits"] = torch.empty((T, E), dtype=torch.float32, device=dev) if logits_out else None
+    L.moe_layer_forward_w8a8(shape, opts, x, w_router, logit_bias, *wq.args(), res["out"],
+                             res["logits"], res["topk_idx"], res["topk_w"], res["counts"],
+                             res["drop_mask"], ws.buf, ws.nbytes, stream)
+    res["ws"] = ws
+    res["C"] = L.moe_capacity(shape)
+    return res

@@ -115,8 +115,9 @@ moe_status moe_align(const moe_shape* shape, const int32_t* topk_idx, int32_t* c
  *   Its scratch (per-chunk histograms, the token-block plan, an error word; about 130 KB) is
  *   a file-scope __device__ array inside libmoe.so that every device loading the library keeps
  *   until the process exits. The first call on a device looks up that array's device address
- *   (cudaGetSymbolAddress) with the device current; make that first call before any stream
- *   capture. The call itself allocates nothing: no cudaMalloc, cudaFree or allocating library
+ *   (cudaGetSymbolAddress) with the device current, and looks it up again when the device's
+ *   context has changed (after cudaDeviceReset); make the first call after any such change
+ *   before any stream capture. The call itself allocates nothing: no cudaMalloc, cudaFree or allocating library
  *   routine.
  *   Limits: T*k <= 262144 assignments and E <= 256; larger batches return MOE_ERR_UNSUPPORTED
  *   (use moe_align with a workspace). All calls share the one scratch array, which keeps the
@@ -235,6 +236,45 @@ moe_status moe_layer_forward_w8(const moe_shape* shape, const moe_layer_opts* op
                                 int32_t* counts, uint8_t* drop_mask, void* ws, size_t ws_bytes,
                                 void* stream);
 
+/* ---- FP8 weights and activations (W8A8).
+ *
+ * [P5] section "4.3 MOE量化方案矩阵": W8A8 with FP8, and offline weight repacking. The reading
+ * taken: the weights as in W8A16 (e4m3, one float32 scale per output channel), repacked with the
+ * reduction dimension contiguous; the activations entering each expert GEMM quantised per row to
+ * e4m3 with the same rule (one float32 scale per token row of x and per slot row of the SwiGLU
+ * intermediate h, which is rounded to bf16 first). Both GEMMs then run as e4m3 x e4m3 products on
+ * the tensor cores, and the fp32 accumulator is multiplied by the channel scale and the row scale:
+ *   y[s,m] = s_act[s] * s_w[e][m] * sum_k decode(q_act[s][k]) * decode(q_w[e][m][k]).
+ * Halves the expert-weight bytes the layer streams and the activation bytes the GEMMs read. */
+
+/* Repacks bf16 weights w [E][K][M] (K the reduction dimension; K, M multiples of 64) into K-major
+ * e4m3 codes [E][M][K] (uint8, 16-byte aligned) and per-channel scales [E][M] (float32), with the
+ * rule of moe_quantize_weights_fp8 (the same codes, transposed). */
+moe_status moe_pack_weights_w8a8(const void* w, int64_t E, int64_t K, int64_t M, uint8_t* codes,
+                                 float* scale, void* stream);
+
+/* Per-row e4m3 quantisation of bf16 rows a [N][K] (K a multiple of 8): scale[n] = max_k
+ * |a[n][k]| / 448 (1 for an all-zero row, float32 division), codes[n][k] = e4m3(a[n][k] /
+ * scale[n]) (float32 division, nearest-even, saturating). codes [N][K] uint8, scale [N] float32. */
+moe_status moe_quantize_rows_fp8(const void* a, int64_t N, int64_t K, uint8_t* codes,
+                                 float* scale, void* stream);
+
+/* moe_grouped_ffn / moe_layer_forward_ex with W8A8 expert GEMMs (bf16 shapes only): qk_gate, qk_up
+ * [E][I][H] and s_gate, s_up [E][I]; qk_down [E][H][I] and s_down [E][H] (moe_pack_weights_w8a8
+ * of w_gate, w_up [E][H][I] and w_down [E][I][H]). y_slots and out stay bf16. */
+moe_status moe_grouped_ffn_w8a8(const moe_shape* shape, const void* x, const int32_t* sorted_ids,
+                                const int32_t* offsets, const uint8_t* qk_gate,
+                                const uint8_t* qk_up, const uint8_t* qk_down, const float* s_gate,
+                                const float* s_up, const float* s_down, void* y_slots, void* ws,
+                                size_t ws_bytes, void* stream);
+moe_status moe_layer_forward_w8a8(const moe_shape* shape, const moe_layer_opts* opts,
+                                  const void* x, const void* w_router, const float* logit_bias,
+                                  const uint8_t* qk_gate, const uint8_t* qk_up,
+                                  const uint8_t* qk_down, const float* s_gate, const float* s_up,
+                                  const float* s_down, void* out, float* logits_out,
+                                  int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                  uint8_t* drop_mask, void* ws, size_t ws_bytes, void* stream);
+
 /* Expert parallelism over R ranks, [P4] section "Token 分发的通信瓶颈" (rows go to the devices
  * that own their experts and the outputs come back) with the capacity of section
  * "昇腾NPU的通信计算重叠". Rank r holds its own T tokens (shape->T) and the experts
@@ -243,8 +283,11 @@ moe_status moe_layer_forward_w8(const moe_shape* shape, const moe_layer_opts* op
  * drops by the global token order, each expert's rows expert-major in that order at its owner.
  * Steps on rank r: moe_route; moe_align with capacity_factor <= 0 (the local grouping);
  * gather every rank's `counts` into counts_all [R,E] (a collective between devices);
- * moe_ep_plan; moe_ep_dispatch on every rank; moe_grouped_ffn on the owner's rows (E/R
- * experts, k = 1, identity sorted_ids, own_offsets); moe_ep_combine on every rank.
+ * moe_ep_plan; moe_ep_dispatch; moe_ep_signal (rows sent) and moe_ep_wait (every rank's rows
+ * arrived); moe_grouped_ffn on the owner's rows (E/R experts, k = 1, identity sorted_ids,
+ * own_offsets); moe_ep_signal (outputs ready) and moe_ep_wait; moe_ep_combine. Before a buffer
+ * is reused by the next step, a third signal/wait pair (or a host barrier) orders the reuse
+ * after the last remote read. Rows move only by plain loads and stores through peer pointers.
  *
  * moe_ep_plan: owner [T*k] (rank owning the expert, -1 if dropped) and slot [T*k] (row in the
  * owner's slot-major buffer, -1 if dropped) of this rank's assignments, and own_offsets
@@ -263,10 +306,30 @@ moe_status moe_ep_plan(const moe_shape* shape, int32_t R, int32_t rank, int64_t 
  * slot[a]. peer_xs is a device array of R device pointers to the ranks' slot-major row buffers
  * ([rows, H] dtype, 16-byte aligned; the other ranks' buffers mapped into this device's address
  * space, or other buffers of the same device when ranks are emulated on one device). The
- * stores are plain global stores; the caller orders them before the owners read. */
+ * stores are plain global stores, fenced at system scope by each block before it exits; the
+ * owners read them after moe_ep_signal / moe_ep_wait. */
 moe_status moe_ep_dispatch(const moe_shape* shape, int32_t R, const void* x,
                            const int32_t* owner, const int32_t* slot, void* const* peer_xs,
                            void* stream);
+
+/* Step signal between ranks (the ordering of [P4] section "昇腾NPU的通信计算重叠", where compute
+ * on arrived rows overlaps the transfer of the rest): after all earlier work on `stream`, stores
+ * `epoch` into word `rank` of every rank's flag array, with a system-scope fence before it and
+ * release semantics. peer_flags is a device array of R device pointers; peer_flags[q] points to
+ * rank q's flag array of R uint32 words (mapped into this device's address space). Use a new
+ * epoch per step and per kind of signal (flag arrays start at 0; epochs compare modulo 2^32). */
+moe_status moe_ep_signal(int32_t R, int32_t rank, uint32_t epoch, uint32_t* const* peer_flags,
+                         void* stream);
+
+/* Waits on `stream` until every one of the R words of this rank's flag array `flags` (device
+ * memory, 4-byte aligned; the flag arrays are exempt from the 16-byte rule) holds at least
+ * `epoch` (system-scope acquire loads). The wait is bounded: if a rank
+ * has not signalled within 2 s, the kernel records device error 2 in the error word at the start
+ * of `ws` (ws_bytes >= 256) and returns; moe_check_error then reports MOE_ERR_DEVICE. Launch it
+ * only after every signal it waits for has been launched, on this device or another: kernels
+ * that wait on one another are never run as separate launches that must overlap on one GPU. */
+moe_status moe_ep_wait(int32_t R, uint32_t epoch, const uint32_t* flags, void* ws,
+                       size_t ws_bytes, void* stream);
 
 /* out[t,:] = sum over kept j, ascending, of topk_w[t,j] * peer_y[owner][slot,:], accumulated in
  * float32 and rounded once (a fully dropped token gives a zero row): moe_combine with each

@@ -59,6 +59,23 @@ class DequantExpertWeights:
         return self.w.shape[0]
 
 
+class W8A8ExpertWeights:
+    """Expert e's weights as the oracle's (codes, scale) pair of the FP8 quantisation, computed
+    on demand from the seeded bf16 weights of a (device) [E, K, M] tensor; the argument form that
+    orc.swiglu_expert_w8a8 takes."""
+
+    def __init__(self, w):
+        self.w = w
+
+    def __getitem__(self, e):
+        w = self.w[int(e)].detach().float().cpu().numpy()[None]
+        q, sc = orc.quantize_weights_fp8(w)
+        return q[0], sc[0]
+
+    def __len__(self):
+        return self.w.shape[0]
+
+
 def rel_err(got, ref):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)

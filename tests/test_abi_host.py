@@ -177,3 +177,17 @@ def test_stalled_wait_probe_refuses_a_missing_or_small_workspace(lib):
     buf = ctypes.create_string_buffer(512)
     addr = (ctypes.addressof(buf) + 15) & ~15
     assert L.moe_probe_stalled_wait(addr, 128, check=False) == L.MOE_ERR_WORKSPACE
+
+
+def test_expert_parallel_calls_reject_bad_arguments_before_any_launch(lib):
+    shape = L.make_shape(64, 128, 8, 2, 128, 1.25, "bf16")
+    bogus = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    # R must divide E
+    assert lib.moe_ep_dispatch(ctypes.byref(shape), 3, bogus, bogus, bogus, bogus, None) == \
+        L.MOE_ERR_INVALID_ARG
+    # rank outside [0, R)
+    assert lib.moe_ep_signal(2, 2, 1, bogus, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_signal(2, 0, 1, None, None) == L.MOE_ERR_INVALID_ARG
+    # the wait needs a workspace for its error word
+    assert lib.moe_ep_wait(2, 1, bogus, None, 0, None) == L.MOE_ERR_WORKSPACE
+    assert lib.moe_ep_wait(0, 1, bogus, bogus, 256, None) == L.MOE_ERR_INVALID_ARG

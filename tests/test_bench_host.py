@@ -48,12 +48,15 @@ def test_stage_costs_fp8_weights_are_one_byte_plus_channel_scales():
 
 
 def test_launches_per_step():
-    # router GEMM + top-k, one grouping launch, the row copy, two expert GEMMs, the combine
-    assert bench.launches_per_step(W.WORKLOADS["fine"]) == 7
+    # fused router, one grouping launch, the row copy, two expert GEMMs, the combine
+    assert bench.launches_per_step(W.WORKLOADS["fine"]) == 6
+    # decode: at most 64 tokens route through the CUDA-core GEMV + top-k
     assert bench.launches_per_step(W.WORKLOADS["decode"].with_tokens(1)) == 7
+    assert bench.launches_per_step(W.WORKLOADS["decode"].with_tokens(64)) == 7
+    assert bench.launches_per_step(W.WORKLOADS["decode"].with_tokens(256)) == 6
     # skewed: 196608 assignments take the three grouping kernels; every bf16 layer makes the
     # row copy, whatever I
-    assert bench.launches_per_step(W.WORKLOADS["skewed"]) == 2 + 3 + 1 + 2 + 1
+    assert bench.launches_per_step(W.WORKLOADS["skewed"]) == 1 + 3 + 1 + 2 + 1
     # tiny f32: one fused CUDA-core router kernel
     assert bench.launches_per_step(W.WORKLOADS["tiny"]) == 1 + 1 + 0 + 2 + 1
 
@@ -71,7 +74,7 @@ def test_reference_arm_line_matches_our_config_and_reports_its_own_wall_time():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     wl = W.WORKLOADS["tiny"]
     assert line["impl"] == "reference" and line["metric"] == bench.METRIC
-    assert line["config"] == bench.layer_config(wl, 64, 1, False)
+    assert line["config"] == bench.layer_config(wl, 64, 1)
     assert line["ms_per_step"] <= line["ms_per_step_extrapolated_to_T"] * 10
     assert line["cpu_baseline"]["value"] == line["value"] == line["e2e"]["value"]
     assert "8 sampled tokens" in line["cpu_baseline"]["sample"]

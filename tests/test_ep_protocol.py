@@ -8,6 +8,7 @@ code runs with all ranks as threads of one process and as two gloo processes; in
 collectives are the only way data moves between ranks.
 """
 import datetime
+import time
 import os
 import socket
 import threading
@@ -210,3 +211,78 @@ def test_expert_parallel_two_gloo_ranks():
     R, T_list, H, E, k, I, cf, zipf = case
     host, _ = _problem(T_list, H, E, k, I, zipf, seed=R + len(T_list) + E)
     _check_against_one_device(host, [got[0], got[1]], E, k, cf)
+
+
+def _leaving_worker(rank, world, port, store_port, case, q):
+    """Two gloo ranks run one expert-parallel step; rank 1 then leaves between steps. Rank 0
+    learns of it on the host before launching step 2."""
+    from expert_dispatch_gate_b200.ep_host import RankLost, StepHeartbeat
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=30))
+    store = dist.TCPStore("127.0.0.1", store_port, world, rank == 0,
+                          timeout=datetime.timedelta(seconds=30))
+    hb = StepHeartbeat(store, rank, world, timeout_s=10.0)
+    try:
+        R, T_list, H, E, k, I, cf, zipf = case
+        host, xs = _problem(T_list, H, E, k, I, zipf, seed=R + len(T_list) + E)
+        hb.begin_step(1)
+        res = _rank_fn(host, xs, E, k, cf)(DistComm(), rank)
+        dist.barrier()  # step 1 done on both ranks: nothing of it is in flight
+        if rank == 1:
+            hb.leave()
+            q.put((rank, "left", res))
+            # keep the store's host alive until rank 0 has seen the mark
+            return
+        t0 = time.monotonic()
+        try:
+            hb.begin_step(2)
+            q.put((rank, "step 2 started", None))
+        except RankLost as e:
+            q.put((rank, f"lost {e.rank} at step {e.step} after {time.monotonic() - t0:.2f} s",
+                   res))
+    except Exception as e:  # reported to the test instead of a silent exit
+        q.put((rank, f"error {type(e).__name__}: {e}", None))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_rank_leaving_between_steps_is_seen_on_the_host_before_the_next_step():
+    case = (2, [20, 17], 32, 8, 2, 16, 1.0, 0.0)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port, store_port = _free_port(), _free_port()
+    procs = [ctx.Process(target=_leaving_worker, args=(r, 2, port, store_port, case, q))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(2):
+        r, msg, res = q.get(timeout=180)
+        got[r] = (msg, res)
+    for p in procs:
+        p.join(60)
+    assert got[1][0] == "left", got[1][0]
+    assert got[0][0].startswith("lost 1 at step 2"), got[0][0]
+    assert float(got[0][0].split(" after ")[1].split(" s")[0]) < 5.0  # seen at once, no deadline
+    # step 1 itself was complete and correct on both ranks
+    R, T_list, H, E, k, I, cf, zipf = case
+    host, _ = _problem(T_list, H, E, k, I, zipf, seed=R + len(T_list) + E)
+    _check_against_one_device(host, [got[0][1], got[1][1]], E, k, cf)
+    assert all(p.exitcode == 0 for p in procs)
+
+
+def test_step_heartbeat_deadline_for_a_rank_that_never_arrives():
+    from expert_dispatch_gate_b200.ep_host import RankLost, StepHeartbeat
+    store = dist.HashStore()
+    hb0 = StepHeartbeat(store, 0, 3, timeout_s=0.2)
+    hb1 = StepHeartbeat(store, 1, 3, timeout_s=0.2)
+    store.set("moe_ep/rank2", "4")          # rank 2 is still at step 4
+    hb1.store.set("moe_ep/rank1", "5")      # rank 1 has published step 5
+    t0 = time.monotonic()
+    with pytest.raises(RankLost) as ei:
+        hb0.begin_step(5)
+    assert ei.value.rank == 2 and ei.value.step == 5
+    assert 0.2 <= time.monotonic() - t0 < 2.0
+    store.set("moe_ep/rank2", "5")
+    hb0.begin_step(5)                        # everyone at step 5 now

@@ -1,7 +1,9 @@
 """Expert parallelism emulated on one GPU (moe_ep_plan / moe_ep_dispatch / moe_ep_combine).
 
 R ranks' buffers live on one device and each rank's "peer" pointers point at the other ranks'
-buffers. The kernels are launched rank after rank, and no kernel waits on another. The routing is
+buffers. The kernels are launched rank after rank on one stream. Every rank's step signal
+(moe_ep_signal) is launched before any rank's wait (moe_ep_wait), so each wait finds its flags
+already set and no kernel waits on a later one. The routing is
 computed once for the concatenated batch and sliced per rank, so the emulated ranks and the
 one-device layer group exactly the same assignments. Then:
 
@@ -71,9 +73,17 @@ def test_ep_emulated_matches_one_device(R, T_list, H, E, k, I, cf, dtype, zipf):
     rows_cap = El * C
     xs = [torch.zeros((rows_cap, H), dtype=dev["x"].dtype, device="cuda") for _ in range(R)]
     peer_xs = _ptr_table(xs)
+    # one flag array of R words per rank and per kind of signal (rows sent, outputs ready)
+    flags = torch.zeros((2, R, R), dtype=torch.int32, device="cuda")
+    sent = _ptr_table([flags[0, q] for q in range(R)])
+    ready = _ptr_table([flags[1, q] for q in range(R)])
+    epoch = 7
     for r in range(R):
         L.moe_ep_dispatch(shapes[r], R, dev["x"][cuts[r]:cuts[r + 1]], plans[r][0], plans[r][1],
                           peer_xs)
+        L.moe_ep_signal(R, r, epoch, sent)
+    for r in range(R):
+        L.moe_ep_wait(R, epoch, flags[0, r], plans[r][3].buf, plans[r][3].nbytes)
     ys = []
     ident = torch.arange(rows_cap, dtype=torch.int32, device="cuda")
     for r in range(R):
@@ -81,6 +91,10 @@ def test_ep_emulated_matches_one_device(R, T_list, H, E, k, I, cf, dtype, zipf):
         ys.append(M.grouped_ffn(xs[r], ident, plans[r][2], dev["w_gate"][sl].contiguous(),
                                 dev["w_up"][sl].contiguous(), dev["w_down"][sl].contiguous(), 1,
                                 0.0))
+    for r in range(R):
+        L.moe_ep_signal(R, r, epoch, ready)
+    for r in range(R):
+        L.moe_ep_wait(R, epoch, flags[1, r], plans[r][3].buf, plans[r][3].nbytes)
     peer_y = _ptr_table(ys)
     outs = []
     for r in range(R):
@@ -91,6 +105,7 @@ def test_ep_emulated_matches_one_device(R, T_list, H, E, k, I, cf, dtype, zipf):
     torch.cuda.synchronize()
     for r in range(R):
         assert plans[r][3].check() == L.MOE_OK
+    assert torch.all(flags == epoch)
 
     # plan: the protocol oracle's owners and slots for the same routing
     idx_np = idx_all.cpu().numpy()
@@ -107,3 +122,29 @@ def test_ep_emulated_matches_one_device(R, T_list, H, E, k, I, cf, dtype, zipf):
         lo, hi = int(offsets1[r * El]), int(offsets1[(r + 1) * El])
         assert torch.equal(ys[r][:hi - lo], y1[lo:hi])
     assert torch.equal(torch.cat(outs), out1)
+
+
+def test_ep_wait_for_a_rank_that_never_signals_ends_with_a_device_error():
+    """Rank 1 of 2 never signals: rank 0's wait runs to its 2 s limit, records device error 2 and
+    returns; the next step's wait, after both ranks signal a new epoch, succeeds."""
+    import time
+    R = 2
+    shape = L.make_shape(64, 128, 8, 2, 128, 1.25, "bf16")
+    ws = M.Workspace(shape, "cuda")
+    flags = torch.zeros((R, R), dtype=torch.int32, device="cuda")
+    table = _ptr_table([flags[q] for q in range(R)])
+    L.moe_ep_signal(R, 0, 1, table)          # rank 0 announces epoch 1; rank 1 does not
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    L.moe_ep_wait(R, 1, flags[0], ws.buf, ws.nbytes)
+    with pytest.raises(L.MoeError) as ei:
+        ws.check()
+    elapsed = time.perf_counter() - t0
+    assert ei.value.status == L.MOE_ERR_DEVICE and "device error 2" in str(ei.value)
+    assert 1.5 < elapsed < 60
+    assert flags[0].tolist() == [1, 0] and flags[1].tolist() == [1, 0]
+    for r in range(R):
+        L.moe_ep_signal(R, r, 2, table)
+    L.moe_ep_wait(R, 2, flags[0], ws.buf, ws.nbytes)
+    assert ws.check() == L.MOE_OK
+    assert torch.all(flags == 2)

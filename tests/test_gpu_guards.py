@@ -1,13 +1,17 @@
 """Out-of-bounds writes. Every output of the layer and of the grouping, and the workspace, sits
 inside a byte buffer with 256-byte guard regions on both sides filled with 0xA5. After the call
-the guards must be intact, and the results must equal those of an ordinary call."""
+the guards must be intact, the results must equal those of an ordinary call, and they must match
+the oracle (grouping bit for bit; the layer by the parity rules of the layer tests), so that a
+write that lands inside the outputs but in the wrong place fails too."""
+import numpy as np
 import pytest
 import torch
 
 from expert_dispatch_gate_b200 import _lib as L
 from expert_dispatch_gate_b200 import layer as M
 from expert_dispatch_gate_b200 import workloads as W
-from tests.test_gpu_parity import small_inputs
+from oracle import moe_oracle as orc
+from tests.test_gpu_parity import compare_layer, small_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -64,6 +68,9 @@ def test_layer_writes_stay_inside_their_buffers(name):
     torch.cuda.synchronize()
     for key in b:
         assert torch.equal(b[key][1], ref[key]), key
+    got = {key: view for key, (_, view) in b.items()}
+    got["C"] = L.moe_capacity(shape)
+    compare_layer(wl, cpu, dev, got)
 
 
 # one 256-thread block (2048 assignments), the 8-CTA cluster (32768), chunked kernels (65544)
@@ -91,3 +98,6 @@ def test_grouping_writes_stay_inside_their_buffers(T, E, k):
     torch.cuda.synchronize()
     for key in b:
         assert torch.equal(b[key][1], ref[key]), key
+    al = orc.align(idx.cpu().numpy(), E, orc.capacity(T, k, E, 1.25))
+    for key in b:
+        assert np.array_equal(b[key][1].cpu().numpy(), al[key]), key

@@ -32,8 +32,10 @@ SMALL = {
     # accumulators); I = 640 leaves the last GEMM1 pair tile half outside the weight; H = 384
     # runs GEMM2 with one feature block per tile
     "e96_partial_tiles": W.Workload("e96", 19, 333, 384, 96, 4, 640, "bf16", 1.25),
-    # T = 50, H = 1024: one token tile, the router's K split into 4 ranges
-    "e128_router_ksplit": W.Workload("e128", 20, 50, 1024, 128, 6, 256, "bf16", 1.25),
+    # T = 50, H = 1024: few tokens, the router's split-K CUDA-core GEMV
+    "e128_router_gemv": W.Workload("e128", 20, 50, 1024, 128, 6, 256, "bf16", 1.25),
+    # T = 90: one token tile of the tensor-core router, its K split into 4 ranges
+    "e128_router_ksplit": W.Workload("e128k", 21, 90, 1024, 128, 6, 256, "bf16", 1.25),
 }
 
 
@@ -95,6 +97,14 @@ ROUTER = {
     "pairs_short_peer": W.Workload("r3", 23, 129, 256, 256, 8, 128, "bf16", 1.25),
     "pairs_t2_ksplit16": W.Workload("r4", 24, 2, 4096, 256, 8, 128, "bf16", 1.25),
     "single_e192": W.Workload("r5", 25, 513, 4096, 192, 8, 128, "bf16", 1.25),
+    # just above the CUDA-core GEMV's token limit (64): tensor cores with the K split in 4 / 16
+    "tc_t100_ksplit4": W.Workload("r6", 26, 100, 1024, 128, 6, 128, "bf16", 1.25),
+    "tc_t65_ksplit16": W.Workload("r7", 27, 65, 4096, 256, 8, 128, "bf16", 1.25),
+    # a few tokens: the split-K CUDA-core GEMV, each of its token-count tiers (4, 16, 64)
+    "gemv_t1": W.Workload("r8", 28, 1, 4096, 256, 8, 128, "bf16", 0.0),
+    "gemv_t3_e128": W.Workload("r9", 29, 3, 2048, 128, 4, 128, "bf16", 0.0),
+    "gemv_t16_e96": W.Workload("r10", 30, 16, 1024, 96, 6, 128, "bf16", 1.25),
+    "gemv_t64_e64_zipf": W.Workload("r11", 31, 64, 2048, 64, 6, 128, "bf16", 1.25, zipf_s=1.2),
 }
 
 
@@ -227,7 +237,7 @@ def test_combine(name):
 # ----------------------------------------------------------------- whole layer
 
 def compare_layer(wl, cpu_or_dev, dev, res, sample=None, seed=0, n_group=1, topk_group=1,
-                  shared=None, shared_factor=0.0, out_bias=None, weights=None):
+                  shared=None, shared_factor=0.0, out_bias=None, weights=None, expert_fn=None):
     """Compare moe_layer_forward's outputs with the oracle (see module docstring of parity).
     With n_group > 1 the routing is group-limited; shared / out_bias (host numpy) add the
     combine's shared-expert and bias terms."""
@@ -290,7 +300,7 @@ def compare_layer(wl, cpu_or_dev, dev, res, sample=None, seed=0, n_group=1, topk
     ref = orc.layer_forward(host["x"], host["w_router"], weights[0], weights[1], weights[2], k,
                             wl.capacity_factor, logit_bias=host["logit_bias"], tokens=comparable,
                             n_group=n_group, topk_group=topk_group, shared=shared,
-                            shared_factor=shared_factor, out_bias=out_bias)
+                            shared_factor=shared_factor, out_bias=out_bias, expert_fn=expert_fn)
     got = np32(res["out"])[comparable]
     r = assert_close_rel(got, ref["out"], TOL_OUT[wl.dtype], "layer output")
     return {"delta_logits": delta, "fragile": int((~dec).sum()), "compared": len(comparable),
@@ -359,7 +369,7 @@ def test_layer_workload_sizes(name, T):
                           wl.k, wl.capacity_factor, logit_bias=dev["logit_bias"])
     torch.cuda.synchronize()
     assert res["ws"].check() == L.MOE_OK
-    info = compare_layer(wl, dev, dev, res, sample=12 if wl.E > 8 else 24)
+    info = compare_layer(wl, dev, dev, res, sample=64)
     print(name, T, info)
     # per-stage checks on oracle-made inputs at this size
     host = inputs_np(dev)
@@ -380,3 +390,53 @@ def test_layer_workload_sizes(name, T):
     slots = [s for e in pick for s in range(al_o["offsets"][e], al_o["offsets"][e + 1])]
     _ffn_check(wl, dev["x"], (dev["w_gate"], dev["w_up"], dev["w_down"]), al_o, slots,
                x_host=host["x"])
+
+
+# ----------------------------------------------------------------- the bench's schedule, in full
+
+def test_layer_fine_e32_every_token_and_slot():
+    """The fine-grained layer's per-expert shapes and load (H = 4096, I = 2048, k = 8, C = 160,
+    about 128 tokens per expert) with 32 experts: the expert GEMMs run the same persistent CTA-pair
+    schedule over all SMs as the bench (several tiles per CTA pair), and every token's output and
+    every kept slot's expert output is compared with the oracle."""
+    wl = W.PROFILE_WORKLOADS["fine_e32"]
+    dev = W.make_inputs(wl, "cuda")
+    res = M.layer_forward(dev["x"], dev["w_router"], dev["w_gate"], dev["w_up"], dev["w_down"],
+                          wl.k, wl.capacity_factor, logit_bias=dev["logit_bias"])
+    torch.cuda.synchronize()
+    assert res["ws"].check() == L.MOE_OK
+    info = compare_layer(wl, dev, dev, res)
+    print("fine_e32 layer", info)
+    assert info["compared"] >= wl.T // 2
+    host = inputs_np(dev)
+    L_o = orc.router_logits(host["x"], host["w_router"], host["logit_bias"])
+    idx_o = orc.select_topk(L_o, wl.k)
+    C = orc.capacity(wl.T, wl.k, wl.E, wl.capacity_factor)
+    al_o = orc.align(idx_o, wl.E, C)
+    kept = int(al_o["offsets"][-1])
+    r = _ffn_check(wl, dev["x"], (dev["w_gate"], dev["w_up"], dev["w_down"]), al_o,
+                   list(range(kept)), x_host=host["x"])
+    print("fine_e32 expert outputs: %d slots, max rel err %.3e" % (kept, r))
+
+
+def test_combine_fine_every_token():
+    """moe_combine at the fine-grained size (T = 4096, k = 8, H = 4096, C = 160) over every token,
+    on the oracle's grouping of seeded logits and seeded expert outputs."""
+    wl = W.WORKLOADS["fine"]
+    logits = W.random_logits(wl.T, wl.E, seed=99)
+    l32 = logits.numpy()
+    idx_o = orc.select_topk(l32, wl.k)
+    w32 = orc.route_weights(l32, idx_o).astype(np.float32)
+    C = orc.capacity(wl.T, wl.k, wl.E, wl.capacity_factor)
+    al = orc.align(idx_o, wl.E, C)
+    y = W.make_y_slots(wl, "cpu")
+    out = M.combine(y.cuda(), to_dev(al["slot_of"]), to_dev(w32, torch.float32), wl.E)
+    torch.cuda.synchronize()
+    ref = orc.combine(np32(y), al["slot_of"], w32)
+    got = np32(out)
+    r = assert_close_rel(got, ref, TOL_OUT[wl.dtype], "combine")
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6 * np.abs(ref).max())
+    dropped_all = np.all(al["slot_of"].reshape(wl.T, wl.k) < 0, axis=1)
+    assert np.all(got[dropped_all] == 0.0)
+    print("combine fine: %d tokens, %d dropped assignments, max rel err %.3e"
+          % (wl.T, int(al["drop_mask"].sum()), r))

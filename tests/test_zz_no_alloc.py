@@ -38,8 +38,10 @@ def _noalloc(idx, E, cf, H=4096, I=2048):
 
 
 @pytest.mark.parametrize("T,E,k,cf,mode", [
+    (256, 16, 8, 1.25, "zipf"),        # 2048 assignments: the one-block form
     (4096, 256, 8, 1.25, "uniform"),   # the fine-grained layer's routing size
     (32768, 64, 6, 1.25, "zipf"),      # 196608 assignments, heavy drops
+    (32768, 256, 8, 1.25, "zipf"),     # 262144: the limit, every chunk histogram in use
 ])
 def test_noalloc_matches_workspace_align_twice(T, E, k, cf, mode):
     assert torch.cuda.is_available()
@@ -60,3 +62,43 @@ def test_noalloc_rejects_batches_beyond_its_scratch():
     st = L.moe_align_noalloc(shape, buf, buf, buf, buf, buf, buf, check=False)
     assert st == L.MOE_ERR_UNSUPPORTED
     assert "262144" in L.last_error_detail()
+
+
+def test_noalloc_empty_batch_gives_zero_counts_and_offsets():
+    E = 64
+    shape = L.make_shape(0, 4096, E, 6, 2048, 1.25, "bf16")
+    counts = torch.full((E,), -7, dtype=torch.int32, device="cuda")
+    offsets = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
+    other = torch.full((16,), -7, dtype=torch.int32, device="cuda")
+    assert L.moe_align_noalloc(shape, other, counts, offsets, other, other, other,
+                               check=False) == L.MOE_OK
+    torch.cuda.synchronize()
+    assert torch.all(counts == 0) and torch.all(offsets == 0)
+    assert torch.all(other == -7)  # no assignment: nothing else is written
+
+
+G = 256  # guard bytes on each side of every output (keeps 16-byte alignment)
+
+
+def _guarded(n, dtype):
+    es = torch.empty((), dtype=dtype).element_size()
+    buf = torch.full((G + n * es + G,), 0xA5, dtype=torch.uint8, device="cuda")
+    return buf, buf[G:G + n * es].view(dtype)
+
+
+@pytest.mark.parametrize("T,E,k", [(256, 16, 8), (4096, 256, 8), (8193, 256, 8)])
+def test_noalloc_writes_stay_inside_their_buffers(T, E, k):
+    """Each output between 0xA5 guard regions, at each launch form of the grouping; the guards
+    stay intact and the results equal the workspace call's."""
+    idx = W.random_topk_idx(T, E, k, seed=T + 3 * E, mode="zipf").cuda()
+    shape = L.make_shape(T, 4096, E, k, 2048, 1.25, "bf16")
+    A = T * k
+    b = {"counts": _guarded(E, torch.int32), "offsets": _guarded(E + 1, torch.int32),
+         "sorted_ids": _guarded(A, torch.int32), "slot_of": _guarded(A, torch.int32),
+         "drop_mask": _guarded(A, torch.uint8)}
+    L.moe_align_noalloc(shape, idx, *(b[key][1] for key in KEYS))
+    ref = M.align(idx, E, 1.25, H=4096, I=2048)
+    torch.cuda.synchronize()
+    for key, (buf, view) in b.items():
+        assert bool((buf[:G] == 0xA5).all()) and bool((buf[-G:] == 0xA5).all()), key
+        assert torch.equal(view, ref[key]), key
