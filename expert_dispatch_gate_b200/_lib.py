@@ -11,7 +11,9 @@ import os
 import re
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libmoe.so")
+# MOE_DEBUG_LIB=1 selects the debug build (device-side bounds checks, see moe_debug_checks).
+LIB_PATH = os.path.join(HERE, "libmoe_debug.so" if os.environ.get("MOE_DEBUG_LIB") == "1"
+                        else "libmoe.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "moe.h")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE = range(6)
@@ -83,6 +85,7 @@ def _signatures(lib):
         "moe_layer_forward_w8": (st, [S, O] + [_P] * 16 + [sz, _P]),
         "moe_probe_stalled_wait": (st, [_P, sz, _P]),
         "moe_pack_weights_w8a8": (st, [_P, i64, i64, i64, _P, _P, _P]),
+        "moe_debug_checks": (ctypes.c_int32, []),
         "moe_quantize_rows_fp8": (st, [_P, i64, i64, _P, _P, _P]),
         "moe_grouped_ffn_w8a8": (st, [S] + [_P] * 11 + [sz, _P]),
         "moe_layer_forward_w8a8": (st, [S, O] + [_P] * 16 + [sz, _P]),

@@ -19,6 +19,10 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmoe.so")
+# Debug variant (-DMOE_DEBUG): every slot, token-row and group-table index a kernel reads from
+# device data is checked before use; a failure is recorded in the workspace error word.
+BUILD_DEBUG = os.path.join(HERE, "_build_debug")
+LIB_DEBUG = os.path.join(HERE, "libmoe_debug.so")
 SOURCES = ["moe_api.cu", "route.cu", "route_tc.cu", "align.cu", "combine.cu", "ffn_simt.cu",
            "ffn_tc.cu", "quant.cu", "probe.cu", "ep.cu"]
 # every header under csrc/: a change to any of them rebuilds every object
@@ -41,43 +45,46 @@ def _deps_mtime():
     return max(os.path.getmtime(p) for p in paths)
 
 
-def _compile(src, force):
-    obj = os.path.join(BUILD, src.replace(".cu", ".o"))
+def _compile(src, force, debug=False):
+    obj = os.path.join(BUILD_DEBUG if debug else BUILD, src.replace(".cu", ".o"))
     srcp = os.path.join(CSRC, src)
     if (not force and os.path.exists(obj)
             and os.path.getmtime(obj) >= max(os.path.getmtime(srcp), _deps_mtime())):
         return obj, ""
-    cmd = [nvcc()] + FLAGS + ["-c", srcp, "-o", obj]
+    cmd = [nvcc()] + FLAGS + (["-DMOE_DEBUG"] if debug else []) + ["-c", srcp, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
     return obj, r.stderr
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    bdir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD, LIB)
+    os.makedirs(bdir, exist_ok=True)
     with cf.ThreadPoolExecutor(max_workers=min(8, len(SOURCES))) as ex:
-        results = list(ex.map(lambda s: _compile(s, force), SOURCES))
+        results = list(ex.map(lambda s: _compile(s, force, debug), SOURCES))
     objs = [o for o, _ in results]
     logs = "".join(l for _, l in results)
     if logs:
-        with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
+        with open(os.path.join(bdir, "ptxas.log"), "w") as f:
             f.write(logs)
-    if (force or not os.path.exists(LIB)
-            or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs)):
-        cmd = [nvcc()] + ARCH + ["-shared", "-o", LIB] + objs
+    if (force or not os.path.exists(lib)
+            or os.path.getmtime(lib) < max(os.path.getmtime(o) for o in objs)):
+        cmd = [nvcc()] + ARCH + ["-shared", "-o", lib] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
     if verbose:
         print(logs)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
+    ap.add_argument("--debug", action="store_true",
+                    help="build libmoe_debug.so with the device-side bounds checks")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, debug=a.debug))
     sys.exit(0)

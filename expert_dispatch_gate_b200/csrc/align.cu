@@ -73,8 +73,19 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
   const int64_t base = static_cast<int64_t>(blockIdx.x) * chunk;
   const int64_t end = min(A, base + chunk);
-  for (int64_t a = base + threadIdx.x; a < end; a += kThreads) {
-    const int e = idx[a];
+  // a thread's ids of the chunk (at most kAlignChunkMax / kThreads = 8) are loaded together
+  constexpr int kPer = kAlignChunkMax / kThreads;
+  int ids[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int64_t a = base + threadIdx.x + static_cast<int64_t>(i) * kThreads;
+    ids[i] = (a < end) ? __ldg(idx + a) : -1;
+  }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int64_t a = base + threadIdx.x + static_cast<int64_t>(i) * kThreads;
+    if (a >= end) continue;
+    const int e = ids[i];
     if (e >= 0 && e < E) atomicAdd(&h[e], 1);
     else flag_error(err, kDevBadExpert);
   }
@@ -195,19 +206,38 @@ __global__ void __launch_bounds__(kThreads)
   pdl_enter<false>();
   __shared__ int wrun[kWarps][kMaxE];
   __shared__ int s_off[kMaxE];
+  __shared__ uint16_t code[kAlignChunkMax];  // the chunk's ids (0xFFFF: none or invalid)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kWarps * kMaxE; i += kThreads) (&wrun[0][0])[i] = 0;
   for (int e = threadIdx.x; e < E; e += kThreads) s_off[e] = offsets[e];
-  __syncthreads();
   const int per_warp = chunk / kWarps;  // a multiple of 32
-  const int64_t wbase = static_cast<int64_t>(blockIdx.x) * chunk + warp * per_warp;
+  const int64_t cbase = static_cast<int64_t>(blockIdx.x) * chunk;
+  const int64_t wbase = cbase + warp * per_warp;
+  {
+    // the chunk's ids, read once (a thread's loads in flight together)
+    constexpr int kPer = kAlignChunkMax / kThreads;
+    int ids[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int o = threadIdx.x + i * kThreads;
+      const int64_t a = cbase + o;
+      ids[i] = (o < chunk && a < A) ? __ldg(idx + a) : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int o = threadIdx.x + i * kThreads;
+      if (o < chunk)
+        code[o] = (ids[i] >= 0 && ids[i] < E) ? static_cast<uint16_t>(ids[i]) : uint16_t{0xFFFF};
+    }
+  }
+  __syncthreads();
 
   const int nbits = (E > 1) ? 32 - __clz(E - 1) : 0;
+  const int wofs = warp * per_warp;  // this warp's first id in `code`
   // pass 1: per-warp per-expert counts of this warp's assignments
   for (int step = 0; step < per_warp / 32; ++step) {
-    const int64_t a = wbase + step * 32 + lane;
-    const int e = (a < A) ? idx[a] : -1;
-    if (e >= 0 && e < E) atomicAdd(&wrun[warp][e], 1);
+    const uint32_t c = code[wofs + step * 32 + lane];
+    if (c != 0xFFFFu) atomicAdd(&wrun[warp][c], 1);
   }
   __syncthreads();
   // per expert: exclusive prefix across the warps, seeded with this chunk's base
@@ -225,8 +255,9 @@ __global__ void __launch_bounds__(kThreads)
   for (int step = 0; step < per_warp / 32; ++step) {
     const int64_t a = wbase + step * 32 + lane;
     const bool in = a < A;
-    const int e = in ? idx[a] : -1;
-    const bool ok = (e >= 0 && e < E);
+    const uint32_t c = code[wofs + step * 32 + lane];
+    const bool ok = in && c != 0xFFFFu;
+    const int e = ok ? static_cast<int>(c) : -1;
     const uint32_t peers = warp_peers(static_cast<uint32_t>(e), ok, nbits);
     int rank = 0;
     if (ok) rank = wrun[warp][e] + __popc(peers & lanemask_lt());

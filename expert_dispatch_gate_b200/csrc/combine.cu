@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     combine_kernel(const T* __restrict__ y, const int32_t* __restrict__ slot_of,
                    const float* __restrict__ topk_w, const T* __restrict__ shared,
                    float shared_factor, const float* __restrict__ out_bias, T* __restrict__ out,
-                   int64_t Ttok, int H, int k, int segs) {
+                   int64_t Ttok, int H, int k, int segs, int* err) {
   pdl_enter<false>();
   constexpr int N = Vec<T>::N;
   const int lane = threadIdx.x & 31;
@@ -71,7 +71,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int64_t t = wid / segs;
   if (t >= Ttok) return;
   const int seg = static_cast<int>(wid - t * segs);
-  const int my_slot = (lane < k) ? slot_of[t * k + lane] : -1;
+  int my_slot = (lane < k) ? slot_of[t * k + lane] : -1;
+  if (kDebugChecks && my_slot >= Ttok * k) {  // y_slots holds T*k rows
+    if (seg == 0) flag_error(err, kDevDebugBounds);
+    my_slot = -1;
+  }
   const float my_w = (lane < k) ? topk_w[t * k + lane] : 0.f;
   const int nchunk = H / N;
   T* orow = out + static_cast<size_t>(t) * H;
@@ -147,12 +151,16 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
     dispatch_rows_kernel(const T* __restrict__ x, const int32_t* __restrict__ sorted_ids,
                          const int32_t* __restrict__ offsets, int E, int k, int H, int64_t rows,
-                         T* __restrict__ xs) {
+                         int64_t Ttok, T* __restrict__ xs, int* err) {
   pdl_enter<false>();
   const int lane = threadIdx.x & 31;
   const int64_t s = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   if (s >= rows || s >= offsets[E]) return;
   const int64_t t = sorted_ids[s] / k;
+  if (kDebugChecks && (sorted_ids[s] < 0 || t >= Ttok)) {
+    if (lane == 0) flag_error(err, kDevDebugBounds);
+    return;
+  }
   const uint4* src = reinterpret_cast<const uint4*>(x + t * H);
   uint4* dst = reinterpret_cast<uint4*>(xs + s * H);
   const int n = H * static_cast<int>(sizeof(T)) / 16;
@@ -163,22 +171,22 @@ __global__ void __launch_bounds__(kThreads)
 
 cudaError_t launch_dispatch_rows(int dtype, const void* x, const int32_t* sorted_ids,
                                  const int32_t* offsets, int E, int k, int H, int64_t rows,
-                                 void* xs, cudaStream_t stream) {
+                                 int64_t T, void* xs, int* err, cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((rows + kWarps - 1) / kWarps);
   if (dtype == 0)
     return launch_kernel(dispatch_rows_kernel<float>, dim3(grid), dim3(kThreads), 0, stream, 1,
-                         static_cast<const float*>(x), sorted_ids, offsets, E, k, H, rows,
-                         static_cast<float*>(xs));
+                         static_cast<const float*>(x), sorted_ids, offsets, E, k, H, rows, T,
+                         static_cast<float*>(xs), err);
   return launch_kernel(dispatch_rows_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), 0, stream,
                        1, static_cast<const __nv_bfloat16*>(x), sorted_ids, offsets, E, k, H, rows,
-                       static_cast<__nv_bfloat16*>(xs));
+                       T, static_cast<__nv_bfloat16*>(xs), err);
 }
 
 cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_of,
                            const float* topk_w, const void* shared, float shared_factor,
                            const float* out_bias, void* out, int64_t T, int H, int k,
-                           cudaStream_t stream) {
+                           int* err, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const int n = (dtype == 0) ? 4 : 8;  // elements per 16-byte chunk
   const int segs = static_cast<int>((H / n + 32 * kG - 1) / (32 * kG));
@@ -188,11 +196,11 @@ cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_o
     return launch_kernel(combine_kernel<float>, grid, dim3(kThreads), 0, stream, 1,
                          static_cast<const float*>(y_slots), slot_of, topk_w,
                          static_cast<const float*>(shared), shared_factor, out_bias,
-                         static_cast<float*>(out), T, H, k, segs);
+                         static_cast<float*>(out), T, H, k, segs, err);
   return launch_kernel(combine_kernel<__nv_bfloat16>, grid, dim3(kThreads), 0, stream, 1,
                        static_cast<const __nv_bfloat16*>(y_slots), slot_of, topk_w,
                        static_cast<const __nv_bfloat16*>(shared), shared_factor, out_bias,
-                       static_cast<__nv_bfloat16*>(out), T, H, k, segs);
+                       static_cast<__nv_bfloat16*>(out), T, H, k, segs, err);
 }
 
 }  // namespace moe

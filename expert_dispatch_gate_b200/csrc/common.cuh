@@ -21,7 +21,17 @@ enum DeviceError : int {
   kDevOk = 0,
   kDevBadExpert = 1,   // topk_idx held an expert id outside [0, E)
   kDevWaitTimeout = 2, // a bounded mbarrier wait ran out (pipeline stalled)
+  kDevDebugBounds = 3, // debug builds: an index read from device data was out of range
 };
+
+// Debug builds (-DMOE_DEBUG, libmoe_debug.so) check every slot, token-row and group-table index a
+// kernel reads from device data before using it: a failed check records kDevDebugBounds in the
+// error word and the access is skipped, never trapped. Release builds compile the checks away.
+#ifdef MOE_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
 
 // A wait that has not completed after this many nanoseconds is abandoned: the kernel records
 // kDevWaitTimeout and winds down instead of spinning forever.
@@ -133,6 +143,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
       : "memory");
+}
+
+// Prefetch of one 2-D tensor-map box into L2 (no shared-memory destination, no completion).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
 }
 
 // 16-byte global -> shared copy through L2 only (cp.async.cg).
@@ -274,28 +292,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
-// 16-byte load from a CTA's shared memory given by its shared::cluster address (mapa_shared).
-__device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t cluster_addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(cluster_addr)
-               : "memory");
-  return v;
-}
-__device__ __forceinline__ float2 ld_shared_cluster_f32x2(uint32_t cluster_addr) {
-  float2 v;
-  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];"
-               : "=f"(v.x), "=f"(v.y)
-               : "r"(cluster_addr)
-               : "memory");
-  return v;
-}
-__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
-  return v;
-}
 // Arrive (release, cluster scope) on an mbarrier given by its shared::cluster address.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
@@ -420,36 +416,7 @@ constexpr bool kUsePdl = true;  // programmatic dependent launch between the lib
 #endif
 
 // cudaLaunchKernelEx with programmatic stream serialization (unless built with MOE_NO_PDL) and,
-// when the cluster has more than one CTA, clusters of cluster.x * cluster.y CTAs.
-template <typename... KArgs, typename... Args>
-inline cudaError_t launch_kernel_clusters(void (*kernel)(KArgs...), dim3 grid, dim3 block,
-                                          size_t smem, cudaStream_t stream, dim3 cluster,
-                                          Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  unsigned n = 0;
-  if (kUsePdl) {
-    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[n].val.programmaticStreamSerializationAllowed = 1;
-    ++n;
-  }
-  if (cluster.x * cluster.y * cluster.z > 1) {
-    attr[n].id = cudaLaunchAttributeClusterDimension;
-    attr[n].val.clusterDim.x = cluster.x;
-    attr[n].val.clusterDim.y = cluster.y;
-    attr[n].val.clusterDim.z = cluster.z;
-    ++n;
-  }
-  cfg.attrs = attr;
-  cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
-}
-
-// The same with clusters of cluster_x CTAs along x.
+// when cluster_x > 1, clusters of cluster_x CTAs along x.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                                  cudaStream_t stream, int cluster_x, Args&&... args) {

@@ -252,13 +252,29 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
     s_off[i] = p.offsets[i];
     s_blk[i] = p.blk_prefix[i];
   }
+  if constexpr (kDebugChecks) {
+    // the group tables must describe token blocks inside the B rows; otherwise no tile runs
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      bool bad = s_off[0] != 0 || s_blk[0] != 0 || s_off[groups] > p.rows_b;
+      for (int g = 0; g < groups && !bad; ++g) {
+        const int cnt = s_off[g + 1] - s_off[g], nb = s_blk[g + 1] - s_blk[g];
+        bad = cnt < 0 || nb < (cnt + p.TB - 1) / p.TB || nb > cnt;
+      }
+      if (bad) {
+        flag_error(p.err, kDevDebugBounds);
+        for (int g = 0; g <= groups; ++g) s_off[g] = s_blk[g] = 0;
+      }
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if constexpr (PAIR) cluster_sync_all();  // barriers of both CTAs are initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int num_tiles = p.num_fb * s_blk[groups];
-  const int kblocks = p.K / kStageK;
+  // the last stage of an e4m3 operand may reach past K (K % 128 == 64): TMA fills it with zeros
+  const int kblocks = (p.K + kStageK - 1) / kStageK;
   const int tile0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int tstep = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   // B rows of a tile held by this CTA: all npad rows, or half of them per CTA in PAIR mode
@@ -626,10 +642,16 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
       // W8 / F8: channel scales of this lane's feature rows (1 otherwise, and then unused)
       float sc0 = 1.0f, sc1 = 1.0f;
       if constexpr (W8 || F8) {
+        // feature rows past the weight's extent (a partial last tile) have no scale and no
+        // output
         const size_t so = static_cast<size_t>(t.group) * p.scale_ld + m;
-        sc0 = p.scale0[so];
-        if constexpr (kSwiGLU) sc1 = p.scale1[so];
-        else if constexpr (kDual) sc1 = p.scale0[so + 128];
+        if (m < p.m_valid) {
+          sc0 = p.scale0[so];
+          if constexpr (kSwiGLU) sc1 = p.scale1[so];
+        }
+        if constexpr (kDual && !kSwiGLU) {
+          if (m + 128 < p.m_valid) sc1 = p.scale0[so + 128];
+        }
       }
       auto scl0 = [&](uint32_t a) {
         return (W8 || F8) ? __uint_as_float(a) * sc0 : __uint_as_float(a);
@@ -930,7 +952,7 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
     TcParams p{};
     p.b_box_rows = box_rows;
     p.K = H;
-    p.num_fb = pair ? (I + 255) / 256 : I / kBM;
+    p.num_fb = pair ? (I + 255) / 256 : (I + kBM - 1) / kBM;
     p.m_valid = I;
     p.TB = TB;
     p.groups = E;
@@ -958,7 +980,7 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
   TcParams p{};
   p.b_box_rows = 0;
   p.K = H;
-  p.num_fb = I / kBM;
+  p.num_fb = (I + kBM - 1) / kBM;
   p.m_valid = I;
   p.TB = TB;
   p.groups = E;
@@ -993,7 +1015,7 @@ cudaError_t launch_gemm2_tc(const void* hbuf, int64_t hbuf_rows, const int32_t* 
   TcParams p{};
   p.b_box_rows = box_rows;
   p.K = I;
-  p.num_fb = pair ? (H + 511) / 512 : (dual ? H / 256 : H / kBM);
+  p.num_fb = pair ? (H + 511) / 512 : (dual ? H / 256 : (H + kBM - 1) / kBM);
   p.m_valid = H;
   p.TB = TB;
   p.groups = E;
@@ -1029,7 +1051,7 @@ cudaError_t launch_gemm1_w8(const void* xs, const int32_t* offsets, const int32_
   TcParams p{};
   p.b_box_rows = TB;
   p.K = H;
-  p.num_fb = I / kBM;
+  p.num_fb = (I + kBM - 1) / kBM;
   p.m_valid = I;
   p.TB = TB;
   p.groups = E;
@@ -1063,7 +1085,7 @@ cudaError_t launch_gemm2_w8(const void* hbuf, int64_t hbuf_rows, const int32_t* 
   TcParams p{};
   p.b_box_rows = TB;
   p.K = I;
-  p.num_fb = dual ? H / 256 : H / kBM;
+  p.num_fb = dual ? H / 256 : (H + kBM - 1) / kBM;
   p.m_valid = H;
   p.TB = TB;
   p.groups = E;
@@ -1106,7 +1128,7 @@ cudaError_t launch_gemm1_f8(const void* xs8, const float* sx, const int32_t* off
   TcParams p{};
   p.b_box_rows = box_rows;
   p.K = H;
-  p.num_fb = pair ? (I + 255) / 256 : I / kBM;
+  p.num_fb = pair ? (I + 255) / 256 : (I + kBM - 1) / kBM;
   p.m_valid = I;
   p.TB = TB;
   p.groups = E;
@@ -1146,7 +1168,7 @@ cudaError_t launch_gemm2_f8(const void* h8, const float* sh, int64_t hbuf_rows,
   TcParams p{};
   p.b_box_rows = box_rows;
   p.K = I;
-  p.num_fb = pair ? (H + 511) / 512 : (dual ? H / 256 : H / kBM);
+  p.num_fb = pair ? (H + 511) / 512 : (dual ? H / 256 : (H + kBM - 1) / kBM);
   p.m_valid = H;
   p.TB = TB;
   p.groups = E;

@@ -33,16 +33,13 @@ cudaError_t launch_route_gemv(const void* x, const void* w_router, int T, int H,
                               float* partials, cudaStream_t stream);
 
 // ---- route_tc.cu (tcgen05 / TMEM / TMA, bf16)
-// The whole router in one launch for E in [16, 256], E % 8 == 0: gate logits on the tensor
-// cores (tokens on the MMA's M side, experts on N), the K split into `ksplit` ranges whose
-// partial logits are summed (ascending range) inside a thread-block cluster through distributed
-// shared memory, then top-k + renormalised weights (select.cuh) and, when logits_out is non-null,
-// the logits (bias included). The launch layout (CTA pairs or single CTAs, the number of K
-// ranges) is chosen per T so that every cluster fits on the GPU at once when possible.
-cudaError_t launch_route_tc(const void* x, const void* w_router, const float* bias, int T, int H,
-                            int E, int k, int n_group, int topk_group, float* logits_out,
-                            int32_t* topk_idx, float* topk_w, int* err, cudaStream_t stream,
-                            std::string* detail);
+// Gate logits on the tensor cores (tokens on the MMA's M side, experts on N, E in [16, 256],
+// E % 8 == 0), K split into `ksplit` ranges:
+// partials[ks][t][e] = sum over h in range ks of x[t,h] * w_router[h,e].
+int route_ksplit(int64_t T, int H, int E);
+cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int H, int E,
+                                 float* partials, int ksplit, int* err, int num_sms,
+                                 cudaStream_t stream, std::string* detail);
 
 // ---- ffn_tc.cu (tcgen05 / TMEM / TMA, bf16)
 // Expert GEMM1: h[s, :] = silu(x[t] Wg[e]) * (x[t] Wu[e]) for kept slots; h rows = hbuf_rows.
@@ -133,7 +130,8 @@ cudaError_t launch_quantize_rows(const void* a, int64_t N, const int32_t* n_dev,
 // the kept slots s < offsets[E] (H % 16 == 0).
 cudaError_t launch_dispatch_rows_q8(const uint8_t* x8, const float* sxt, const int32_t* sorted_ids,
                                     const int32_t* offsets, int E, int k, int H, int64_t rows,
-                                    uint8_t* xs8, float* sx, cudaStream_t stream);
+                                    int64_t T, uint8_t* xs8, float* sx, int* err,
+                                    cudaStream_t stream);
 
 // ---- probe.cu: one bounded wait that nothing satisfies (failure-detection test)
 cudaError_t launch_stalled_wait(int* err, cudaStream_t stream);
@@ -155,12 +153,14 @@ cudaError_t launch_ep_combine(int dtype, const void* const* peer_y, const int32_
 
 // ---- combine.cu
 // Expert-major copy of the token rows: xs[s,:] = x[sorted_ids[s]/k,:] for kept slots.
+// T: rows of x (debug builds check sorted_ids[s] / k < T; err receives the failure).
 cudaError_t launch_dispatch_rows(int dtype, const void* x, const int32_t* sorted_ids,
                                  const int32_t* offsets, int E, int k, int H, int64_t rows,
-                                 void* xs, cudaStream_t stream);
+                                 int64_t T, void* xs, int* err, cudaStream_t stream);
+// err (may be null): debug builds record a slot outside the T*k rows of y_slots there.
 cudaError_t launch_combine(int dtype, const void* y_slots, const int32_t* slot_of,
                            const float* topk_w, const void* shared, float shared_factor,
-                           const float* out_bias, void* out, int64_t T, int H, int k,
+                           const float* out_bias, void* out, int64_t T, int H, int k, int* err,
                            cudaStream_t stream);
 
 // ---- FP8 (e4m3) expert weights (quant.cu, ffn_tc.cu)

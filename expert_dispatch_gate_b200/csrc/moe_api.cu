@@ -55,8 +55,8 @@ moe_status check_shape(const moe_shape* s) {
     return fail(MOE_ERR_INVALID_ARG, "capacity_factor is NaN");
   if (s->H % 8 != 0) return fail(MOE_ERR_UNSUPPORTED, "H % 8 != 0");
   if (s->dtype == MOE_BF16) {
-    if (s->H % 128 != 0 || s->I % 128 != 0)
-      return fail(MOE_ERR_UNSUPPORTED, "bf16 needs H % 128 == 0 and I % 128 == 0");
+    if (s->H % 64 != 0 || s->I % 64 != 0)
+      return fail(MOE_ERR_UNSUPPORTED, "bf16 needs H % 64 == 0 and I % 64 == 0");
     if (s->E > 64 && s->E % 8 != 0) return fail(MOE_ERR_UNSUPPORTED, "bf16 with E > 64 needs E % 8 == 0");
   } else {
     if (s->E > 64) return fail(MOE_ERR_UNSUPPORTED, "f32 needs E <= 64");
@@ -134,13 +134,13 @@ Layout layout_of(const moe_shape& s) {
   };
   const size_t es = elem_size(s.dtype);
   L.err = take(256);
-  L.ksplit = 1;  // K ranges of the split-K GEMV router (its partial logits live here)
-  if (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0 && moe::route_uses_gemv(s.T, s.H, s.E))
-    L.ksplit = moe::kRouteGemvSplit;
-  // partial logits of the split-K GEMV (a few tokens), or the logits of the CUDA-core router
-  // before a group-limited selection; the tensor-core router keeps its partials on chip
-  const bool gemv = L.ksplit > 1 && moe::route_uses_gemv(s.T, s.H, s.E);
-  L.logits_bytes = static_cast<size_t>(s.T) * s.E * 4 * (gemv ? L.ksplit : 1);
+  L.ksplit = 1;  // K ranges of the router's partial logits (GEMV or tensor-core gate GEMM)
+  if (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0 && s.T > 0)
+    L.ksplit = moe::route_uses_gemv(s.T, s.H, s.E) ? moe::kRouteGemvSplit
+                                                   : moe::route_ksplit(s.T, s.H, s.E);
+  // the router's partial logits [ksplit][T][E] (or the CUDA-core router's logits before a
+  // group-limited selection)
+  L.logits_bytes = static_cast<size_t>(s.T) * s.E * 4 * L.ksplit;
   L.logits = take(L.logits_bytes);
   L.blk_hist = take(static_cast<size_t>(L.nblk) * s.E * 4);
   L.offsets = take(static_cast<size_t>(s.E + 1) * 4);
@@ -247,11 +247,14 @@ moe_status do_route(const moe_shape& s, const Layout& L, const Opts& o, const vo
                            o.n_group, o.topk_group, topk_idx, topk_w, st);
       if (e != cudaSuccess) return cuda_fail(e, "router top-k");
     } else {
+      float* partials = at<float>(ws, L.logits);
       std::string d;
-      e = moe::launch_route_tc(x, w_router, bias, static_cast<int>(s.T), s.H, s.E, s.k,
-                               o.n_group, o.topk_group, logits_out, topk_idx, topk_w,
-                               at<int>(ws, L.err), st, &d);
-      if (e != cudaSuccess) return cuda_fail(e, "router (tcgen05 gate GEMM + top-k)", d);
+      e = moe::launch_route_gemm_tc(x, w_router, static_cast<int>(s.T), s.H, s.E, partials,
+                                    L.ksplit, at<int>(ws, L.err), num_sms(), st, &d);
+      if (e != cudaSuccess) return cuda_fail(e, "router gate GEMM (tcgen05)", d);
+      e = moe::launch_topk(partials, L.ksplit, s.T * s.E, bias, logits_out, s.T, s.E, s.k,
+                           o.n_group, o.topk_group, topk_idx, topk_w, st);
+      if (e != cudaSuccess) return cuda_fail(e, "router top-k");
     }
   } else {
     // the fused CUDA-core router selects plain top-k; with groups its logits (bias included)
@@ -305,8 +308,8 @@ moe_status do_ffn(const moe_shape& s, const Layout& L, const void* x, const int3
     float* sh = reinterpret_cast<float*>(h8 + static_cast<size_t>(L.a_cap) * s.I);
     e = moe::launch_quantize_rows(x, s.T, nullptr, s.H, x8, sxt, st);
     if (e != cudaSuccess) return cuda_fail(e, "e4m3 quantisation of the token rows");
-    e = moe::launch_dispatch_rows_q8(x8, sxt, sorted_ids, offsets, s.E, s.k, s.H, L.a_cap, xs8,
-                                     sx, st);
+    e = moe::launch_dispatch_rows_q8(x8, sxt, sorted_ids, offsets, s.E, s.k, s.H, L.a_cap, s.T,
+                                     xs8, sx, at<int>(ws, L.err), st);
     if (e != cudaSuccess) return cuda_fail(e, "expert-major copy of the e4m3 rows");
     e = moe::launch_gemm1_f8(xs8, sx, offsets, at<int32_t>(ws, L.blk_prefix), fw.q_gate, fw.q_up,
                              fw.s_gate, fw.s_up, at<void>(ws, L.hbuf), L.a_cap, s.H, s.E, s.I,
@@ -323,7 +326,8 @@ moe_status do_ffn(const moe_shape& s, const Layout& L, const void* x, const int3
     const int64_t ub_blocks = (s.E < L.a_cap ? s.E : L.a_cap) + L.a_cap / L.TB;
     std::string d;
     void* xs = at<void>(ws, L.xs);
-    e = moe::launch_dispatch_rows(s.dtype, x, sorted_ids, offsets, s.E, s.k, s.H, L.a_cap, xs, st);
+    e = moe::launch_dispatch_rows(s.dtype, x, sorted_ids, offsets, s.E, s.k, s.H, L.a_cap, s.T,
+                                     xs, at<int>(ws, L.err), st);
     if (e != cudaSuccess) return cuda_fail(e, "expert-major row copy");
     e = moe::launch_gemm1_w8(xs, offsets, at<int32_t>(ws, L.blk_prefix), fw.q_gate, fw.q_up,
                              fw.s_gate, fw.s_up, at<void>(ws, L.hbuf), L.a_cap, s.H, s.E, s.I,
@@ -340,7 +344,8 @@ moe_status do_ffn(const moe_shape& s, const Layout& L, const void* x, const int3
     void* xs = nullptr;
     if (gemm1_from_copy(s)) {
       xs = at<void>(ws, L.xs);
-      e = moe::launch_dispatch_rows(s.dtype, x, sorted_ids, offsets, s.E, s.k, s.H, L.a_cap, xs, st);
+      e = moe::launch_dispatch_rows(s.dtype, x, sorted_ids, offsets, s.E, s.k, s.H, L.a_cap, s.T,
+                                     xs, at<int>(ws, L.err), st);
       if (e != cudaSuccess) return cuda_fail(e, "expert-major row copy");
     }
     e = moe::launch_gemm1_tc(x, static_cast<int>(s.T), xs, sorted_ids, offsets,
@@ -370,6 +375,14 @@ moe_status do_ffn(const moe_shape& s, const Layout& L, const void* x, const int3
 }  // namespace
 
 extern "C" {
+
+int32_t moe_debug_checks(void) {
+#ifdef MOE_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 size_t moe_workspace_bytes(const moe_shape* shape) {
   if (check_shape(shape) != MOE_OK) return 0;
@@ -539,7 +552,7 @@ moe_status moe_combine_ex(const moe_shape* shape, const moe_layer_opts* opts,
   REQUIRE_PTR(out, "out");
   cudaError_t e = moe::launch_combine(shape->dtype, y_slots, slot_of, topk_w, o.shared,
                                       o.shared_factor, o.out_bias, out, shape->T, shape->H,
-                                      shape->k, static_cast<cudaStream_t>(stream));
+                                      shape->k, nullptr, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "combine");
   return MOE_OK;
 }
@@ -711,7 +724,7 @@ moe_status layer_impl(const moe_shape* shape, const moe_layer_opts* opts, const 
   st = do_ffn(s, L, x, sorted_ids, offsets, fw, y, ws, cs, true);
   if (st != MOE_OK) return st;
   e = moe::launch_combine(s.dtype, y, slot_of, topk_w, o.shared, o.shared_factor, o.out_bias, out,
-                          s.T, s.H, s.k, cs);
+                          s.T, s.H, s.k, at<int>(ws, L.err), cs);
   if (e != cudaSuccess) return cuda_fail(e, "combine");
   record_stage(4, cs);
   return MOE_OK;
@@ -919,6 +932,8 @@ moe_status moe_check_error(void* ws, void* stream) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
     if (e != cudaSuccess) return cuda_fail(e, "moe_check_error (clear)");
     const char* what = word == 1 ? "an expert id outside [0, E) in topk_idx"
+                       : word == 3 ? "debug bounds check: a slot, token row or group offset read "
+                                     "from device data was out of range"
                        : word == 2 ? "a bounded wait ran out in a pipelined kernel (stalled pipeline)"
                                    : "unknown device error";
     return fail(MOE_ERR_DEVICE, std::string("device error ") + std::to_string(word) + ": " + what);

@@ -143,12 +143,17 @@ __global__ void __launch_bounds__(kThreads)
     dispatch_rows_q8_kernel(const uint8_t* __restrict__ x8, const float* __restrict__ sxt,
                             const int32_t* __restrict__ sorted_ids,
                             const int32_t* __restrict__ offsets, int E, int k, int H, int64_t rows,
-                            uint8_t* __restrict__ xs8, float* __restrict__ sx) {
+                            int64_t Ttok, uint8_t* __restrict__ xs8, float* __restrict__ sx,
+                            int* err) {
   pdl_enter<false>();
   const int lane = threadIdx.x & 31;
   const int64_t s = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
   if (s >= rows || s >= offsets[E]) return;
   const int64_t t = sorted_ids[s] / k;
+  if (kDebugChecks && (sorted_ids[s] < 0 || t >= Ttok)) {
+    if (lane == 0) flag_error(err, kDevDebugBounds);
+    return;
+  }
   const uint4* src = reinterpret_cast<const uint4*>(x8 + t * H);
   uint4* dst = reinterpret_cast<uint4*>(xs8 + s * H);
   for (int c = lane; c < H / 16; c += 32) dst[c] = __ldg(src + c);
@@ -181,11 +186,12 @@ cudaError_t launch_quantize_rows(const void* a, int64_t N, const int32_t* n_dev,
 
 cudaError_t launch_dispatch_rows_q8(const uint8_t* x8, const float* sxt, const int32_t* sorted_ids,
                                     const int32_t* offsets, int E, int k, int H, int64_t rows,
-                                    uint8_t* xs8, float* sx, cudaStream_t stream) {
+                                    int64_t T, uint8_t* xs8, float* sx, int* err,
+                                    cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((rows + kThreads / 32 - 1) / (kThreads / 32));
   return launch_kernel(dispatch_rows_q8_kernel, dim3(grid), dim3(kThreads), 0, stream, 1, x8, sxt,
-                       sorted_ids, offsets, E, k, H, rows, xs8, sx);
+                       sorted_ids, offsets, E, k, H, rows, T, xs8, sx, err);
 }
 
 cudaError_t launch_quantize_fp8(const void* w, int64_t E, int K, int M, uint8_t* codes,

@@ -265,30 +265,32 @@ cudaError_t route_simt_dispatch(const Tin* x, const Tin* wr, const float* bias, 
 // Gate GEMV for a few tokens (decode), CUDA cores, bf16, E % 32 == 0: the router weight (2 MB
 // at H = 4096, E = 256) is streamed once over ~128 CTAs instead of through 128-token tensor-core
 // tiles that would be almost empty. CTA (ks, ec) takes the H/ksplit rows of K range ks and the
-// 32 experts of chunk ec; lane = expert, warp w = every 8th row of the range (rows ks*R0 + w,
-// + 8, ...). Each thread keeps T <= TMAX running sums (x from shared memory, a broadcast read),
-// the 8 warps' sums are added in ascending warp order, and the CTA writes
-// partials[ks][t][32*ec + lane], the layout topk_kernel sums over ks.
-constexpr int kGemvWarps = 8;
+// 32 experts of chunk ec. It stages its slice of x (widened to float) and of the router weight
+// in shared memory; then warp w takes tokens w*4 ... w*4+3 (then + 64 ...) with lane = expert,
+// and sums over the range's rows in ascending order, each token's sum a separate chain. It
+// writes partials[ks][t][32*ec + lane], the layout topk_kernel sums over ks.
+constexpr int kGemvWarps = 16;
+constexpr int kGemvTok = 4;  // tokens per warp pass
 
-template <int TMAX>
 __global__ void __launch_bounds__(kGemvWarps * 32)
     route_gemv_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
                       int T, int H, int E, int rows_per_split, float* __restrict__ partials) {
   extern __shared__ float gsm[];
-  float* xs = gsm;                                 // [T][rows_per_split], x widened to float
-  float* red = gsm + TMAX * rows_per_split;        // [kGemvWarps][TMAX][32]
+  const int Tp = (T + kGemvTok - 1) / kGemvTok * kGemvTok;         // tokens padded to a pass
+  float* xs = gsm;                                                  // [Tp][rows], float
+  __nv_bfloat16* ws = reinterpret_cast<__nv_bfloat16*>(gsm + static_cast<size_t>(Tp) * rows_per_split);  // [rows][32]
   pdl_enter<false>();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int ks = blockIdx.x;
-  const int e = blockIdx.y * 32 + lane;
+  const int e0 = blockIdx.y * 32;
   const int h0 = ks * rows_per_split;
-  // x[t, h0 .. h0 + rows_per_split) -> shared memory, 8 bf16 per 16-byte load
+  // x[t, h0 .. h0 + rows) -> float, 8 bf16 per 16-byte load; padding tokens read as zero
   const int vec_per_row = rows_per_split / 8;
-  for (int i = threadIdx.x; i < T * vec_per_row; i += blockDim.x) {
+  for (int i = threadIdx.x; i < Tp * vec_per_row; i += blockDim.x) {
     const int t = i / vec_per_row, v = i - t * vec_per_row;
-    const uint4 r = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + h0) + v);
+    uint4 r = make_uint4(0u, 0u, 0u, 0u);
+    if (t < T) r = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + h0) + v);
     const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
     float* dst = xs + t * rows_per_split + v * 8;
 #pragma unroll
@@ -297,46 +299,43 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
       dst[2 * j + 1] = __uint_as_float(w4[j] & 0xffff0000u);
     }
   }
+  // the router weight rows of this range, 32 experts (64 bytes) each, 16-byte loads
+  for (int i = threadIdx.x; i < rows_per_split * 4; i += blockDim.x) {
+    const int r = i >> 2, c = i & 3;
+    reinterpret_cast<uint4*>(ws + r * 32)[c] =
+        __ldg(reinterpret_cast<const uint4*>(wr + static_cast<size_t>(h0 + r) * E + e0) + c);
+  }
   __syncthreads();
-  float acc[TMAX];
+  for (int t0 = warp * kGemvTok; t0 < T; t0 += kGemvWarps * kGemvTok) {
+    float acc[kGemvTok];
 #pragma unroll
-  for (int t = 0; t < TMAX; ++t) acc[t] = 0.f;
-  // the weights of this thread's rows are loaded 16 at a time before they are used, so their
-  // latencies overlap instead of adding up row after row
-  constexpr int kRowBatch = 16;
-  for (int r0 = warp; r0 < rows_per_split; r0 += kGemvWarps * kRowBatch) {
-    float w[kRowBatch];
+    for (int i = 0; i < kGemvTok; ++i) acc[i] = 0.f;
+    const float* xt = xs + t0 * rows_per_split;
+    // four rows at a time: one 16-byte shared-memory load of x per token, four weights
+#pragma unroll 2
+    for (int r = 0; r < rows_per_split; r += 4) {
+      float w[4];
 #pragma unroll
-    for (int i = 0; i < kRowBatch; ++i) {
-      const int r = r0 + i * kGemvWarps;
-      w[i] = (r < rows_per_split) ? __bfloat162float(wr[static_cast<size_t>(h0 + r) * E + e]) : 0.f;
-    }
+      for (int q = 0; q < 4; ++q) w[q] = __bfloat162float(ws[(r + q) * 32 + lane]);
 #pragma unroll
-    for (int i = 0; i < kRowBatch; ++i) {
-      const int r = r0 + i * kGemvWarps;
-      if (r < rows_per_split) {
-#pragma unroll
-        for (int t = 0; t < TMAX; ++t)
-          if (t < T) acc[t] = fmaf(xs[t * rows_per_split + r], w[i], acc[t]);
+      for (int i = 0; i < kGemvTok; ++i) {
+        const float4 xv = *reinterpret_cast<const float4*>(xt + i * rows_per_split + r);
+        acc[i] = fmaf(xv.x, w[0], acc[i]);
+        acc[i] = fmaf(xv.y, w[1], acc[i]);
+        acc[i] = fmaf(xv.z, w[2], acc[i]);
+        acc[i] = fmaf(xv.w, w[3], acc[i]);
       }
     }
-  }
 #pragma unroll
-  for (int t = 0; t < TMAX; ++t)
-    if (t < T) red[(warp * TMAX + t) * 32 + lane] = acc[t];
-  __syncthreads();
-  for (int t = warp; t < T; t += kGemvWarps) {
-    float v = red[t * 32 + lane];
-#pragma unroll
-    for (int w2 = 1; w2 < kGemvWarps; ++w2) v += red[(w2 * TMAX + t) * 32 + lane];
-    partials[(static_cast<size_t>(ks) * T + t) * E + e] = v;
+    for (int i = 0; i < kGemvTok; ++i)
+      if (t0 + i < T) partials[(static_cast<size_t>(ks) * T + t0 + i) * E + e0 + lane] = acc[i];
   }
 }
 
 }  // namespace
 
 bool route_uses_gemv(int64_t T, int H, int E) {
-  // x rows of one K range and the warps' sums fit in shared memory up to 512 rows per range
+  // x rows of one K range (64 tokens) and its weight rows fit in shared memory up to 512 rows
   return T >= 1 && T <= kRouteGemvMaxT && E % 32 == 0 && H % (kRouteGemvSplit * 8) == 0 &&
          H <= kRouteGemvSplit * 512;
 }
@@ -345,20 +344,15 @@ cudaError_t launch_route_gemv(const void* x, const void* w_router, int T, int H,
                               float* partials, cudaStream_t stream) {
   if (!route_uses_gemv(T, H, E)) return cudaErrorInvalidValue;
   const int rows = H / kRouteGemvSplit;
-  const dim3 grid(kRouteGemvSplit, E / 32);
-  const dim3 block(kGemvWarps * 32);
-  const auto* xb = static_cast<const __nv_bfloat16*>(x);
-  const auto* wb = static_cast<const __nv_bfloat16*>(w_router);
-  auto go = [&](auto kernel, int tmax) {
-    const size_t smem = (static_cast<size_t>(tmax) * rows + kGemvWarps * tmax * 32) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    return launch_kernel(kernel, grid, block, smem, stream, 1, xb, wb, T, H, E, rows, partials);
-  };
-  if (T <= 4) return go(route_gemv_kernel<4>, 4);
-  if (T <= 16) return go(route_gemv_kernel<16>, 16);
-  return go(route_gemv_kernel<kRouteGemvMaxT>, kRouteGemvMaxT);
+  const int Tp = (T + kGemvTok - 1) / kGemvTok * kGemvTok;
+  const size_t smem = static_cast<size_t>(Tp) * rows * sizeof(float) + static_cast<size_t>(rows) * 64;
+  cudaError_t e = cudaFuncSetAttribute(route_gemv_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_kernel(route_gemv_kernel, dim3(kRouteGemvSplit, E / 32), dim3(kGemvWarps * 32),
+                       smem, stream, 1, static_cast<const __nv_bfloat16*>(x),
+                       static_cast<const __nv_bfloat16*>(w_router), T, H, E, rows, partials);
 }
 
 cudaError_t launch_route_simt(int dtype, const void* x, const void* w_router, const float* bias,

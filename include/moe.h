@@ -34,7 +34,7 @@
  *     (one tensor per kind with a leading expert dimension, [P1] "手动编译 MoE 融合算子").
  *   - Outputs are the MoE contribution only; the residual add belongs to the caller.
  *   - Limits: 1 <= E <= 256, 1 <= k <= min(E,16), 0 <= T < 2^24, H % 8 == 0, I >= 1.
- *     BF16: H % 128 == 0 and I % 128 == 0 (tensor-core expert GEMMs); E <= 64 or E % 8 == 0.
+ *     BF16: H % 64 == 0 and I % 64 == 0 (tensor-core expert GEMMs); E <= 64 or E % 8 == 0.
  *     F32: E <= 64.
  */
 #ifndef MOE_H_
@@ -351,6 +351,12 @@ moe_status moe_check_error(void* ws, void* stream);
  * context stays usable. Returns MOE_ERR_WORKSPACE without launching when ws is NULL or too
  * small. */
 moe_status moe_probe_stalled_wait(void* ws, size_t ws_bytes, void* stream);
+
+/* 1 in the debug build (libmoe_debug.so, compiled with -DMOE_DEBUG), 0 otherwise. The debug build
+ * checks every slot, token-row and group-table index a kernel reads from device data before
+ * using it; a failed check records device error 3 in the workspace error word (moe_check_error
+ * reports it) and the access is skipped. Its results are otherwise those of the release build. */
+int32_t moe_debug_checks(void);
 
 /* Static description of a status code. */
 const char* moe_status_string(moe_status status);

@@ -69,8 +69,8 @@ ODD = 0x1001  # misaligned
     (16, 128, 300, 8, 128, 1.25, "bf16", L.MOE_ERR_UNSUPPORTED),  # E > 256
     (16, 128, 32, 17, 128, 1.25, "bf16", L.MOE_ERR_UNSUPPORTED),  # k > 16
     (16, 100, 8, 2, 128, 1.25, "bf16", L.MOE_ERR_UNSUPPORTED),   # H % 8
-    (16, 192, 8, 2, 128, 1.25, "bf16", L.MOE_ERR_UNSUPPORTED),   # bf16 H % 128
-    (16, 128, 8, 2, 200, 1.25, "bf16", L.MOE_ERR_UNSUPPORTED),   # bf16 I % 128
+    (16, 136, 8, 2, 128, 1.25, "bf16", L.MOE_ERR_UNSUPPORTED),   # bf16 H % 64
+    (16, 128, 8, 2, 200, 1.25, "bf16", L.MOE_ERR_UNSUPPORTED),   # bf16 I % 64
     (16, 128, 100, 2, 128, 1.25, "bf16", L.MOE_ERR_UNSUPPORTED),  # bf16 E > 64, E % 8
     (16, 128, 72, 2, 128, 1.25, "f32", L.MOE_ERR_UNSUPPORTED),   # f32 E > 64
     (-1, 128, 8, 2, 128, 1.25, "bf16", L.MOE_ERR_INVALID_ARG),   # T < 0
@@ -191,3 +191,8 @@ def test_expert_parallel_calls_reject_bad_arguments_before_any_launch(lib):
     # the wait needs a workspace for its error word
     assert lib.moe_ep_wait(2, 1, bogus, None, 0, None) == L.MOE_ERR_WORKSPACE
     assert lib.moe_ep_wait(0, 1, bogus, bogus, 256, None) == L.MOE_ERR_INVALID_ARG
+
+
+def test_bf16_accepts_multiples_of_64(lib):
+    s = L.make_shape(300, 192, 16, 4, 320, 1.25, "bf16")
+    assert L.moe_workspace_bytes(s) > 0 and L.moe_capacity(s) == 94  # ceil(1.25 * 300 * 4 / 16)

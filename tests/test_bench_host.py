@@ -48,15 +48,16 @@ def test_stage_costs_fp8_weights_are_one_byte_plus_channel_scales():
 
 
 def test_launches_per_step():
-    # fused router, one grouping launch, the row copy, two expert GEMMs, the combine
-    assert bench.launches_per_step(W.WORKLOADS["fine"]) == 6
-    # decode: at most 64 tokens route through the CUDA-core GEMV + top-k
+    # router gate GEMM (or GEMV) + top-k, one grouping launch, the row copy, two expert GEMMs,
+    # the combine
+    assert bench.launches_per_step(W.WORKLOADS["fine"]) == 7
     assert bench.launches_per_step(W.WORKLOADS["decode"].with_tokens(1)) == 7
-    assert bench.launches_per_step(W.WORKLOADS["decode"].with_tokens(64)) == 7
-    assert bench.launches_per_step(W.WORKLOADS["decode"].with_tokens(256)) == 6
+    assert bench.launches_per_step(W.WORKLOADS["decode"].with_tokens(256)) == 7
     # skewed: 196608 assignments take the three grouping kernels; every bf16 layer makes the
     # row copy, whatever I
-    assert bench.launches_per_step(W.WORKLOADS["skewed"]) == 1 + 3 + 1 + 2 + 1
+    assert bench.launches_per_step(W.WORKLOADS["skewed"]) == 2 + 3 + 1 + 2 + 1
+    # W8A8: the token rows and the SwiGLU rows are quantised by one launch each
+    assert bench.launches_per_step(W.WORKLOADS["fine"], "w8a8") == 9
     # tiny f32: one fused CUDA-core router kernel
     assert bench.launches_per_step(W.WORKLOADS["tiny"]) == 1 + 1 + 0 + 2 + 1
 

@@ -36,6 +36,9 @@ SMALL = {
     "e128_router_gemv": W.Workload("e128", 20, 50, 1024, 128, 6, 256, "bf16", 1.25),
     # T = 90: one token tile of the tensor-core router, its K split into 4 ranges
     "e128_router_ksplit": W.Workload("e128k", 21, 90, 1024, 128, 6, 256, "bf16", 1.25),
+    # H = 192 and I = 320, multiples of 64 only: partial last feature blocks in both GEMMs (and
+    # a partial last K stage of the e4m3 operands)
+    "h192_i320": W.Workload("h192", 22, 300, 192, 16, 4, 320, "bf16", 1.25),
 }
 
 
@@ -440,3 +443,49 @@ def test_combine_fine_every_token():
     assert np.all(got[dropped_all] == 0.0)
     print("combine fine: %d tokens, %d dropped assignments, max rel err %.3e"
           % (wl.T, int(al["drop_mask"].sum()), r))
+
+
+def test_layer_call_captured_in_a_cuda_graph_replays_identically():
+    """The layer call makes no host synchronisation and launches only on its stream, so a serving
+    loop can capture it in a CUDA graph: replays give the eager call's results bit for bit, for
+    new inputs copied into the captured buffers too."""
+    wl, cpu, dev = small_inputs("e256_k8")
+    shape = M.shape_of(wl.T, wl.H, wl.E, wl.k, wl.I, wl.capacity_factor, wl.dtype)
+    ws = M.Workspace(shape, "cuda")
+    x = dev["x"].clone()
+    ref = M.layer_forward(x, dev["w_router"], dev["w_gate"], dev["w_up"], dev["w_down"], wl.k,
+                          wl.capacity_factor, ws=ws)
+    torch.cuda.synchronize()
+    outs = {key: torch.empty_like(ref[key]) for key in ("out", "topk_idx", "topk_w", "counts",
+                                                         "drop_mask", "logits")}
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+
+    def call():
+        L.moe_layer_forward(shape, x, dev["w_router"], None, dev["w_gate"], dev["w_up"],
+                            dev["w_down"], outs["out"], outs["logits"], outs["topk_idx"],
+                            outs["topk_w"], outs["counts"], outs["drop_mask"], ws.buf, ws.nbytes,
+                            stream)
+
+    with torch.cuda.stream(stream):
+        call()  # first call on this stream before capture (tensor-map and attribute setup)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        call()
+    for key in outs:
+        outs[key].zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    for key in outs:
+        assert torch.equal(outs[key], ref[key]), key
+    # new activations through the captured buffer
+    x.copy_(torch.flip(dev["x"], dims=[0]))
+    ref2 = M.layer_forward(x, dev["w_router"], dev["w_gate"], dev["w_up"], dev["w_down"], wl.k,
+                           wl.capacity_factor)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert ws.check() == L.MOE_OK
+    for key in outs:
+        assert torch.equal(outs[key], ref2[key]), key
+    del graph
