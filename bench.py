@@ -280,10 +280,10 @@ def oracle_baseline(wl, dev, n_tokens, reps=1):
 # ------------------------------------------------------------------ the GPU arm
 
 def launches_per_step(wl, weights="bf16"):
-    """Kernels one moe_layer_forward launches: router (gate GEMM on the tensor cores, or a
-    CUDA-core GEMV for at most 64 tokens, then the top-k kernel; one fused CUDA-core kernel for
-    E < 64 or f32), align (one launch up to 65536 assignments, else three), the expert-major row
-    copy (bf16), two expert GEMMs, combine."""
+    """Kernels one moe_layer_forward launches: router (tensor-core gate GEMM + top-k, or one
+    fused CUDA-core kernel for E < 64 or f32), align (one launch up to 65536 assignments, else
+    three), the expert-major row copy (bf16), the W8A8 quantisations, two expert GEMMs,
+    combine."""
     route = 2 if (wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0) else 1
     align = 1 if wl.T * wl.k <= 65536 else 3
     # expert-major copy of the token rows before GEMM1: every bf16 layer (GEMM1 runs on CTA

@@ -23,15 +23,6 @@ cudaError_t launch_topk(const float* partials, int ksplit, int64_t split_stride,
                         int n_group, int topk_group, int32_t* topk_idx, float* topk_w,
                         cudaStream_t stream);
 
-// Gate logits for a few tokens (decode) on CUDA cores, bf16, E % 32 == 0, T <= kRouteGemvMaxT:
-// partials[ks][t][e] for kRouteGemvSplit K ranges of H / kRouteGemvSplit rows each (the layout
-// launch_topk sums).
-constexpr int kRouteGemvMaxT = 64;
-constexpr int kRouteGemvSplit = 16;
-bool route_uses_gemv(int64_t T, int H, int E);
-cudaError_t launch_route_gemv(const void* x, const void* w_router, int T, int H, int E,
-                              float* partials, cudaStream_t stream);
-
 // ---- route_tc.cu (tcgen05 / TMEM / TMA, bf16)
 // Gate logits on the tensor cores (tokens on the MMA's M side, experts on N, E in [16, 256],
 // E % 8 == 0), K split into `ksplit` ranges:

@@ -115,7 +115,7 @@ struct Layout {
   int nblk;
   int32_t C;
   int TB;
-  int ksplit;  // K ranges of the split-K GEMV router (1 otherwise)
+  int ksplit;  // router K split (tensor-core router only)
 };
 
 Layout layout_of(const moe_shape& s) {
@@ -134,10 +134,8 @@ Layout layout_of(const moe_shape& s) {
   };
   const size_t es = elem_size(s.dtype);
   L.err = take(256);
-  L.ksplit = 1;  // K ranges of the router's partial logits (GEMV or tensor-core gate GEMM)
-  if (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0 && s.T > 0)
-    L.ksplit = moe::route_uses_gemv(s.T, s.H, s.E) ? moe::kRouteGemvSplit
-                                                   : moe::route_ksplit(s.T, s.H, s.E);
+  L.ksplit = (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0 && s.T > 0)
+                 ? moe::route_ksplit(s.T, s.H, s.E) : 1;
   // the router's partial logits [ksplit][T][E] (or the CUDA-core router's logits before a
   // group-limited selection)
   L.logits_bytes = static_cast<size_t>(s.T) * s.E * 4 * L.ksplit;
@@ -238,24 +236,14 @@ moe_status do_route(const moe_shape& s, const Layout& L, const Opts& o, const vo
                     float* topk_w, void* ws, cudaStream_t st) {
   cudaError_t e;
   if (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0) {
-    if (moe::route_uses_gemv(s.T, s.H, s.E)) {
-      // a few tokens: stream the router weight once on CUDA cores (split-K GEMV), then select
-      float* partials = at<float>(ws, L.logits);
-      e = moe::launch_route_gemv(x, w_router, static_cast<int>(s.T), s.H, s.E, partials, st);
-      if (e != cudaSuccess) return cuda_fail(e, "router gate GEMV (CUDA cores)");
-      e = moe::launch_topk(partials, L.ksplit, s.T * s.E, bias, logits_out, s.T, s.E, s.k,
-                           o.n_group, o.topk_group, topk_idx, topk_w, st);
-      if (e != cudaSuccess) return cuda_fail(e, "router top-k");
-    } else {
-      float* partials = at<float>(ws, L.logits);
-      std::string d;
-      e = moe::launch_route_gemm_tc(x, w_router, static_cast<int>(s.T), s.H, s.E, partials,
-                                    L.ksplit, at<int>(ws, L.err), num_sms(), st, &d);
-      if (e != cudaSuccess) return cuda_fail(e, "router gate GEMM (tcgen05)", d);
-      e = moe::launch_topk(partials, L.ksplit, s.T * s.E, bias, logits_out, s.T, s.E, s.k,
-                           o.n_group, o.topk_group, topk_idx, topk_w, st);
-      if (e != cudaSuccess) return cuda_fail(e, "router top-k");
-    }
+    float* partials = at<float>(ws, L.logits);
+    std::string d;
+    e = moe::launch_route_gemm_tc(x, w_router, static_cast<int>(s.T), s.H, s.E, partials,
+                                  L.ksplit, at<int>(ws, L.err), num_sms(), st, &d);
+    if (e != cudaSuccess) return cuda_fail(e, "router gate GEMM (tcgen05)", d);
+    e = moe::launch_topk(partials, L.ksplit, s.T * s.E, bias, logits_out, s.T, s.E, s.k,
+                         o.n_group, o.topk_group, topk_idx, topk_w, st);
+    if (e != cudaSuccess) return cuda_fail(e, "router top-k");
   } else {
     // the fused CUDA-core router selects plain top-k; with groups its logits (bias included)
     // go through the group-limited top-k kernel

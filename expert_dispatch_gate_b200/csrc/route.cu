@@ -262,98 +262,7 @@ cudaError_t route_simt_dispatch(const Tin* x, const Tin* wr, const float* bias, 
   return route_simt_launch<Tin, 64>(x, wr, bias, T, H, E, k, logits_out, idx, w, st);
 }
 
-// Gate GEMV for a few tokens (decode), CUDA cores, bf16, E % 32 == 0: the router weight (2 MB
-// at H = 4096, E = 256) is streamed once over ~128 CTAs instead of through 128-token tensor-core
-// tiles that would be almost empty. CTA (ks, ec) takes the H/ksplit rows of K range ks and the
-// 32 experts of chunk ec. It stages its slice of x (widened to float) and of the router weight
-// in shared memory; then warp w takes tokens w*4 ... w*4+3 (then + 64 ...) with lane = expert,
-// and sums over the range's rows in ascending order, each token's sum a separate chain. It
-// writes partials[ks][t][32*ec + lane], the layout topk_kernel sums over ks.
-constexpr int kGemvWarps = 16;
-constexpr int kGemvTok = 4;  // tokens per warp pass
-
-__global__ void __launch_bounds__(kGemvWarps * 32)
-    route_gemv_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
-                      int T, int H, int E, int rows_per_split, float* __restrict__ partials) {
-  extern __shared__ float gsm[];
-  const int Tp = (T + kGemvTok - 1) / kGemvTok * kGemvTok;         // tokens padded to a pass
-  float* xs = gsm;                                                  // [Tp][rows], float
-  __nv_bfloat16* ws = reinterpret_cast<__nv_bfloat16*>(gsm + static_cast<size_t>(Tp) * rows_per_split);  // [rows][32]
-  pdl_enter<false>();
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int ks = blockIdx.x;
-  const int e0 = blockIdx.y * 32;
-  const int h0 = ks * rows_per_split;
-  // x[t, h0 .. h0 + rows) -> float, 8 bf16 per 16-byte load; padding tokens read as zero
-  const int vec_per_row = rows_per_split / 8;
-  for (int i = threadIdx.x; i < Tp * vec_per_row; i += blockDim.x) {
-    const int t = i / vec_per_row, v = i - t * vec_per_row;
-    uint4 r = make_uint4(0u, 0u, 0u, 0u);
-    if (t < T) r = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + h0) + v);
-    const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
-    float* dst = xs + t * rows_per_split + v * 8;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      dst[2 * j] = __uint_as_float(w4[j] << 16);
-      dst[2 * j + 1] = __uint_as_float(w4[j] & 0xffff0000u);
-    }
-  }
-  // the router weight rows of this range, 32 experts (64 bytes) each, 16-byte loads
-  for (int i = threadIdx.x; i < rows_per_split * 4; i += blockDim.x) {
-    const int r = i >> 2, c = i & 3;
-    reinterpret_cast<uint4*>(ws + r * 32)[c] =
-        __ldg(reinterpret_cast<const uint4*>(wr + static_cast<size_t>(h0 + r) * E + e0) + c);
-  }
-  __syncthreads();
-  for (int t0 = warp * kGemvTok; t0 < T; t0 += kGemvWarps * kGemvTok) {
-    float acc[kGemvTok];
-#pragma unroll
-    for (int i = 0; i < kGemvTok; ++i) acc[i] = 0.f;
-    const float* xt = xs + t0 * rows_per_split;
-    // four rows at a time: one 16-byte shared-memory load of x per token, four weights
-#pragma unroll 2
-    for (int r = 0; r < rows_per_split; r += 4) {
-      float w[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) w[q] = __bfloat162float(ws[(r + q) * 32 + lane]);
-#pragma unroll
-      for (int i = 0; i < kGemvTok; ++i) {
-        const float4 xv = *reinterpret_cast<const float4*>(xt + i * rows_per_split + r);
-        acc[i] = fmaf(xv.x, w[0], acc[i]);
-        acc[i] = fmaf(xv.y, w[1], acc[i]);
-        acc[i] = fmaf(xv.z, w[2], acc[i]);
-        acc[i] = fmaf(xv.w, w[3], acc[i]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kGemvTok; ++i)
-      if (t0 + i < T) partials[(static_cast<size_t>(ks) * T + t0 + i) * E + e0 + lane] = acc[i];
-  }
-}
-
 }  // namespace
-
-bool route_uses_gemv(int64_t T, int H, int E) {
-  // x rows of one K range (64 tokens) and its weight rows fit in shared memory up to 512 rows
-  return T >= 1 && T <= kRouteGemvMaxT && E % 32 == 0 && H % (kRouteGemvSplit * 8) == 0 &&
-         H <= kRouteGemvSplit * 512;
-}
-
-cudaError_t launch_route_gemv(const void* x, const void* w_router, int T, int H, int E,
-                              float* partials, cudaStream_t stream) {
-  if (!route_uses_gemv(T, H, E)) return cudaErrorInvalidValue;
-  const int rows = H / kRouteGemvSplit;
-  const int Tp = (T + kGemvTok - 1) / kGemvTok * kGemvTok;
-  const size_t smem = static_cast<size_t>(Tp) * rows * sizeof(float) + static_cast<size_t>(rows) * 64;
-  cudaError_t e = cudaFuncSetAttribute(route_gemv_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  return launch_kernel(route_gemv_kernel, dim3(kRouteGemvSplit, E / 32), dim3(kGemvWarps * 32),
-                       smem, stream, 1, static_cast<const __nv_bfloat16*>(x),
-                       static_cast<const __nv_bfloat16*>(w_router), T, H, E, rows, partials);
-}
 
 cudaError_t launch_route_simt(int dtype, const void* x, const void* w_router, const float* bias,
                               int64_t T, int H, int E, int k, float* logits_out, int32_t* topk_idx,

@@ -114,9 +114,6 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       const int c0 = static_cast<int>(rank) * p.nch;  // first expert chunk this CTA loads
       bool ok = true;
       int issued = 0;
-      // the CTA's token rows of x for the k-blocks past the first ring's worth go to L2 now,
-      // so their loads meet L2 latency instead of DRAM latency when the ring reaches them
-      for (int i = S; i < nkb; ++i) tma_prefetch_2d(&tmX, (kb0 + i) * kRtBK, row0);
       for (int i = 0; i < nkb; ++i) {
         if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag)) {
           ok = false;

@@ -32,8 +32,8 @@ SMALL = {
     # accumulators); I = 640 leaves the last GEMM1 pair tile half outside the weight; H = 384
     # runs GEMM2 with one feature block per tile
     "e96_partial_tiles": W.Workload("e96", 19, 333, 384, 96, 4, 640, "bf16", 1.25),
-    # T = 50, H = 1024: few tokens, the router's split-K CUDA-core GEMV
-    "e128_router_gemv": W.Workload("e128", 20, 50, 1024, 128, 6, 256, "bf16", 1.25),
+    # T = 50, H = 1024: one token tile, the router's K split into 4 ranges
+    "e128_router_t50": W.Workload("e128", 20, 50, 1024, 128, 6, 256, "bf16", 1.25),
     # T = 90: one token tile of the tensor-core router, its K split into 4 ranges
     "e128_router_ksplit": W.Workload("e128k", 21, 90, 1024, 128, 6, 256, "bf16", 1.25),
     # H = 192 and I = 320, multiples of 64 only: partial last feature blocks in both GEMMs (and
@@ -100,14 +100,14 @@ ROUTER = {
     "pairs_short_peer": W.Workload("r3", 23, 129, 256, 256, 8, 128, "bf16", 1.25),
     "pairs_t2_ksplit16": W.Workload("r4", 24, 2, 4096, 256, 8, 128, "bf16", 1.25),
     "single_e192": W.Workload("r5", 25, 513, 4096, 192, 8, 128, "bf16", 1.25),
-    # just above the CUDA-core GEMV's token limit (64): tensor cores with the K split in 4 / 16
+    # the K split at 4 and 16 ranges with one or two token tiles
     "tc_t100_ksplit4": W.Workload("r6", 26, 100, 1024, 128, 6, 128, "bf16", 1.25),
     "tc_t65_ksplit16": W.Workload("r7", 27, 65, 4096, 256, 8, 128, "bf16", 1.25),
-    # a few tokens: the split-K CUDA-core GEMV, each of its token-count tiers (4, 16, 64)
-    "gemv_t1": W.Workload("r8", 28, 1, 4096, 256, 8, 128, "bf16", 0.0),
-    "gemv_t3_e128": W.Workload("r9", 29, 3, 2048, 128, 4, 128, "bf16", 0.0),
-    "gemv_t16_e96": W.Workload("r10", 30, 16, 1024, 96, 6, 128, "bf16", 1.25),
-    "gemv_t64_e64_zipf": W.Workload("r11", 31, 64, 2048, 64, 6, 128, "bf16", 1.25, zipf_s=1.2),
+    # decode-sized batches: one token, a few, and E not a multiple of 128 (single CTAs)
+    "tc_t1": W.Workload("r8", 28, 1, 4096, 256, 8, 128, "bf16", 0.0),
+    "tc_t3_e128": W.Workload("r9", 29, 3, 2048, 128, 4, 128, "bf16", 0.0),
+    "tc_t16_e96": W.Workload("r10", 30, 16, 1024, 96, 6, 128, "bf16", 1.25),
+    "tc_t64_e64_zipf": W.Workload("r11", 31, 64, 2048, 64, 6, 128, "bf16", 1.25, zipf_s=1.2),
 }
 
 
