@@ -10,7 +10,9 @@
 // Rank of assignment a = t*k + j inside expert e = idx[t,j]: number of earlier assignments (in
 // a order, i.e. token order) routed to e. Kept iff rank < C. The result is deterministic and
 // identical to the sequential definition. Up to kAlignCluster assignments one launch does all
-// of it (one block up to kAlignSingle, one cluster of CTAs above); beyond that three kernels:
+// of it (one block up to kAlignSingle, one cluster of CTAs above); beyond that one cooperative
+// launch with a grid barrier (align_grid_kernel), or, when its CTAs cannot all be resident,
+// three kernels:
 //   1. hist:    per chunk of align_chunk(A) assignments, per-expert counts (shared-memory
 //               atomics).
 //   2. scan:    one block; per expert, exclusive prefix over chunks (chunk bases; the chunks
@@ -425,6 +427,183 @@ __global__ void __launch_bounds__(NT, 1)
   if constexpr (CS > 1) cluster_wait();
 }
 
+// Whole grouping in one cooperative launch of G CTAs (at most one per SM, all resident at
+// once), for kAlignCluster < A <= G * kGridThreads * kGridMaxSteps. Same steps as the cluster
+// form; the per-CTA expert totals go through global memory (hist[r][e]) and a grid barrier
+// instead of distributed shared memory:
+//   1. ids into 16-bit codes in shared memory, per-warp per-expert counts;
+//   2. per expert, the exclusive prefix over this CTA's warps; the CTA's totals to hist[r];
+//   3. grid barrier (bounded wait); each CTA sums hist over the CTAs before it (its base) and
+//      over all of them (raw totals), in CTA order, split over several threads per expert;
+//      counts, offsets and the token-block plan as in the cluster form (CTA 0 writes them);
+//   4. stable ranks in assignment order and the scatter.
+// The barrier's two counters (arrivals, departures; bar[0], bar[1]) are zero between launches:
+// the last CTA to leave the barrier resets both.
+constexpr int kGridThreads = 1024;
+constexpr int kGridMaxSteps = 64;  // rounds of 32 ids per warp: 128 KB of codes per CTA
+
+__global__ void __launch_bounds__(kGridThreads, 1)
+    align_grid_kernel(const int32_t* __restrict__ idx, int64_t A, int E, int C, int TB,
+                      int32_t* __restrict__ hist, int* bar, int32_t* __restrict__ counts,
+                      int32_t* __restrict__ offsets, int32_t* __restrict__ blk_prefix,
+                      int32_t* __restrict__ sorted_ids, int32_t* __restrict__ slot_of,
+                      uint8_t* __restrict__ drop_mask, int* err) {
+  constexpr int NT = kGridThreads, NW = NT / 32, kBatch = 8;
+  pdl_enter<false>();
+  __shared__ int wrun[NW][kMaxE];
+  __shared__ int s_off[kMaxE];
+  __shared__ int part[2][NT];
+  __shared__ int sh[NW];
+  __shared__ int s_ok;
+  extern __shared__ uint16_t code_sm[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r = static_cast<int>(blockIdx.x), G = static_cast<int>(gridDim.x);
+  for (int i = threadIdx.x; i < NW * kMaxE; i += NT) (&wrun[0][0])[i] = 0;
+  // A <= G * NT * kGridMaxSteps (checked by the launcher): 32-bit indices suffice
+  const int An = static_cast<int>(A);
+  const int steps = ((An + G * NW - 1) / (G * NW) + 31) / 32;
+  const int wbase = (r * NW + warp) * steps * 32;
+  const int nbits = (E > 1) ? 32 - __clz(E - 1) : 0;
+  for (int s0 = 0; s0 < steps; s0 += kBatch) {  // uniform across the block
+    int raw[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int a = wbase + (s0 + j) * 32 + lane;
+      raw[j] = (s0 + j < steps && a < An) ? __ldg(idx + a) : -1;
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int st = s0 + j;
+      const int a = wbase + st * 32 + lane;
+      const bool ok = (raw[j] >= 0 && raw[j] < E);
+      if (st < steps && a < An && !ok) flag_error(err, kDevBadExpert);
+      if (st < steps)
+        code_sm[st * NT + threadIdx.x] = ok ? static_cast<uint16_t>(raw[j]) : uint16_t{0xFFFF};
+    }
+  }
+  __syncthreads();
+  // 1. per-warp per-expert counts
+  for (int st = 0; st < steps; ++st) {
+    const uint32_t c = code_sm[st * NT + threadIdx.x];
+    if (c != 0xFFFFu) atomicAdd(&wrun[warp][c], 1);
+  }
+  __syncthreads();
+  // 2. per expert: exclusive prefix across this CTA's warps; the CTA's total to hist[r]
+  if (threadIdx.x < E) {
+    const int e = threadIdx.x;
+    int mine = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const int c = wrun[w][e];
+      wrun[w][e] = mine;
+      mine += c;
+    }
+    hist[static_cast<size_t>(r) * E + e] = mine;
+  }
+  // 3. grid barrier: every CTA's totals are written before any CTA reads them
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(&bar[0], 1);
+    const unsigned long long t0 = global_ns();
+    int ok = 1, v;
+    for (;;) {
+      asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+      if (v >= G) break;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+    if (!ok) flag_error(err, kDevWaitTimeout);
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  if (!s_ok) return;  // the grouping is abandoned; the error word says so
+  // thread (sp, e), tid = sp * Ep + e, sums the totals of CTAs [sp * per, (sp + 1) * per)
+  int Ep = 1;
+  while (Ep < E) Ep <<= 1;
+  const int S = NT / Ep;
+  const int e = threadIdx.x % Ep, sp = threadIdx.x / Ep;
+  const int per = (G + S - 1) / S;
+  int below = 0, all = 0;
+  if (e < E) {
+    const int q1 = min(G, (sp + 1) * per);
+#pragma unroll 8
+    for (int q = sp * per; q < q1; ++q) {
+      const int v = __ldcg(hist + static_cast<size_t>(q) * E + e);
+      all += v;
+      below += (q < r) ? v : 0;
+    }
+  }
+  part[0][threadIdx.x] = below;
+  part[1][threadIdx.x] = all;
+  __syncthreads();
+  // every CTA has read what it needs from the counters: the last one out resets them
+  if (threadIdx.x == 0 && atomicAdd(&bar[1], 1) == G - 1) {
+    bar[0] = 0;
+    bar[1] = 0;
+  }
+  int before = 0, raw_tot = 0;
+  if (threadIdx.x < E) {
+    for (int q = 0; q < S; ++q) {
+      before += part[0][q * Ep + threadIdx.x];
+      raw_tot += part[1][q * Ep + threadIdx.x];
+    }
+  }
+  const int cnt = (threadIdx.x < E) ? min(raw_tot, C) : 0;
+  const int nb = (cnt + TB - 1) / TB;
+  int tot_cnt, tot_nb;
+  const int off = block_exclusive_scan<NW>(cnt, sh, tot_cnt);
+  const int bp = block_exclusive_scan<NW>(nb, sh, tot_nb);
+  if (threadIdx.x < E) {
+    const int ee = threadIdx.x;
+    s_off[ee] = off;
+    if (r == 0) {
+      counts[ee] = cnt;
+      offsets[ee] = off;
+      if (blk_prefix != nullptr) blk_prefix[ee] = bp;
+    }
+    if (before != 0) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) wrun[w][ee] += before;
+    }
+  }
+  if (threadIdx.x == 0 && r == 0) {
+    offsets[E] = tot_cnt;
+    if (blk_prefix != nullptr) blk_prefix[E] = tot_nb;
+  }
+  __syncthreads();
+  // 4. stable ranks in assignment order, then the scatter
+  for (int st = 0; st < steps; ++st) {  // uniform across the block
+    const int a = wbase + st * 32 + lane;
+    const bool in = a < An;
+    const uint32_t c = code_sm[st * NT + threadIdx.x];
+    const bool ok = c != 0xFFFFu;
+    const int ea = static_cast<int>(c);
+    const uint32_t peers = warp_peers(c, ok, nbits);
+    int rank = 0;
+    if (ok) rank = wrun[warp][ea] + __popc(peers & lanemask_lt());
+    __syncwarp();
+    if (ok && lane == __ffs(peers) - 1) wrun[warp][ea] += __popc(peers);
+    __syncwarp();
+    if (in) {
+      if (ok && rank < C) {
+        const int slot = s_off[ea] + rank;
+        sorted_ids[slot] = a;
+        slot_of[a] = slot;
+        drop_mask[a] = 0;
+      } else {
+        slot_of[a] = -1;
+        drop_mask[a] = 1;
+      }
+    }
+  }
+  for (int sl = tot_cnt + r * NT + threadIdx.x; sl < An; sl += G * NT) sorted_ids[sl] = -1;
+}
+
 __global__ void __launch_bounds__(kThreads)
     plan_from_offsets_kernel(const int32_t* __restrict__ offsets, int E, int TB,
                              int32_t* __restrict__ blk_prefix) {
@@ -466,6 +645,44 @@ cudaError_t launch_align(const int32_t* topk_idx, int64_t A, int E, int C, int T
   }
   const int chunk = align_chunk(A);
   const int nblk = static_cast<int>((A + chunk - 1) / chunk);
+  // one cooperative launch when every CTA (one per SM, at most one per chunk histogram row of
+  // blk_hist) can be resident and hold its share of the codes
+  {
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int G = nblk < sms ? nblk : sms;
+    const int64_t steps = ((A + int64_t{G} * (kGridThreads / 32) - 1) /
+                               (int64_t{G} * (kGridThreads / 32)) + 31) / 32;
+    if (G > 0 && steps <= kGridMaxSteps) {
+      const size_t code_bytes = static_cast<size_t>(steps) * kGridThreads * 2;
+      e = cudaFuncSetAttribute(align_grid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(code_bytes));
+      if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, align_grid_kernel,
+                                                          kGridThreads, code_bytes);
+      if (e != cudaSuccess) return e;
+      if (per_sm >= 1) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(G));
+        cfg.blockDim = dim3(kGridThreads);
+        cfg.dynamicSmemBytes = code_bytes;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, align_grid_kernel, topk_idx, A, E, C, TB, blk_hist,
+                               err + kAlignBarrierWord, counts, offsets, blk_prefix, sorted_ids,
+                               slot_of, drop_mask, err);
+        // the GPU cannot hold every CTA at once (other work resident): the chunked kernels
+        if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+        (void)cudaGetLastError();
+      }
+    }
+  }
   cudaError_t e = launch_kernel(align_hist_kernel, dim3(nblk), dim3(kThreads), 0, stream, 1,
                                 topk_idx, A, E, chunk, blk_hist, err);
   if (e == cudaSuccess)
@@ -545,8 +762,9 @@ cudaError_t launch_align_noalloc(const int32_t* topk_idx, int64_t A, int E, int 
     base = g_noalloc_ptr[dev];
   }
   NoAllocScratch* sc = static_cast<NoAllocScratch*>(base);
-  // The error word must start at zero; the histograms and the plan are fully rewritten.
-  e = cudaMemsetAsync(sc->err, 0, sizeof(int), stream);
+  // The error word and the grid barrier's counters must start at zero; the histograms and the
+  // plan are fully rewritten.
+  e = cudaMemsetAsync(sc->err, 0, sizeof(sc->err), stream);
   if (e != cudaSuccess) return e;
   return launch_align(topk_idx, A, E, C, TB, sc->blk_hist, counts, offsets, sc->blk_prefix,
                       sorted_ids, slot_of, drop_mask, sc->err, stream);

@@ -73,11 +73,12 @@ cudaError_t launch_gemm2_simt(const float* hbuf, const int32_t* offsets, const f
 
 // ---- align.cu
 // Grouping: one launch does everything up to kAlignCluster assignments (one 256-thread block up
-// to kAlignSingle, one cluster of 8 CTAs of 1024 threads above); beyond that the histogram /
-// scatter blocks take align_chunk(A) assignments each (a multiple of 256 between
-// kAlignChunkMin and kAlignChunkMax, aiming at about 128 blocks). Measured on B200, the
-// cluster's time grows by about 0.11 us per 1000 assignments on its 8 SMs and the chunked
-// kernels' by far less, so the cluster form stops where the two meet.
+// to kAlignSingle, one cluster of 8 CTAs of 1024 threads above); beyond that one cooperative
+// launch of min(chunks, SMs) CTAs with a grid barrier, or, when those CTAs cannot all be
+// resident, three kernels (histogram / scan / scatter) whose blocks take align_chunk(A)
+// assignments each (a multiple of 256 between kAlignChunkMin and kAlignChunkMax, aiming at
+// about 128 blocks). Measured on B200, the cluster's time grows by about 0.11 us per 1000
+// assignments on its 8 SMs, so the cluster form stops at 65536.
 constexpr int kAlignSingle = 2048;
 constexpr int kAlignCluster = 65536;
 constexpr int kAlignChunkMin = 512;
@@ -89,6 +90,10 @@ inline int align_chunk(int64_t A) {
   if (c > kAlignChunkMax) c = kAlignChunkMax;
   return static_cast<int>(c);
 }
+// `err` points at the error word, the first of 64 ints (256 bytes) that start out zero:
+// err[kAlignBarrierWord] and the int after it are the one-launch grid barrier's counters, which
+// the grouping leaves at zero.
+constexpr int kAlignBarrierWord = 32;
 cudaError_t launch_align(const int32_t* topk_idx, int64_t A, int E, int C, int TB,
                          int32_t* blk_hist, int32_t* counts, int32_t* offsets,
                          int32_t* blk_prefix, int32_t* sorted_ids, int32_t* slot_of,

@@ -916,7 +916,9 @@ moe_status moe_check_error(void* ws, void* stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
   if (e != cudaSuccess) return cuda_fail(e, "moe_check_error");
   if (word != 0) {
-    e = cudaMemsetAsync(ws, 0, sizeof(int), cs);
+    // the whole 256-byte control block: a wait that ran out may have left the grouping's grid
+    // barrier counters (words 32 and 33) off zero
+    e = cudaMemsetAsync(ws, 0, 256, cs);
     if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
     if (e != cudaSuccess) return cuda_fail(e, "moe_check_error (clear)");
     const char* what = word == 1 ? "an expert id outside [0, E) in topk_idx"

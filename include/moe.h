@@ -28,6 +28,10 @@
  *     status and launches nothing. A failed launch returns MOE_ERR_CUDA. Device-side faults
  *     that the kernels detect (an expert id out of range, a bounded wait that ran out) are
  *     recorded in the first word of `ws` and reported by moe_check_error.
+ *   - The first 256 bytes of `ws` are the library's control block (the error word, and the
+ *     counters of the grid barrier the one-launch grouping uses above 65536 assignments). They
+ *     must be zero before the first call on a workspace; the library leaves them zero, and
+ *     moe_check_error clears all of them when it reports a device error.
  *   - Float dtype: MOE_F32 or MOE_BF16 for x, the weights, y_slots and out. Gate logits,
  *     routing weights and the logit bias are always float32.
  *   - Weight layout (x @ W convention): w_router [H,E]; w_gate, w_up [E,H,I]; w_down [E,I,H]

@@ -76,6 +76,8 @@ def oracle_routing(wl, cpu):
     (257, 256, 16, False), (33, 16, 16, True), (4096, 256, 8, False), (129, 128, 4, True),
     # experts not a multiple of the per-lane run (scalar loads, lanes past E)
     (50, 37, 3, True), (64, 5, 2, True), (100, 200, 8, True), (77, 104, 7, True),
+    # large batches: 2 lanes per token at E = 256, one thread per token at E = 64
+    (40000, 256, 8, True), (100000, 64, 6, True),
 ])
 def test_route_from_logits_bitexact(T, E, k, ties):
     logits = W.random_logits(T, E, seed=T * 7 + E + k, ties=ties)
@@ -87,6 +89,25 @@ def test_route_from_logits_bitexact(T, E, k, ties):
     assert np.array_equal(npi(idx_g), idx_o)
     np.testing.assert_allclose(npi(w_g), w_o, atol=TOL_W, rtol=0)
     np.testing.assert_allclose(npi(w_g).astype(np.float64).sum(1), 1.0, atol=k * 2.0 ** -23 * 2)
+
+
+@pytest.mark.parametrize("T,E,k", [
+    (3000, 64, 6), (1000, 64, 8), (513, 32, 2), (700, 16, 16), (300, 60, 5), (257, 64, 1),
+    (100000, 64, 6),                    # one lane per token
+    (4096, 256, 8), (40000, 256, 8),   # 16 and 2 lanes per token
+    (77, 256, 16), (129, 200, 7), (3, 62, 4),
+])
+def test_lane_and_warp_selection_agree_bitwise(T, E, k):
+    """Plain top-k runs G lanes per token (topk_lanes_kernel, G from 1 to 16 by T and E); the
+    group-limited form with every group kept (no expert excluded) runs the warp-per-token
+    kernel on the same rule. Indices and weights (the renormalising sum is taken in the same
+    pairwise order) agree bit for bit."""
+    logits = W.random_logits(T, E, seed=5 * T + E + k, ties=True).cuda()
+    idx_t, w_t = M.route_from_logits(logits, k)
+    idx_w, w_w = M.route_from_logits(logits, k, n_group=2, topk_group=2)
+    torch.cuda.synchronize()
+    assert torch.equal(idx_t, idx_w)
+    assert torch.equal(w_t.view(torch.int32), w_w.view(torch.int32))
 
 
 # ----------------------------------------------------------------- route (gate GEMM + selection)
@@ -108,6 +129,11 @@ ROUTER = {
     "tc_t3_e128": W.Workload("r9", 29, 3, 2048, 128, 4, 128, "bf16", 0.0),
     "tc_t16_e96": W.Workload("r10", 30, 16, 1024, 96, 6, 128, "bf16", 1.25),
     "tc_t64_e64_zipf": W.Workload("r11", 31, 64, 2048, 64, 6, 128, "bf16", 1.25, zipf_s=1.2),
+    # the CUDA-core router (E < 64 or f32) over several 256-row slabs of Wr, the last one
+    # partial, in bf16 and f32, and a single token
+    "simt_e8_slabs": W.Workload("r12", 32, 300, 1088, 8, 2, 128, "bf16", 1.25),
+    "simt_e64_f32_slabs": W.Workload("r13", 33, 129, 520, 64, 6, 128, "f32", 1.25),
+    "simt_e16_t1": W.Workload("r14", 34, 1, 4096, 16, 4, 128, "bf16", 0.0),
 }
 
 
@@ -144,12 +170,14 @@ def test_router(name):
     (4096, 256, 8, 1.25, "uniform"), (4096, 256, 8, 1.25, "zipf"), (3000, 64, 6, 1.25, "zipf"),
     (2500, 16, 4, 1.0, "one"), (777, 32, 3, 0.5, "uniform"), (2049, 1, 1, 1.25, "one"),
     (20000, 64, 6, 1.25, "zipf"),
-    # the grouping's three launch forms and their edges: one 256-thread block up to 2048
-    # assignments, one cluster of 8 CTAs up to 65536, chunked kernels beyond
+    # the grouping's launch forms and their edges: one 256-thread block up to 2048
+    # assignments, one cluster of 8 CTAs up to 65536, one cooperative grid beyond (86 CTAs
+    # just above 65536, one per SM from about 300000)
     (256, 16, 8, 1.25, "zipf"), (1024, 128, 2, 1.0, "uniform"), (1025, 128, 2, 1.0, "uniform"),
     (4097, 256, 8, 1.25, "zipf"), (8192, 256, 8, 1.25, "zipf"), (5462, 96, 6, 0.75, "uniform"),
     (8193, 256, 8, 1.25, "uniform"), (10923, 64, 6, 1.25, "zipf"),
     (32768, 256, 8, 1.25, "zipf"), (40000, 64, 8, 1.25, "zipf"), (43691, 64, 6, 0.0, "uniform"),
+    (49152, 256, 8, 1.25, "zipf"), (131072, 64, 6, 1.25, "zipf"),
 ])
 def test_align_bitexact(T, E, k, cf, mode):
     idx = W.random_topk_idx(T, E, k, seed=T + 31 * E + k, mode=mode)
@@ -160,6 +188,35 @@ def test_align_bitexact(T, E, k, cf, mode):
     al = orc.align(idx.numpy(), E, C)
     for key in ("counts", "offsets", "sorted_ids", "slot_of", "drop_mask"):
         assert np.array_equal(npi(res[key]), al[key]), key
+    assert res["ws"].check() == L.MOE_OK
+
+
+def test_align_chunked_form_beyond_the_grid_properties():
+    """10 M assignments: more than the cooperative grid holds (148 SMs x 1024 threads x 64
+    rounds), so the three chunked kernels run. Checked by the grouping's defining properties
+    (numpy, any size): counts = min(histogram, C), offsets their prefix, each expert's slots the
+    first C of its assignments in assignment order, everything else dropped."""
+    T, E, k, cf = 1250000, 256, 8, 1.25
+    idx = W.random_topk_idx(T, E, k, seed=77, mode="zipf")
+    res = M.align(idx.cuda(), E, cf)
+    torch.cuda.synchronize()
+    C = orc.capacity(T, k, E, cf)
+    flat = idx.numpy().reshape(-1).astype(np.int64)
+    A = flat.size
+    counts = np.minimum(np.bincount(flat, minlength=E), C)
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    order = np.argsort(flat, kind="stable")          # expert-major, assignment order inside
+    start = np.concatenate([[0], np.cumsum(np.bincount(flat, minlength=E))])[flat[order]]
+    keep = (np.arange(A) - start) < C
+    sorted_ids = np.full(A, -1, np.int64)
+    sorted_ids[:offsets[-1]] = order[keep]
+    slot_of = np.full(A, -1, np.int64)
+    slot_of[order[keep]] = np.arange(offsets[-1])
+    assert np.array_equal(npi(res["counts"]), counts)
+    assert np.array_equal(npi(res["offsets"]), offsets)
+    assert np.array_equal(npi(res["sorted_ids"]), sorted_ids)
+    assert np.array_equal(npi(res["slot_of"]), slot_of)
+    assert np.array_equal(npi(res["drop_mask"]), (slot_of < 0).astype(np.uint8))
     assert res["ws"].check() == L.MOE_OK
 
 
