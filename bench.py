@@ -279,13 +279,28 @@ def oracle_baseline(wl, dev, n_tokens, reps=1):
 
 # ------------------------------------------------------------------ the GPU arm
 
+def route_ksplit(T, H, E):
+    """K ranges of the tensor-core gate GEMM (the library's rule): split while about 128 CTAs
+    or fewer run and each range keeps at least 4 k-blocks of 64."""
+    kb_total = H // 64
+    ctas = 2 * ((T + 255) // 256) if E % 128 == 0 else (T + 127) // 128
+    ks = 1
+    while (ks * 2 <= 16 and kb_total % (ks * 2) == 0 and kb_total // (ks * 2) >= 4
+           and ctas * ks * 2 <= 128):
+        ks *= 2
+    return ks
+
+
 def launches_per_step(wl, weights="bf16"):
-    """Kernels one moe_layer_forward launches: router (tensor-core gate GEMM + top-k, or one
-    fused CUDA-core kernel for E < 64 or f32), align (one launch up to 65536 assignments, else
-    three), the expert-major row copy (bf16), the W8A8 quantisations, two expert GEMMs,
-    combine."""
-    route = 2 if (wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0) else 1
-    align = 1 if wl.T * wl.k <= 65536 else 3
+    """Kernels one moe_layer_forward launches: router (tensor-core gate GEMM + top-k; one
+    persistent kernel for both when E = 64 and the hidden dimension is one K range; one
+    CUDA-core kernel for E < 64 or f32), align (one launch; three past the cooperative grid's
+    capacity of SMs x 1024 threads x 64 rounds of 32), the expert-major row copy (bf16), the
+    W8A8 quantisations, two expert GEMMs, combine."""
+    tc = wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0
+    fused = tc and wl.E == 64 and wl.k <= 16 and route_ksplit(wl.T, wl.H, wl.E) == 1
+    route = 2 if tc and not fused else 1
+    align = 1 if wl.T * wl.k <= 148 * 1024 * 64 * 32 else 3
     # expert-major copy of the token rows before GEMM1: every bf16 layer (GEMM1 runs on CTA
     # pairs, and the e4m3-weight GEMM1 reads the copy too)
     copy = 1 if wl.dtype == "bf16" else 0

@@ -31,6 +31,13 @@ int route_ksplit(int64_t T, int H, int E);
 cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int H, int E,
                                  float* partials, int ksplit, int* err, int num_sms,
                                  cudaStream_t stream, std::string* detail);
+// Gate GEMM + plain top-k in one persistent kernel (E = 64, one K range, n_group = 1, k <= 16):
+// the same logits, picks and weights as launch_route_gemm_tc followed by launch_topk.
+bool route_fuses_topk(int64_t T, int H, int E, int k, int n_group);
+cudaError_t launch_route_gemm_topk_tc(const void* x, const void* w_router, int T, int H, int E,
+                                      int k, const float* bias, float* logits_out,
+                                      int32_t* topk_idx, float* topk_w, int* err, int num_sms,
+                                      cudaStream_t stream, std::string* detail);
 
 // ---- ffn_tc.cu (tcgen05 / TMEM / TMA, bf16)
 // Expert GEMM1: h[s, :] = silu(x[t] Wg[e]) * (x[t] Wu[e]) for kept slots; h rows = hbuf_rows.

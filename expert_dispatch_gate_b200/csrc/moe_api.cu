@@ -235,7 +235,14 @@ moe_status do_route(const moe_shape& s, const Layout& L, const Opts& o, const vo
                     const void* w_router, const float* bias, float* logits_out, int32_t* topk_idx,
                     float* topk_w, void* ws, cudaStream_t st) {
   cudaError_t e;
-  if (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0) {
+  if (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0 &&
+      moe::route_fuses_topk(s.T, s.H, s.E, s.k, o.n_group)) {
+    std::string d;
+    e = moe::launch_route_gemm_topk_tc(x, w_router, static_cast<int>(s.T), s.H, s.E, s.k, bias,
+                                       logits_out, topk_idx, topk_w, at<int>(ws, L.err),
+                                       num_sms(), st, &d);
+    if (e != cudaSuccess) return cuda_fail(e, "router gate GEMM + top-k (tcgen05)", d);
+  } else if (s.dtype == MOE_BF16 && s.E >= 64 && s.E % 8 == 0) {
     float* partials = at<float>(ws, L.logits);
     std::string d;
     e = moe::launch_route_gemm_tc(x, w_router, static_cast<int>(s.T), s.H, s.E, partials,

@@ -128,7 +128,6 @@ __global__ void __launch_bounds__(256)
                       const float* __restrict__ bias, float* __restrict__ logits_out, int64_t T,
                       int E, int k, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   constexpr int TPB = 256 / G;
-  constexpr int PW = KL <= 2 ? 2 : KL <= 4 ? 4 : KL <= 8 ? 8 : 16;  // butterfly width
   extern __shared__ float s_log[];
   pdl_enter<false>();
   const int stride = E + G;
@@ -217,31 +216,11 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   const int g = static_cast<int>(threadIdx.x) % G;
   const int tl = static_cast<int>(threadIdx.x) / G;
-  uint32_t tk[KL];
-  int ti[KL];
-#pragma unroll
-  for (int j = 0; j < KL; ++j) {
-    tk[j] = 0u;  // key 0 belongs to no finite float: an empty place
-    ti[j] = 0x7fffffff;
-  }
+  TopList<KL> L;
+  L.clear();
   if (tl < nt) {
     const float* row = s_log + tl * stride;
-    for (int e = g; e < E; e += G) {
-      uint32_t ck = order_key(row[e]);
-      int ci = e;
-      bool shift = false;
-#pragma unroll
-      for (int q = 0; q < KL; ++q) {
-        const bool gt = shift || ck > tk[q];
-        shift = gt;
-        const uint32_t hk = gt ? ck : tk[q];
-        const int hi = gt ? ci : ti[q];
-        ck = gt ? tk[q] : ck;
-        ci = gt ? ti[q] : ci;
-        tk[q] = hk;
-        ti[q] = hi;
-      }
-    }
+    for (int e = g; e < E; e += G) L.insert(order_key(row[e]), e);
   }
   // k merge rounds over the token's G lanes (every lane of the warp takes part)
   uint32_t pk[KL];
@@ -251,8 +230,8 @@ __global__ void __launch_bounds__(256)
     pk[j] = 0u;
     pi[j] = 0;
     if (j < k) {
-      uint32_t hk = tk[0];
-      int hi = ti[0];
+      uint32_t hk = L.key[0];
+      int hi = L.idx[0];
 #pragma unroll
       for (int off = 1; off < G; off <<= 1) {
         const uint32_t ok = __shfl_xor_sync(0xffffffffu, hk, off);
@@ -263,42 +242,19 @@ __global__ void __launch_bounds__(256)
       }
       pk[j] = hk;
       pi[j] = hi;
-      const bool pop = ti[0] == hi;  // expert ids are unique: only the holder pops
+      const bool pop = L.idx[0] == hi;  // expert ids are unique: only the holder pops
 #pragma unroll
       for (int q = 0; q + 1 < KL; ++q) {
-        tk[q] = pop ? tk[q + 1] : tk[q];
-        ti[q] = pop ? ti[q + 1] : ti[q];
+        L.key[q] = pop ? L.key[q + 1] : L.key[q];
+        L.idx[q] = pop ? L.idx[q + 1] : L.idx[q];
       }
-      tk[KL - 1] = pop ? 0u : tk[KL - 1];
-      ti[KL - 1] = pop ? 0x7fffffff : ti[KL - 1];
+      L.key[KL - 1] = pop ? 0u : L.key[KL - 1];
+      L.idx[KL - 1] = pop ? 0x7fffffff : L.idx[KL - 1];
     }
   }
   if (tl >= nt) return;
-  // renormalised weights over the k picks: exp(l_j - l_0) / sum_i exp(l_i - l_0). The sum is
-  // taken in the pairwise order of write_selection's butterfly (halving strides; adding the
-  // zeros of unused places is exact), so this kernel and topk_kernel agree bit for bit.
-  const float top = key_value(pk[0]);
-  float ex[KL], acc[PW];
-#pragma unroll
-  for (int j = 0; j < PW; ++j) acc[j] = 0.f;
-#pragma unroll
-  for (int j = 0; j < KL; ++j) {
-    ex[j] = (j < k) ? expf(key_value(pk[j]) - top) : 0.f;
-    acc[j] = ex[j];
-  }
-#pragma unroll
-  for (int off = PW / 2; off > 0; off >>= 1) {
-#pragma unroll
-    for (int j = 0; j < off; ++j) acc[j] += acc[j + off];
-  }
   const int64_t t = t0 + tl;
-#pragma unroll
-  for (int j = 0; j < KL; ++j) {
-    if (j < k && j % G == g) {
-      topk_idx[t * k + j] = pi[j];
-      topk_w[t * k + j] = ex[j] / acc[0];
-    }
-  }
+  thread_write_selection<KL>(pk, pi, k, g, G, topk_idx + t * k, topk_w + t * k);
 }
 
 template <int G>

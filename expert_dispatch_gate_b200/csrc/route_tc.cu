@@ -23,6 +23,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "select.cuh"
 
 namespace moe {
 namespace {
@@ -259,6 +260,217 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   }
 }
 
+// Gate GEMM and plain top-k in one persistent kernel, for E = 64 with the whole hidden
+// dimension in one K range (large T) on single CTAs: the selection that topk_lanes_kernel would
+// run after a round trip of fp32 logits through memory runs in the epilogue warps instead, on
+// one tile's logits while the MMAs of the CTA's next tile run (two TMEM accumulator sets, each
+// the even/odd K-step pair of route_gemm_kernel). Epilogue thread q * 32 + lane owns TMEM lane
+// (token) q * 32 + lane of the tile: it reads its E logits (the two K-step accumulators added,
+// as in route_gemm_kernel), adds the bias, writes the logits when asked, inserts them in
+// ascending expert order into a TopList and writes the picks and their weights, so the result
+// equals the two-kernel router's bit for bit.
+template <int KL>
+__global__ void __launch_bounds__(kRtThreads, 1)
+    route_gemm_topk_kernel(const __grid_constant__ CUtensorMap tmX,
+                           const __grid_constant__ CUtensorMap tmW, const RtParams p,
+                           const float* __restrict__ bias, float* __restrict__ logits_out, int k,
+                           int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int b_bytes = p.nch * 8192;
+  const int stage_bytes = 16384 + b_bytes;
+  const int S = p.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * stage_bytes);
+  uint64_t* empty = full + kRtMaxStages;
+  uint64_t* tfull = empty + kRtMaxStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&tfull[b]), 1);
+      mbar_init(smem_u32(&tempty[b]), 4);  // one arrival per epilogue warp
+    }
+    mbar_init(smem_u32(done), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), kRtTmemCols);
+    tmem_relinquish();
+  }
+  pdl_enter<false>();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int ntiles = (p.T + kRtM - 1) / kRtM;
+  const int nkb = p.kb_per_split;  // the whole hidden dimension
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t s = 0, ph = 0;
+      const uint32_t tx = static_cast<uint32_t>(stage_bytes);
+      bool ok = true;
+      int issued = 0;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+        for (int i = 0; i < nkb; ++i) {
+          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+          const uint32_t fb = smem_u32(&full[s]);
+          const int kc = i * kRtBK;
+          mbar_arrive_expect_tx(fb, tx);
+          tma_load_2d(sa, &tmX, kc, tile * kRtM, fb);
+          for (int c = 0; c < p.nch; ++c) tma_load_2d(sa + 16384 + c * 8192, &tmW, c * 64, kc, fb);
+          ++issued;
+          if (++s == static_cast<uint32_t>(S)) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        flag_error(p.err, kDevWaitTimeout);
+      }
+      // every load issued lands before the CTA may exit
+      for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
+        mbar_wait(smem_u32(&full[i % S]), static_cast<uint32_t>(i / S) & 1u, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (whole warp)
+    constexpr uint32_t kFull = 0xffffffffu;
+    const uint32_t sbase = smem_u32(smem);
+    const uint64_t adesc0 = smem_desc_sw128(sbase, 16, 1024);            // x rows, K-major
+    const uint64_t bdesc0 = smem_desc_sw128(sbase + 16384, 8192, 1024);  // Wr, MN-major
+    const uint32_t idesc = idesc_bf16(kRtM, p.npad, /*a_mn_major=*/false, /*b_mn_major=*/true);
+    uint32_t s = 0, ph = 0, soff = 0;
+    bool ok = true;
+    int tc = 0;
+    for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tc) {
+      const int buf = tc & 1;
+      const uint32_t use = static_cast<uint32_t>(tc >> 1);
+      if (!__all_sync(kFull, mbar_wait(smem_u32(&tempty[buf]), (use & 1u) ^ 1u, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // two accumulators per buffer: even and odd K steps (npad <= 64 columns each)
+      const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * 128);
+      const uint32_t d1 = d0 + static_cast<uint32_t>(p.npad);
+      uint32_t acc0 = 0, acc1 = 0;
+      for (int i = 0; i < nkb; ++i) {
+        if (!__all_sync(kFull, mbar_wait(smem_u32(&full[s]), ph, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t ad = adesc0 + (soff >> 4);
+        const uint64_t bd = bdesc0 + (soff >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kRtBK / 16; ++kk) {
+          const bool second = kk & 1;
+          tc_mma_bf16_elect(second ? d1 : d0, ad + kk * 2, bd + kk * 128, idesc,
+                            second ? acc1 : acc0);
+          if (second) acc1 = 1u;
+          else acc0 = 1u;
+        }
+        tc_commit_elect(smem_u32(&empty[s]));
+        if (++s == static_cast<uint32_t>(S)) {
+          s = 0;
+          ph ^= 1u;
+          soff = 0;
+        } else {
+          soff += static_cast<uint32_t>(stage_bytes);
+        }
+      }
+      if (!ok) break;
+      tc_commit_elect(smem_u32(&tfull[buf]));
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      flag_error(p.err, kDevWaitTimeout);
+    }
+    // completes once every MMA issued has finished (also when the loop stopped early)
+    tc_commit_elect(smem_u32(done));
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue + top-k (warps 2..5)
+    const int q = warp & 3;
+    int tc = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+      const int buf = tc & 1;
+      const uint32_t use = static_cast<uint32_t>(tc >> 1);
+      int got = 1;
+      if (lane == 0) got = mbar_wait(smem_u32(&tfull[buf]), use & 1u, abort_flag) ? 1 : 0;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          flag_error(p.err, kDevWaitTimeout);
+        }
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                          static_cast<uint32_t>(buf * 128);
+      float lg[64];
+#pragma unroll
+      for (int c0 = 0; c0 < 64; c0 += 32) {
+        if (c0 < p.E) {  // uniform
+          uint32_t v[32], u[32];
+          tmem_ld32(tb + static_cast<uint32_t>(c0), v);
+          tmem_ld32(tb + static_cast<uint32_t>(p.npad + c0), u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) lg[c0 + j] = __uint_as_float(v[j]) + __uint_as_float(u[j]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
+      const int64_t t = static_cast<int64_t>(tile) * kRtM + q * 32 + lane;
+      if (t < p.T) {
+        TopList<KL> L;
+        L.clear();
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          if (e < p.E) {
+            float v = lg[e];
+            if (bias != nullptr) v += __ldg(bias + e);
+            if (logits_out != nullptr) logits_out[t * p.E + e] = v;
+            L.insert(order_key(v), e);
+          }
+        }
+        thread_write_selection<KL>(L.key, L.idx, k, 0, 1, topk_idx + t * k, topk_w + t * k);
+      }
+    }
+  }
+
+  // TMEM is released only after every MMA issued has completed
+  if (warp == 1 && lane == 0) mbar_wait(smem_u32(done), 0u, nullptr);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kRtTmemCols);
+  }
+}
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -357,6 +569,55 @@ cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int
                               : static_cast<unsigned>((T + kRtM - 1) / kRtM);
   const dim3 grid(tiles, static_cast<unsigned>(ksplit));
   return launch_kernel(kernel, grid, dim3(kRtThreads), smem, stream, pair ? 2 : 1, mx, mw, p);
+}
+
+bool route_fuses_topk(int64_t T, int H, int E, int k, int n_group) {
+  return E == 64 && n_group <= 1 && k <= 16 && H % kRtBK == 0 && route_ksplit(T, H, E) == 1;
+}
+
+cudaError_t launch_route_gemm_topk_tc(const void* x, const void* w_router, int T, int H, int E,
+                                      int k, const float* bias, float* logits_out,
+                                      int32_t* topk_idx, float* topk_w, int* err, int num_sms,
+                                      cudaStream_t stream, std::string* detail) {
+  if (T == 0) return cudaSuccess;
+  if (E != 64 || H % kRtBK != 0 || k < 1 || k > 16) {
+    if (detail) *detail = "fused router shape outside the tensor-core path";
+    return cudaErrorInvalidValue;
+  }
+  CUtensorMap mx, mw;
+  if (!map_2d(&mx, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), kRtM, detail) ||
+      !map_2d(&mw, w_router, static_cast<uint64_t>(E), static_cast<uint64_t>(H), kRtBK, detail))
+    return cudaErrorInvalidValue;
+  RtParams p{};
+  p.T = T;
+  p.H = H;
+  p.E = E;
+  p.npad = E;
+  p.nch = 1;
+  p.kb_per_split = H / kRtBK;
+  p.two_acc = 1;
+  p.split_stride = 0;
+  p.out = nullptr;
+  p.err = err;
+  const int stage_bytes = 16384 + 8192;
+  int stages = (kRtSmemLimit - 1024 - kRtCtrl) / stage_bytes;
+  if (stages > kRtMaxStages) stages = kRtMaxStages;
+  if (stages > p.kb_per_split) stages = p.kb_per_split;
+  if (stages < 2) stages = 2;
+  p.stages = stages;
+  const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + kRtCtrl;
+  auto kernel = route_gemm_topk_kernel<16>;
+  if (k <= 2) kernel = route_gemm_topk_kernel<2>;
+  else if (k <= 4) kernel = route_gemm_topk_kernel<4>;
+  else if (k <= 6) kernel = route_gemm_topk_kernel<6>;
+  else if (k <= 8) kernel = route_gemm_topk_kernel<8>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int tiles = (T + kRtM - 1) / kRtM;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  return launch_kernel(kernel, dim3(static_cast<unsigned>(grid)), dim3(kRtThreads), smem, stream,
+                       1, mx, mw, p, bias, logits_out, k, topk_idx, topk_w);
 }
 
 }  // namespace moe

@@ -113,6 +113,70 @@ __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
+// A thread's list of its KL largest candidates in (key descending, index ascending) order.
+// Candidates must arrive in ascending index order: an entry moves ahead of a listed one only on
+// a strictly larger key, and from the place it takes the entries below shift down one place
+// each, so equal keys keep the lower index first. Key 0 (no finite float) marks an empty place.
+template <int KL>
+struct TopList {
+  uint32_t key[KL];
+  int idx[KL];
+  __device__ __forceinline__ void clear() {
+#pragma unroll
+    for (int j = 0; j < KL; ++j) {
+      key[j] = 0u;
+      idx[j] = 0x7fffffff;
+    }
+  }
+  __device__ __forceinline__ void insert(uint32_t ck, int ci) {
+    bool shift = false;
+#pragma unroll
+    for (int q = 0; q < KL; ++q) {
+      const bool gt = shift || ck > key[q];
+      shift = gt;
+      const uint32_t hk = gt ? ck : key[q];
+      const int hi = gt ? ci : idx[q];
+      ck = gt ? key[q] : ck;
+      ci = gt ? idx[q] : ci;
+      key[q] = hk;
+      idx[q] = hi;
+    }
+  }
+};
+
+// Renormalised weights of k picks held by one thread (keys pk, indices pi; k <= KL):
+// w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0), the sum taken in the pairwise order of
+// write_selection's butterfly (halving strides; adding the zeros of unused places is exact), so
+// the weights equal the warp kernels' bit for bit. Writes the picks j with j % stride == first.
+template <int KL>
+__device__ __forceinline__ void thread_write_selection(const uint32_t (&pk)[KL],
+                                                       const int (&pi)[KL], int k, int first,
+                                                       int stride, int32_t* idx_row,
+                                                       float* w_row) {
+  constexpr int PW = KL <= 2 ? 2 : KL <= 4 ? 4 : KL <= 8 ? 8 : 16;
+  const float top = key_value(pk[0]);
+  float ex[KL], acc[PW];
+#pragma unroll
+  for (int j = 0; j < PW; ++j) acc[j] = 0.f;
+#pragma unroll
+  for (int j = 0; j < KL; ++j) {
+    ex[j] = (j < k) ? expf(key_value(pk[j]) - top) : 0.f;
+    acc[j] = ex[j];
+  }
+#pragma unroll
+  for (int off = PW / 2; off > 0; off >>= 1) {
+#pragma unroll
+    for (int j = 0; j < off; ++j) acc[j] += acc[j + off];
+  }
+#pragma unroll
+  for (int j = 0; j < KL; ++j) {
+    if (j < k && j % stride == first) {
+      idx_row[j] = pi[j];
+      w_row[j] = ex[j] / acc[0];
+    }
+  }
+}
+
 // This lane's two best entries not yet taken, in (key descending, index ascending) order:
 // entries are scanned in ascending index order and only a strictly larger key displaces one.
 // Lane l holds experts VPL*l + i. Key 0 (no finite float) marks "none".

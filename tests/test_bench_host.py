@@ -48,14 +48,18 @@ def test_stage_costs_fp8_weights_are_one_byte_plus_channel_scales():
 
 
 def test_launches_per_step():
-    # router gate GEMM (or GEMV) + top-k, one grouping launch, the row copy, two expert GEMMs,
-    # the combine
+    # router gate GEMM + top-k, one grouping launch, the row copy, two expert GEMMs, the combine
     assert bench.launches_per_step(W.WORKLOADS["fine"]) == 7
     assert bench.launches_per_step(W.WORKLOADS["decode"].with_tokens(1)) == 7
     assert bench.launches_per_step(W.WORKLOADS["decode"].with_tokens(256)) == 7
-    # skewed: 196608 assignments take the three grouping kernels; every bf16 layer makes the
-    # row copy, whatever I
-    assert bench.launches_per_step(W.WORKLOADS["skewed"]) == 2 + 3 + 1 + 2 + 1
+    # skewed: E = 64 with the hidden dimension in one K range (T = 32768) runs the gate GEMM and
+    # the top-k as one kernel; 196608 assignments group in one cooperative launch; every bf16
+    # layer makes the row copy, whatever I
+    assert bench.route_ksplit(32768, 2048, 64) == 1
+    assert bench.launches_per_step(W.WORKLOADS["skewed"]) == 1 + 1 + 1 + 2 + 1
+    # a short E = 64 batch splits K, so gate GEMM and top-k run separately
+    assert bench.route_ksplit(4096, 2048, 64) == 4
+    assert bench.launches_per_step(W.WORKLOADS["skewed"].with_tokens(4096)) == 2 + 1 + 1 + 2 + 1
     # W8A8: the token rows and the SwiGLU rows are quantised by one launch each
     assert bench.launches_per_step(W.WORKLOADS["fine"], "w8a8") == 9
     # tiny f32: one fused CUDA-core router kernel

@@ -134,6 +134,10 @@ ROUTER = {
     "simt_e8_slabs": W.Workload("r12", 32, 300, 1088, 8, 2, 128, "bf16", 1.25),
     "simt_e64_f32_slabs": W.Workload("r13", 33, 129, 520, 64, 6, 128, "f32", 1.25),
     "simt_e16_t1": W.Workload("r14", 34, 1, 4096, 16, 4, 128, "bf16", 0.0),
+    # E = 64 with one K range: the persistent gate GEMM with the top-k in its epilogue, over
+    # about three tiles per CTA (both TMEM buffers reused) with a ragged last tile
+    "fused_e64_t60000": W.Workload("r15", 35, 60000, 256, 64, 6, 128, "bf16", 1.25),
+    "fused_e64_h2048_k8": W.Workload("r16", 36, 20000, 2048, 64, 8, 128, "bf16", 1.25),
 }
 
 
@@ -158,9 +162,10 @@ def test_router(name):
     check_topk_valid(L_o, idx_g, wl.k, delta, np.nonzero(~dec)[0])
     np.testing.assert_allclose(npi(w_g)[dec], w_o[dec], atol=TOL_W + wl.k * delta, rtol=0)
     # the selection the kernel made is exactly the rule applied to the logits it exported
-    # (checked by the selection-only kernel on the same values, bit for bit)
+    # (checked by the selection-only kernel on the same values, bit for bit, weights included)
     idx_s, w_s = M.route_from_logits(logits_g, wl.k)
     assert torch.equal(idx_s.cpu(), torch.as_tensor(idx_g))
+    assert torch.equal(w_s.view(torch.int32), w_g.view(torch.int32))
 
 
 # ----------------------------------------------------------------- align
