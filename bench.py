@@ -293,12 +293,13 @@ def route_ksplit(T, H, E):
 
 def launches_per_step(wl, weights="bf16"):
     """Kernels one moe_layer_forward launches: router (tensor-core gate GEMM + top-k; one
-    persistent kernel for both when E = 64 and the hidden dimension is one K range; one
-    CUDA-core kernel for E < 64 or f32), align (one launch; three past the cooperative grid's
+    persistent kernel for both when E is 64, 128 or 256 and the hidden dimension is one K range;
+    one CUDA-core kernel for E < 64 or f32), align (one launch; three past the cooperative grid's
     capacity of SMs x 1024 threads x 64 rounds of 32), the expert-major row copy (bf16), the
     W8A8 quantisations, two expert GEMMs, combine."""
     tc = wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0
-    fused = tc and wl.E == 64 and wl.k <= 16 and route_ksplit(wl.T, wl.H, wl.E) == 1
+    fused = (tc and (wl.E == 64 or (wl.E % 128 == 0 and wl.E <= 256)) and wl.k <= 16
+             and route_ksplit(wl.T, wl.H, wl.E) == 1)
     route = 2 if tc and not fused else 1
     align = 1 if wl.T * wl.k <= 148 * 1024 * 64 * 32 else 3
     # expert-major copy of the token rows before GEMM1: every bf16 layer (GEMM1 runs on CTA
@@ -373,6 +374,37 @@ class LayerRun:
 
     def step(self):
         self.forward(self.inp["x"], self.outs)
+
+    def graph_time(self, steps, warmup, world):
+        """The same layer call captured once in a CUDA graph (on a side stream) and replayed
+        per step, as a serving loop for short batches would run it: the launches' host cost and
+        the gaps between them leave the timed region. Returns ms per step (max over ranks)."""
+        side = torch.cuda.Stream(self.dev)
+        side.wait_stream(torch.cuda.current_stream(self.dev))
+        saved = self.stream
+        self.stream = side
+        with torch.cuda.stream(side):
+            self.step()  # first call on this stream: tensor maps and attributes set up
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            self.step()
+        self.stream = saved
+        for _ in range(warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(steps):
+            graph.replay()
+        b.record()
+        torch.cuda.synchronize()
+        self.ws.check()
+        del graph
+        return max_over_ranks(a.elapsed_time(b), world, "cuda") / steps
 
     def time_stages(self, steps, warmup, world, local, peaks):
         """Device-resident timing: total CUDA-event time over `steps` layer calls (max over
@@ -481,6 +513,15 @@ def other_workloads(args, dev, world, local, peaks):
                     "kept_assignments": int(t["cnt"].sum()),
                     "experts_used": int((t["cnt"] > 0).sum()),
                     "gpu_launches": launches_per_step(wl) * args.steps}
+        if wl.T <= 256:
+            # decode batches are launch-bound: also the call captured in a CUDA graph
+            ms = run.graph_time(args.steps, args.warmup, world)
+            res[key]["graph"] = {"value": round(aggregate_throughput(wl.T * args.steps, world,
+                                                                     ms * args.steps / 1e3), 1),
+                                 "unit": "tokens/s", "ms_per_step": round(ms, 4),
+                                 "how": "the layer call captured once in a CUDA graph on a side "
+                                        "stream and replayed per step; CUDA events around the "
+                                        "replays"}
         run.release()
     return res
 

@@ -20,6 +20,7 @@
 
 #include <mutex>
 #include <string>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -260,21 +261,24 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   }
 }
 
-// Gate GEMM and plain top-k in one persistent kernel, for E = 64 with the whole hidden
-// dimension in one K range (large T) on single CTAs: the selection that topk_lanes_kernel would
-// run after a round trip of fp32 logits through memory runs in the epilogue warps instead, on
-// one tile's logits while the MMAs of the CTA's next tile run (two TMEM accumulator sets, each
-// the even/odd K-step pair of route_gemm_kernel). Epilogue thread q * 32 + lane owns TMEM lane
-// (token) q * 32 + lane of the tile: it reads its E logits (the two K-step accumulators added,
-// as in route_gemm_kernel), adds the bias, writes the logits when asked, inserts them in
-// ascending expert order into a TopList and writes the picks and their weights, so the result
-// equals the two-kernel router's bit for bit.
-template <int KL>
+// Gate GEMM and plain top-k in one persistent kernel, for the whole hidden dimension in one K
+// range (large T): E = 64 on single CTAs, or E = 128 / 256 on CTA pairs (the pair protocol of
+// route_gemm_kernel). The selection that a top-k kernel would run after a round trip of fp32
+// logits through memory runs in the epilogue warps instead, on one tile's logits while the MMAs
+// of the CTA's next tile run: two TMEM accumulator buffers (each the even/odd K-step pair of
+// route_gemm_kernel when N <= 128, else one accumulator of N columns). Epilogue thread
+// q * 32 + lane owns TMEM lane (token) q * 32 + lane of its CTA's rows: it reads its logits 32
+// experts at a time (the two K-step accumulators added, as in route_gemm_kernel), adds the
+// bias, writes the logits when asked and inserts them in ascending expert order into a
+// TopList, then writes the picks and their weights; the result equals the two-kernel router's
+// bit for bit. The buffer goes back to the MMA issuer after the last 32-expert chunk is read.
+template <int KL, bool PAIR>
 __global__ void __launch_bounds__(kRtThreads, 1)
     route_gemm_topk_kernel(const __grid_constant__ CUtensorMap tmX,
                            const __grid_constant__ CUtensorMap tmW, const RtParams p,
-                           const float* __restrict__ bias, float* __restrict__ logits_out, int k,
-                           int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+                           int tmem_cols, const float* __restrict__ bias,
+                           float* __restrict__ logits_out, int k, int32_t* __restrict__ topk_idx,
+                           float* __restrict__ topk_w) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -291,6 +295,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = (rank == 0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
@@ -298,43 +304,66 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&tfull[b]), 1);
-      mbar_init(smem_u32(&tempty[b]), 4);  // one arrival per epilogue warp
+      // one arrival per epilogue warp (of both CTAs in PAIR mode, on the even CTA's barrier)
+      mbar_init(smem_u32(&tempty[b]), PAIR ? 8 : 4);
     }
     mbar_init(smem_u32(done), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), kRtTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_holder), static_cast<uint32_t>(tmem_cols));
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_holder), static_cast<uint32_t>(tmem_cols));
+      tmem_relinquish();
+    }
   }
   pdl_enter<false>();
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // both CTAs' barriers are initialised
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int ntiles = (p.T + kRtM - 1) / kRtM;
+  constexpr int kTileRows = PAIR ? 2 * kRtM : kRtM;
+  const int ntiles = (p.T + kTileRows - 1) / kTileRows;
+  const int tile0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int tstep = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   const int nkb = p.kb_per_split;  // the whole hidden dimension
+  const int cb = p.two_acc ? 2 * p.npad : p.npad;  // TMEM columns per accumulator buffer
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t s = 0, ph = 0;
-      const uint32_t tx = static_cast<uint32_t>(stage_bytes);
+      // in PAIR mode the even CTA's barrier expects both CTAs' bytes
+      const uint32_t tx = static_cast<uint32_t>(stage_bytes) * (PAIR ? 2u : 1u);
+      const int c0 = static_cast<int>(rank) * p.nch;  // first expert chunk this CTA loads
       bool ok = true;
       int issued = 0;
-      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+      for (int tile = tile0; ok && tile < ntiles; tile += tstep) {
+        const int row0 = tile * kTileRows + static_cast<int>(rank) * kRtM;
         for (int i = 0; i < nkb; ++i) {
           if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
           const uint32_t sa = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
-          const uint32_t fb = smem_u32(&full[s]);
           const int kc = i * kRtBK;
-          mbar_arrive_expect_tx(fb, tx);
-          tma_load_2d(sa, &tmX, kc, tile * kRtM, fb);
-          for (int c = 0; c < p.nch; ++c) tma_load_2d(sa + 16384 + c * 8192, &tmW, c * 64, kc, fb);
+          if constexpr (PAIR) {
+            const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
+            if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), tx);
+            tma_load_2d_pair(sa, &tmX, kc, row0, fb);
+            for (int c = 0; c < p.nch; ++c)
+              tma_load_2d_pair(sa + 16384 + c * 8192, &tmW, (c0 + c) * 64, kc, fb);
+          } else {
+            const uint32_t fb = smem_u32(&full[s]);
+            mbar_arrive_expect_tx(fb, tx);
+            tma_load_2d(sa, &tmX, kc, row0, fb);
+            for (int c = 0; c < p.nch; ++c)
+              tma_load_2d(sa + 16384 + c * 8192, &tmW, (c0 + c) * 64, kc, fb);
+          }
           ++issued;
           if (++s == static_cast<uint32_t>(S)) {
             s = 0;
@@ -346,77 +375,88 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         *abort_flag = 1;
         flag_error(p.err, kDevWaitTimeout);
       }
-      // every load issued lands before the CTA may exit
-      for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
-        mbar_wait(smem_u32(&full[i % S]), static_cast<uint32_t>(i / S) & 1u, nullptr);
+      // Every load issued lands before the CTA may exit. In PAIR mode the loads complete on the
+      // even CTA's barriers; the cluster barrier at the end keeps the odd CTA alive until then.
+      if (!PAIR || leader) {
+        for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
+          mbar_wait_cluster(smem_u32(&full[i % S]), static_cast<uint32_t>(i / S) & 1u, nullptr);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (whole warp)
-    constexpr uint32_t kFull = 0xffffffffu;
-    const uint32_t sbase = smem_u32(smem);
-    const uint64_t adesc0 = smem_desc_sw128(sbase, 16, 1024);            // x rows, K-major
-    const uint64_t bdesc0 = smem_desc_sw128(sbase + 16384, 8192, 1024);  // Wr, MN-major
-    const uint32_t idesc = idesc_bf16(kRtM, p.npad, /*a_mn_major=*/false, /*b_mn_major=*/true);
-    uint32_t s = 0, ph = 0, soff = 0;
-    bool ok = true;
-    int tc = 0;
-    for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tc) {
-      const int buf = tc & 1;
-      const uint32_t use = static_cast<uint32_t>(tc >> 1);
-      if (!__all_sync(kFull, mbar_wait(smem_u32(&tempty[buf]), (use & 1u) ^ 1u, abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // two accumulators per buffer: even and odd K steps (npad <= 64 columns each)
-      const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * 128);
-      const uint32_t d1 = d0 + static_cast<uint32_t>(p.npad);
-      uint32_t acc0 = 0, acc1 = 0;
-      for (int i = 0; i < nkb; ++i) {
-        if (!__all_sync(kFull, mbar_wait(smem_u32(&full[s]), ph, abort_flag))) {
+    if (leader) {
+      constexpr uint32_t kFull = 0xffffffffu;
+      const uint32_t sbase = smem_u32(smem);
+      const uint64_t adesc0 = smem_desc_sw128(sbase, 16, 1024);            // x rows, K-major
+      const uint64_t bdesc0 = smem_desc_sw128(sbase + 16384, 8192, 1024);  // Wr, MN-major
+      const uint32_t idesc = idesc_bf16(kTileRows, p.npad, /*a_mn_major=*/false,
+                                        /*b_mn_major=*/true);
+      uint32_t s = 0, ph = 0, soff = 0;
+      bool ok = true;
+      int tc = 0;
+      for (int tile = tile0; ok && tile < ntiles; tile += tstep, ++tc) {
+        const int buf = tc & 1;
+        const uint32_t use = static_cast<uint32_t>(tc >> 1);
+        if (!__all_sync(kFull, mbar_wait_cluster(smem_u32(&tempty[buf]), (use & 1u) ^ 1u,
+                                                 abort_flag))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t ad = adesc0 + (soff >> 4);
-        const uint64_t bd = bdesc0 + (soff >> 4);
+        const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf * cb);
+        const uint32_t d1 = d0 + static_cast<uint32_t>(p.npad);
+        uint32_t acc0 = 0, acc1 = 0;
+        for (int i = 0; i < nkb; ++i) {
+          if (!__all_sync(kFull, mbar_wait_cluster(smem_u32(&full[s]), ph, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = adesc0 + (soff >> 4);
+          const uint64_t bd = bdesc0 + (soff >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kRtBK / 16; ++kk) {
-          const bool second = kk & 1;
-          tc_mma_bf16_elect(second ? d1 : d0, ad + kk * 2, bd + kk * 128, idesc,
-                            second ? acc1 : acc0);
-          if (second) acc1 = 1u;
-          else acc0 = 1u;
+          for (int kk = 0; kk < kRtBK / 16; ++kk) {
+            const bool second = p.two_acc && (kk & 1);
+            const uint32_t d = second ? d1 : d0;
+            const uint32_t acc = second ? acc1 : acc0;
+            if constexpr (PAIR) tc_mma_bf16_pair_elect(d, ad + kk * 2, bd + kk * 128, idesc, acc);
+            else tc_mma_bf16_elect(d, ad + kk * 2, bd + kk * 128, idesc, acc);
+            if (second) acc1 = 1u;
+            else acc0 = 1u;
+          }
+          if constexpr (PAIR) tc_commit_pair_mc_elect(smem_u32(&empty[s]), 0x3);
+          else tc_commit_elect(smem_u32(&empty[s]));
+          if (++s == static_cast<uint32_t>(S)) {
+            s = 0;
+            ph ^= 1u;
+            soff = 0;
+          } else {
+            soff += static_cast<uint32_t>(stage_bytes);
+          }
         }
-        tc_commit_elect(smem_u32(&empty[s]));
-        if (++s == static_cast<uint32_t>(S)) {
-          s = 0;
-          ph ^= 1u;
-          soff = 0;
-        } else {
-          soff += static_cast<uint32_t>(stage_bytes);
-        }
+        if (!ok) break;
+        if constexpr (PAIR) tc_commit_pair_mc_elect(smem_u32(&tfull[buf]), 0x3);
+        else tc_commit_elect(smem_u32(&tfull[buf]));
       }
-      if (!ok) break;
-      tc_commit_elect(smem_u32(&tfull[buf]));
+      if (!ok && lane == 0) {
+        *abort_flag = 1;
+        flag_error(p.err, kDevWaitTimeout);
+      }
+      // completes once every MMA issued has finished (also when the loop stopped early)
+      if constexpr (PAIR) tc_commit_pair_mc_elect(smem_u32(done), 0x3);
+      else tc_commit_elect(smem_u32(done));
     }
-    if (!ok && lane == 0) {
-      *abort_flag = 1;
-      flag_error(p.err, kDevWaitTimeout);
-    }
-    // completes once every MMA issued has finished (also when the loop stopped early)
-    tc_commit_elect(smem_u32(done));
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue + top-k (warps 2..5)
     const int q = warp & 3;
     int tc = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+    for (int tile = tile0; tile < ntiles; tile += tstep, ++tc) {
       const int buf = tc & 1;
       const uint32_t use = static_cast<uint32_t>(tc >> 1);
       int got = 1;
-      if (lane == 0) got = mbar_wait(smem_u32(&tfull[buf]), use & 1u, abort_flag) ? 1 : 0;
+      if (lane == 0) got = mbar_wait_cluster(smem_u32(&tfull[buf]), use & 1u, abort_flag) ? 1 : 0;
       got = __shfl_sync(0xffffffffu, got, 0);
       if (!got) {
         if (lane == 0) {
@@ -427,47 +467,55 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       }
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                          static_cast<uint32_t>(buf * 128);
-      float lg[64];
-#pragma unroll
-      for (int c0 = 0; c0 < 64; c0 += 32) {
-        if (c0 < p.E) {  // uniform
-          uint32_t v[32], u[32];
-          tmem_ld32(tb + static_cast<uint32_t>(c0), v);
+                          static_cast<uint32_t>(buf * cb);
+      const int64_t t = static_cast<int64_t>(tile) * kTileRows + static_cast<int>(rank) * kRtM +
+                        q * 32 + lane;
+      const bool mine = t < p.T;
+      TopList<KL> L;
+      L.clear();
+      for (int c0 = 0; c0 < p.E; c0 += 32) {  // uniform; E % 32 == 0
+        uint32_t v[32];
+        tmem_ld32(tb + static_cast<uint32_t>(c0), v);
+        if (p.two_acc) {
+          uint32_t u[32];
           tmem_ld32(tb + static_cast<uint32_t>(p.npad + c0), u);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) lg[c0 + j] = __uint_as_float(v[j]) + __uint_as_float(u[j]);
+          for (int j = 0; j < 32; ++j)
+            v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(u[j]));
+        } else {
+          tmem_wait_ld();
+        }
+        if (mine) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int e = c0 + j;
+            float val = __uint_as_float(v[j]);
+            if (bias != nullptr) val += __ldg(bias + e);
+            if (logits_out != nullptr) logits_out[t * p.E + e] = val;
+            L.insert(order_key(val), e);
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
-      const int64_t t = static_cast<int64_t>(tile) * kRtM + q * 32 + lane;
-      if (t < p.T) {
-        TopList<KL> L;
-        L.clear();
-#pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          if (e < p.E) {
-            float v = lg[e];
-            if (bias != nullptr) v += __ldg(bias + e);
-            if (logits_out != nullptr) logits_out[t * p.E + e] = v;
-            L.insert(order_key(v), e);
-          }
-        }
-        thread_write_selection<KL>(L.key, L.idx, k, 0, 1, topk_idx + t * k, topk_w + t * k);
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
+        else mbar_arrive(smem_u32(&tempty[buf]));
       }
+      if (mine) thread_write_selection<KL>(L.key, L.idx, k, 0, 1, topk_idx + t * k, topk_w + t * k);
     }
   }
 
-  // TMEM is released only after every MMA issued has completed
-  if (warp == 1 && lane == 0) mbar_wait(smem_u32(done), 0u, nullptr);
+  // TMEM is released only after every MMA issued has completed (the commit reaches both CTAs)
+  if (warp == 1 && lane == 0) mbar_wait_cluster(smem_u32(done), 0u, nullptr);
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // no CTA leaves while its peer may still signal it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kRtTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, static_cast<uint32_t>(tmem_cols));
+    else tmem_dealloc(tmem_base, static_cast<uint32_t>(tmem_cols));
   }
 }
 
@@ -572,7 +620,8 @@ cudaError_t launch_route_gemm_tc(const void* x, const void* w_router, int T, int
 }
 
 bool route_fuses_topk(int64_t T, int H, int E, int k, int n_group) {
-  return E == 64 && n_group <= 1 && k <= 16 && H % kRtBK == 0 && route_ksplit(T, H, E) == 1;
+  const bool shape_ok = E == 64 || (E % 128 == 0 && E <= 256);
+  return shape_ok && n_group <= 1 && k <= 16 && H % kRtBK == 0 && route_ksplit(T, H, E) == 1;
 }
 
 cudaError_t launch_route_gemm_topk_tc(const void* x, const void* w_router, int T, int H, int E,
@@ -580,7 +629,8 @@ cudaError_t launch_route_gemm_topk_tc(const void* x, const void* w_router, int T
                                       int32_t* topk_idx, float* topk_w, int* err, int num_sms,
                                       cudaStream_t stream, std::string* detail) {
   if (T == 0) return cudaSuccess;
-  if (E != 64 || H % kRtBK != 0 || k < 1 || k > 16) {
+  const bool pair = route_uses_pairs(E);
+  if (!(E == 64 || (pair && E <= 256)) || H % kRtBK != 0 || k < 1 || k > 16) {
     if (detail) *detail = "fused router shape outside the tensor-core path";
     return cudaErrorInvalidValue;
   }
@@ -593,31 +643,39 @@ cudaError_t launch_route_gemm_topk_tc(const void* x, const void* w_router, int T
   p.H = H;
   p.E = E;
   p.npad = E;
-  p.nch = 1;
+  p.nch = pair ? E / 128 : E / 64;
   p.kb_per_split = H / kRtBK;
-  p.two_acc = 1;
+  p.two_acc = (E <= 128) ? 1 : 0;  // two K-step accumulators per buffer while 2E <= 256
   p.split_stride = 0;
   p.out = nullptr;
   p.err = err;
-  const int stage_bytes = 16384 + 8192;
+  // two accumulator buffers: 2 * (2E or E) columns, a power of two (256 or 512)
+  const int tmem_cols = 2 * (p.two_acc ? 2 * E : E);
+  const int stage_bytes = 16384 + p.nch * 8192;
   int stages = (kRtSmemLimit - 1024 - kRtCtrl) / stage_bytes;
   if (stages > kRtMaxStages) stages = kRtMaxStages;
   if (stages > p.kb_per_split) stages = p.kb_per_split;
   if (stages < 2) stages = 2;
   p.stages = stages;
   const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + kRtCtrl;
-  auto kernel = route_gemm_topk_kernel<16>;
-  if (k <= 2) kernel = route_gemm_topk_kernel<2>;
-  else if (k <= 4) kernel = route_gemm_topk_kernel<4>;
-  else if (k <= 6) kernel = route_gemm_topk_kernel<6>;
-  else if (k <= 8) kernel = route_gemm_topk_kernel<8>;
+  auto pick = [&](auto tag) {
+    constexpr bool P = decltype(tag)::value;
+    auto kernel = route_gemm_topk_kernel<16, P>;
+    if (k <= 2) kernel = route_gemm_topk_kernel<2, P>;
+    else if (k <= 4) kernel = route_gemm_topk_kernel<4, P>;
+    else if (k <= 6) kernel = route_gemm_topk_kernel<6, P>;
+    else if (k <= 8) kernel = route_gemm_topk_kernel<8, P>;
+    return kernel;
+  };
+  auto kernel = pair ? pick(std::true_type{}) : pick(std::false_type{});
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int tiles = (T + kRtM - 1) / kRtM;
-  const int grid = tiles < num_sms ? tiles : num_sms;
+  const int tiles = pair ? (T + 2 * kRtM - 1) / (2 * kRtM) : (T + kRtM - 1) / kRtM;
+  const int units = pair ? num_sms / 2 : num_sms;
+  const int grid = (tiles < units ? tiles : units) * (pair ? 2 : 1);
   return launch_kernel(kernel, dim3(static_cast<unsigned>(grid)), dim3(kRtThreads), smem, stream,
-                       1, mx, mw, p, bias, logits_out, k, topk_idx, topk_w);
+                       pair ? 2 : 1, mx, mw, p, tmem_cols, bias, logits_out, k, topk_idx, topk_w);
 }
 
 }  // namespace moe

@@ -57,6 +57,9 @@ def test_launches_per_step():
     # layer makes the row copy, whatever I
     assert bench.route_ksplit(32768, 2048, 64) == 1
     assert bench.launches_per_step(W.WORKLOADS["skewed"]) == 1 + 1 + 1 + 2 + 1
+    # fine-grained at T = 32768: one K range on CTA pairs, gate GEMM and top-k fused
+    assert bench.route_ksplit(32768, 4096, 256) == 1
+    assert bench.launches_per_step(W.WORKLOADS["fine"].with_tokens(32768)) == 1 + 1 + 1 + 2 + 1
     # a short E = 64 batch splits K, so gate GEMM and top-k run separately
     assert bench.route_ksplit(4096, 2048, 64) == 4
     assert bench.launches_per_step(W.WORKLOADS["skewed"].with_tokens(4096)) == 2 + 1 + 1 + 2 + 1

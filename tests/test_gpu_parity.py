@@ -138,6 +138,9 @@ ROUTER = {
     # about three tiles per CTA (both TMEM buffers reused) with a ragged last tile
     "fused_e64_t60000": W.Workload("r15", 35, 60000, 256, 64, 6, 128, "bf16", 1.25),
     "fused_e64_h2048_k8": W.Workload("r16", 36, 20000, 2048, 64, 8, 128, "bf16", 1.25),
+    # the same on CTA pairs: E = 256 over about three 256-token tiles per pair, E = 128
+    "fused_pairs_e256_t60000": W.Workload("r17", 38, 60000, 256, 256, 8, 128, "bf16", 1.25),
+    "fused_pairs_e128": W.Workload("r18", 39, 40000, 512, 128, 6, 128, "bf16", 1.25),
 }
 
 
@@ -507,11 +510,25 @@ def test_combine_fine_every_token():
           % (wl.T, int(al["drop_mask"].sum()), r))
 
 
-def test_layer_call_captured_in_a_cuda_graph_replays_identically():
+GRAPH_SHAPES = {
+    "e256_k8": None,
+    # E = 64 with one K range and 72000 assignments: the fused gate GEMM + top-k and the
+    # cooperative one-launch grouping inside the graph
+    "fused_router_grid_align": W.Workload("g1", 37, 12000, 256, 64, 6, 128, "bf16", 1.25),
+}
+
+
+@pytest.mark.parametrize("name", list(GRAPH_SHAPES))
+def test_layer_call_captured_in_a_cuda_graph_replays_identically(name):
     """The layer call makes no host synchronisation and launches only on its stream, so a serving
     loop can capture it in a CUDA graph: replays give the eager call's results bit for bit, for
     new inputs copied into the captured buffers too."""
-    wl, cpu, dev = small_inputs("e256_k8")
+    if GRAPH_SHAPES[name] is None:
+        wl, cpu, dev = small_inputs(name)
+    else:
+        wl = GRAPH_SHAPES[name]
+        cpu = W.make_inputs(wl, "cpu")
+        dev = {k: (None if v is None else v.cuda()) for k, v in cpu.items()}
     shape = M.shape_of(wl.T, wl.H, wl.E, wl.k, wl.I, wl.capacity_factor, wl.dtype)
     ws = M.Workspace(shape, "cuda")
     x = dev["x"].clone()
