@@ -124,6 +124,46 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int& total) 
   return warp_base + inc - v;
 }
 
+// Two exclusive block-wide scans at once (NW warps, NW <= 32; sh2 holds NW int2): returns the
+// prefix of a, sets b_prefix, and the totals of a and b.
+template <int NW>
+__device__ __forceinline__ int block_exclusive_scan2(int a, int b, int2* sh2, int& total_a,
+                                                     int& total_b, int& b_prefix) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int ia = a, ib = b;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int oa = __shfl_up_sync(0xffffffffu, ia, off);
+    const int ob = __shfl_up_sync(0xffffffffu, ib, off);
+    if (lane >= off) {
+      ia += oa;
+      ib += ob;
+    }
+  }
+  if (lane == 31) sh2[warp] = make_int2(ia, ib);
+  __syncthreads();
+  if (warp == 0) {
+    int2 w = (lane < NW) ? sh2[lane] : make_int2(0, 0);
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int oa = __shfl_up_sync(0xffffffffu, w.x, off);
+      const int ob = __shfl_up_sync(0xffffffffu, w.y, off);
+      if (lane >= off) {
+        w.x += oa;
+        w.y += ob;
+      }
+    }
+    if (lane < NW) sh2[lane] = w;  // inclusive warp totals
+  }
+  __syncthreads();
+  const int2 wb = (warp > 0) ? sh2[warp - 1] : make_int2(0, 0);
+  total_a = sh2[NW - 1].x;
+  total_b = sh2[NW - 1].y;
+  __syncthreads();
+  b_prefix = wb.y + ib - b;
+  return wb.x + ia - a;
+}
+
 // Chunk bases, counts, offsets and the token-block plan, one block of kScanThreads threads.
 // Thread (s, e), tid = s * Ep + e (Ep = E rounded up to a power of two, S = kScanThreads / Ep
 // splits capped at kScanMaxSplit), owns the chunks [s*per, (s+1)*per) of expert e: it sums them
@@ -450,15 +490,16 @@ __global__ void __launch_bounds__(kGridThreads, 1)
                       uint8_t* __restrict__ drop_mask, int* err) {
   constexpr int NT = kGridThreads, NW = NT / 32, kBatch = 8;
   pdl_enter<false>();
-  __shared__ int wrun[NW][kMaxE];
+  __shared__ int wrun[NW][kMaxE + 1];  // padded: a warp reads one column without conflicts
   __shared__ int s_off[kMaxE];
+  __shared__ int s_base[kMaxE];        // this CTA's base per expert (totals of CTAs before it)
   __shared__ int part[2][NT];
-  __shared__ int sh[NW];
+  __shared__ int2 sh2[NW];
   __shared__ int s_ok;
   extern __shared__ uint16_t code_sm[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = static_cast<int>(blockIdx.x), G = static_cast<int>(gridDim.x);
-  for (int i = threadIdx.x; i < NW * kMaxE; i += NT) (&wrun[0][0])[i] = 0;
+  for (int i = threadIdx.x; i < NW * (kMaxE + 1); i += NT) (&wrun[0][0])[i] = 0;
   // A <= G * NT * kGridMaxSteps (checked by the launcher): 32-bit indices suffice
   const int An = static_cast<int>(A);
   const int steps = ((An + G * NW - 1) / (G * NW) + 31) / 32;
@@ -488,17 +529,18 @@ __global__ void __launch_bounds__(kGridThreads, 1)
     if (c != 0xFFFFu) atomicAdd(&wrun[warp][c], 1);
   }
   __syncthreads();
-  // 2. per expert: exclusive prefix across this CTA's warps; the CTA's total to hist[r]
-  if (threadIdx.x < E) {
-    const int e = threadIdx.x;
-    int mine = 0;
+  // 2. per expert: exclusive prefix across this CTA's warps, warp-parallel (warp w takes
+  //    experts w, w + 32, ...; lane = source warp); the CTA's total to hist[r]
+  for (int e = warp; e < E; e += NW) {
+    const int c = wrun[lane][e];
+    int inc = c;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const int c = wrun[w][e];
-      wrun[w][e] = mine;
-      mine += c;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += o;
     }
-    hist[static_cast<size_t>(r) * E + e] = mine;
+    wrun[lane][e] = inc - c;
+    if (lane == 31) hist[static_cast<size_t>(r) * E + e] = inc;
   }
   // 3. grid barrier: every CTA's totals are written before any CTA reads them
   __syncthreads();
@@ -556,19 +598,16 @@ __global__ void __launch_bounds__(kGridThreads, 1)
   const int cnt = (threadIdx.x < E) ? min(raw_tot, C) : 0;
   const int nb = (cnt + TB - 1) / TB;
   int tot_cnt, tot_nb;
-  const int off = block_exclusive_scan<NW>(cnt, sh, tot_cnt);
-  const int bp = block_exclusive_scan<NW>(nb, sh, tot_nb);
+  int bp;
+  const int off = block_exclusive_scan2<NW>(cnt, nb, sh2, tot_cnt, tot_nb, bp);
   if (threadIdx.x < E) {
     const int ee = threadIdx.x;
     s_off[ee] = off;
+    s_base[ee] = before;
     if (r == 0) {
       counts[ee] = cnt;
       offsets[ee] = off;
       if (blk_prefix != nullptr) blk_prefix[ee] = bp;
-    }
-    if (before != 0) {
-#pragma unroll
-      for (int w = 0; w < NW; ++w) wrun[w][ee] += before;
     }
   }
   if (threadIdx.x == 0 && r == 0) {
@@ -585,7 +624,7 @@ __global__ void __launch_bounds__(kGridThreads, 1)
     const int ea = static_cast<int>(c);
     const uint32_t peers = warp_peers(c, ok, nbits);
     int rank = 0;
-    if (ok) rank = wrun[warp][ea] + __popc(peers & lanemask_lt());
+    if (ok) rank = s_base[ea] + wrun[warp][ea] + __popc(peers & lanemask_lt());
     __syncwarp();
     if (ok && lane == __ffs(peers) - 1) wrun[warp][ea] += __popc(peers);
     __syncwarp();

@@ -48,12 +48,14 @@ __device__ __forceinline__ void load_run(const float* p, bool vec, bool in, floa
   }
 }
 
-// Partial sums in ascending K-range order. Four K ranges are loaded per group with no branch
-// between the loads, so one group costs one memory latency. vec: E % VPL == 0, so a lane's run
-// of VPL logits is one or two aligned vector loads (rows start on 16-byte boundaries then);
-// otherwise a lane with experts past E reads only those below E.
-template <int VPL>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
+// Partial sums in ascending K-range order. GROUP K ranges are loaded per group with no branch
+// between the loads, so one group costs one memory latency: 4 for the usual split, 16 (every
+// range of a short batch at once, where few warps run and registers are plentiful) when the
+// K split is deeper. vec: E % VPL == 0, so a lane's run of VPL logits is one or two aligned
+// vector loads (rows start on 16-byte boundaries then); otherwise a lane with experts past E
+// reads only those below E.
+template <int VPL, int GROUP>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, GROUP == 4 ? 4 : 1)
     topk_kernel(const float* __restrict__ partials, int ksplit, int64_t split_stride,
                 const float* __restrict__ bias, float* __restrict__ logits_out, int64_t T, int E,
                 int k, int n_group, int topk_group, int32_t* __restrict__ topk_idx,
@@ -73,10 +75,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
     v[i] = 0.f;
     if (e0 + i >= E) taken |= 1u << i;
   }
-  for (int ks0 = 0; ks0 < ksplit; ks0 += 4) {
-    float p[4][VPL];
+  for (int ks0 = 0; ks0 < ksplit; ks0 += GROUP) {
+    float p[GROUP][VPL];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < GROUP; ++j) {
       const bool in = ks0 + j < ksplit;
       if (full) {
         load_run<VPL>(row + (ks0 + j) * split_stride, vec, in, p[j]);
@@ -87,7 +89,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 4)
       }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < GROUP; ++j) {
       if (ks0 + j < ksplit) {
 #pragma unroll
         for (int i = 0; i < VPL; ++i) v[i] = (ks0 + j == 0) ? p[j][i] : v[i] + p[j][i];
@@ -673,10 +675,13 @@ cudaError_t launch_topk(const float* partials, int ksplit, int64_t split_stride,
   }
   const unsigned grid = static_cast<unsigned>((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
   const unsigned block = kWarpsPerBlock * 32;
-  auto kernel = topk_kernel<8>;
-  if (E <= 32) kernel = topk_kernel<1>;
-  else if (E <= 64) kernel = topk_kernel<2>;
-  else if (E <= 128) kernel = topk_kernel<4>;
+  // short batch (at most one warp per token for 1024 tokens: one block per SM suffices): every
+  // K range in one batch of loads
+  const bool deep = ksplit > 4 && T <= 1024;
+  auto kernel = deep ? topk_kernel<8, 16> : topk_kernel<8, 4>;
+  if (E <= 32) kernel = deep ? topk_kernel<1, 16> : topk_kernel<1, 4>;
+  else if (E <= 64) kernel = deep ? topk_kernel<2, 16> : topk_kernel<2, 4>;
+  else if (E <= 128) kernel = deep ? topk_kernel<4, 16> : topk_kernel<4, 4>;
   return launch_kernel(kernel, dim3(grid), dim3(block), 0, stream, 1, partials, ksplit,
                        split_stride, bias, logits_out, T, E, k, n_group, topk_group, topk_idx,
                        topk_w);

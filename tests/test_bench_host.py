@@ -50,8 +50,8 @@ def test_stage_costs_fp8_weights_are_one_byte_plus_channel_scales():
 def test_launches_per_step():
     # router gate GEMM + top-k, one grouping launch, the row copy, two expert GEMMs, the combine
     assert bench.launches_per_step(W.WORKLOADS["fine"]) == 7
-    assert bench.launches_per_step(W.WORKLOADS["decode"].with_tokens(1)) == 7
     assert bench.launches_per_step(W.WORKLOADS["decode"].with_tokens(256)) == 7
+    assert bench.launches_per_step(W.WORKLOADS["decode"].with_tokens(1)) == 7
     # skewed: E = 64 with the hidden dimension in one K range (T = 32768) runs the gate GEMM and
     # the top-k as one kernel; 196608 assignments group in one cooperative launch; every bf16
     # layer makes the row copy, whatever I

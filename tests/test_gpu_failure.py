@@ -35,3 +35,30 @@ def test_stalled_wait_ends_with_a_device_error_and_the_context_stays_usable():
     assert ws.check() == L.MOE_OK
     al = orc.align(idx.cpu().numpy(), 8, orc.capacity(64, 2, 8, 1.25))
     assert np.array_equal(res["slot_of"].cpu().numpy(), al["slot_of"])
+
+
+def test_check_error_clears_the_whole_control_block():
+    """A device error may leave the one-launch grouping's grid-barrier counters (control-block
+    words 32 and 33) off zero; moe_check_error clears all 256 bytes with the error word. Planted
+    on the host: an error code and stale counters written into the block, no kernel faulted.
+    After the check, a grouping that uses the grid barrier (98304 assignments) matches the
+    oracle and leaves the block at zero."""
+    T, E, k = 16384, 64, 6
+    shape = L.make_shape(T, 128, E, k, 128, 1.25, "bf16")
+    ws = M.Workspace(shape, "cuda")
+    block = ws.buf[:256].view(torch.int32)
+    block[0] = 2
+    block[32] = 77
+    block[33] = 5
+    with pytest.raises(L.MoeError) as ei:
+        ws.check()
+    assert ei.value.status == L.MOE_ERR_DEVICE
+    assert torch.count_nonzero(ws.buf[:256]).item() == 0
+    idx = W.random_topk_idx(T, E, k, seed=11, mode="zipf").cuda()
+    res = M.align(idx, E, 1.25, ws=ws)
+    torch.cuda.synchronize()
+    assert ws.check() == L.MOE_OK
+    al = orc.align(idx.cpu().numpy(), E, orc.capacity(T, k, E, 1.25))
+    for key in ("counts", "offsets", "sorted_ids", "slot_of", "drop_mask"):
+        assert np.array_equal(res[key].cpu().numpy(), al[key]), key
+    assert torch.count_nonzero(ws.buf[:256]).item() == 0

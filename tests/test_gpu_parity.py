@@ -138,6 +138,9 @@ ROUTER = {
     # about three tiles per CTA (both TMEM buffers reused) with a ragged last tile
     "fused_e64_t60000": W.Workload("r15", 35, 60000, 256, 64, 6, 128, "bf16", 1.25),
     "fused_e64_h2048_k8": W.Workload("r16", 36, 20000, 2048, 64, 8, 128, "bf16", 1.25),
+    # short batches: every K range's partials summed in one batch of loads
+    "short_t5_e64": W.Workload("r19", 40, 5, 2048, 64, 6, 128, "bf16", 0.0),
+    "short_t16_e256_pairs": W.Workload("r20", 41, 16, 4096, 256, 8, 128, "bf16", 1.25),
     # the same on CTA pairs: E = 256 over about three 256-token tiles per pair, E = 128
     "fused_pairs_e256_t60000": W.Workload("r17", 38, 60000, 256, 256, 8, 128, "bf16", 1.25),
     "fused_pairs_e128": W.Workload("r18", 39, 40000, 512, 128, 6, 128, "bf16", 1.25),

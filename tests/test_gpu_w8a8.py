@@ -33,7 +33,8 @@ def test_pack_w8a8_bitexact(E, K, N):
     assert np.array_equal(npi(codes), np.ascontiguousarray(q_o.transpose(0, 2, 1)))
 
 
-@pytest.mark.parametrize("N,K", [(1, 8), (37, 4096), (300, 2048), (5, 14336)])
+@pytest.mark.parametrize("N,K", [(1, 8), (37, 4096), (300, 2048), (5, 14336), (9, 1000), (3, 4104),
+                                 (7, 8192)])
 def test_quantize_rows_fp8_bitexact(N, K):
     g = torch.Generator().manual_seed(N * 31 + K)
     a = torch.randn((N, K), generator=g) * torch.exp(4 * torch.randn((N, 1), generator=g))
