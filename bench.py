@@ -296,7 +296,7 @@ def launches_per_step(wl, weights="bf16"):
     persistent kernel for both when E is 64, 128 or 256 and the hidden dimension is one K range;
     one CUDA-core kernel for E < 64 or f32), align (one launch; three past the cooperative grid's
     capacity of SMs x 1024 threads x 64 rounds of 32), the expert-major row copy (bf16), the
-    W8A8 quantisations, two expert GEMMs, combine."""
+    W8A8 quantisations, the expert GEMMs, combine."""
     tc = wl.dtype == "bf16" and wl.E >= 64 and wl.E % 8 == 0
     fused = (tc and (wl.E == 64 or (wl.E % 128 == 0 and wl.E <= 256)) and wl.k <= 16
              and route_ksplit(wl.T, wl.H, wl.E) == 1)
@@ -307,7 +307,10 @@ def launches_per_step(wl, weights="bf16"):
     copy = 1 if wl.dtype == "bf16" else 0
     # W8A8: the token rows and the SwiGLU rows are quantised by one launch each
     quant = 2 if weights == "w8a8" else 0
-    return route + align + copy + quant + 2 + 1
+    # bf16 GEMM1 on CTA pairs with I % 256 == 128: the last 128 features on single CTAs
+    gemm1 = 2 if (wl.dtype == "bf16" and weights == "bf16" and wl.I % 256 == 128
+                  and wl.I >= 384) else 1
+    return route + align + copy + quant + gemm1 + 1 + 1
 
 
 def workload_of(args):

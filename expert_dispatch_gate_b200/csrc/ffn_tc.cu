@@ -77,6 +77,7 @@ struct TcParams {
   int K;          // reduction length (multiple of 64)
   int num_fb;     // feature blocks of 128
   int m_valid;    // features stored by the epilogue
+  int m_base;     // first feature of feature block 0
   int TB;         // max tokens per tile, multiple of 32, <= 256
   int groups;     // experts
   int k_top;      // GEMM1: B row = sorted_ids[slot] / k_top
@@ -301,7 +302,7 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
           }
         }
       }
-      const int m0 = t.fb * kTileFeatures + static_cast<int>(rank) * kCtaFeatures;
+      const int m0 = p.m_base + t.fb * kTileFeatures + static_cast<int>(rank) * kCtaFeatures;
       // A: one box per weight operand (all feature chunks of this CTA's rows); B: one box of
       // b_box_rows token rows, or npad gathered rows
       uint32_t tx = static_cast<uint32_t>(W8 ? a8_bytes : a_bytes);
@@ -631,7 +632,8 @@ __global__ void __launch_bounds__(threads_of<BMODE, W8>(), 1)
         break;
       }
       tc_fence_after();
-      const int m = t.fb * kTileFeatures + static_cast<int>(rank) * kCtaFeatures + q * 32 + lane;
+      const int m = p.m_base + t.fb * kTileFeatures + static_cast<int>(rank) * kCtaFeatures +
+                    q * 32 + lane;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(buf * 256);
       // Read every accumulator chunk this warp owns into registers, already rounded to bf16
@@ -942,9 +944,11 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
   if (xs != nullptr) {
     // token rows already in expert-major order: contiguous rows like GEMM2's B operand, so
     // both CTAs of a pair can take their halves by TMA, one box per stage
-    // CTA pairs cover 256 features; when I % 256 == 128 the last pair tile's second CTA reads
-    // only zero-filled weight rows and stores nothing
+    // CTA pairs cover 256 features. When I % 256 == 128 a last pair tile would give its second
+    // CTA only zero-filled weight rows (an eighth of the work wasted at I = 1408), so the pairs
+    // take the first I - 128 features and a second launch of single CTAs the last 128.
     const bool pair = kUsePairs;
+    const bool split = pair && I % 256 == 128 && I >= 384;
     const int box_rows = b_rows_smem(pair, TB);
     if (!map_row_boxes(&b, xs, static_cast<uint64_t>(H), static_cast<uint64_t>(hbuf_rows), detail,
                        static_cast<uint32_t>(box_rows)))
@@ -952,8 +956,9 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
     TcParams p{};
     p.b_box_rows = box_rows;
     p.K = H;
-    p.num_fb = pair ? (I + 255) / 256 : (I + kBM - 1) / kBM;
-    p.m_valid = I;
+    p.num_fb = pair ? (split ? I / 256 : (I + 255) / 256) : (I + kBM - 1) / kBM;
+    p.m_valid = split ? I - 128 : I;
+    p.m_base = 0;
     p.TB = TB;
     p.groups = E;
     p.k_top = 1;
@@ -966,9 +971,24 @@ cudaError_t launch_gemm1_tc(const void* x, int T, const void* xs, const int32_t*
     p.err = err;
     p.b_ptr = nullptr;
     const int64_t tiles = static_cast<int64_t>(p.num_fb) * ub_blocks;
-    if (pair)
-      return launch_mode<kEpiSwiGLU, kBTiled, true>(a0, a1, b, p, tiles, num_sms, stream, detail);
-    return launch_mode<kEpiSwiGLU, kBTiled, false>(a0, a1, b, p, tiles, num_sms, stream, detail);
+    if (!pair)
+      return launch_mode<kEpiSwiGLU, kBTiled, false>(a0, a1, b, p, tiles, num_sms, stream, detail);
+    cudaError_t e =
+        launch_mode<kEpiSwiGLU, kBTiled, true>(a0, a1, b, p, tiles, num_sms, stream, detail);
+    if (e != cudaSuccess || !split) return e;
+    // the last 128 features on single CTAs, each taking its token block's rows whole
+    CUtensorMap b1;
+    const int box1 = b_rows_smem(false, TB);
+    if (!map_row_boxes(&b1, xs, static_cast<uint64_t>(H), static_cast<uint64_t>(hbuf_rows),
+                       detail, static_cast<uint32_t>(box1)))
+      return cudaErrorInvalidValue;
+    TcParams p1 = p;
+    p1.b_box_rows = box1;
+    p1.num_fb = 1;
+    p1.m_base = I - 128;
+    p1.m_valid = I;
+    return launch_mode<kEpiSwiGLU, kBTiled, false>(a0, a1, b1, p1, ub_blocks, num_sms, stream,
+                                                    detail);
   }
   if (!map_rows(&b, x, static_cast<uint64_t>(H), static_cast<uint64_t>(T), detail))
     return cudaErrorInvalidValue;

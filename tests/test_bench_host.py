@@ -56,13 +56,14 @@ def test_launches_per_step():
     # the top-k as one kernel; 196608 assignments group in one cooperative launch; every bf16
     # layer makes the row copy, whatever I
     assert bench.route_ksplit(32768, 2048, 64) == 1
-    assert bench.launches_per_step(W.WORKLOADS["skewed"]) == 1 + 1 + 1 + 2 + 1
+    # I = 1408 = 5 x 256 + 128: GEMM1's last 128 features run as a second, single-CTA launch
+    assert bench.launches_per_step(W.WORKLOADS["skewed"]) == 1 + 1 + 1 + 3 + 1
     # fine-grained at T = 32768: one K range on CTA pairs, gate GEMM and top-k fused
     assert bench.route_ksplit(32768, 4096, 256) == 1
     assert bench.launches_per_step(W.WORKLOADS["fine"].with_tokens(32768)) == 1 + 1 + 1 + 2 + 1
     # a short E = 64 batch splits K, so gate GEMM and top-k run separately
     assert bench.route_ksplit(4096, 2048, 64) == 4
-    assert bench.launches_per_step(W.WORKLOADS["skewed"].with_tokens(4096)) == 2 + 1 + 1 + 2 + 1
+    assert bench.launches_per_step(W.WORKLOADS["skewed"].with_tokens(4096)) == 2 + 1 + 1 + 3 + 1
     # W8A8: the token rows and the SwiGLU rows are quantised by one launch each
     assert bench.launches_per_step(W.WORKLOADS["fine"], "w8a8") == 9
     # tiny f32: one fused CUDA-core router kernel
