@@ -654,3 +654,44 @@ def test_layer_w8a8_close_to_the_exact_layer():
     assert np.array_equal(quant["topk_idx"], exact["topk_idx"])
     err = np.abs(quant["out"] - exact["out"]).max() / np.abs(exact["out"]).max()
     assert 1e-4 < err < 0.1
+
+
+def _torch_swiglu(xr, wg, wu, wd):
+    """Independent float64 composition with torch's own SiLU: (silu(x Wg) * (x Wu)) Wd."""
+    xt = torch.as_tensor(xr, dtype=torch.float64)
+    g = xt @ torch.as_tensor(wg, dtype=torch.float64)
+    u = xt @ torch.as_tensor(wu, dtype=torch.float64)
+    return (torch.nn.functional.silu(g) * u) @ torch.as_tensor(wd, dtype=torch.float64)
+
+
+def test_grouped_ffn_slots_pinned_per_slot():
+    """grouped_ffn_slots: slot s of expert e holds expert e's SwiGLU FFN of token
+    sorted_ids[s] // k ([P1] step 4), checked slot by slot against a torch composition, on a
+    grouping with drops (so slots and assignments are not the identity). Planted mistakes fail:
+    gate and up exchanged, the expert of the neighbouring range, the assignment index taken as
+    the token."""
+    g = np.random.default_rng(7)
+    T, H, E, k, I = 11, 6, 4, 2, 5
+    x = g.standard_normal((T, H))
+    wg, wu, wd = (g.standard_normal((E, H, I)), g.standard_normal((E, H, I)),
+                  g.standard_normal((E, I, H)))
+    idx = np.stack([g.choice(E, k, replace=False) for _ in range(T)])
+    al = orc.align(idx, E, 4)  # capacity 4 of 5.5 mean: drops
+    assert al["drop_mask"].sum() > 0
+    y = orc.grouped_ffn_slots(x, al["sorted_ids"], al["offsets"], k, wg, wu, wd)
+    offs = al["offsets"]
+
+    def expected(s, e, tok_of=lambda a: a // k, gate=wg, up=wu):
+        a = int(al["sorted_ids"][s])
+        return _torch_swiglu(x[tok_of(a)][None], gate[e], up[e], wd[e])[0].numpy()
+
+    for e in range(E):
+        for s in range(int(offs[e]), int(offs[e + 1])):
+            np.testing.assert_allclose(y[s], expected(s, e), rtol=1e-12, atol=1e-12)
+    # planted mistakes, each caught on at least one slot
+    def differs(fn):
+        return any(not np.allclose(y[s], fn(s, e), rtol=1e-9, atol=1e-9)
+                   for e in range(E) for s in range(int(offs[e]), int(offs[e + 1])))
+    assert differs(lambda s, e: expected(s, e, gate=wu, up=wg))
+    assert differs(lambda s, e: expected(s, (e + 1) % E))
+    assert differs(lambda s, e: expected(s, e, tok_of=lambda a: a % T))
