@@ -410,14 +410,36 @@ class LayerRun:
         return max_over_ranks(a.elapsed_time(b), world, "cuda") / steps
 
     def time_stages(self, steps, warmup, world, local, peaks):
-        """Device-resident timing: total CUDA-event time over `steps` layer calls (max over
-        ranks) and the per-stage times the library records on its stream; returns the layer
-        line's timing keys."""
+        """Device-resident timing. Pass 1: total CUDA-event time over `steps` layer calls (max
+        over ranks), the calls as a user makes them, so each kernel's launch still overlaps
+        the end of the one before it (programmatic dependent launch). Pass 2: the same calls
+        with the per-stage events the library records on its stream; an event between two
+        kernels ends that overlap, so the stage times sum to a little more than pass 1's
+        step. Returns the layer line's timing keys."""
         wl, stream = self.wl, self.stream
         for _ in range(warmup):
             self.step()
         torch.cuda.synchronize()
         self.ws.check()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clk:
+            t_start.record(stream)
+            for i in range(steps):
+                # an NVTX range per layer call, for timeline profilers
+                torch.cuda.nvtx.range_push(f"moe_layer_forward step {i}")
+                self.step()
+                torch.cuda.nvtx.range_pop()
+            t_end.record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        ms = t_start.elapsed_time(t_end)
+        self.ws.check()
+        ms_max = max_over_ranks(ms, world, "cuda")
+        value = aggregate_throughput(wl.T * steps, world, ms_max / 1e3)
+        # pass 2: per-stage events
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
         ev = [[torch.cuda.Event(enable_timing=True) for _ in STAGES] for _ in range(steps)]
         for e in ev:
@@ -426,27 +448,13 @@ class LayerRun:
         for s in starts:
             s.record(stream)
         torch.cuda.synchronize()
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        barrier(world)
+        for i in range(steps):
+            starts[i].record(stream)
+            L.moe_set_stage_events(ev[i])
+            self.step()
         torch.cuda.synchronize()
-        with ClockSampler(local) as clk:
-            t_start.record(stream)
-            for i in range(steps):
-                starts[i].record(stream)
-                L.moe_set_stage_events(ev[i])
-                # an NVTX range per layer call, for timeline profilers
-                torch.cuda.nvtx.range_push(f"moe_layer_forward step {i}")
-                self.step()
-                torch.cuda.nvtx.range_pop()
-            t_end.record(stream)
-            torch.cuda.synchronize()
         L.moe_set_stage_events(None)
-        barrier(world)
-        ms = t_start.elapsed_time(t_end)
         self.ws.check()
-        ms_max = max_over_ranks(ms, world, "cuda")
-        value = aggregate_throughput(wl.T * steps, world, ms_max / 1e3)
         st_ms = {s: 0.0 for s in STAGES}
         for i in range(steps):
             prev = starts[i]
