@@ -5,8 +5,11 @@
 // [P5] "大模型推理加速200%+？…", section "3.1 Moe Fuse Gate & Softmax TopK": gate + softmax + top-k
 // in one kernel, a warp-level arg-max with the winner erased each round, exp evaluated only for
 // the k selected logits (exp(l - m) / sum over the selection equals the renormalised softmax).
-// With E >= 64 in bf16 the gate GEMM runs on the tensor cores (route_tc.cu) and topk_kernel
-// below does the selection; the CUDA-core kernel further down fuses both for small E.
+// With E >= 64 in bf16 the gate GEMM runs on the tensor cores (route_tc.cu); with the hidden
+// dimension in one K range it also selects, otherwise a kernel below does: topk_kernel (one
+// warp per token) for E > 64, topk_lanes_kernel (G lanes per token) for E <= 64. For smaller E
+// or float32 the CUDA-core kernels further down (route_slab_kernel, route_simt_kernel) compute
+// the logits and select in one pass.
 //
 // Selection rule: the k largest float32 logits, ties to the lower expert index (-0 == +0);
 // listed by descending logit then ascending index. Logits must be finite.
