@@ -378,6 +378,32 @@ class LayerRun:
     def step(self):
         self.forward(self.inp["x"], self.outs)
 
+    def _stage_pass(self, steps):
+        """`steps` layer calls with the library's stage events; mean ms per stage."""
+        stream = self.stream
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in STAGES] for _ in range(steps)]
+        for e in ev:
+            for x in e:
+                x.record(stream)
+        for s in starts:
+            s.record(stream)
+        torch.cuda.synchronize()
+        for i in range(steps):
+            starts[i].record(stream)
+            L.moe_set_stage_events(ev[i])
+            self.step()
+        torch.cuda.synchronize()
+        L.moe_set_stage_events(None)
+        self.ws.check()
+        st_ms = {s: 0.0 for s in STAGES}
+        for i in range(steps):
+            prev = starts[i]
+            for j, s in enumerate(STAGES):
+                st_ms[s] += prev.elapsed_time(ev[i][j]) / steps
+                prev = ev[i][j]
+        return st_ms
+
     def graph_time(self, steps, warmup, world):
         """The same layer call captured once in a CUDA graph (on a side stream) and replayed
         per step, as a serving loop for short batches would run it: the launches' host cost and
@@ -410,17 +436,19 @@ class LayerRun:
         return max_over_ranks(a.elapsed_time(b), world, "cuda") / steps
 
     def time_stages(self, steps, warmup, world, local, peaks):
-        """Device-resident timing. Pass 1: total CUDA-event time over `steps` layer calls (max
-        over ranks), the calls as a user makes them, so each kernel's launch still overlaps
-        the end of the one before it (programmatic dependent launch). Pass 2: the same calls
-        with the per-stage events the library records on its stream; an event between two
-        kernels ends that overlap, so the stage times sum to a little more than pass 1's
-        step. Returns the layer line's timing keys."""
+        """Device-resident timing. Pass 1, the timed region: total CUDA-event time over `steps`
+        layer calls (max over ranks), the calls as a user makes them, so each kernel's launch
+        still overlaps the end of the one before it (programmatic dependent launch). Pass 2
+        (once before and once after pass 1, the smaller total kept): the same calls with the
+        per-stage events the library records on its stream; an event between two kernels ends
+        that overlap, so the stage times sum to a little more than pass 1's step. Returns the
+        layer line's timing keys."""
         wl, stream = self.wl, self.stream
         for _ in range(warmup):
             self.step()
         torch.cuda.synchronize()
         self.ws.check()
+        stages_before = self._stage_pass(steps)
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         barrier(world)
@@ -439,28 +467,11 @@ class LayerRun:
         self.ws.check()
         ms_max = max_over_ranks(ms, world, "cuda")
         value = aggregate_throughput(wl.T * steps, world, ms_max / 1e3)
-        # pass 2: per-stage events
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in STAGES] for _ in range(steps)]
-        for e in ev:
-            for x in e:
-                x.record(stream)
-        for s in starts:
-            s.record(stream)
-        torch.cuda.synchronize()
-        for i in range(steps):
-            starts[i].record(stream)
-            L.moe_set_stage_events(ev[i])
-            self.step()
-        torch.cuda.synchronize()
-        L.moe_set_stage_events(None)
-        self.ws.check()
-        st_ms = {s: 0.0 for s in STAGES}
-        for i in range(steps):
-            prev = starts[i]
-            for j, s in enumerate(STAGES):
-                st_ms[s] += prev.elapsed_time(ev[i][j]) / steps
-                prev = ev[i][j]
+        # pass 2, run once before and once after pass 1: per-stage events. A pass disturbed by
+        # something outside the layer (the box's power or clock state) shows as a larger total;
+        # the breakdown reported is the pass with the smaller total.
+        stages_after = self._stage_pass(steps)
+        st_ms = min(stages_before, stages_after, key=lambda d: sum(d.values()))
         cnt = self.outs[3].cpu().numpy()
         fp8 = self.fp8 is not None or self.w8a8 is not None
         # the tensor-core peak of the MMA's own operand type: e4m3 x e4m3 (W8A8) runs at the
@@ -500,6 +511,9 @@ class LayerRun:
                                                     3)},
             "route_align_combine_gbs": round(rac_bytes / rac_t / 1e9, 1),
             "route_align_combine_frac": round(rac_bytes / rac_t / 1e9 / peaks["hbm_gbs"], 3),
+            # per-step sums of the two stage passes (before, after the timed pass), in ms
+            "stage_passes_ms": [round(sum(stages_before.values()), 4),
+                                round(sum(stages_after.values()), 4)],
         }
 
     def release(self):
@@ -636,6 +650,7 @@ def run_ours(args, world, rank, local):
         "route_align_combine_gbs": t["route_align_combine_gbs"],
         "route_align_combine_frac": t["route_align_combine_frac"],
         "kernels": t["kernels"],
+        "stage_passes_ms": t["stage_passes_ms"],
         "e2e": {"value": round(aggregate_throughput(wl.T * args.steps, world, e2e_ms / 1e3), 1),
                 "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "copies": "each step's copies overlap the neighbouring steps' forward passes "
